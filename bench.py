@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Benchmark of the Muon step on B200: GPT-2-small hidden set, full muon_step.
+
+One "step" = one full Muon update (momentum, Frobenius normalisation, five
+Newton-Schulz iterations, scale and apply) of all 72 hidden matrices of GPT-2
+small (12 layers x [4 x 768x768, 768x3072, 3072x768]); bf16 gradients drawn
+iid N(0, 0.01^2), fp32 momentum (beta 0.95, Nesterov), lr 0.05, wd 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` is matrices/s over all ranks with
+inputs resident in HBM; `e2e` repeats the measurement with the gradients
+copied in from pinned host memory and the updated weights copied back every
+step.  Per-kernel device times are taken live with CUDA events on the
+launching stream (the library's timing hooks); `roofline` reports the
+dominant kernel against the measured peaks in MEASURED_PEAKS.json.
+`--impl reference` times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Muon NS-5 matrices/s and TFLOP/s (% of B200 BF16 peak), GPT-2-small set"
+UNIT = "matrices/s"
+WORKLOAD = ("GPT-2-small hidden set: 12 layers x (4x 768x768, 768x3072, 3072x768) = 72 matrices; "
+            "bf16 grads iid N(0,1e-2^2), fp32 momentum beta=0.95 Nesterov, T=5, lr 0.05, wd 0")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+REASON_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+    0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+    0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- workload
+def gpt2_shapes():
+    from newton_schulz_12_b200 import workloads
+    return workloads.gpt2_small_shapes()
+
+
+def nominal_flops(shapes, steps=5):
+    """steps * (4 m^2 n + 2 m^3) per matrix, m = min, n = max."""
+    tot = 0
+    for r, c in shapes:
+        m, n = min(r, c), max(r, c)
+        tot += steps * (4 * m * m * n + 2 * m ** 3)
+    return tot
+
+
+def stage_work(shapes):
+    """Algorithmic work of one launch of each kernel kind over the whole set.
+
+    GEMMs: nominal FLOPs (X X^T: 2 m^2 n, A A: 2 m^3, B X: 2 m^2 n).
+    Memory-bound kernels: bytes that must cross HBM per element -- momentum
+    g(2)+buf(4) read, buf(4) written = 10 B; cast g(2)+buf(4) read, fp32 X(4) +
+    bf16 X(2) written = 12 B; apply W(4)+O(4) read, W(4) written = 12 B.
+    """
+    elems = sum(r * c for r, c in shapes)
+    g = sum(2 * min(r, c) ** 2 * max(r, c) for r, c in shapes)
+    p = sum(2 * min(r, c) ** 3 for r, c in shapes)
+    return {
+        "gram": ("tensor", g), "poly": ("tensor", p), "bx": ("tensor", g),
+        "flat": ("hbm", 10 * elems), "cast": ("hbm", 12 * elems), "out": ("hbm", 12 * elems),
+    }
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, torch_device):
+        self.samples, self.reasons, self.max_mhz, self.err = [], set(), None, None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = f"nvml unavailable: {e}"
+            self.h = None
+
+    def _run(self):
+        nv = self.nvml
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = get_reasons(self.h)
+                for b, name in REASON_BITS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception as e:  # pragma: no cover
+                self.err = str(e)
+                break
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.h is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+               "samples": len(self.samples)}
+        if self.err:
+            out["note"] = self.err
+        return out
+
+
+# ---------------------------------------------------------------- oracle legs
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_matrix_step(shape, idx):
+    """One fp64 oracle Muon step of one GPT-2 hidden matrix (seeded as in the GPU run)."""
+    import numpy as np
+    from newton_schulz_12_b200 import workloads
+    from oracle import muon as oracle
+    Ws, Gs = workloads.muon_set([shape], step=0, grad_seed=1000 + idx, w_seed=2000 + idx)
+    W = Ws[0].double().numpy()
+    g = Gs[0].float().numpy()
+    return oracle.muon_step(W, g, np.zeros(shape), beta=0.95, nesterov=True, lr=0.05, wd=0.0)
+
+
+def cpu_baseline(shapes, budget_s=12.0):
+    """The oracle on whole layers (4 square + wide + tall) until ~budget_s of CPU time."""
+    layer = shapes[:6]
+    done, t0 = 0, time.perf_counter()
+    while True:
+        for i, s in enumerate(layer):
+            oracle_matrix_step(s, i)
+        done += len(layer)
+        if time.perf_counter() - t0 >= budget_s or done >= len(shapes):
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{done // 6} of 12 GPT-2-small layers ({done} of 72 matrices), full Muon "
+                      f"step in fp64 (numpy, BLAS matmul), {dt:.1f} s"}
+
+
+def run_reference(args):
+    """`--impl reference`: the fp64 oracle as it stands, on host cores, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    shapes = gpt2_shapes()
+    layer = shapes[:6]
+    for w in range(args.warmup):
+        oracle_matrix_step(layer[w % 6], w % 6)
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        oracle_matrix_step(layer[k % 6], k % 6)
+    dt = time.perf_counter() - t0
+    value = args.steps / dt
+    cores = _blas_threads()
+    sample = (f"each step = one matrix of GPT-2-small layer 0, cycling through its 6 shapes "
+              f"(4x 768x768, 768x3072, 3072x768), full Muon step in fp64 numpy")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * dt / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "matrices_per_step": 1, "parallelism": "none (host cores)"},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def traffic_record():
+    """Per-launch DRAM bytes of the dominant kernel from a committed ncu summary, if current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for name in rec.get("sources", []):
+        with open(os.path.join(ROOT, name), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec.get("sources_sha256"):
+        return None
+    return rec
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import newton_schulz_12_b200 as nsb
+    from newton_schulz_12_b200 import workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    peaks, peak_src = load_peaks()
+    shapes = gpt2_shapes()
+    counts = [r * c for r, c in shapes]
+    total = sum(counts)
+    offs = [0]
+    for n in counts:
+        offs.append(offs[-1] + n)
+    # one flat allocation per tensor kind; every matrix a view (all 16-byte aligned)
+    Ws, Gs = workloads.muon_set(shapes, step=0)
+    W_flat = torch.empty(total, dtype=torch.float32, device=dev)
+    G_flat = torch.empty(total, dtype=torch.bfloat16, device=dev)
+    M_flat = torch.zeros(total, dtype=torch.float32, device=dev)
+    for i in range(len(shapes)):
+        W_flat[offs[i]:offs[i + 1]].copy_(Ws[i].reshape(-1))
+        G_flat[offs[i]:offs[i + 1]].copy_(Gs[i].reshape(-1))
+    W = [W_flat[offs[i]:offs[i + 1]].view(shapes[i]) for i in range(len(shapes))]
+    G = [G_flat[offs[i]:offs[i + 1]].view(shapes[i]) for i in range(len(shapes))]
+    M = [M_flat[offs[i]:offs[i + 1]].view(shapes[i]) for i in range(len(shapes))]
+    stream = torch.cuda.current_stream(dev)
+
+    plan = nsb.MuonStepPlan(W, G, M, beta=0.95, nesterov=True, lr=0.05, wd=0.0, steps=5)
+
+    def step():
+        plan(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if nsb.muon_get_status(stream) != 0:
+        raise RuntimeError("device status after warm-up: " + nsb.muon_last_error())
+
+    # ---- timed region: inputs resident in HBM
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev) as clocks:
+        nsb.muon_profile_begin()
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    prof = nsb.muon_profile_end()
+    barrier()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if nsb.muon_get_status(stream) != 0:
+        raise RuntimeError("device status after timed region: " + nsb.muon_last_error())
+    launches = sum(n for _, n in prof.values())
+
+    # ---- end to end: pinned host grads in, updated weights out, every step
+    G_host = G_flat.cpu().pin_memory()
+    W_host = torch.empty(total, dtype=torch.float32).pin_memory()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = args.steps
+    barrier()
+    torch.cuda.synchronize(dev)
+    e_start.record(stream)
+    for _ in range(e2e_steps):
+        G_flat.copy_(G_host, non_blocking=True)
+        step()
+        W_host.copy_(W_flat, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e_ms = e_start.elapsed_time(e_end)
+    if world > 1:
+        t = torch.tensor([e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+
+    nmat = len(shapes) * world
+    value = nmat * args.steps / (ms / 1000.0)
+    flops_step = nominal_flops(shapes)
+    tflops = flops_step * world * args.steps / (ms / 1000.0) / 1e12
+
+    # ---- per-kernel roofline from the live event timings (rank 0's)
+    work = stage_work(shapes)
+    kernels = {}
+    for kind, (tot_ms, n) in prof.items():
+        if n == 0:
+            continue
+        per = tot_ms / n
+        entry = {"launches": n, "ms_per_launch": per, "ms_per_step": tot_ms / args.steps}
+        if kind in work:
+            bound, amount = work[kind]
+            if bound == "tensor":
+                ach = amount / (per / 1000.0) / 1e12
+                entry.update(bound="tensor", achieved=ach, unit="TFLOP/s",
+                             frac=ach / peaks["bf16_tflops"])
+            else:
+                ach = amount / (per / 1000.0) / 1e9
+                entry.update(bound="hbm", achieved=ach, unit="GB/s", frac=ach / peaks["hbm_gbs"])
+        kernels[kind] = entry
+    dom = max((k for k in kernels if k in work), key=lambda k: kernels[k]["ms_per_step"])
+    d = kernels[dom]
+    trec = traffic_record()
+    traffic = None
+    if trec and trec.get("kernel_kind") == dom:
+        traffic = trec.get("bytes_per_launch")
+    roofline = {"bound": d["bound"], "achieved": d["achieved"],
+                "peak": peaks["bf16_tflops"] if d["bound"] == "tensor" else peaks["hbm_gbs"],
+                "unit": d["unit"], "frac": d["frac"], "traffic": traffic, "kernel": dom,
+                "peak_source": f"{peak_src} ({'bf16 burst' if d['bound'] == 'tensor' else 'copy'})"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "matrices_per_step": len(shapes) * world,
+                       "parallelism": f"replicas x{world} (one independent 72-matrix set per GPU)",
+                       "l2": "inputs larger than L2 (W 340 MB + momentum 340 MB + grads 170 MB "
+                             "per GPU, plus an 850 MB workspace); no flush"},
+            "tflops": tflops,
+            "pct_of_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
+            "pct_of_bf16_peak_sustained": 100.0 * tflops / peaks["bf16_tflops_sustained"],
+            "roofline": roofline,
+            "kernels": kernels,
+            "gpu_launches": launches,
+            "e2e": {"value": nmat * e2e_steps / (e_ms / 1000.0), "unit": UNIT,
+                    "h2d_bytes_per_step": G_host.numel() * G_host.element_size(),
+                    "d2h_bytes_per_step": W_host.numel() * W_host.element_size()},
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(shapes)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,216 @@
+/*
+ * muon.h -- C ABI of the B200 (sm_100a) Muon update library.
+ *
+ * The Muon optimizer step of the NanoGPT speedrun: each hidden weight
+ * matrix's Nesterov-momentum update is orthogonalised by Newton-Schulz
+ * iteration and then applied ("NanoGPT Speedrun: The Ultimate Guide to
+ * Pushing LLM Training Efficiency to Its Limits", section "Optimizer and
+ * Training Strategy Tuning"); the update is replaced by its nearest
+ * semi-orthogonal matrix through five Newton-Schulz steps ("The NanoGPT
+ * speedrun", paragraph "Six records account for most of the speedup",
+ * record #3).  The iteration is X <- aX + (bA + cA^2)X with A = X X^T, on the
+ * Frobenius-normalised update, transposed so that rows <= cols.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Pointer arrays (X_ptrs, params, grads, ...) are HOST arrays of DEVICE
+ *   pointers.  Each matrix is one contiguous row-major buffer owned by the
+ *   caller; every device pointer must be 16-byte aligned.
+ * - `stream` is a cudaStream_t (NULL = legacy default stream).  All calls are
+ *   asynchronous on it: they validate, enqueue kernels and return.
+ * - Argument and shape errors return a negative muon_status synchronously,
+ *   before anything is enqueued; nothing is modified.  muon_last_error()
+ *   then holds a message (thread-local).
+ * - Errors found on the device (a bounded wait that ran out) are recorded in
+ *   a per-(device, stream) status word and reported by muon_get_status().
+ * - The library owns a workspace per (device, stream), grown on demand with
+ *   stream-ordered allocation and freed by muon_release().  Calls that share a
+ *   stream share the workspace; calls on different streams do not.
+ * - Results are deterministic: no floating-point atomics anywhere, fixed
+ *   reduction orders, so a rerun on the same inputs is bit-identical.
+ */
+#ifndef MUON_B200_H
+#define MUON_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Storage / arithmetic type of muon_ns_orthogonalize's matrices. */
+typedef enum {
+  MUON_BF16 = 0, /* bf16 storage; bf16 tensor-core operands, fp32 accumulate,
+                    fp32 master copy of X between steps */
+  MUON_FP32 = 1  /* fp32 storage; fp32 SIMT FMA verification path */
+} muon_dtype;
+
+typedef enum {
+  MUON_OK = 0,
+  MUON_ERR_ARG = -1,            /* null pointer, bad count/steps/dtype, misaligned */
+  MUON_ERR_SHAPE = -2,          /* non-positive or too large dimensions */
+  MUON_ERR_CUDA = -3,           /* a CUDA runtime call failed (message has the name) */
+  MUON_ERR_ALLOC = -4,          /* workspace allocation failed */
+  MUON_ERR_DEVICE_TIMEOUT = -5, /* a bounded device-side wait ran out */
+  MUON_ERR_UNSUPPORTED = -6     /* device is not sm_100 or feature not built */
+} muon_status;
+
+/*
+ * muon_ns_orthogonalize -- Newton-Schulz orthogonalisation of a batch, in place.
+ *
+ * Source: "The NanoGPT speedrun", paragraph "Six records account for most of
+ * the speedup" (nearest semi-orthogonal matrix through five Newton-Schulz
+ * steps); the form X <- aX + (bA + cA^2)X is the library's specification.
+ *
+ * batch   number of matrices (>= 0; 0 is a no-op).
+ * m, n    rows and columns of EVERY matrix (1 <= m, n <= 32768).  When m > n
+ *         the matrix is processed as its transpose (a view; no copy is made
+ *         in the caller's memory) and written back in its own layout.
+ * X_ptrs  host array of `batch` device pointers, each to an m x n row-major
+ *         matrix of bf16 (dtype MUON_BF16) or fp32 (MUON_FP32).  On return
+ *         (stream order) each holds NS(X / (||X||_F + 1e-7)) after `steps`
+ *         iterations, rounded to the storage type.
+ * a, b, c coefficients of the quintic; the speedrun's are 3.4445, -4.7750, 2.0315.
+ * steps   number of iterations T (0 <= steps <= 100; 0 = normalise only).
+ * dtype   a muon_dtype.
+ * Returns MUON_OK or a negative muon_status.
+ */
+int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a, float b,
+                          float c, int steps, int dtype, void* stream);
+
+/*
+ * muon_step -- one full Muon optimizer step over `count` hidden matrices.
+ *
+ * Source: "NanoGPT Speedrun: The Ultimate Guide...", section "Optimizer and
+ * Training Strategy Tuning" (orthogonalise after a Nesterov-momentum update;
+ * hidden matrices only) and "The NanoGPT speedrun", record #3 (T = 5).
+ *
+ * Per matrix i with shape (r, s) = (shapes[2i], shapes[2i+1]):
+ *   buf' = beta*buf + (1-beta)*g                       (fp32, written in place)
+ *   u    = (1-beta)*g + beta*buf'   if nesterov, else buf'
+ *   X0   = u / (||u||_F + 1e-7), transposed when r > s
+ *   X    = NS(X0) with (a,b,c) = (3.4445, -4.7750, 2.0315), `steps` iterations
+ *   W'   = (W - fl(lr*wd)*W) - fl(lr*scale)*O,   O = X in (r, s) layout,
+ *          scale = sqrt(max(1, r/s)) in fp32      (fp32, written in place)
+ * params         host array of device pointers to fp32 W (r x s, row-major).
+ * grads          host array of device pointers to bf16 g (r x s).
+ * momentum_bufs  host array of device pointers to fp32 buf (r x s).
+ * shapes         host array of 2*count int64: rows, cols of each matrix.
+ * Matrices of equal (min, max) dimensions are batched into one group; any mix
+ * of shapes is accepted.  Returns MUON_OK or a negative muon_status.
+ */
+int muon_step(int count, float* const* params, const void* const* grads,
+              float* const* momentum_bufs, const int64_t* shapes, float beta, int nesterov,
+              float lr, float wd, int steps, void* stream);
+
+/*
+ * muon_momentum -- the momentum stage of muon_step on its own.
+ *
+ * Source: "Nesterov momentum" in "NanoGPT Speedrun: The Ultimate Guide...",
+ * section "Optimizer and Training Strategy Tuning" (lerp reading, as in
+ * muon_step).  Writes buf' in place, bit-exact with the fp32 order
+ *   buf' = fl(fl(beta*buf) + fl(fl(1-beta)*g)),
+ * and, if `sumsq_out` is not NULL, sumsq_out[i] = sum of u^2 over matrix i
+ * (fp32, fixed two-stage order; u as in muon_step).  sumsq_out is a DEVICE
+ * pointer to `count` floats.
+ */
+int muon_momentum(int count, const void* const* grads, float* const* momentum_bufs,
+                  const int64_t* shapes, float beta, int nesterov, float* sumsq_out,
+                  void* stream);
+
+/*
+ * muon_apply -- the apply stage of muon_step on its own.
+ *
+ * W' = fl(fl(W - fl(fl(lr*wd)*W)) - fl(fl(lr*scale)*O)), scale as in
+ * muon_step, all fp32 with no fused multiply-add.  updates[i] is a device
+ * pointer to the fp32 update O (r x s, same layout as W).
+ */
+int muon_apply(int count, float* const* params, const float* const* updates,
+               const int64_t* shapes, float lr, float wd, void* stream);
+
+/*
+ * Stage calls on contiguous bf16 batches (the tensor-core kernels of the
+ * iteration, exposed for testing and for callers that run their own loop).
+ * Every pointer is a DEVICE pointer to `batch` contiguous row-major matrices;
+ * m and k (or n) must be multiples of 8 (16-byte row strides for the bulk
+ * tensor copies).
+ *
+ * muon_gram_bf16:  A = X X^T          X: batch x m x k bf16, A: batch x m x m bf16.
+ *                  Only upper 128x128 tiles are computed; A is exactly symmetric.
+ * muon_poly_bf16:  B = b*A + c*(A A)   A, B: batch x m x m bf16, A symmetric.
+ * muon_bx_bf16:    X' = a*X + B X      B: m x m bf16; Xb: bf16 operand copy of X;
+ *                  Xf: fp32 master X (read, then overwritten by X');
+ *                  Xb_out: bf16 copy of X' (must not alias Xb).
+ */
+int muon_gram_bf16(int batch, int m, int k, const void* X, void* A, void* stream);
+int muon_poly_bf16(int batch, int m, const void* A, void* B, float b, float c, void* stream);
+int muon_bx_bf16(int batch, int m, int n, const void* B, const void* Xb, float* Xf,
+                 void* Xb_out, float a, void* stream);
+
+/*
+ * muon_get_status -- synchronise `stream`, then return and clear the device
+ * status word of (current device, stream): MUON_OK or MUON_ERR_DEVICE_TIMEOUT,
+ * or MUON_ERR_CUDA if the synchronisation itself failed.
+ */
+int muon_get_status(void* stream);
+
+/* Thread-local message of the last failed call on this thread ("" if none). */
+const char* muon_last_error(void);
+
+/*
+ * muon_release -- synchronise the device and free every workspace and status
+ * word the library holds on the current device.  Safe to call at any time
+ * outside stream capture; later calls re-allocate on demand.
+ */
+int muon_release(void);
+
+/*
+ * muon_set_wait_timeout_ms -- limit of every device-side wait (default 2000 ms).
+ * A wait that runs out records MUON_ERR_DEVICE_TIMEOUT, the kernel drains
+ * what it has in flight, frees its tensor memory and returns.
+ */
+int muon_set_wait_timeout_ms(int ms);
+
+/*
+ * muon_set_fault_injection -- host-controlled fault injection for tests.
+ * mode 0: off.  mode 1: the next tensor-core GEMM launch withholds one
+ * operand copy, so one device wait runs out and the timeout path is taken.
+ * The mode resets to 0 after one launch.
+ */
+int muon_set_fault_injection(int mode);
+
+/*
+ * Kernel timing for measurement harnesses (off by default).
+ *
+ * muon_profile_begin: from now on every kernel this library launches is
+ *   bracketed by two CUDA events recorded on the stream it is launched on
+ *   (previous records are discarded).
+ * muon_profile_end: stop recording, wait for the recorded events, and write,
+ *   for each kernel kind k < kinds, the summed device time in milliseconds to
+ *   total_ms[k] and the number of launches to launches[k] (host arrays of
+ *   `kinds` entries; either may be NULL).  Returns the total launch count or a
+ *   negative muon_status.
+ */
+typedef enum {
+  MUON_KERNEL_FLAT = 0, /* momentum / sum of squares (flat, 128-bit vectors) */
+  MUON_KERNEL_CAST = 1, /* normalise + transpose + cast to the iteration layout */
+  MUON_KERNEL_GRAM = 2, /* tensor cores: A = X X^T */
+  MUON_KERNEL_POLY = 3, /* tensor cores: B = bA + cA^2 */
+  MUON_KERNEL_BX = 4,   /* tensor cores: X' = aX + BX */
+  MUON_KERNEL_OUT = 5,  /* apply / write-back */
+  MUON_KERNEL_SIMT = 6, /* fp32 verification GEMMs */
+  MUON_KERNEL_SUMS = 7, /* per-matrix sums of partials */
+  MUON_KERNEL_KINDS = 8
+} muon_kernel_kind;
+
+int muon_profile_begin(void);
+int muon_profile_end(int kinds, double* total_ms, int* launches);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int muon_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_B200_H */

@@ -1,0 +1,242 @@
+"""Muon update (Newton-Schulz orthogonalisation) for B200 / sm_100a.
+
+Thin binding over the C ABI of ``libmuon_b200.so`` (include/muon.h): argument
+marshalling only -- every step of the update runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.
+
+The update is the Muon step of the NanoGPT speedrun: orthogonalise each hidden
+matrix's Nesterov-momentum update by Newton-Schulz iteration, then apply it
+("NanoGPT Speedrun: The Ultimate Guide to Pushing LLM Training Efficiency to Its
+Limits", section "Optimizer and Training Strategy Tuning"; "The NanoGPT
+speedrun", paragraph "Six records account for most of the speedup", record #3).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import MUON_BF16, MUON_FP32, MuonError, check, ptr_array, shape_array
+
+__all__ = [
+    "NS_COEFFS", "MuonError", "MuonStepPlan", "muon_ns_orthogonalize", "muon_step", "muon_momentum",
+    "muon_apply", "muon_gram_bf16", "muon_poly_bf16", "muon_bx_bf16", "muon_get_status",
+    "muon_last_error", "muon_release", "muon_set_wait_timeout_ms", "muon_set_fault_injection",
+    "muon_profile_begin", "muon_profile_end", "muon_version", "MUON_BF16", "MUON_FP32",
+]
+
+#: Default quintic coefficients (a, b, c) of X <- aX + (bA + cA^2)X.
+NS_COEFFS = (3.4445, -4.7750, 2.0315)
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check_cuda(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def muon_ns_orthogonalize(xs, a=NS_COEFFS[0], b=NS_COEFFS[1], c=NS_COEFFS[2], steps=5,
+                          stream=None):
+    """Orthogonalise every matrix of ``xs`` in place (list of equal-shape CUDA tensors).
+
+    bf16 tensors take the tensor-core path; fp32 tensors take the fp32 SIMT
+    verification path.  Returns ``xs``.
+    """
+    xs = list(xs)
+    if not xs:
+        return xs
+    shape, dtype = tuple(xs[0].shape), xs[0].dtype
+    if len(shape) != 2:
+        raise ValueError("matrices must be 2-D")
+    if dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("matrices must be bf16 or fp32")
+    for i, x in enumerate(xs):
+        _check_cuda(x, f"xs[{i}]", dtype)
+        if tuple(x.shape) != shape:
+            raise ValueError("all matrices must have the same shape")
+    mode = MUON_BF16 if dtype == torch.bfloat16 else MUON_FP32
+    arr = ptr_array([x.data_ptr() for x in xs])
+    check(_lib.lib().muon_ns_orthogonalize(len(xs), shape[0], shape[1], arr, a, b, c, steps, mode,
+                                           _stream(stream)))
+    return xs
+
+
+def muon_step(params, grads, momentum_bufs, beta=0.95, nesterov=True, lr=0.05, wd=0.0, steps=5,
+              stream=None):
+    """One Muon step: fp32 ``params`` and ``momentum_bufs`` updated in place from bf16 ``grads``."""
+    params, grads, bufs = list(params), list(grads), list(momentum_bufs)
+    if not (len(params) == len(grads) == len(bufs)):
+        raise ValueError("params, grads and momentum_bufs must have the same length")
+    shapes = []
+    for i, (w, g, m) in enumerate(zip(params, grads, bufs)):
+        _check_cuda(w, f"params[{i}]", torch.float32)
+        _check_cuda(g, f"grads[{i}]", torch.bfloat16)
+        _check_cuda(m, f"momentum_bufs[{i}]", torch.float32)
+        if w.dim() != 2 or w.shape != g.shape or w.shape != m.shape:
+            raise ValueError(f"matrix {i}: params, grads and buffers must be equal 2-D shapes")
+        shapes.append(tuple(w.shape))
+    check(_lib.lib().muon_step(len(params), ptr_array([w.data_ptr() for w in params]),
+                               ptr_array([g.data_ptr() for g in grads]),
+                               ptr_array([m.data_ptr() for m in bufs]), shape_array(shapes),
+                               beta, int(bool(nesterov)), lr, wd, steps, _stream(stream)))
+
+
+class MuonStepPlan:
+    """muon_step with its arguments marshalled once, for a fixed set of tensors.
+
+    Checks dtypes, shapes and contiguity at construction; each call then passes
+    the cached pointer arrays straight to the C ABI.  The tensors must stay
+    alive and keep their storage while the plan is used.
+    """
+
+    def __init__(self, params, grads, momentum_bufs, beta=0.95, nesterov=True, lr=0.05, wd=0.0,
+                 steps=5):
+        self.params, self.grads, self.bufs = list(params), list(grads), list(momentum_bufs)
+        if not (len(self.params) == len(self.grads) == len(self.bufs)):
+            raise ValueError("params, grads and momentum_bufs must have the same length")
+        shapes = []
+        for i, (w, g, m) in enumerate(zip(self.params, self.grads, self.bufs)):
+            _check_cuda(w, f"params[{i}]", torch.float32)
+            _check_cuda(g, f"grads[{i}]", torch.bfloat16)
+            _check_cuda(m, f"momentum_bufs[{i}]", torch.float32)
+            if w.dim() != 2 or w.shape != g.shape or w.shape != m.shape:
+                raise ValueError(f"matrix {i}: params, grads and buffers must be equal 2-D shapes")
+            shapes.append(tuple(w.shape))
+        self.shapes = shapes
+        self._p = ptr_array([w.data_ptr() for w in self.params])
+        self._g = ptr_array([g.data_ptr() for g in self.grads])
+        self._m = ptr_array([m.data_ptr() for m in self.bufs])
+        self._s = shape_array(shapes)
+        self._hyper = (float(beta), int(bool(nesterov)), float(lr), float(wd), int(steps))
+        self._fn = _lib.lib().muon_step
+
+    def __call__(self, stream=None):
+        beta, nest, lr, wd, steps = self._hyper
+        check(self._fn(len(self.params), self._p, self._g, self._m, self._s, beta, nest, lr, wd,
+                       steps, _stream(stream)))
+
+
+def muon_momentum(grads, momentum_bufs, beta=0.95, nesterov=True, sumsq_out=None, stream=None):
+    """Momentum stage alone: buffers updated in place; optional per-matrix sum(u^2) (fp32 CUDA)."""
+    grads, bufs = list(grads), list(momentum_bufs)
+    shapes = []
+    for i, (g, m) in enumerate(zip(grads, bufs)):
+        _check_cuda(g, f"grads[{i}]", torch.bfloat16)
+        _check_cuda(m, f"momentum_bufs[{i}]", torch.float32)
+        if g.shape != m.shape or g.dim() != 2:
+            raise ValueError(f"matrix {i}: grads and buffers must be equal 2-D shapes")
+        shapes.append(tuple(g.shape))
+    out = None
+    if sumsq_out is not None:
+        _check_cuda(sumsq_out, "sumsq_out", torch.float32)
+        if sumsq_out.numel() < len(grads):
+            raise ValueError("sumsq_out is too small")
+        out = sumsq_out.data_ptr()
+    check(_lib.lib().muon_momentum(len(grads), ptr_array([g.data_ptr() for g in grads]),
+                                   ptr_array([m.data_ptr() for m in bufs]), shape_array(shapes),
+                                   beta, int(bool(nesterov)), out, _stream(stream)))
+
+
+def muon_apply(params, updates, lr=0.05, wd=0.0, stream=None):
+    """Apply stage alone: W <- (W - lr*wd*W) - lr*scale*O, fp32, in place."""
+    params, updates = list(params), list(updates)
+    shapes = []
+    for i, (w, o) in enumerate(zip(params, updates)):
+        _check_cuda(w, f"params[{i}]", torch.float32)
+        _check_cuda(o, f"updates[{i}]", torch.float32)
+        if w.shape != o.shape or w.dim() != 2:
+            raise ValueError(f"matrix {i}: params and updates must be equal 2-D shapes")
+        shapes.append(tuple(w.shape))
+    check(_lib.lib().muon_apply(len(params), ptr_array([w.data_ptr() for w in params]),
+                                ptr_array([o.data_ptr() for o in updates]), shape_array(shapes),
+                                lr, wd, _stream(stream)))
+
+
+def muon_gram_bf16(X, A=None, stream=None):
+    """A = X X^T for a contiguous bf16 batch X (batch, m, k); returns A (batch, m, m)."""
+    _check_cuda(X, "X", torch.bfloat16)
+    bsz, m, k = X.shape
+    if A is None:
+        A = torch.empty(bsz, m, m, dtype=torch.bfloat16, device=X.device)
+    _check_cuda(A, "A", torch.bfloat16)
+    check(_lib.lib().muon_gram_bf16(bsz, m, k, X.data_ptr(), A.data_ptr(), _stream(stream)))
+    return A
+
+
+def muon_poly_bf16(A, b=NS_COEFFS[1], c=NS_COEFFS[2], B=None, stream=None):
+    """B = b A + c A A for a contiguous symmetric bf16 batch A (batch, m, m)."""
+    _check_cuda(A, "A", torch.bfloat16)
+    bsz, m, _ = A.shape
+    if B is None:
+        B = torch.empty_like(A)
+    _check_cuda(B, "B", torch.bfloat16)
+    check(_lib.lib().muon_poly_bf16(bsz, m, A.data_ptr(), B.data_ptr(), b, c, _stream(stream)))
+    return B
+
+
+def muon_bx_bf16(B, Xb, Xf, a=NS_COEFFS[0], Xb_out=None, stream=None):
+    """X' = a X + B X: Xf (fp32 master) updated in place; returns the bf16 copy of X'."""
+    _check_cuda(B, "B", torch.bfloat16)
+    _check_cuda(Xb, "Xb", torch.bfloat16)
+    _check_cuda(Xf, "Xf", torch.float32)
+    bsz, m, n = Xb.shape
+    if Xb_out is None:
+        Xb_out = torch.empty_like(Xb)
+    _check_cuda(Xb_out, "Xb_out", torch.bfloat16)
+    check(_lib.lib().muon_bx_bf16(bsz, m, n, B.data_ptr(), Xb.data_ptr(), Xf.data_ptr(),
+                                  Xb_out.data_ptr(), a, _stream(stream)))
+    return Xb_out
+
+
+def muon_get_status(stream=None):
+    """Synchronise the stream and return (and clear) its device status word."""
+    return _lib.lib().muon_get_status(_stream(stream))
+
+
+def muon_last_error():
+    msg = _lib.lib().muon_last_error()
+    return msg.decode() if msg else ""
+
+
+def muon_release():
+    check(_lib.lib().muon_release())
+
+
+def muon_set_wait_timeout_ms(ms):
+    check(_lib.lib().muon_set_wait_timeout_ms(int(ms)))
+
+
+def muon_set_fault_injection(mode):
+    check(_lib.lib().muon_set_fault_injection(int(mode)))
+
+
+def muon_profile_begin():
+    """Start bracketing every library kernel launch with CUDA events."""
+    check(_lib.lib().muon_profile_begin())
+
+
+def muon_profile_end():
+    """Stop timing; returns {kind: (total_ms, launches)} over the recorded launches."""
+    k = len(_lib.KERNEL_KINDS)
+    ms = (ctypes.c_double * k)()
+    n = (ctypes.c_int * k)()
+    rc = _lib.lib().muon_profile_end(k, ms, n)
+    if rc < 0:
+        check(rc)
+    return {name: (ms[i], n[i]) for i, name in enumerate(_lib.KERNEL_KINDS)}
+
+
+def muon_version():
+    return _lib.lib().muon_version()

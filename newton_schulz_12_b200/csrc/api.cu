@@ -1,0 +1,958 @@
+// C ABI of the Muon update library: argument checking, shape grouping,
+// workspace ownership and the launch sequence of one step.
+//
+// Launch sequence of muon_step (all on the caller's stream):
+//   flat_kernel (momentum + partial norms) -> cast_kernel (normalise,
+//   transpose to rows <= cols, fp32 master + bf16 operand) -> T x
+//   [kGram, kPoly, kBx] tensor-core launches over every shape group ->
+//   out_kernel (scale and apply).
+// Sources: "NanoGPT Speedrun: The Ultimate Guide to Pushing LLM Training
+// Efficiency to Its Limits", section "Optimizer and Training Strategy Tuning"
+// (orthogonalise the Nesterov-momentum update of hidden matrices by
+// Newton-Schulz), and "The NanoGPT speedrun", paragraph "Six records account
+// for most of the speedup" (five Newton-Schulz steps, nearest semi-orthogonal
+// matrix).
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "muon.h"
+
+using namespace muon;
+typedef __nv_bfloat16 bf16;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxDim = 32768;
+constexpr int kMaxStepsArg = 100;
+constexpr float kNormEps = 1e-7f;
+constexpr float kCoefA = 3.4445f, kCoefB = -4.7750f, kCoefC = 2.0315f;
+
+thread_local std::string t_err;
+
+int set_err(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return code;
+}
+
+#define CUDA_TRY(call)                                                                     \
+  do {                                                                                     \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess)                                                                 \
+      return set_err(MUON_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));       \
+  } while (0)
+
+#define MUON_TRY(expr)           \
+  do {                           \
+    int r_ = (expr);             \
+    if (r_ != MUON_OK) return r_; \
+  } while (0)
+
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+  int* status = nullptr;
+};
+
+struct DevInfo {
+  int sms = 0, major = 0, minor = 0;
+};
+
+std::mutex g_mu;
+std::map<std::pair<int, uintptr_t>, Workspace> g_ws;
+std::map<int, DevInfo> g_dev;
+unsigned long long g_timeout_ns = 2000000000ull;
+int g_inject = 0;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int get_encoder() {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  static cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSuccess;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  if (!g_encode)
+    return set_err(MUON_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s, query %d)",
+                   cudaGetErrorString(err), static_cast<int>(q));
+  return MUON_OK;
+}
+
+// ------------------------------------------------------------ kernel timing
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+};
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Brackets one launch with events on its stream while timing is on.
+struct ProfScope {
+  int kind;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  ProfScope(int k, cudaStream_t st) : kind(k), s(st) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_prof_on) return;
+    a = take_event();
+    if (a) cudaEventRecord(a, s);
+  }
+  ~ProfScope() {
+    if (!a) return;
+    std::lock_guard<std::mutex> lk(g_mu);
+    cudaEvent_t b = take_event();
+    if (!b) return;
+    cudaEventRecord(b, s);
+    g_prof.push_back({kind, a, b});
+  }
+};
+
+int device_info(DevInfo* out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_dev.find(dev);
+    if (it != g_dev.end()) {
+      *out = it->second;
+      return MUON_OK;
+    }
+  }
+  DevInfo d;
+  CUDA_TRY(cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev));
+  CUDA_TRY(cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev));
+  CUDA_TRY(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+  if (d.major != 10 || d.minor != 0)
+    return set_err(MUON_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                   dev, d.major, d.minor);
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_dev[dev] = d;
+  *out = d;
+  return MUON_OK;
+}
+
+// Workspace of (current device, stream), grown stream-ordered to >= need bytes.
+int get_workspace(cudaStream_t s, size_t need, Workspace** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[{dev, reinterpret_cast<uintptr_t>(s)}];
+  if (!w.status) {
+    CUDA_TRY(cudaMalloc(&w.status, 256));
+    CUDA_TRY(cudaMemset(w.status, 0, 256));
+  }
+  if (w.bytes < need) {
+    if (w.ptr) {
+      CUDA_TRY(cudaFreeAsync(w.ptr, s));
+      w.ptr = nullptr;
+      w.bytes = 0;
+    }
+    size_t nb = std::max(need, static_cast<size_t>(1) << 21);
+    nb = (nb + (static_cast<size_t>(1) << 21) - 1) & ~((static_cast<size_t>(1) << 21) - 1);
+    cudaError_t e = cudaMallocAsync(&w.ptr, nb, s);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      w.ptr = nullptr;
+      return set_err(MUON_ERR_ALLOC, "workspace of %zu bytes: %s", nb, cudaGetErrorString(e));
+    }
+    w.bytes = nb;
+  }
+  *out = &w;
+  return MUON_OK;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline long long round8(long long x) { return (x + 7) / 8 * 8; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+int make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
+             uint64_t ld, uint64_t mat_stride, uint32_t box_inner, uint32_t box_rows) {
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {ld * 2, mat_stride * 2};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return set_err(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %llux%llux%llu ld %llu",
+                   static_cast<int>(r), (unsigned long long)inner, (unsigned long long)rows,
+                   (unsigned long long)batch, (unsigned long long)ld);
+  return MUON_OK;
+}
+
+// One shape class of the iteration: `batch` matrices X (m x n, m <= n) laid
+// out contiguously in the workspace with padded row strides.
+struct NsGroup {
+  int batch = 0, m = 0, n = 0;
+  long long ldn = 0, ldm = 0;
+  float* xf = nullptr;          // fp32 master X (bf16 path) / ping buffer (fp32 path)
+  float* xf1 = nullptr;         // fp32 pong buffer (fp32 path)
+  bf16* xb[2] = {nullptr, nullptr};
+  bf16* A = nullptr;
+  bf16* B = nullptr;
+  float* Af = nullptr;
+  float* Bf = nullptr;
+};
+
+// Bytes of workspace a group needs; assigns its offsets from `base` (or counts
+// only, when base is null).
+size_t layout_group(NsGroup& g, char* base, size_t off, bool fp32) {
+  g.ldn = round8(g.n);
+  g.ldm = round8(g.m);
+  const size_t xe = static_cast<size_t>(g.batch) * g.m * g.ldn;
+  const size_t ae = static_cast<size_t>(g.batch) * g.m * g.ldm;
+  auto take = [&](size_t bytes) {
+    off = align_up(off, 1024);
+    char* p = base ? base + off : nullptr;
+    off += bytes;
+    return p;
+  };
+  if (!fp32) {
+    g.xf = reinterpret_cast<float*>(take(xe * 4));
+    g.xb[0] = reinterpret_cast<bf16*>(take(xe * 2));
+    g.xb[1] = reinterpret_cast<bf16*>(take(xe * 2));
+    g.A = reinterpret_cast<bf16*>(take(ae * 2));
+    g.B = reinterpret_cast<bf16*>(take(ae * 2));
+  } else {
+    g.xf = reinterpret_cast<float*>(take(xe * 4));
+    g.xf1 = reinterpret_cast<float*>(take(xe * 4));
+    g.Af = reinterpret_cast<float*>(take(ae * 4));
+    g.Bf = reinterpret_cast<float*>(take(ae * 4));
+  }
+  return off;
+}
+
+tc::Group tc_group(int batch, int m, int n, int k, bool sym, int tile_begin, long long ld,
+                   long long mat_stride, void* d, const void* e, float* xf) {
+  tc::Group G{};
+  G.batch = batch;
+  G.m = m;
+  G.n = n;
+  G.k = k;
+  G.tiles_m = (m + tc::BM - 1) / tc::BM;
+  G.tiles_n = sym ? G.tiles_m : (n + tc::BN - 1) / tc::BN;
+  G.tiles_per_mat = sym ? G.tiles_m * (G.tiles_m + 1) / 2 : G.tiles_m * G.tiles_n;
+  G.tile_begin = tile_begin;
+  G.ld = ld;
+  G.mat_stride = mat_stride;
+  G.d = d;
+  G.e = e;
+  G.xf = xf;
+  return G;
+}
+
+void init_tc_params(tc::Params& P, int* status, float a, float b, float c) {
+  P.ngroups = 0;
+  P.total_tiles = 0;
+  P.a = a;
+  P.b = b;
+  P.c = c;
+  P.status = status;
+  P.timeout_ns = g_timeout_ns;
+  P.inject = 0;
+}
+
+int launch_tc(int epi, tc::Params& P, int sms, cudaStream_t s) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_inject) {
+      P.inject = g_inject;
+      g_inject = 0;
+    }
+  }
+  const int grid = std::min(P.total_tiles, sms);
+  ProfScope prof(MUON_KERNEL_GRAM + epi, s);
+  CUDA_TRY(tc::launch(epi, P, grid, s));
+  P.inject = 0;
+  return MUON_OK;
+}
+
+// T steps of X <- aX + (bA + cA^2)X on bf16 operands with fp32 master X.
+// On entry each group's xf / xb[0] hold X0; on exit xf holds X_T.
+int run_ns_bf16(std::vector<NsGroup>& gs, int steps, float a, float b, float c, int* status,
+                int sms, cudaStream_t s) {
+  if (steps <= 0 || gs.empty()) return MUON_OK;
+  MUON_TRY(get_encoder());
+  for (size_t g0 = 0; g0 < gs.size(); g0 += tc::kMaxGroups) {
+    const size_t g1 = std::min(gs.size(), g0 + tc::kMaxGroups);
+    tc::Params gram[2], poly, bx[2];
+    for (int par = 0; par < 2; ++par) {
+      init_tc_params(gram[par], status, a, b, c);
+      init_tc_params(bx[par], status, a, b, c);
+    }
+    init_tc_params(poly, status, a, b, c);
+    for (size_t gi = g0; gi < g1; ++gi) {
+      NsGroup& G = gs[gi];
+      const int k = static_cast<int>(gi - g0);
+      const long long xs = static_cast<long long>(G.m) * G.ldn;
+      const long long as = static_cast<long long>(G.m) * G.ldm;
+      for (int par = 0; par < 2; ++par) {
+        gram[par].grp[k] = tc_group(G.batch, G.m, G.m, G.n, true, gram[par].total_tiles, G.ldm,
+                                    as, G.A, nullptr, nullptr);
+        MUON_TRY(make_map(&gram[par].map_p[k], G.xb[par], G.n, G.m, G.batch, G.ldn, xs, 64, 128));
+        gram[par].map_q[k] = gram[par].map_p[k];
+        gram[par].total_tiles += G.batch * gram[par].grp[k].tiles_per_mat;
+        gram[par].ngroups = k + 1;
+
+        bx[par].grp[k] = tc_group(G.batch, G.m, G.n, G.m, false, bx[par].total_tiles, G.ldn, xs,
+                                  G.xb[par ^ 1], nullptr, G.xf);
+        MUON_TRY(make_map(&bx[par].map_p[k], G.B, G.m, G.m, G.batch, G.ldm, as, 64, 128));
+        MUON_TRY(make_map(&bx[par].map_q[k], G.xb[par], G.n, G.m, G.batch, G.ldn, xs, 64, 64));
+        bx[par].total_tiles += G.batch * bx[par].grp[k].tiles_per_mat;
+        bx[par].ngroups = k + 1;
+      }
+      poly.grp[k] = tc_group(G.batch, G.m, G.m, G.m, true, poly.total_tiles, G.ldm, as, G.B, G.A,
+                             nullptr);
+      MUON_TRY(make_map(&poly.map_p[k], G.A, G.m, G.m, G.batch, G.ldm, as, 64, 128));
+      poly.map_q[k] = poly.map_p[k];
+      poly.total_tiles += G.batch * poly.grp[k].tiles_per_mat;
+      poly.ngroups = k + 1;
+    }
+    int cur = 0;
+    for (int t = 0; t < steps; ++t) {
+      MUON_TRY(launch_tc(tc::kGram, gram[cur], sms, s));
+      MUON_TRY(launch_tc(tc::kPoly, poly, sms, s));
+      MUON_TRY(launch_tc(tc::kBx, bx[cur], sms, s));
+      cur ^= 1;
+    }
+  }
+  return MUON_OK;
+}
+
+// fp32 SIMT verification path; on exit *final_xf of each group holds X_T.
+int run_ns_fp32(std::vector<NsGroup>& gs, int steps, float a, float b, float c, cudaStream_t s,
+                std::vector<float*>& final_xf) {
+  final_xf.clear();
+  for (NsGroup& G : gs) {
+    float* x[2] = {G.xf, G.xf1};
+    int cur = 0;
+    const long long xs = static_cast<long long>(G.m) * G.ldn;
+    const long long as = static_cast<long long>(G.m) * G.ldm;
+    for (int t = 0; t < steps; ++t) {
+      simt::Params p{};
+      p.batch = G.batch;
+      p.a = a;
+      p.b = b;
+      p.c = c;
+      // A = X X^T
+      p.m = G.m; p.n = G.m; p.k = G.n;
+      p.P = x[cur]; p.ldp = G.ldn; p.sp = xs;
+      p.Q = x[cur]; p.ldq = G.ldn; p.sq = xs;
+      p.E = nullptr; p.lde = 0; p.se = 0;
+      p.D = G.Af; p.ldd = G.ldm; p.sd = as;
+      {
+        ProfScope prof(MUON_KERNEL_SIMT, s);
+        CUDA_TRY(simt::launch(simt::kGram, p, s));
+      }
+      // B = bA + c A A
+      p.k = G.m;
+      p.P = G.Af; p.ldp = G.ldm; p.sp = as;
+      p.Q = G.Af; p.ldq = G.ldm; p.sq = as;
+      p.E = G.Af; p.lde = G.ldm; p.se = as;
+      p.D = G.Bf;
+      {
+        ProfScope prof(MUON_KERNEL_SIMT, s);
+        CUDA_TRY(simt::launch(simt::kPoly, p, s));
+      }
+      // X' = aX + B X
+      p.n = G.n; p.k = G.m;
+      p.P = G.Bf; p.ldp = G.ldm; p.sp = as;
+      p.Q = x[cur]; p.ldq = G.ldn; p.sq = xs;
+      p.E = x[cur]; p.lde = G.ldn; p.se = xs;
+      p.D = x[cur ^ 1]; p.ldd = G.ldn; p.sd = xs;
+      {
+        ProfScope prof(MUON_KERNEL_SIMT, s);
+        CUDA_TRY(simt::launch(simt::kBx, p, s));
+      }
+      cur ^= 1;
+    }
+    final_xf.push_back(x[cur]);
+  }
+  return MUON_OK;
+}
+
+bool finite(float v) { return std::isfinite(v); }
+
+struct MatInfo {
+  int rows, cols, m, n, transposed, group, index;
+};
+
+// Group matrices by (m, n) = (min, max); larger n first (longer K in kGram).
+void group_shapes(const std::vector<std::pair<int, int>>& shapes, std::vector<MatInfo>& mats,
+                  std::vector<NsGroup>& groups) {
+  std::map<std::pair<int, int>, int, std::greater<std::pair<int, int>>> key;
+  mats.resize(shapes.size());
+  for (size_t i = 0; i < shapes.size(); ++i) {
+    MatInfo& M = mats[i];
+    M.rows = shapes[i].first;
+    M.cols = shapes[i].second;
+    M.transposed = M.rows > M.cols;
+    M.m = std::min(M.rows, M.cols);
+    M.n = std::max(M.rows, M.cols);
+    key.emplace(std::make_pair(M.n, M.m), 0);
+  }
+  groups.clear();
+  for (auto& kv : key) {
+    kv.second = static_cast<int>(groups.size());
+    NsGroup g;
+    g.n = kv.first.first;
+    g.m = kv.first.second;
+    groups.push_back(g);
+  }
+  for (size_t i = 0; i < shapes.size(); ++i) {
+    MatInfo& M = mats[i];
+    M.group = key[std::make_pair(M.n, M.m)];
+    M.index = groups[M.group].batch++;
+  }
+}
+
+// Flat momentum / sum-of-squares pass over matrices [i0, i1) of `srcs`.
+int launch_flat_chunked(const std::vector<const void*>& srcs, const std::vector<float*>& bufs,
+                        const std::vector<long long>& numels, int src_kind, float beta,
+                        int nesterov, float* partials, std::vector<int>& part_begin,
+                        std::vector<int>& part_count, cudaStream_t s) {
+  const int count = static_cast<int>(srcs.size());
+  part_begin.assign(count, 0);
+  part_count.assign(count, 0);
+  int global_blk = 0;
+  for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
+    const int i1 = std::min(count, i0 + ew::kMaxMats);
+    ew::FlatParams fp{};
+    fp.src_kind = src_kind;
+    fp.beta = beta;
+    fp.omb = 1.0f - beta;
+    fp.nesterov = nesterov;
+    fp.partials = partials + global_blk;
+    int blk = 0;
+    for (int i = i0; i < i1; ++i) {
+      ew::FlatMat& F = fp.mat[i - i0];
+      F.src = srcs[i];
+      F.buf = bufs.empty() ? nullptr : bufs[i];
+      F.numel = numels[i];
+      F.blk_begin = blk;
+      const int nb = static_cast<int>((numels[i] + ew::kFlatChunk - 1) / ew::kFlatChunk);
+      part_begin[i] = global_blk + blk;
+      part_count[i] = nb;
+      blk += nb;
+    }
+    fp.nmat = i1 - i0;
+    fp.nblocks = blk;
+    ProfScope prof(MUON_KERNEL_FLAT, s);
+    CUDA_TRY(ew::launch_flat(fp, s));
+    global_blk += blk;
+  }
+  return MUON_OK;
+}
+
+int count_flat_blocks(const std::vector<long long>& numels) {
+  long long nb = 0;
+  for (long long n : numels) nb += (n + ew::kFlatChunk - 1) / ew::kFlatChunk;
+  return static_cast<int>(nb);
+}
+
+// Normalise (+ transpose) every matrix into its group's workspace buffers.
+int launch_cast_chunked(const std::vector<MatInfo>& mats, std::vector<NsGroup>& groups,
+                        const std::vector<const void*>& src0, const std::vector<const float*>& src1,
+                        int src_kind, float beta, int nesterov, const float* partials,
+                        const std::vector<int>& part_begin, const std::vector<int>& part_count,
+                        bool with_bf16, cudaStream_t s) {
+  const int count = static_cast<int>(mats.size());
+  for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
+    const int i1 = std::min(count, i0 + ew::kMaxMats);
+    ew::CastParams cp{};
+    cp.src_kind = src_kind;
+    cp.beta = beta;
+    cp.omb = 1.0f - beta;
+    cp.nesterov = nesterov;
+    cp.eps = kNormEps;
+    cp.partials = partials;
+    int tiles = 0;
+    for (int i = i0; i < i1; ++i) {
+      const MatInfo& M = mats[i];
+      const NsGroup& G = groups[M.group];
+      ew::CastMat& C = cp.mat[i - i0];
+      C.src0 = src0[i];
+      C.src1 = src1.empty() ? nullptr : src1[i];
+      C.rows = M.rows;
+      C.cols = M.cols;
+      C.transposed = M.transposed;
+      C.tiles_n = (M.n + ew::kTile - 1) / ew::kTile;
+      C.tile_begin = tiles;
+      C.part_begin = part_begin[i];
+      C.part_count = part_count[i];
+      const long long off = static_cast<long long>(M.index) * G.m * G.ldn;
+      C.xf = G.xf + off;
+      C.xb = with_bf16 ? static_cast<void*>(G.xb[0] + off) : nullptr;
+      C.ld = G.ldn;
+      tiles += ((M.m + ew::kTile - 1) / ew::kTile) * C.tiles_n;
+    }
+    cp.nmat = i1 - i0;
+    cp.ntiles = tiles;
+    ProfScope prof(MUON_KERNEL_CAST, s);
+    CUDA_TRY(ew::launch_cast(cp, s));
+  }
+  return MUON_OK;
+}
+
+// mode 0: apply into W; 1: bf16 write-back; 2: fp32 write-back.  O of matrix i
+// is read from its group's buffer `final_xf[group]` (X layout, transposed back).
+int launch_out_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGroup>& groups,
+                       const std::vector<float*>& final_xf, const std::vector<void*>& ys, int mode,
+                       float lr, float wd, cudaStream_t s) {
+  const int count = static_cast<int>(mats.size());
+  for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
+    const int i1 = std::min(count, i0 + ew::kMaxMats);
+    ew::OutParams op{};
+    op.mode = mode;
+    op.lw = lr * wd;
+    int tiles = 0;
+    for (int i = i0; i < i1; ++i) {
+      const MatInfo& M = mats[i];
+      const NsGroup& G = groups[M.group];
+      ew::OutMat& O = op.mat[i - i0];
+      O.y = ys[i];
+      O.o = final_xf[M.group] + static_cast<long long>(M.index) * G.m * G.ldn;
+      O.rows = M.rows;
+      O.cols = M.cols;
+      O.o_transposed = M.transposed;
+      O.ld = G.ldn;
+      O.tiles_c = (M.cols + ew::kTile - 1) / ew::kTile;
+      O.tile_begin = tiles;
+      const float ratio = static_cast<float>(M.rows) / static_cast<float>(M.cols);
+      const float scale = ratio > 1.0f ? sqrtf(ratio) : 1.0f;
+      O.ls = lr * scale;
+      tiles += ((M.rows + ew::kTile - 1) / ew::kTile) * O.tiles_c;
+    }
+    op.nmat = i1 - i0;
+    op.ntiles = tiles;
+    ProfScope prof(MUON_KERNEL_OUT, s);
+    CUDA_TRY(ew::launch_out(op, s));
+  }
+  return MUON_OK;
+}
+
+int check_shape(long long r, long long c, int i) {
+  if (r < 1 || c < 1 || r > kMaxDim || c > kMaxDim)
+    return set_err(MUON_ERR_SHAPE, "matrix %d has shape %lldx%lld (each side must be in 1..%d)", i,
+                   r, c, kMaxDim);
+  return MUON_OK;
+}
+
+int check_ptr(const void* p, const char* what, int i) {
+  if (!p) return set_err(MUON_ERR_ARG, "%s[%d] is NULL", what, i);
+  if (!aligned16(p)) return set_err(MUON_ERR_ARG, "%s[%d] is not 16-byte aligned", what, i);
+  return MUON_OK;
+}
+
+}  // namespace
+
+// =============================================================================
+extern "C" {
+
+int muon_version(void) { return kVersion; }
+
+const char* muon_last_error(void) { return t_err.c_str(); }
+
+int muon_set_wait_timeout_ms(int ms) {
+  if (ms < 1 || ms > 600000) return set_err(MUON_ERR_ARG, "timeout %d ms out of range 1..600000", ms);
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_timeout_ns = static_cast<unsigned long long>(ms) * 1000000ull;
+  return MUON_OK;
+}
+
+int muon_set_fault_injection(int mode) {
+  if (mode < 0 || mode > 1) return set_err(MUON_ERR_ARG, "fault injection mode %d unknown", mode);
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_inject = mode;
+  return MUON_OK;
+}
+
+int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a, float b, float c,
+                          int steps, int dtype, void* stream) {
+  t_err.clear();
+  if (batch < 0 || batch > 65535) return set_err(MUON_ERR_ARG, "batch %d out of range 0..65535", batch);
+  if (steps < 0 || steps > kMaxStepsArg) return set_err(MUON_ERR_ARG, "steps %d out of range 0..%d", steps, kMaxStepsArg);
+  if (dtype != MUON_BF16 && dtype != MUON_FP32) return set_err(MUON_ERR_ARG, "dtype %d unknown", dtype);
+  if (!finite(a) || !finite(b) || !finite(c)) return set_err(MUON_ERR_ARG, "coefficients must be finite");
+  MUON_TRY(check_shape(m, n, 0));
+  if (batch == 0) return MUON_OK;
+  if (!X_ptrs) return set_err(MUON_ERR_ARG, "X_ptrs is NULL");
+  for (int i = 0; i < batch; ++i) MUON_TRY(check_ptr(X_ptrs[i], "X_ptrs", i));
+  DevInfo dev;
+  MUON_TRY(device_info(&dev));
+  cudaStream_t s = as_stream(stream);
+  const bool fp32 = (dtype == MUON_FP32);
+
+  std::vector<std::pair<int, int>> shapes(batch, std::make_pair(m, n));
+  std::vector<MatInfo> mats;
+  std::vector<NsGroup> groups;
+  group_shapes(shapes, mats, groups);
+  std::vector<long long> numels(batch, static_cast<long long>(m) * n);
+  const int nblk = count_flat_blocks(numels);
+  size_t off = align_up(static_cast<size_t>(nblk) * 4, 1024);
+  for (NsGroup& g : groups) off = layout_group(g, nullptr, off, fp32);
+  Workspace* ws = nullptr;
+  MUON_TRY(get_workspace(s, off, &ws));
+  char* base = static_cast<char*>(ws->ptr);
+  float* partials = reinterpret_cast<float*>(base);
+  off = align_up(static_cast<size_t>(nblk) * 4, 1024);
+  for (NsGroup& g : groups) off = layout_group(g, base, off, fp32);
+
+  std::vector<const void*> src(X_ptrs, X_ptrs + batch);
+  std::vector<int> pb, pc;
+  const int kind = fp32 ? ew::kFromF32 : ew::kFromBf16;
+  MUON_TRY(launch_flat_chunked(src, {}, numels, kind, 0.f, 0, partials, pb, pc, s));
+  MUON_TRY(launch_cast_chunked(mats, groups, src, {}, kind, 0.f, 0, partials, pb, pc, !fp32, s));
+  std::vector<float*> final_xf;
+  if (fp32) {
+    MUON_TRY(run_ns_fp32(groups, steps, a, b, c, s, final_xf));
+  } else {
+    MUON_TRY(run_ns_bf16(groups, steps, a, b, c, ws->status, dev.sms, s));
+    for (NsGroup& g : groups) final_xf.push_back(g.xf);
+  }
+  std::vector<void*> ys(X_ptrs, X_ptrs + batch);
+  MUON_TRY(launch_out_chunked(mats, groups, final_xf, ys, fp32 ? 2 : 1, 0.f, 0.f, s));
+  return MUON_OK;
+}
+
+int muon_step(int count, float* const* params, const void* const* grads,
+              float* const* momentum_bufs, const int64_t* shapes, float beta, int nesterov,
+              float lr, float wd, int steps, void* stream) {
+  t_err.clear();
+  if (count < 0) return set_err(MUON_ERR_ARG, "count %d < 0", count);
+  if (steps < 0 || steps > kMaxStepsArg) return set_err(MUON_ERR_ARG, "steps %d out of range 0..%d", steps, kMaxStepsArg);
+  if (!finite(beta) || beta < 0.f || beta > 1.f) return set_err(MUON_ERR_ARG, "beta must be in [0, 1]");
+  if (!finite(lr) || !finite(wd)) return set_err(MUON_ERR_ARG, "lr and wd must be finite");
+  if (count == 0) return MUON_OK;
+  if (!params || !grads || !momentum_bufs || !shapes)
+    return set_err(MUON_ERR_ARG, "params, grads, momentum_bufs and shapes must be non-NULL");
+  std::vector<std::pair<int, int>> shp(count);
+  for (int i = 0; i < count; ++i) {
+    MUON_TRY(check_shape(shapes[2 * i], shapes[2 * i + 1], i));
+    shp[i] = std::make_pair(static_cast<int>(shapes[2 * i]), static_cast<int>(shapes[2 * i + 1]));
+    MUON_TRY(check_ptr(params[i], "params", i));
+    MUON_TRY(check_ptr(grads[i], "grads", i));
+    MUON_TRY(check_ptr(momentum_bufs[i], "momentum_bufs", i));
+  }
+  DevInfo dev;
+  MUON_TRY(device_info(&dev));
+  cudaStream_t s = as_stream(stream);
+
+  std::vector<MatInfo> mats;
+  std::vector<NsGroup> groups;
+  group_shapes(shp, mats, groups);
+  std::vector<long long> numels(count);
+  for (int i = 0; i < count; ++i) numels[i] = static_cast<long long>(shp[i].first) * shp[i].second;
+  const int nblk = count_flat_blocks(numels);
+  size_t off = align_up(static_cast<size_t>(nblk) * 4, 1024);
+  for (NsGroup& g : groups) off = layout_group(g, nullptr, off, false);
+  Workspace* ws = nullptr;
+  MUON_TRY(get_workspace(s, off, &ws));
+  char* base = static_cast<char*>(ws->ptr);
+  float* partials = reinterpret_cast<float*>(base);
+  off = align_up(static_cast<size_t>(nblk) * 4, 1024);
+  for (NsGroup& g : groups) off = layout_group(g, base, off, false);
+
+  std::vector<const void*> gsrc(grads, grads + count);
+  std::vector<float*> bufs(momentum_bufs, momentum_bufs + count);
+  std::vector<const float*> cbufs(momentum_bufs, momentum_bufs + count);
+  std::vector<int> pb, pc;
+  MUON_TRY(launch_flat_chunked(gsrc, bufs, numels, ew::kFromMomentum, beta, nesterov, partials, pb,
+                               pc, s));
+  MUON_TRY(launch_cast_chunked(mats, groups, gsrc, cbufs, ew::kFromMomentum, beta, nesterov,
+                               partials, pb, pc, true, s));
+  MUON_TRY(run_ns_bf16(groups, steps, kCoefA, kCoefB, kCoefC, ws->status, dev.sms, s));
+  std::vector<float*> final_xf;
+  for (NsGroup& g : groups) final_xf.push_back(g.xf);
+  std::vector<void*> ys(params, params + count);
+  MUON_TRY(launch_out_chunked(mats, groups, final_xf, ys, 0, lr, wd, s));
+  return MUON_OK;
+}
+
+int muon_momentum(int count, const void* const* grads, float* const* momentum_bufs,
+                  const int64_t* shapes, float beta, int nesterov, float* sumsq_out,
+                  void* stream) {
+  t_err.clear();
+  if (count < 0) return set_err(MUON_ERR_ARG, "count %d < 0", count);
+  if (!finite(beta) || beta < 0.f || beta > 1.f) return set_err(MUON_ERR_ARG, "beta must be in [0, 1]");
+  if (count == 0) return MUON_OK;
+  if (!grads || !momentum_bufs || !shapes) return set_err(MUON_ERR_ARG, "grads, momentum_bufs and shapes must be non-NULL");
+  std::vector<long long> numels(count);
+  for (int i = 0; i < count; ++i) {
+    MUON_TRY(check_shape(shapes[2 * i], shapes[2 * i + 1], i));
+    numels[i] = shapes[2 * i] * shapes[2 * i + 1];
+    MUON_TRY(check_ptr(grads[i], "grads", i));
+    MUON_TRY(check_ptr(momentum_bufs[i], "momentum_bufs", i));
+  }
+  DevInfo dev;
+  MUON_TRY(device_info(&dev));
+  cudaStream_t s = as_stream(stream);
+  const int nblk = count_flat_blocks(numels);
+  Workspace* ws = nullptr;
+  MUON_TRY(get_workspace(s, static_cast<size_t>(nblk) * 4, &ws));
+  float* partials = static_cast<float*>(ws->ptr);
+  std::vector<const void*> gsrc(grads, grads + count);
+  std::vector<float*> bufs(momentum_bufs, momentum_bufs + count);
+  std::vector<int> pb, pc;
+  MUON_TRY(launch_flat_chunked(gsrc, bufs, numels, ew::kFromMomentum, beta, nesterov, partials, pb,
+                               pc, s));
+  if (sumsq_out) {
+    for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
+      const int i1 = std::min(count, i0 + ew::kMaxMats);
+      ew::SumParams sp{};
+      sp.partials = partials;
+      sp.out = sumsq_out + i0;
+      sp.nmat = i1 - i0;
+      for (int i = i0; i < i1; ++i) {
+        sp.part_begin[i - i0] = pb[i];
+        sp.part_count[i - i0] = pc[i];
+      }
+      ProfScope prof(MUON_KERNEL_SUMS, s);
+      CUDA_TRY(ew::launch_sums(sp, s));
+    }
+  }
+  return MUON_OK;
+}
+
+int muon_apply(int count, float* const* params, const float* const* updates, const int64_t* shapes,
+               float lr, float wd, void* stream) {
+  t_err.clear();
+  if (count < 0) return set_err(MUON_ERR_ARG, "count %d < 0", count);
+  if (!finite(lr) || !finite(wd)) return set_err(MUON_ERR_ARG, "lr and wd must be finite");
+  if (count == 0) return MUON_OK;
+  if (!params || !updates || !shapes) return set_err(MUON_ERR_ARG, "params, updates and shapes must be non-NULL");
+  for (int i = 0; i < count; ++i) {
+    MUON_TRY(check_shape(shapes[2 * i], shapes[2 * i + 1], i));
+    MUON_TRY(check_ptr(params[i], "params", i));
+    MUON_TRY(check_ptr(updates[i], "updates", i));
+  }
+  DevInfo dev;
+  MUON_TRY(device_info(&dev));
+  cudaStream_t s = as_stream(stream);
+  for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
+    const int i1 = std::min(count, i0 + ew::kMaxMats);
+    ew::OutParams op{};
+    op.mode = 0;
+    op.lw = lr * wd;
+    int tiles = 0;
+    for (int i = i0; i < i1; ++i) {
+      const int r = static_cast<int>(shapes[2 * i]), c = static_cast<int>(shapes[2 * i + 1]);
+      ew::OutMat& O = op.mat[i - i0];
+      O.y = params[i];
+      O.o = updates[i];
+      O.rows = r;
+      O.cols = c;
+      O.o_transposed = 0;
+      O.ld = c;
+      O.tiles_c = (c + ew::kTile - 1) / ew::kTile;
+      O.tile_begin = tiles;
+      const float ratio = static_cast<float>(r) / static_cast<float>(c);
+      const float scale = ratio > 1.0f ? sqrtf(ratio) : 1.0f;
+      O.ls = lr * scale;
+      tiles += ((r + ew::kTile - 1) / ew::kTile) * O.tiles_c;
+    }
+    op.nmat = i1 - i0;
+    op.ntiles = tiles;
+    ProfScope prof(MUON_KERNEL_OUT, s);
+    CUDA_TRY(ew::launch_out(op, s));
+  }
+  return MUON_OK;
+}
+
+static int stage_common(int batch, int m, int k, DevInfo* dev, Workspace** ws, cudaStream_t s) {
+  if (batch < 0 || batch > 65535) return set_err(MUON_ERR_ARG, "batch %d out of range", batch);
+  MUON_TRY(check_shape(m, k, 0));
+  if (m % 8 || k % 8) return set_err(MUON_ERR_SHAPE, "m (%d) and k/n (%d) must be multiples of 8", m, k);
+  MUON_TRY(device_info(dev));
+  MUON_TRY(get_encoder());
+  MUON_TRY(get_workspace(s, 0, ws));
+  return MUON_OK;
+}
+
+int muon_gram_bf16(int batch, int m, int k, const void* X, void* A, void* stream) {
+  t_err.clear();
+  if (batch == 0) return MUON_OK;
+  if (!X || !A || !aligned16(X) || !aligned16(A)) return set_err(MUON_ERR_ARG, "X and A must be non-NULL and 16-byte aligned");
+  cudaStream_t s = as_stream(stream);
+  DevInfo dev;
+  Workspace* ws = nullptr;
+  MUON_TRY(stage_common(batch, m, k, &dev, &ws, s));
+  tc::Params P;
+  init_tc_params(P, ws->status, 0.f, 0.f, 0.f);
+  P.grp[0] = tc_group(batch, m, m, k, true, 0, m, static_cast<long long>(m) * m, A, nullptr, nullptr);
+  MUON_TRY(make_map(&P.map_p[0], X, k, m, batch, k, static_cast<uint64_t>(m) * k, 64, 128));
+  P.map_q[0] = P.map_p[0];
+  P.ngroups = 1;
+  P.total_tiles = batch * P.grp[0].tiles_per_mat;
+  return launch_tc(tc::kGram, P, dev.sms, s);
+}
+
+int muon_poly_bf16(int batch, int m, const void* A, void* B, float b, float c, void* stream) {
+  t_err.clear();
+  if (batch == 0) return MUON_OK;
+  if (!A || !B || !aligned16(A) || !aligned16(B)) return set_err(MUON_ERR_ARG, "A and B must be non-NULL and 16-byte aligned");
+  if (A == B) return set_err(MUON_ERR_ARG, "B must not alias A");
+  cudaStream_t s = as_stream(stream);
+  DevInfo dev;
+  Workspace* ws = nullptr;
+  MUON_TRY(stage_common(batch, m, m, &dev, &ws, s));
+  tc::Params P;
+  init_tc_params(P, ws->status, 0.f, b, c);
+  const long long as = static_cast<long long>(m) * m;
+  P.grp[0] = tc_group(batch, m, m, m, true, 0, m, as, B, A, nullptr);
+  MUON_TRY(make_map(&P.map_p[0], A, m, m, batch, m, as, 64, 128));
+  P.map_q[0] = P.map_p[0];
+  P.ngroups = 1;
+  P.total_tiles = batch * P.grp[0].tiles_per_mat;
+  return launch_tc(tc::kPoly, P, dev.sms, s);
+}
+
+int muon_bx_bf16(int batch, int m, int n, const void* B, const void* Xb, float* Xf, void* Xb_out,
+                 float a, void* stream) {
+  t_err.clear();
+  if (batch == 0) return MUON_OK;
+  if (!B || !Xb || !Xf || !Xb_out || !aligned16(B) || !aligned16(Xb) || !aligned16(Xf) || !aligned16(Xb_out))
+    return set_err(MUON_ERR_ARG, "B, Xb, Xf and Xb_out must be non-NULL and 16-byte aligned");
+  if (Xb == Xb_out) return set_err(MUON_ERR_ARG, "Xb_out must not alias Xb");
+  if (m > n) return set_err(MUON_ERR_SHAPE, "muon_bx_bf16 expects m <= n (got %dx%d)", m, n);
+  cudaStream_t s = as_stream(stream);
+  DevInfo dev;
+  Workspace* ws = nullptr;
+  MUON_TRY(stage_common(batch, m, n, &dev, &ws, s));
+  tc::Params P;
+  init_tc_params(P, ws->status, a, 0.f, 0.f);
+  const long long xs = static_cast<long long>(m) * n, as = static_cast<long long>(m) * m;
+  P.grp[0] = tc_group(batch, m, n, m, false, 0, n, xs, Xb_out, nullptr, Xf);
+  MUON_TRY(make_map(&P.map_p[0], B, m, m, batch, m, as, 64, 128));
+  MUON_TRY(make_map(&P.map_q[0], Xb, n, m, batch, n, xs, 64, 64));
+  P.ngroups = 1;
+  P.total_tiles = batch * P.grp[0].tiles_per_mat;
+  return launch_tc(tc::kBx, P, dev.sms, s);
+}
+
+int muon_get_status(void* stream) {
+  t_err.clear();
+  cudaStream_t s = as_stream(stream);
+  CUDA_TRY(cudaStreamSynchronize(s));
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  int* st = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto it = g_ws.find({dev, reinterpret_cast<uintptr_t>(s)});
+    if (it == g_ws.end() || !it->second.status) return MUON_OK;
+    st = it->second.status;
+  }
+  int v = 0;
+  CUDA_TRY(cudaMemcpy(&v, st, sizeof(int), cudaMemcpyDeviceToHost));
+  if (v != 0) {
+    CUDA_TRY(cudaMemset(st, 0, sizeof(int)));
+    set_err(v, "device status %d (a bounded device-side wait ran out)", v);
+  }
+  return v;
+}
+
+int muon_profile_begin(void) {
+  t_err.clear();
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (ProfRec& r : g_prof) {
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_prof.clear();
+  g_prof_on = true;
+  return MUON_OK;
+}
+
+int muon_profile_end(int kinds, double* total_ms, int* launches) {
+  t_err.clear();
+  std::vector<ProfRec> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_prof_on = false;
+    recs.swap(g_prof);
+  }
+  for (int k = 0; k < kinds; ++k) {
+    if (total_ms) total_ms[k] = 0.0;
+    if (launches) launches[k] = 0;
+  }
+  int n = 0;
+  int rc = MUON_OK;
+  for (ProfRec& r : recs) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess && rc == MUON_OK)
+      rc = set_err(MUON_ERR_CUDA, "kernel timing: %s", cudaGetErrorString(e));
+    if (r.kind >= 0 && r.kind < kinds) {
+      if (total_ms) total_ms[r.kind] += ms;
+      if (launches) launches[r.kind] += 1;
+    }
+    ++n;
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (ProfRec& r : recs) {
+      g_event_pool.push_back(r.a);
+      g_event_pool.push_back(r.b);
+    }
+  }
+  return rc == MUON_OK ? n : rc;
+}
+
+int muon_release(void) {
+  t_err.clear();
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  CUDA_TRY(cudaDeviceSynchronize());
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (auto it = g_ws.begin(); it != g_ws.end();) {
+    if (it->first.first == dev) {
+      if (it->second.ptr) cudaFree(it->second.ptr);
+      if (it->second.status) cudaFree(it->second.status);
+      it = g_ws.erase(it);
+    } else {
+      ++it;
+    }
+  }
+  return MUON_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,157 @@
+// Host-side interface between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace muon {
+
+// ----------------------------------------------------------------- tcgen05 GEMMs
+namespace tc {
+
+constexpr int kMaxGroups = 4;  // shape groups per launch
+constexpr int BM = 128;        // tile rows (TMEM lanes)
+constexpr int BN = 128;        // tile columns (TMEM fp32 columns per accumulator)
+constexpr int BK = 64;         // K per stage: one 128-byte swizzle row of bf16
+constexpr int kStages = 6;
+constexpr int kThreads = 192;  // warp 0 copies, warp 1 issues MMAs, warps 2-5 epilogue
+
+enum Epi : int { kGram = 0, kPoly = 1, kBx = 2 };
+
+struct Group {
+  int batch;        // matrices in the group
+  int m;            // rows of D
+  int n;            // columns of D (= m for kGram / kPoly)
+  int k;            // reduction length
+  int tiles_m, tiles_n, tiles_per_mat, tile_begin;
+  long long ld;          // row stride (elements) of D and of the epilogue operands
+  long long mat_stride;  // elements between consecutive matrices of D / operands
+  void* d;               // output: A (kGram), B (kPoly), bf16 X' (kBx)
+  const void* e;         // kPoly: A (bf16) for the b*A term
+  float* xf;             // kBx: fp32 master X, read then overwritten
+};
+
+struct Params {
+  CUtensorMap map_p[kMaxGroups];  // rows of D: X (kGram), A (kPoly), B (kBx); K-major
+  CUtensorMap map_q[kMaxGroups];  // columns of D: X / A K-major, or X MN-major (kBx)
+  Group grp[kMaxGroups];
+  int ngroups;
+  int total_tiles;
+  float a, b, c;
+  int* status;
+  unsigned long long timeout_ns;
+  int inject;  // 1: withhold one operand copy in CTA 0 (timeout-path test)
+};
+
+size_t smem_bytes();
+cudaError_t launch(int epi, const Params& p, int grid, cudaStream_t stream);
+
+}  // namespace tc
+
+// ----------------------------------------------------------- fp32 SIMT GEMMs
+namespace simt {
+
+enum Mode : int { kGram = 0, kPoly = 1, kBx = 2 };
+
+struct Params {
+  int batch, m, n;  // D is m x n (n = m for kGram / kPoly); K = k
+  int k;
+  const float* P;   // rows of D: X (kGram), A (kPoly), B (kBx)
+  const float* Q;   // X (kGram, k-contiguous rows), A (kPoly), X (kBx, n-contiguous rows)
+  const float* E;   // epilogue operand: A (kPoly), X (kBx)
+  float* D;
+  long long ldp, ldq, lde, ldd;  // row strides (elements)
+  long long sp, sq, se, sd;      // matrix strides (elements)
+  float a, b, c;
+};
+
+cudaError_t launch(int mode, const Params& p, cudaStream_t stream);
+
+}  // namespace simt
+
+// ----------------------------------------------------------- elementwise steps
+namespace ew {
+
+constexpr int kMaxMats = 128;  // matrices per launch
+constexpr int kFlatThreads = 256;
+constexpr int kFlatChunk = 8192;  // elements per block of the flat kernels
+constexpr int kTile = 64;         // tile edge of the transposing kernels
+
+enum SrcKind : int { kFromMomentum = 0, kFromBf16 = 1, kFromF32 = 2 };
+
+struct FlatMat {
+  const void* src;  // grad (bf16) for momentum; X (bf16/f32) for sumsq
+  float* buf;       // momentum buffer (in/out), momentum only
+  long long numel;
+  int blk_begin;    // first block of this matrix
+};
+
+struct FlatParams {
+  FlatMat mat[kMaxMats];
+  int nmat, nblocks;
+  int src_kind;       // kFromMomentum, kFromBf16, kFromF32
+  float beta, omb;
+  int nesterov;
+  float* partials;    // one per block
+};
+
+struct CastMat {
+  const void* src0;   // grad (bf16) or X (bf16 / f32)
+  const float* src1;  // updated momentum buffer (kFromMomentum) or null
+  int rows, cols;     // source layout
+  int transposed;     // rows > cols: X = U^T
+  int tiles_n;        // 64-wide tiles along X's columns
+  int tile_begin;
+  int part_begin, part_count;
+  float* xf;          // fp32 X (m x n, row stride ld)
+  void* xb;           // bf16 X or null
+  long long ld;
+};
+
+struct CastParams {
+  CastMat mat[kMaxMats];
+  int nmat, ntiles;
+  int src_kind;
+  float beta, omb;
+  int nesterov;
+  float eps;
+  const float* partials;
+};
+
+// Apply (W' = (W - lw W) - ls O) or write-back (Y = cast(O)) over tiles of the
+// caller's matrix; O is read from an m x n buffer, transposed when needed.
+struct OutMat {
+  void* y;            // W (fp32, in/out) or destination X (bf16 / f32)
+  const float* o;     // update / result in X layout (or in W layout if !o_transposed)
+  int rows, cols;     // caller layout of y
+  int o_transposed;   // O[r][s] = o[s * ld + r]
+  long long ld;
+  int tiles_c;        // 64-wide tiles along y's columns
+  int tile_begin;
+  float ls;           // fl(lr * scale)
+};
+
+struct OutParams {
+  OutMat mat[kMaxMats];
+  int nmat, ntiles;
+  int mode;           // 0: apply, 1: write bf16, 2: write f32
+  float lw;           // fl(lr * wd)
+};
+
+struct SumParams {
+  const float* partials;
+  int part_begin[kMaxMats];
+  int part_count[kMaxMats];
+  float* out;
+  int nmat;
+};
+
+cudaError_t launch_flat(const FlatParams& p, cudaStream_t s);
+cudaError_t launch_cast(const CastParams& p, cudaStream_t s);
+cudaError_t launch_out(const OutParams& p, cudaStream_t s);
+cudaError_t launch_sums(const SumParams& p, cudaStream_t s);
+
+}  // namespace ew
+
+}  // namespace muon

@@ -1,0 +1,117 @@
+"""The C-ABI library loads without a GPU, exports every symbol include/muon.h
+declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from newton_schulz_12_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "muon.h")
+
+
+def declared_functions():
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(muon_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _lib.lib()
+
+
+def test_header_lists_the_boundary():
+    names = declared_functions()
+    for required in ("muon_ns_orthogonalize", "muon_step", "muon_get_status", "muon_last_error"):
+        assert required in names
+    assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_build_targets_sm100a_only():
+    from newton_schulz_12_b200 import build
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    assert os.path.exists(_lib.LIB_PATH)
+
+
+def test_version(lib):
+    assert lib.muon_version() == 100
+
+
+def _err(lib):
+    return lib.muon_last_error().decode()
+
+
+def test_argument_errors_need_no_device(lib):
+    null = ctypes.c_void_p(0)
+    # negative batch, too many steps, unknown dtype, bad shape, null array
+    assert lib.muon_ns_orthogonalize(-1, 4, 4, None, 1.0, 0.0, 0.0, 5, 0, null) == -1
+    assert "batch" in _err(lib)
+    assert lib.muon_ns_orthogonalize(1, 4, 4, None, 1.0, 0.0, 0.0, 101, 0, null) == -1
+    assert lib.muon_ns_orthogonalize(1, 4, 4, None, 1.0, 0.0, 0.0, 5, 7, null) == -1
+    assert lib.muon_ns_orthogonalize(1, 0, 4, None, 1.0, 0.0, 0.0, 5, 0, null) == -2
+    assert lib.muon_ns_orthogonalize(1, 4, 40000, None, 1.0, 0.0, 0.0, 5, 0, null) == -2
+    assert lib.muon_ns_orthogonalize(1, 4, 4, None, 1.0, 0.0, 0.0, 5, 0, null) == -1
+    assert lib.muon_ns_orthogonalize(1, 4, 4, None, float("nan"), 0.0, 0.0, 5, 0, null) == -1
+    # misaligned / null device pointers are caught on the host
+    arr = _lib.ptr_array([0x1001])
+    assert lib.muon_ns_orthogonalize(1, 4, 4, arr, 1.0, 0.0, 0.0, 5, 0, null) == -1
+    assert "aligned" in _err(lib)
+    arr = _lib.ptr_array([0])
+    assert lib.muon_ns_orthogonalize(1, 4, 4, arr, 1.0, 0.0, 0.0, 5, 0, null) == -1
+    assert "NULL" in _err(lib)
+    # batch 0 is a no-op that succeeds without a device
+    assert lib.muon_ns_orthogonalize(0, 4, 4, None, 1.0, 0.0, 0.0, 5, 0, null) == 0
+
+
+def test_step_argument_errors(lib):
+    null = ctypes.c_void_p(0)
+    p = _lib.ptr_array([0x1000])
+    shapes = _lib.shape_array([(4, 4)])
+    assert lib.muon_step(-1, p, p, p, shapes, 0.9, 1, 0.1, 0.0, 5, null) == -1
+    assert lib.muon_step(0, None, None, None, None, 0.9, 1, 0.1, 0.0, 5, null) == 0
+    assert lib.muon_step(1, None, p, p, shapes, 0.9, 1, 0.1, 0.0, 5, null) == -1
+    assert lib.muon_step(1, p, p, p, shapes, 1.5, 1, 0.1, 0.0, 5, null) == -1
+    assert "beta" in _err(lib)
+    assert lib.muon_step(1, p, p, p, shapes, 0.9, 1, float("inf"), 0.0, 5, null) == -1
+    bad = _lib.shape_array([(4, -3)])
+    assert lib.muon_step(1, p, p, p, bad, 0.9, 1, 0.1, 0.0, 5, null) == -2
+    assert "shape" in _err(lib)
+    mis = _lib.ptr_array([0x1008])
+    assert lib.muon_step(1, p, mis, p, shapes, 0.9, 1, 0.1, 0.0, 5, null) == -1
+    assert "grads[0]" in _err(lib)
+    assert lib.muon_momentum(1, p, p, shapes, -0.1, 1, None, null) == -1
+    assert lib.muon_apply(1, p, None, shapes, 0.1, 0.0, null) == -1
+
+
+def test_stage_argument_errors(lib):
+    null = ctypes.c_void_p(0)
+    assert lib.muon_gram_bf16(1, 8, 8, None, None, null) == -1
+    assert lib.muon_poly_bf16(1, 8, 0x1000, 0x1000, 1.0, 1.0, null) == -1  # aliasing
+    assert lib.muon_bx_bf16(1, 8, 8, 0x1000, 0x2000, 0x3000, 0x2000, 1.0, null) == -1
+    assert lib.muon_gram_bf16(0, 8, 8, None, None, null) == 0
+
+
+def test_setters(lib):
+    assert lib.muon_set_wait_timeout_ms(0) == -1
+    assert lib.muon_set_wait_timeout_ms(2000) == 0
+    assert lib.muon_set_fault_injection(5) == -1
+    assert lib.muon_set_fault_injection(0) == 0
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    import newton_schulz_12_b200 as nsb
+    with pytest.raises(ValueError):
+        nsb.muon_ns_orthogonalize([torch.zeros(4, 4)])
+    with pytest.raises(ValueError):
+        nsb.muon_step([torch.zeros(4, 4)], [torch.zeros(4, 4, dtype=torch.bfloat16)],
+                      [torch.zeros(4, 4)])

@@ -1,0 +1,84 @@
+"""Tensor-core stage kernels against plain fp64 products of the same bf16 values.
+
+Each stage (A = X X^T, B = bA + cA^2, X' = aX + BX) is called through the C ABI
+and compared element by element with torch's fp64 CPU product of the very same
+operands.  Bounds: bf16 output rounding (2^-8 relative) plus fp32 accumulation
+(2^-16 of the sum of absolute products); the symmetric outputs must be exactly
+symmetric, and the bf16 copy of X' must be the round-to-nearest of its fp32 value.
+"""
+import pytest
+import torch
+
+import newton_schulz_12_b200 as nsb
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def rnd_bf16(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(*shape, generator=g) * scale).to(torch.bfloat16)
+
+
+def check_close(got, ref, absref, rel=2.0 ** -8, acc=2.0 ** -16):
+    got = got.double()
+    bound = rel * ref.abs() + acc * absref + 1e-30
+    err = (got - ref).abs()
+    bad = err > bound
+    assert not bad.any(), f"{int(bad.sum())} elements out of bound; worst {float((err - bound).max())}"
+
+
+@pytest.mark.parametrize("batch,m,k", [(1, 128, 64), (2, 256, 320), (3, 200, 328), (1, 8, 8),
+                                       (2, 768, 3072), (5, 384, 768), (1, 136, 24), (1, 1024, 200)])
+def test_gram(batch, m, k):
+    X = rnd_bf16((batch, m, k), seed=m * 7 + k)
+    A = nsb.muon_gram_bf16(X.to(DEV)).cpu()
+    Xd = X.double()
+    ref = Xd @ Xd.transpose(1, 2)
+    absref = Xd.abs() @ Xd.abs().transpose(1, 2)
+    check_close(A, ref, absref)
+    assert torch.equal(A, A.transpose(1, 2)), "A must be exactly symmetric"
+
+
+@pytest.mark.parametrize("batch,m", [(1, 128), (2, 200), (3, 768), (1, 8), (2, 392), (1, 1024)])
+def test_poly(batch, m):
+    G = torch.randn(batch, m, m, generator=torch.Generator().manual_seed(m)) / m ** 0.5
+    A = ((G + G.transpose(1, 2)) / 2).to(torch.bfloat16)
+    assert torch.equal(A, A.transpose(1, 2))
+    b, c = -4.7750, 2.0315
+    B = nsb.muon_poly_bf16(A.to(DEV), b, c).cpu()
+    Ad = A.double()
+    b32, c32 = float(torch.tensor(b, dtype=torch.float32)), float(torch.tensor(c, dtype=torch.float32))
+    ref = b32 * Ad + c32 * (Ad @ Ad)
+    absref = abs(b32) * Ad.abs() + abs(c32) * (Ad.abs() @ Ad.abs())
+    check_close(B, ref, absref)
+    assert torch.equal(B, B.transpose(1, 2)), "B must be exactly symmetric"
+
+
+@pytest.mark.parametrize("batch,m,n", [(1, 128, 128), (2, 200, 328), (1, 768, 3072), (3, 8, 72),
+                                       (2, 384, 384), (1, 136, 520), (1, 1024, 4096)])
+def test_bx(batch, m, n):
+    B = rnd_bf16((batch, m, m), seed=m, scale=m ** -0.5)
+    Xf = torch.randn(batch, m, n, generator=torch.Generator().manual_seed(n)) / n ** 0.5
+    Xb = Xf.to(torch.bfloat16)
+    a = 3.4445
+    a32 = float(torch.tensor(a, dtype=torch.float32))
+    Xf_dev = Xf.to(DEV)
+    out_b = nsb.muon_bx_bf16(B.to(DEV), Xb.to(DEV), Xf_dev, a).cpu()
+    got = Xf_dev.cpu()
+    ref = a32 * Xf.double() + B.double() @ Xb.double()
+    absref = abs(a32) * Xf.double().abs() + B.double().abs() @ Xb.double().abs()
+    check_close(got, ref, absref, rel=2.0 ** -23, acc=2.0 ** -16)
+    assert torch.equal(out_b, got.to(torch.bfloat16)), "bf16 copy must be RNE of the fp32 result"
+
+
+def test_stage_kernels_are_deterministic():
+    X = rnd_bf16((4, 768, 3072), seed=1).to(DEV)
+    A1 = nsb.muon_gram_bf16(X)
+    A2 = nsb.muon_gram_bf16(X)
+    assert torch.equal(A1, A2)
+    B1 = nsb.muon_poly_bf16(A1)
+    B2 = nsb.muon_poly_bf16(A1)
+    assert torch.equal(B1, B2)
+    assert nsb.muon_get_status() == 0

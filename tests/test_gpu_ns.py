@@ -1,0 +1,98 @@
+"""muon_ns_orthogonalize (C ABI) against the fp64 oracle on the same inputs.
+
+bf16 mode: relative Frobenius error <= 3e-2 (bf16 tensor-core operands, fp32
+accumulation); fp32 mode: <= 1e-4 (fp32 SIMT FMA).  The oracle receives the
+exact values the GPU receives (bf16 inputs are widened exactly).
+"""
+import numpy as np
+import pytest
+import torch
+
+import newton_schulz_12_b200 as nsb
+from newton_schulz_12_b200 import workloads
+from oracle import muon as oracle
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16 = 3e-2
+TOL_FP32 = 1e-4
+
+
+def rel_fro(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    return np.linalg.norm(got - ref) / np.linalg.norm(ref)
+
+
+def run_ns(mats, steps=5, coeffs=oracle.NS_COEFFS):
+    dev = [m.clone().cuda() for m in mats]
+    nsb.muon_ns_orthogonalize(dev, *coeffs, steps=steps)
+    assert nsb.muon_get_status() == 0
+    return [d.float().cpu().numpy() for d in dev]
+
+
+def test_config1_single_768_fp32_and_bf16():
+    """768x768 fp32, iid N(0,1) from seed 0, T=5, in both modes."""
+    X = workloads.gaussian((768, 768), 1.0, seed=0)
+    ref = oracle.newton_schulz(X.double().numpy())
+    got32 = run_ns([X])[0]
+    assert rel_fro(got32, ref) <= TOL_FP32
+    Xb = X.to(torch.bfloat16)
+    ref_b = oracle.newton_schulz(Xb.double().numpy())
+    got16 = run_ns([Xb])[0]
+    assert rel_fro(got16, ref_b) <= TOL_BF16
+
+
+@pytest.mark.parametrize("rows,cols,batch", [
+    (768, 768, 2), (768, 3072, 2), (3072, 768, 1), (200, 328, 3), (328, 200, 2), (130, 390, 1),
+    (8, 8, 4), (1, 17, 1), (17, 1, 1), (1, 1, 2), (64, 1000, 1), (1024, 1024, 1), (256, 4096, 1)])
+def test_bf16_shapes(rows, cols, batch):
+    mats = [workloads.gaussian((rows, cols), 1.0, seed=100 + i, dtype=torch.bfloat16)
+            for i in range(batch)]
+    got = run_ns(mats)
+    for g, x in zip(got, mats):
+        assert g.shape == (rows, cols)
+        assert rel_fro(g, oracle.newton_schulz(x.double().numpy())) <= TOL_BF16
+
+
+@pytest.mark.parametrize("rows,cols", [(768, 3072), (200, 328), (328, 200), (8, 8), (1, 5), (96, 96)])
+def test_fp32_shapes(rows, cols):
+    X = workloads.gaussian((rows, cols), 1.0, seed=rows + cols)
+    got = run_ns([X])[0]
+    assert rel_fro(got, oracle.newton_schulz(X.double().numpy())) <= TOL_FP32
+
+
+@pytest.mark.parametrize("steps", [0, 1, 2, 7])
+def test_step_counts(steps):
+    X = workloads.gaussian((384, 640), 1.0, seed=steps, dtype=torch.bfloat16)
+    ref = oracle.newton_schulz(X.double().numpy(), steps=steps)
+    assert rel_fro(run_ns([X], steps=steps)[0], ref) <= TOL_BF16
+    X32 = X.float()
+    assert rel_fro(run_ns([X32], steps=steps)[0], ref) <= TOL_FP32
+
+
+def test_other_coefficients():
+    """A different (a, b, c): the classic cubic 1.5 X - 0.5 X X^T X."""
+    X = workloads.gaussian((256, 512), 1.0, seed=3, dtype=torch.bfloat16)
+    coeffs = (1.5, -0.5, 0.0)
+    ref = oracle.newton_schulz(X.double().numpy(), steps=5, coeffs=coeffs)
+    assert rel_fro(run_ns([X], steps=5, coeffs=coeffs)[0], ref) <= TOL_BF16
+
+
+def test_zero_matrix_gives_zero():
+    for dt in (torch.bfloat16, torch.float32):
+        got = run_ns([torch.zeros(64, 96, dtype=dt)])[0]
+        assert np.all(got == 0.0)
+
+
+def test_hard_spectrum_band():
+    """Log-uniform spectrum with a x100 spike: still within tolerance of the oracle."""
+    G = workloads.hard_spectrum(768, 768, seed=5, spike=True)
+    ref = oracle.newton_schulz(G.double().numpy())
+    assert rel_fro(run_ns([G])[0], ref) <= TOL_BF16
+
+
+def test_deterministic():
+    X = workloads.gaussian((768, 3072), 1.0, seed=9, dtype=torch.bfloat16)
+    a = run_ns([X])[0]
+    b = run_ns([X])[0]
+    assert np.array_equal(a, b)

@@ -1,0 +1,142 @@
+"""muon_step / muon_momentum / muon_apply (C ABI) against the oracle.
+
+* momentum buffers: bit-exact against the fp32 restatement of the same order;
+* apply: bit-exact against the fp32 restatement given the same update;
+* the full step: the weight update W' - W within relative Frobenius 3e-2 of the
+  fp64 oracle run on the GPU's own pre-step state (so no drift accumulates);
+* the GPT-2-small hidden set (72 matrices, 768 wide) at full size, with
+  Gaussian and with hard (log-uniform, spiked) gradient spectra.
+"""
+import numpy as np
+import pytest
+import torch
+
+import newton_schulz_12_b200 as nsb
+from newton_schulz_12_b200 import workloads
+from oracle import muon as oracle
+from oracle.fp32_ref import apply_f32, momentum_f32, update_scale_f32
+
+pytestmark = pytest.mark.gpu
+
+TOL = 3e-2
+
+
+def rel_fro(got, ref):
+    return float(np.linalg.norm(np.asarray(got, np.float64) - ref) / np.linalg.norm(ref))
+
+
+class State:
+    def __init__(self, shapes, hard=False, w_seed=2000):
+        self.shapes = shapes
+        self.hard = hard
+        Ws, _ = workloads.muon_set(shapes, step=0, w_seed=w_seed)
+        self.W = [w.cuda() for w in Ws]
+        self.M = [torch.zeros(r, c, device="cuda") for r, c in shapes]
+
+    def grads(self, step):
+        _, Gs = workloads.muon_set(self.shapes, step=step, hard=self.hard)
+        return Gs
+
+
+def check_step(st, step, beta=0.95, nesterov=True, lr=0.05, wd=0.0, steps=5, check=None):
+    Gs = st.grads(step)
+    W0 = [w.cpu().numpy() for w in st.W]
+    M0 = [m.cpu().numpy() for m in st.M]
+    nsb.muon_step(st.W, [g.cuda() for g in Gs], st.M, beta=beta, nesterov=nesterov, lr=lr, wd=wd,
+                  steps=steps)
+    assert nsb.muon_get_status() == 0
+    idx = range(len(st.shapes)) if check is None else check
+    worst = 0.0
+    for i in idx:
+        g32 = Gs[i].float().numpy()
+        nb32, _ = momentum_f32(g32, M0[i], beta, nesterov)
+        assert np.array_equal(st.M[i].cpu().numpy().view(np.uint32), nb32.view(np.uint32)), \
+            f"momentum of matrix {i} not bit-exact"
+        Wn, _, _ = oracle.muon_step(W0[i], g32, M0[i], beta=np.float32(beta), nesterov=nesterov,
+                                    lr=np.float32(lr), wd=np.float32(wd), steps=steps)
+        dW_ref = Wn - W0[i]
+        dW = st.W[i].cpu().numpy().astype(np.float64) - W0[i]
+        err = rel_fro(dW, dW_ref)
+        worst = max(worst, err)
+        assert err <= TOL, f"matrix {i} {st.shapes[i]}: rel err {err:.3e}"
+    return worst
+
+
+def test_small_set_three_steps():
+    shapes = workloads.gpt2_small_shapes(layers=2, width=256) + [(200, 328), (328, 200), (72, 72), (1, 40)]
+    st = State(shapes)
+    for step in range(3):
+        check_step(st, step)
+
+
+def test_weight_decay_and_plain_momentum():
+    shapes = [(256, 256), (256, 1024), (1024, 256)]
+    st = State(shapes)
+    check_step(st, 0, wd=0.01)
+    check_step(st, 1, nesterov=False, beta=0.9, lr=0.02, wd=0.1)
+
+
+def test_zero_steps_applies_normalised_update():
+    st = State([(300, 200), (128, 256)])
+    check_step(st, 0, steps=0)
+
+
+def test_gpt2_small_full_set():
+    """All 72 hidden matrices of GPT-2 small, two steps, every matrix checked."""
+    st = State(workloads.gpt2_small_shapes())
+    for step in range(2):
+        worst = check_step(st, step)
+    assert worst < TOL
+
+
+def test_gpt2_small_hard_spectra():
+    st = State(workloads.gpt2_small_shapes(), hard=True)
+    check_step(st, 0)
+
+
+def test_scaled_set_sampled():
+    """144-matrix 1024-wide set with wd 0.01; one matrix of each shape checked."""
+    shapes = workloads.scaled_shapes()
+    st = State(shapes)
+    check_step(st, 0, wd=0.01, check=[0, 4, 5, 142, 143])
+
+
+def test_momentum_stage_bit_exact_and_sumsq():
+    shapes = [(768, 768), (333, 77), (5, 3), (1, 1)]
+    _, Gs = workloads.muon_set(shapes, step=0)
+    M = [workloads.gaussian(s, 1e-2, seed=50 + i).cuda() for i, s in enumerate(shapes)]
+    M0 = [m.cpu().numpy() for m in M]
+    out = torch.zeros(len(shapes), device="cuda")
+    nsb.muon_momentum([g.cuda() for g in Gs], M, beta=0.95, nesterov=True, sumsq_out=out)
+    for i in range(len(shapes)):
+        nb, u = momentum_f32(Gs[i].float().numpy(), M0[i], 0.95, True)
+        assert np.array_equal(M[i].cpu().numpy().view(np.uint32), nb.view(np.uint32))
+        ref = float(np.sum(u.astype(np.float64) ** 2))
+        assert abs(float(out[i]) - ref) <= 1e-6 * ref
+
+
+def test_apply_stage_bit_exact():
+    shapes = [(768, 3072), (3072, 768), (77, 5)]
+    W = [workloads.gaussian(s, 2e-2, seed=i).cuda() for i, s in enumerate(shapes)]
+    O = [workloads.gaussian(s, 1.0, seed=10 + i).cuda() for i, s in enumerate(shapes)]
+    W0 = [w.cpu().numpy() for w in W]
+    nsb.muon_apply(W, O, lr=0.05, wd=0.01)
+    for i, (r, c) in enumerate(shapes):
+        ref = apply_f32(W0[i], O[i].cpu().numpy(), 0.05, 0.01, update_scale_f32(r, c))
+        assert np.array_equal(W[i].cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+def test_step_is_deterministic():
+    shapes = [(768, 768), (768, 3072), (3072, 768)]
+    outs = []
+    for _ in range(2):
+        st = State(shapes)
+        nsb.muon_step(st.W, [g.cuda() for g in st.grads(0)], st.M)
+        outs.append([w.cpu().numpy() for w in st.W])
+    for a, b in zip(*outs):
+        assert np.array_equal(a, b)
+
+
+def test_empty_count_is_noop():
+    nsb.muon_step([], [], [])
+    assert nsb.muon_get_status() == 0
