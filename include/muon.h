@@ -79,6 +79,48 @@ int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a,
                           float c, int steps, int dtype, void* stream);
 
 /*
+ * muon_ns_orthogonalize_static -- muon_ns_orthogonalize (bf16 storage, the
+ * tensor-core path) for callers that cannot allocate device memory.
+ *
+ * The source pages have no counterpart for this call; it exists for library
+ * users.  Some callers cannot call cudaMalloc (or any allocator) where they
+ * call us: plug-ins whose host engine hands out all device memory up front and
+ * forbids allocation inside its execution callback, processes that run under a
+ * fixed, pre-planned memory budget, and latency-critical loops that must never
+ * wait on, or fail in, an allocator.  This call allocates nothing: its
+ * workspace is a static device array of 24 MiB that the library defines, so
+ * every GPU that loads the library holds those 24 MiB until the process exits.
+ *
+ * Arguments and result are those of muon_ns_orthogonalize with dtype
+ * MUON_BF16 (X_ptrs: host array of device pointers to bf16 m x n matrices,
+ * overwritten in place), plus:
+ * status_dev  DEVICE pointer to an int owned by the caller, or NULL.  If a
+ *             bounded device-side wait runs out during this call, the kernels
+ *             store MUON_ERR_DEVICE_TIMEOUT there (only if it holds 0; the
+ *             library never clears it).  With NULL the code goes to a slot of
+ *             the static array, which each call clears first, and is not
+ *             reported.
+ * Limits: the workspace of the batch -- 8*batch*m*n + 4*batch*min(m,n)^2
+ * bytes with the row strides rounded up to 8 elements, plus ~1 KiB -- must fit
+ * in the 24 MiB; larger requests return MUON_ERR_SHAPE with the byte counts
+ * and do nothing.  One 768 x 3072 matrix (about 20.3 MiB) fits; so do three
+ * 768 x 768 matrices.
+ * Sharing: every call on every stream of a device uses the same array and
+ * leaves its last contents there.  No byte of it needs to start at zero (each
+ * call writes everything it later reads).  Calls whose work overlaps on the
+ * GPU -- on different streams, or from different host threads -- race on the
+ * array and corrupt each other's results: order them on one stream or with
+ * events.
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current, and caches it; make that
+ * first call before any stream capture begins.
+ * If kernel timing (muon_profile_begin) is on, this call's launches are not
+ * timed, so no CUDA event objects are created on its behalf.
+ */
+int muon_ns_orthogonalize_static(int batch, int m, int n, void* const* X_ptrs, float a, float b,
+                                 float c, int steps, int* status_dev, void* stream);
+
+/*
  * muon_step -- one full Muon optimizer step over `count` hidden matrices.
  *
  * Source: "NanoGPT Speedrun: The Ultimate Guide...", section "Optimizer and

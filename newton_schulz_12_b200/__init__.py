@@ -20,7 +20,8 @@ from . import _lib
 from ._lib import MUON_BF16, MUON_FP32, MuonError, check, ptr_array, shape_array
 
 __all__ = [
-    "NS_COEFFS", "MuonError", "MuonStepPlan", "muon_ns_orthogonalize", "muon_step", "muon_momentum",
+    "NS_COEFFS", "MuonError", "MuonStepPlan", "muon_ns_orthogonalize",
+    "muon_ns_orthogonalize_static", "muon_step", "muon_momentum",
     "muon_apply", "muon_gram_bf16", "muon_poly_bf16", "muon_bx_bf16", "muon_get_status",
     "muon_last_error", "muon_release", "muon_set_wait_timeout_ms", "muon_set_fault_injection",
     "muon_profile_begin", "muon_profile_end", "muon_version", "MUON_BF16", "MUON_FP32",
@@ -70,6 +71,37 @@ def muon_ns_orthogonalize(xs, a=NS_COEFFS[0], b=NS_COEFFS[1], c=NS_COEFFS[2], st
     arr = ptr_array([x.data_ptr() for x in xs])
     check(_lib.lib().muon_ns_orthogonalize(len(xs), shape[0], shape[1], arr, a, b, c, steps, mode,
                                            _stream(stream)))
+    return xs
+
+
+def muon_ns_orthogonalize_static(xs, a=NS_COEFFS[0], b=NS_COEFFS[1], c=NS_COEFFS[2], steps=5,
+                                 status=None, stream=None):
+    """muon_ns_orthogonalize for bf16 matrices without any device allocation.
+
+    For callers that may not allocate device memory at the call site (an
+    engine that owns all device memory, a fixed memory budget, a loop that
+    must not touch an allocator): the library's workspace is a 24 MiB static
+    device array instead.  ``status`` is an optional int32 CUDA tensor in which
+    a device-side wait timeout is recorded.  Calls that overlap on the GPU
+    share that array and must be serialised by the caller.  Returns ``xs``.
+    """
+    xs = list(xs)
+    if not xs:
+        return xs
+    shape = tuple(xs[0].shape)
+    if len(shape) != 2:
+        raise ValueError("matrices must be 2-D")
+    for i, x in enumerate(xs):
+        _check_cuda(x, f"xs[{i}]", torch.bfloat16)
+        if tuple(x.shape) != shape:
+            raise ValueError("all matrices must have the same shape")
+    st = None
+    if status is not None:
+        _check_cuda(status, "status", torch.int32)
+        st = status.data_ptr()
+    arr = ptr_array([x.data_ptr() for x in xs])
+    check(_lib.lib().muon_ns_orthogonalize_static(len(xs), shape[0], shape[1], arr, a, b, c, steps,
+                                                  st, _stream(stream)))
     return xs
 
 

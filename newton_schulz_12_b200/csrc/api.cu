@@ -106,6 +106,9 @@ struct ProfRec {
   cudaEvent_t a, b;
 };
 bool g_prof_on = false;
+// While set on a thread, the timing hooks stay inert on that thread (they
+// would otherwise create CUDA event objects); used by the allocation-free call.
+thread_local bool t_hooks_off = false;
 std::vector<ProfRec> g_prof;
 std::vector<cudaEvent_t> g_event_pool;
 
@@ -126,6 +129,7 @@ struct ProfScope {
   cudaStream_t s;
   cudaEvent_t a = nullptr;
   ProfScope(int k, cudaStream_t st) : kind(k), s(st) {
+    if (t_hooks_off) return;
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_prof_on) return;
     a = take_event();
@@ -581,6 +585,48 @@ int check_ptr(const void* p, const char* what, int i) {
   return MUON_OK;
 }
 
+// ------------------------------------------------- allocation-free variant
+// Device scratch of muon_ns_orthogonalize_static.  A file-scope __device__
+// array: every GPU that loads this library holds it until the process exits.
+// Host code must not pass `g_static_scratch` itself to a kernel (on the host it
+// is only a stand-in symbol); its device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(24) << 20;  // 24 MiB
+constexpr size_t kStaticStatusBytes = 1024;  // status slot used when the caller passes none
+
+struct HooksOff {
+  HooksOff() { t_hooks_off = true; }
+  ~HooksOff() { t_hooks_off = false; }
+};
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+
+std::mutex g_static_mu;
+std::map<int, char*> g_static_addr;  // device ordinal -> device address of g_static_scratch
+
+int static_scratch_address(char** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  auto it = g_static_addr.find(dev);
+  if (it != g_static_addr.end()) {
+    *out = it->second;
+    return MUON_OK;
+  }
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (e != cudaSuccess || !p)
+    return set_err(MUON_ERR_CUDA, "cudaGetSymbolAddress of the static scratch on device %d: %s", dev,
+                   cudaGetErrorString(e));
+  g_static_addr[dev] = static_cast<char*>(p);
+  *out = static_cast<char*>(p);
+  return MUON_OK;
+}
+
 }  // namespace
 
 // =============================================================================
@@ -649,6 +695,60 @@ int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a,
   }
   std::vector<void*> ys(X_ptrs, X_ptrs + batch);
   MUON_TRY(launch_out_chunked(mats, groups, final_xf, ys, fp32 ? 2 : 1, 0.f, 0.f, s));
+  return MUON_OK;
+}
+
+int muon_ns_orthogonalize_static(int batch, int m, int n, void* const* X_ptrs, float a, float b,
+                                 float c, int steps, int* status_dev, void* stream) {
+  t_err.clear();
+  if (batch < 0 || batch > 65535) return set_err(MUON_ERR_ARG, "batch %d out of range 0..65535", batch);
+  if (steps < 0 || steps > kMaxStepsArg) return set_err(MUON_ERR_ARG, "steps %d out of range 0..%d", steps, kMaxStepsArg);
+  if (!finite(a) || !finite(b) || !finite(c)) return set_err(MUON_ERR_ARG, "coefficients must be finite");
+  MUON_TRY(check_shape(m, n, 0));
+  if (status_dev && (reinterpret_cast<uintptr_t>(status_dev) & 3u))
+    return set_err(MUON_ERR_ARG, "status_dev is not 4-byte aligned");
+  if (batch == 0) return MUON_OK;
+  if (!X_ptrs) return set_err(MUON_ERR_ARG, "X_ptrs is NULL");
+  for (int i = 0; i < batch; ++i) MUON_TRY(check_ptr(X_ptrs[i], "X_ptrs", i));
+
+  std::vector<std::pair<int, int>> shapes(batch, std::make_pair(m, n));
+  std::vector<MatInfo> mats;
+  std::vector<NsGroup> groups;
+  group_shapes(shapes, mats, groups);
+  std::vector<long long> numels(batch, static_cast<long long>(m) * n);
+  const int nblk = count_flat_blocks(numels);
+  size_t need = align_up(static_cast<size_t>(nblk) * 4, 1024);
+  for (NsGroup& g : groups) need = layout_group(g, nullptr, need, false);
+  if (need + kStaticStatusBytes > kStaticScratchBytes)
+    return set_err(MUON_ERR_SHAPE,
+                   "batch %d of %dx%d needs %zu bytes of scratch; the static scratch holds %zu "
+                   "(use muon_ns_orthogonalize, which allocates its workspace)",
+                   batch, m, n, need + kStaticStatusBytes, kStaticScratchBytes);
+  DevInfo dev;
+  MUON_TRY(device_info(&dev));
+  char* scratch = nullptr;
+  MUON_TRY(static_scratch_address(&scratch));
+  cudaStream_t s = as_stream(stream);
+  int* status = status_dev;
+  if (!status) {
+    status = reinterpret_cast<int*>(scratch);
+    CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
+  }
+  HooksOff no_hooks;
+  char* base = scratch + kStaticStatusBytes;
+  float* partials = reinterpret_cast<float*>(base);
+  size_t off = align_up(static_cast<size_t>(nblk) * 4, 1024);
+  for (NsGroup& g : groups) off = layout_group(g, base, off, false);
+
+  std::vector<const void*> src(X_ptrs, X_ptrs + batch);
+  std::vector<int> pb, pc;
+  MUON_TRY(launch_flat_chunked(src, {}, numels, ew::kFromBf16, 0.f, 0, partials, pb, pc, s));
+  MUON_TRY(launch_cast_chunked(mats, groups, src, {}, ew::kFromBf16, 0.f, 0, partials, pb, pc, true, s));
+  MUON_TRY(run_ns_bf16(groups, steps, a, b, c, status, dev.sms, s));
+  std::vector<float*> final_xf;
+  for (NsGroup& g : groups) final_xf.push_back(g.xf);
+  std::vector<void*> ys(X_ptrs, X_ptrs + batch);
+  MUON_TRY(launch_out_chunked(mats, groups, final_xf, ys, 1, 0.f, 0.f, s));
   return MUON_OK;
 }
 
