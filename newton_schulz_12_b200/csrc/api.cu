@@ -204,20 +204,54 @@ inline long long round8(long long x) { return (x + 7) / 8 * 8; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
-int make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
-             uint64_t ld, uint64_t mat_stride, uint32_t box_inner, uint32_t box_rows) {
+// 3-D tensor map {inner, rows, batch} over a contiguous batch with row stride
+// `ld` and matrix stride `mat_stride` (elements); `esize` 2 = bf16, 4 = fp32.
+int make_map(CUtensorMap* map, const void* base, int esize, uint64_t inner, uint64_t rows,
+             uint64_t batch, uint64_t ld, uint64_t mat_stride, uint32_t box_inner, uint32_t box_rows,
+             CUtensorMapSwizzle swz) {
   cuuint64_t dims[3] = {inner, rows, batch};
-  cuuint64_t strides[2] = {ld * 2, mat_stride * 2};
+  cuuint64_t strides[2] = {ld * esize, mat_stride * esize};
   cuuint32_t box[3] = {box_inner, box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
-                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  const CUtensorMapDataType dt =
+      esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  CUresult r = g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
-    return set_err(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %llux%llux%llu ld %llu",
+    return set_err(MUON_ERR_CUDA,
+                   "cuTensorMapEncodeTiled failed (%d) for %llux%llux%llu ld %llu box %ux%u",
                    static_cast<int>(r), (unsigned long long)inner, (unsigned long long)rows,
-                   (unsigned long long)batch, (unsigned long long)ld);
+                   (unsigned long long)batch, (unsigned long long)ld, box_inner, box_rows);
+  return MUON_OK;
+}
+
+// Maps of the symmetric-output GEMMs: D (m x m) from an operand S (m x k, K-major),
+// D = S S^T (kGram) or b S + c S S (kPoly, with S = A symmetric and e = A).
+int sym_maps(tc::Maps& M, const void* S, int m, int k, long long lds, long long ss, void* D,
+             long long ldd, long long sd, int batch, bool with_e) {
+  MUON_TRY(make_map(&M.p, S, 2, k, m, batch, lds, ss, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
+  MUON_TRY(make_map(&M.q, S, 2, k, m, batch, lds, ss, 64, tc::BN, CU_TENSOR_MAP_SWIZZLE_128B));
+  if (with_e)
+    MUON_TRY(make_map(&M.e, S, 2, m, m, batch, lds, ss, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
+  else
+    M.e = M.p;
+  MUON_TRY(make_map(&M.d, D, 2, m, m, batch, ldd, sd, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
+  MUON_TRY(make_map(&M.mt, D, 2, m, m, batch, ldd, sd, tc::BM, tc::kChunk, CU_TENSOR_MAP_SWIZZLE_NONE));
+  MUON_TRY(make_map(&M.s, D, 2, m, m, batch, ldd, sd, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
+  return MUON_OK;
+}
+
+// Maps of X' = a X + B X: B (m x m), X bf16 operand (m x n, read MN-major),
+// X fp32 master (m x n, read and written), X' bf16 (m x n).
+int bx_maps(tc::Maps& M, const void* B, long long ldb, long long sb, const void* Xb, float* Xf,
+            void* Xout, int m, int n, long long ldx, long long sx, int batch) {
+  MUON_TRY(make_map(&M.p, B, 2, m, m, batch, ldb, sb, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
+  MUON_TRY(make_map(&M.q, Xb, 2, n, m, batch, ldx, sx, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+  MUON_TRY(make_map(&M.e, Xf, 4, n, m, batch, ldx, sx, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
+  MUON_TRY(make_map(&M.d, Xout, 2, n, m, batch, ldx, sx, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
+  M.mt = M.d;
+  M.s = M.d;
   return MUON_OK;
 }
 
@@ -263,22 +297,16 @@ size_t layout_group(NsGroup& g, char* base, size_t off, bool fp32) {
   return off;
 }
 
-tc::Group tc_group(int batch, int m, int n, int k, bool sym, int tile_begin, long long ld,
-                   long long mat_stride, void* d, const void* e, float* xf) {
+tc::Group tc_group(int batch, int m, int n, int k, bool sym, int tile_begin) {
   tc::Group G{};
   G.batch = batch;
   G.m = m;
   G.n = n;
   G.k = k;
   G.tiles_m = (m + tc::BM - 1) / tc::BM;
-  G.tiles_n = sym ? G.tiles_m : (n + tc::BN - 1) / tc::BN;
-  G.tiles_per_mat = sym ? G.tiles_m * (G.tiles_m + 1) / 2 : G.tiles_m * G.tiles_n;
+  G.tiles_n = sym ? (m + tc::BN - 1) / tc::BN : (n + tc::BN - 1) / tc::BN;
+  G.tiles_per_mat = sym ? tc::sym_tiles(m) : G.tiles_m * G.tiles_n;
   G.tile_begin = tile_begin;
-  G.ld = ld;
-  G.mat_stride = mat_stride;
-  G.d = d;
-  G.e = e;
-  G.xf = xf;
   return G;
 }
 
@@ -328,24 +356,20 @@ int run_ns_bf16(std::vector<NsGroup>& gs, int steps, float a, float b, float c, 
       const long long xs = static_cast<long long>(G.m) * G.ldn;
       const long long as = static_cast<long long>(G.m) * G.ldm;
       for (int par = 0; par < 2; ++par) {
-        gram[par].grp[k] = tc_group(G.batch, G.m, G.m, G.n, true, gram[par].total_tiles, G.ldm,
-                                    as, G.A, nullptr, nullptr);
-        MUON_TRY(make_map(&gram[par].map_p[k], G.xb[par], G.n, G.m, G.batch, G.ldn, xs, 64, 128));
-        gram[par].map_q[k] = gram[par].map_p[k];
+        gram[par].grp[k] = tc_group(G.batch, G.m, G.m, G.n, true, gram[par].total_tiles);
+        MUON_TRY(sym_maps(gram[par].map[k], G.xb[par], G.m, G.n, G.ldn, xs, G.A, G.ldm, as,
+                          G.batch, false));
         gram[par].total_tiles += G.batch * gram[par].grp[k].tiles_per_mat;
         gram[par].ngroups = k + 1;
 
-        bx[par].grp[k] = tc_group(G.batch, G.m, G.n, G.m, false, bx[par].total_tiles, G.ldn, xs,
-                                  G.xb[par ^ 1], nullptr, G.xf);
-        MUON_TRY(make_map(&bx[par].map_p[k], G.B, G.m, G.m, G.batch, G.ldm, as, 64, 128));
-        MUON_TRY(make_map(&bx[par].map_q[k], G.xb[par], G.n, G.m, G.batch, G.ldn, xs, 64, 64));
+        bx[par].grp[k] = tc_group(G.batch, G.m, G.n, G.m, false, bx[par].total_tiles);
+        MUON_TRY(bx_maps(bx[par].map[k], G.B, G.ldm, as, G.xb[par], G.xf, G.xb[par ^ 1], G.m, G.n,
+                         G.ldn, xs, G.batch));
         bx[par].total_tiles += G.batch * bx[par].grp[k].tiles_per_mat;
         bx[par].ngroups = k + 1;
       }
-      poly.grp[k] = tc_group(G.batch, G.m, G.m, G.m, true, poly.total_tiles, G.ldm, as, G.B, G.A,
-                             nullptr);
-      MUON_TRY(make_map(&poly.map_p[k], G.A, G.m, G.m, G.batch, G.ldm, as, 64, 128));
-      poly.map_q[k] = poly.map_p[k];
+      poly.grp[k] = tc_group(G.batch, G.m, G.m, G.m, true, poly.total_tiles);
+      MUON_TRY(sym_maps(poly.map[k], G.A, G.m, G.m, G.ldm, as, G.B, G.ldm, as, G.batch, true));
       poly.total_tiles += G.batch * poly.grp[k].tiles_per_mat;
       poly.ngroups = k + 1;
     }
@@ -916,9 +940,9 @@ int muon_gram_bf16(int batch, int m, int k, const void* X, void* A, void* stream
   MUON_TRY(stage_common(batch, m, k, &dev, &ws, s));
   tc::Params P;
   init_tc_params(P, ws->status, 0.f, 0.f, 0.f);
-  P.grp[0] = tc_group(batch, m, m, k, true, 0, m, static_cast<long long>(m) * m, A, nullptr, nullptr);
-  MUON_TRY(make_map(&P.map_p[0], X, k, m, batch, k, static_cast<uint64_t>(m) * k, 64, 128));
-  P.map_q[0] = P.map_p[0];
+  P.grp[0] = tc_group(batch, m, m, k, true, 0);
+  MUON_TRY(sym_maps(P.map[0], X, m, k, k, static_cast<long long>(m) * k, A, m,
+                    static_cast<long long>(m) * m, batch, false));
   P.ngroups = 1;
   P.total_tiles = batch * P.grp[0].tiles_per_mat;
   return launch_tc(tc::kGram, P, dev.sms, s);
@@ -936,9 +960,8 @@ int muon_poly_bf16(int batch, int m, const void* A, void* B, float b, float c, v
   tc::Params P;
   init_tc_params(P, ws->status, 0.f, b, c);
   const long long as = static_cast<long long>(m) * m;
-  P.grp[0] = tc_group(batch, m, m, m, true, 0, m, as, B, A, nullptr);
-  MUON_TRY(make_map(&P.map_p[0], A, m, m, batch, m, as, 64, 128));
-  P.map_q[0] = P.map_p[0];
+  P.grp[0] = tc_group(batch, m, m, m, true, 0);
+  MUON_TRY(sym_maps(P.map[0], A, m, m, m, as, B, m, as, batch, true));
   P.ngroups = 1;
   P.total_tiles = batch * P.grp[0].tiles_per_mat;
   return launch_tc(tc::kPoly, P, dev.sms, s);
@@ -959,9 +982,8 @@ int muon_bx_bf16(int batch, int m, int n, const void* B, const void* Xb, float* 
   tc::Params P;
   init_tc_params(P, ws->status, a, 0.f, 0.f);
   const long long xs = static_cast<long long>(m) * n, as = static_cast<long long>(m) * m;
-  P.grp[0] = tc_group(batch, m, n, m, false, 0, n, xs, Xb_out, nullptr, Xf);
-  MUON_TRY(make_map(&P.map_p[0], B, m, m, batch, m, as, 64, 128));
-  MUON_TRY(make_map(&P.map_q[0], Xb, n, m, batch, n, xs, 64, 64));
+  P.grp[0] = tc_group(batch, m, n, m, false, 0);
+  MUON_TRY(bx_maps(P.map[0], B, m, as, Xb, Xf, Xb_out, m, n, n, xs, batch));
   P.ngroups = 1;
   P.total_tiles = batch * P.grp[0].tiles_per_mat;
   return launch_tc(tc::kBx, P, dev.sms, s);

@@ -10,31 +10,37 @@ namespace muon {
 // ----------------------------------------------------------------- tcgen05 GEMMs
 namespace tc {
 
-constexpr int kMaxGroups = 4;  // shape groups per launch
-constexpr int BM = 128;        // tile rows (TMEM lanes)
-constexpr int BN = 128;        // tile columns (TMEM fp32 columns per accumulator)
-constexpr int BK = 64;         // K per stage: one 128-byte swizzle row of bf16
-constexpr int kStages = 6;
-constexpr int kThreads = 192;  // warp 0 copies, warp 1 issues MMAs, warps 2-5 epilogue
+constexpr int kMaxGroups = 4;        // shape groups per launch
+constexpr int BM = 128;              // tile rows (TMEM lanes)
+constexpr int BN = 256;              // tile columns (fp32 TMEM columns per accumulator)
+constexpr int BK = 64;               // K per stage: one 128-byte swizzle row of bf16
+constexpr int kChunk = 32;           // epilogue columns handled per step
+constexpr int kChunks = BN / kChunk;
+constexpr int kEpiSlots = 4;         // ring of prefetched epilogue operand chunks
+constexpr int kThreads = 192;        // warp 0 copies, warp 1 issues MMAs, warps 2-5 epilogue
 
 enum Epi : int { kGram = 0, kPoly = 1, kBx = 2 };
 
 struct Group {
-  int batch;        // matrices in the group
-  int m;            // rows of D
-  int n;            // columns of D (= m for kGram / kPoly)
-  int k;            // reduction length
+  int batch;  // matrices in the group
+  int m;      // rows of D
+  int n;      // columns of D (= m for kGram / kPoly)
+  int k;      // reduction length
   int tiles_m, tiles_n, tiles_per_mat, tile_begin;
-  long long ld;          // row stride (elements) of D and of the epilogue operands
-  long long mat_stride;  // elements between consecutive matrices of D / operands
-  void* d;               // output: A (kGram), B (kPoly), bf16 X' (kBx)
-  const void* e;         // kPoly: A (bf16) for the b*A term
-  float* xf;             // kBx: fp32 master X, read then overwritten
+};
+
+// Tensor maps of one group (3-D: {inner, rows, batch}).
+struct Maps {
+  CUtensorMap p;   // rows of D: X (kGram), A (kPoly), B (kBx); K-major, box 64 x 128
+  CUtensorMap q;   // columns of D: X / A K-major box 64 x 256; X MN-major box 64 x 64 (kBx)
+  CUtensorMap e;   // epilogue input chunk: A bf16 32 x 128 (kPoly); fp32 X 32 x 128 (kBx, also stored)
+  CUtensorMap d;   // direct output chunk, bf16 32 x 128: A (kGram), B (kPoly), bf16 X' (kBx)
+  CUtensorMap mt;  // mirrored output chunk, bf16 128 x 32 (kGram / kPoly)
+  CUtensorMap s;   // symmetrised diagonal block, bf16 64 x 128 (kGram / kPoly)
 };
 
 struct Params {
-  CUtensorMap map_p[kMaxGroups];  // rows of D: X (kGram), A (kPoly), B (kBx); K-major
-  CUtensorMap map_q[kMaxGroups];  // columns of D: X / A K-major, or X MN-major (kBx)
+  Maps map[kMaxGroups];
   Group grp[kMaxGroups];
   int ngroups;
   int total_tiles;
@@ -44,7 +50,15 @@ struct Params {
   int inject;  // 1: withhold one operand copy in CTA 0 (timeout-path test)
 };
 
-size_t smem_bytes();
+// Symmetric-output tiles per m x m matrix (128 x 256 tiles touching the upper triangle).
+inline int sym_tiles(int m) {
+  const int tm = (m + BM - 1) / BM, tn = (m + BN - 1) / BN;
+  int t = 0;
+  for (int r = 0; r < tm; ++r) t += tn - (r >> 1);
+  return t;
+}
+
+size_t smem_bytes(int epi);
 cudaError_t launch(int epi, const Params& p, int grid, cudaStream_t stream);
 
 }  // namespace tc

@@ -29,8 +29,10 @@ def check_close(got, ref, absref, rel=2.0 ** -8, acc=2.0 ** -16):
     assert not bad.any(), f"{int(bad.sum())} elements out of bound; worst {float((err - bound).max())}"
 
 
+# the last cases give every CTA several tiles (persistent loop, both accumulators)
 @pytest.mark.parametrize("batch,m,k", [(1, 128, 64), (2, 256, 320), (3, 200, 328), (1, 8, 8),
-                                       (2, 768, 3072), (5, 384, 768), (1, 136, 24), (1, 1024, 200)])
+                                       (2, 768, 3072), (5, 384, 768), (1, 136, 24), (1, 1024, 200),
+                                       (160, 256, 136), (40, 768, 768)])
 def test_gram(batch, m, k):
     X = rnd_bf16((batch, m, k), seed=m * 7 + k)
     A = nsb.muon_gram_bf16(X.to(DEV)).cpu()
@@ -41,7 +43,8 @@ def test_gram(batch, m, k):
     assert torch.equal(A, A.transpose(1, 2)), "A must be exactly symmetric"
 
 
-@pytest.mark.parametrize("batch,m", [(1, 128), (2, 200), (3, 768), (1, 8), (2, 392), (1, 1024)])
+@pytest.mark.parametrize("batch,m", [(1, 128), (2, 200), (3, 768), (1, 8), (2, 392), (1, 1024),
+                                     (170, 200), (40, 768)])
 def test_poly(batch, m):
     G = torch.randn(batch, m, m, generator=torch.Generator().manual_seed(m)) / m ** 0.5
     A = ((G + G.transpose(1, 2)) / 2).to(torch.bfloat16)
@@ -57,7 +60,8 @@ def test_poly(batch, m):
 
 
 @pytest.mark.parametrize("batch,m,n", [(1, 128, 128), (2, 200, 328), (1, 768, 3072), (3, 8, 72),
-                                       (2, 384, 384), (1, 136, 520), (1, 1024, 4096)])
+                                       (2, 384, 384), (1, 136, 520), (1, 1024, 4096),
+                                       (80, 256, 520), (6, 768, 3072)])
 def test_bx(batch, m, n):
     B = rnd_bf16((batch, m, m), seed=m, scale=m ** -0.5)
     Xf = torch.randn(batch, m, n, generator=torch.Generator().manual_seed(n)) / n ** 0.5
