@@ -84,15 +84,16 @@ def stage_work(shapes):
 
     GEMMs: nominal FLOPs (X X^T: 2 m^2 n, A A: 2 m^3, B X: 2 m^2 n).
     Memory-bound kernels: bytes that must cross HBM per element -- momentum
-    g(2)+buf(4) read, buf(4) written = 10 B; cast g(2)+buf(4) read, fp32 X(4) +
-    bf16 X(2) written = 12 B; apply W(4)+O(4) read, W(4) written = 12 B.
+    g(2)+buf(4) read, buf(4) written = 10 B; cast g(2)+buf(4) read, the bf16
+    pair hi(2)+lo(2) of X written = 10 B; apply W(4) + O as hi(2)+lo(2) read,
+    W(4) written = 12 B.
     """
     elems = sum(r * c for r, c in shapes)
     g = sum(2 * min(r, c) ** 2 * max(r, c) for r, c in shapes)
     p = sum(2 * min(r, c) ** 3 for r, c in shapes)
     return {
         "gram": ("tensor", g), "poly": ("tensor", p), "bx": ("tensor", g),
-        "flat": ("hbm", 10 * elems), "cast": ("hbm", 12 * elems), "out": ("hbm", 12 * elems),
+        "flat": ("hbm", 10 * elems), "cast": ("hbm", 10 * elems), "out": ("hbm", 12 * elems),
     }
 
 
@@ -373,7 +374,7 @@ def run_ours(args):
             "config": {"workload": WORKLOAD, "matrices_per_step": len(shapes) * world,
                        "parallelism": f"replicas x{world} (one independent 72-matrix set per GPU)",
                        "l2": "inputs larger than L2 (W 340 MB + momentum 340 MB + grads 170 MB "
-                             "per GPU, plus an 850 MB workspace); no flush"},
+                             "per GPU, plus a 680 MB workspace); no flush"},
             "tflops": tflops,
             "pct_of_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
             "pct_of_bf16_peak_sustained": 100.0 * tflops / peaks["bf16_tflops_sustained"],

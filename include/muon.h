@@ -41,7 +41,7 @@ extern "C" {
 /* Storage / arithmetic type of muon_ns_orthogonalize's matrices. */
 typedef enum {
   MUON_BF16 = 0, /* bf16 storage; bf16 tensor-core operands, fp32 accumulate,
-                    fp32 master copy of X between steps */
+                    X kept between steps as a pair of bf16 matrices hi + lo */
   MUON_FP32 = 1  /* fp32 storage; fp32 SIMT FMA verification path */
 } muon_dtype;
 
@@ -100,10 +100,10 @@ int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a,
  *             library never clears it).  With NULL the code goes to a slot of
  *             the static array, which each call clears first, and is not
  *             reported.
- * Limits: the workspace of the batch -- 8*batch*m*n + 4*batch*min(m,n)^2
+ * Limits: the workspace of the batch -- 6*batch*m*n + 4*batch*min(m,n)^2
  * bytes with the row strides rounded up to 8 elements, plus ~1 KiB -- must fit
  * in the 24 MiB; larger requests return MUON_ERR_SHAPE with the byte counts
- * and do nothing.  One 768 x 3072 matrix (about 20.3 MiB) fits; so do three
+ * and do nothing.  One 768 x 3072 matrix (about 15.8 MiB) fits; so do four
  * 768 x 768 matrices.
  * Sharing: every call on every stream of a device uses the same array and
  * leaves its last contents there.  No byte of it needs to start at zero (each
@@ -178,16 +178,19 @@ int muon_apply(int count, float* const* params, const float* const* updates,
  * tensor copies).
  *
  * muon_gram_bf16:  A = X X^T          X: batch x m x k bf16, A: batch x m x m bf16.
- *                  Only upper 128x128 tiles are computed; A is exactly symmetric.
+ *                  Only 128x256 tiles touching the upper triangle are computed;
+ *                  A is exactly symmetric.
  * muon_poly_bf16:  B = b*A + c*(A A)   A, B: batch x m x m bf16, A symmetric.
- * muon_bx_bf16:    X' = a*X + B X      B: m x m bf16; Xb: bf16 operand copy of X;
- *                  Xf: fp32 master X (read, then overwritten by X');
- *                  Xb_out: bf16 copy of X' (must not alias Xb).
+ * muon_bx_bf16:    X' = a*X + B X, with X carried as the bf16 pair hi + lo (the
+ *                  representation the iteration keeps between steps, about 16
+ *                  significant bits): B m x m bf16; Xhi: bf16(X), the operand;
+ *                  Xlo: bf16(X - Xhi), read then overwritten by bf16(X' - bf16(X'));
+ *                  Xhi_out: bf16(X') (must not alias Xhi).
  */
 int muon_gram_bf16(int batch, int m, int k, const void* X, void* A, void* stream);
 int muon_poly_bf16(int batch, int m, const void* A, void* B, float b, float c, void* stream);
-int muon_bx_bf16(int batch, int m, int n, const void* B, const void* Xb, float* Xf,
-                 void* Xb_out, float a, void* stream);
+int muon_bx_bf16(int batch, int m, int n, const void* B, const void* Xhi, void* Xlo,
+                 void* Xhi_out, float a, void* stream);
 
 /*
  * muon_get_status -- synchronise `stream`, then return and clear the device

@@ -218,18 +218,21 @@ def muon_poly_bf16(A, b=NS_COEFFS[1], c=NS_COEFFS[2], B=None, stream=None):
     return B
 
 
-def muon_bx_bf16(B, Xb, Xf, a=NS_COEFFS[0], Xb_out=None, stream=None):
-    """X' = a X + B X: Xf (fp32 master) updated in place; returns the bf16 copy of X'."""
+def muon_bx_bf16(B, Xhi, Xlo, a=NS_COEFFS[0], Xhi_out=None, stream=None):
+    """X' = a X + B X with X = Xhi + Xlo (bf16 pair).
+
+    Xlo is overwritten by bf16(X' - bf16(X')); returns Xhi_out = bf16(X').
+    """
     _check_cuda(B, "B", torch.bfloat16)
-    _check_cuda(Xb, "Xb", torch.bfloat16)
-    _check_cuda(Xf, "Xf", torch.float32)
-    bsz, m, n = Xb.shape
-    if Xb_out is None:
-        Xb_out = torch.empty_like(Xb)
-    _check_cuda(Xb_out, "Xb_out", torch.bfloat16)
-    check(_lib.lib().muon_bx_bf16(bsz, m, n, B.data_ptr(), Xb.data_ptr(), Xf.data_ptr(),
-                                  Xb_out.data_ptr(), a, _stream(stream)))
-    return Xb_out
+    _check_cuda(Xhi, "Xhi", torch.bfloat16)
+    _check_cuda(Xlo, "Xlo", torch.bfloat16)
+    bsz, m, n = Xhi.shape
+    if Xhi_out is None:
+        Xhi_out = torch.empty_like(Xhi)
+    _check_cuda(Xhi_out, "Xhi_out", torch.bfloat16)
+    check(_lib.lib().muon_bx_bf16(bsz, m, n, B.data_ptr(), Xhi.data_ptr(), Xlo.data_ptr(),
+                                  Xhi_out.data_ptr(), a, _stream(stream)))
+    return Xhi_out
 
 
 def muon_get_status(stream=None):

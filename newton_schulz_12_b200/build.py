@@ -37,8 +37,9 @@ def nvcc():
     return exe
 
 
-def _digest():
+def _digest(extra_flags=()):
     h = hashlib.sha256()
+    h.update(" ".join(extra_flags).encode())
     for name in SOURCES + HEADERS:
         with open(os.path.join(CSRC, name), "rb") as f:
             h.update(name.encode() + f.read())
@@ -48,35 +49,41 @@ def _digest():
     return h.hexdigest()
 
 
-def build(verbose=False, force=False):
-    """Compile every source and link the library; skipped when up to date."""
-    os.makedirs(BUILD_DIR, exist_ok=True)
-    stamp = os.path.join(BUILD_DIR, "libmuon_b200.sha256")
-    digest = _digest()
-    if not force and os.path.exists(LIB) and os.path.exists(stamp):
+def build(verbose=False, force=False, extra_flags=(), out=None, build_dir=None):
+    """Compile every source and link the library; skipped when up to date.
+
+    `extra_flags`, `out` and `build_dir` produce a variant library (for
+    example an instrumented one) elsewhere without touching the product.
+    """
+    out = out or LIB
+    bdir = build_dir or BUILD_DIR
+    os.makedirs(bdir, exist_ok=True)
+    stamp = os.path.join(bdir, os.path.basename(out) + ".sha256")
+    digest = _digest(extra_flags)
+    if not force and os.path.exists(out) and os.path.exists(stamp):
         with open(stamp) as f:
             if f.read().strip() == digest:
-                return LIB
+                return out
     objs = []
     for src in SOURCES:
-        obj = os.path.join(BUILD_DIR, src.replace(".cu", ".o"))
-        cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
+        obj = os.path.join(bdir, src.replace(".cu", ".o"))
+        cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *extra_flags, "-c", os.path.join(CSRC, src), "-o", obj]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if verbose or res.returncode != 0:
             sys.stderr.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)
         if res.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}")
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    tmp = out + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, "-ldl", "-lpthread", "-lrt"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(" ".join(cmd) + "\n" + res.stdout + res.stderr)
         raise RuntimeError("link of libmuon_b200.so failed")
-    os.replace(tmp, LIB)
+    os.replace(tmp, out)
     with open(stamp, "w") as f:
         f.write(digest)
-    return LIB
+    return out
 
 
 if __name__ == "__main__":

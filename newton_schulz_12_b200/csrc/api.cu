@@ -242,16 +242,17 @@ int sym_maps(tc::Maps& M, const void* S, int m, int k, long long lds, long long 
   return MUON_OK;
 }
 
-// Maps of X' = a X + B X: B (m x m), X bf16 operand (m x n, read MN-major),
-// X fp32 master (m x n, read and written), X' bf16 (m x n).
-int bx_maps(tc::Maps& M, const void* B, long long ldb, long long sb, const void* Xb, float* Xf,
-            void* Xout, int m, int n, long long ldx, long long sx, int batch) {
+// Maps of X' = a X + B X with X carried as the bf16 pair hi + lo: B (m x m),
+// hi of X (m x n: MN-major operand and epilogue chunks), lo of X (read and
+// written in place), hi of X' (written).
+int bx_maps(tc::Maps& M, const void* B, long long ldb, long long sb, const void* Xhi,
+            void* Xlo, void* Xhi_out, int m, int n, long long ldx, long long sx, int batch) {
   MUON_TRY(make_map(&M.p, B, 2, m, m, batch, ldb, sb, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
-  MUON_TRY(make_map(&M.q, Xb, 2, n, m, batch, ldx, sx, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
-  MUON_TRY(make_map(&M.e, Xf, 4, n, m, batch, ldx, sx, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
-  MUON_TRY(make_map(&M.d, Xout, 2, n, m, batch, ldx, sx, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
-  M.mt = M.d;
-  M.s = M.d;
+  MUON_TRY(make_map(&M.q, Xhi, 2, n, m, batch, ldx, sx, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+  MUON_TRY(make_map(&M.e, Xhi, 2, n, m, batch, ldx, sx, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
+  MUON_TRY(make_map(&M.mt, Xlo, 2, n, m, batch, ldx, sx, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
+  MUON_TRY(make_map(&M.d, Xhi_out, 2, n, m, batch, ldx, sx, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
+  M.s = M.d;  // unused
   return MUON_OK;
 }
 
@@ -260,9 +261,10 @@ int bx_maps(tc::Maps& M, const void* B, long long ldb, long long sb, const void*
 struct NsGroup {
   int batch = 0, m = 0, n = 0;
   long long ldn = 0, ldm = 0;
-  float* xf = nullptr;          // fp32 master X (bf16 path) / ping buffer (fp32 path)
-  float* xf1 = nullptr;         // fp32 pong buffer (fp32 path)
-  bf16* xb[2] = {nullptr, nullptr};
+  float* xf = nullptr;          // fp32 path: ping buffer of X
+  float* xf1 = nullptr;         // fp32 path: pong buffer of X
+  bf16* xb[2] = {nullptr, nullptr};  // bf16 path: hi of X (ping-pong; the GEMM operand)
+  bf16* xlo = nullptr;               // bf16 path: lo of X, X = hi + lo
   bf16* A = nullptr;
   bf16* B = nullptr;
   float* Af = nullptr;
@@ -283,9 +285,9 @@ size_t layout_group(NsGroup& g, char* base, size_t off, bool fp32) {
     return p;
   };
   if (!fp32) {
-    g.xf = reinterpret_cast<float*>(take(xe * 4));
     g.xb[0] = reinterpret_cast<bf16*>(take(xe * 2));
     g.xb[1] = reinterpret_cast<bf16*>(take(xe * 2));
+    g.xlo = reinterpret_cast<bf16*>(take(xe * 2));
     g.A = reinterpret_cast<bf16*>(take(ae * 2));
     g.B = reinterpret_cast<bf16*>(take(ae * 2));
   } else {
@@ -310,6 +312,10 @@ tc::Group tc_group(int batch, int m, int n, int k, bool sym, int tile_begin) {
   return G;
 }
 
+#ifdef MUON_TRACE
+unsigned long long* g_trace = nullptr;  // device buffer for kernel timestamps
+#endif
+
 void init_tc_params(tc::Params& P, int* status, float a, float b, float c) {
   P.ngroups = 0;
   P.total_tiles = 0;
@@ -319,6 +325,10 @@ void init_tc_params(tc::Params& P, int* status, float a, float b, float c) {
   P.status = status;
   P.timeout_ns = g_timeout_ns;
   P.inject = 0;
+  P.trace = nullptr;
+#ifdef MUON_TRACE
+  P.trace = g_trace;
+#endif
 }
 
 int launch_tc(int epi, tc::Params& P, int sms, cudaStream_t s) {
@@ -336,8 +346,8 @@ int launch_tc(int epi, tc::Params& P, int sms, cudaStream_t s) {
   return MUON_OK;
 }
 
-// T steps of X <- aX + (bA + cA^2)X on bf16 operands with fp32 master X.
-// On entry each group's xf / xb[0] hold X0; on exit xf holds X_T.
+// T steps of X <- aX + (bA + cA^2)X on bf16 operands, X carried as hi + lo.
+// On entry each group's xb[0] / xlo hold X0; on exit xb[T % 2] / xlo hold X_T.
 int run_ns_bf16(std::vector<NsGroup>& gs, int steps, float a, float b, float c, int* status,
                 int sms, cudaStream_t s) {
   if (steps <= 0 || gs.empty()) return MUON_OK;
@@ -363,7 +373,7 @@ int run_ns_bf16(std::vector<NsGroup>& gs, int steps, float a, float b, float c, 
         gram[par].ngroups = k + 1;
 
         bx[par].grp[k] = tc_group(G.batch, G.m, G.n, G.m, false, bx[par].total_tiles);
-        MUON_TRY(bx_maps(bx[par].map[k], G.B, G.ldm, as, G.xb[par], G.xf, G.xb[par ^ 1], G.m, G.n,
+        MUON_TRY(bx_maps(bx[par].map[k], G.B, G.ldm, as, G.xb[par], G.xlo, G.xb[par ^ 1], G.m, G.n,
                          G.ldn, xs, G.batch));
         bx[par].total_tiles += G.batch * bx[par].grp[k].tiles_per_mat;
         bx[par].ngroups = k + 1;
@@ -382,6 +392,20 @@ int run_ns_bf16(std::vector<NsGroup>& gs, int steps, float a, float b, float c, 
     }
   }
   return MUON_OK;
+}
+
+// Where a group's result X_T lives: fp32, or the bf16 pair hi + lo.
+struct Result {
+  const float* f = nullptr;
+  const bf16* hi = nullptr;
+  const bf16* lo = nullptr;
+};
+
+Result bf16_result(const NsGroup& g, int steps) {
+  Result r;
+  r.hi = g.xb[steps & 1];
+  r.lo = g.xlo;
+  return r;
 }
 
 // fp32 SIMT verification path; on exit *final_xf of each group holds X_T.
@@ -546,9 +570,11 @@ int launch_cast_chunked(const std::vector<MatInfo>& mats, std::vector<NsGroup>& 
       C.part_begin = part_begin[i];
       C.part_count = part_count[i];
       const long long off = static_cast<long long>(M.index) * G.m * G.ldn;
-      C.xf = G.xf + off;
+      C.xf = with_bf16 ? nullptr : G.xf + off;
       C.xb = with_bf16 ? static_cast<void*>(G.xb[0] + off) : nullptr;
+      C.xlo = with_bf16 ? static_cast<void*>(G.xlo + off) : nullptr;
       C.ld = G.ldn;
+      C.vec = (M.cols % 8 == 0) && aligned16(src0[i]) && (src1.empty() || aligned16(src1[i]));
       tiles += ((M.m + ew::kTile - 1) / ew::kTile) * C.tiles_n;
     }
     cp.nmat = i1 - i0;
@@ -560,9 +586,9 @@ int launch_cast_chunked(const std::vector<MatInfo>& mats, std::vector<NsGroup>& 
 }
 
 // mode 0: apply into W; 1: bf16 write-back; 2: fp32 write-back.  O of matrix i
-// is read from its group's buffer `final_xf[group]` (X layout, transposed back).
+// is read from its group's result (X layout, transposed back).
 int launch_out_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGroup>& groups,
-                       const std::vector<float*>& final_xf, const std::vector<void*>& ys, int mode,
+                       const std::vector<Result>& res, const std::vector<void*>& ys, int mode,
                        float lr, float wd, cudaStream_t s) {
   const int count = static_cast<int>(mats.size());
   for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
@@ -576,7 +602,11 @@ int launch_out_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGro
       const NsGroup& G = groups[M.group];
       ew::OutMat& O = op.mat[i - i0];
       O.y = ys[i];
-      O.o = final_xf[M.group] + static_cast<long long>(M.index) * G.m * G.ldn;
+      const long long roff = static_cast<long long>(M.index) * G.m * G.ldn;
+      const Result& R = res[M.group];
+      O.o = R.f ? R.f + roff : nullptr;
+      O.o_hi = R.f ? nullptr : static_cast<const void*>(R.hi + roff);
+      O.o_lo = R.f ? nullptr : static_cast<const void*>(R.lo + roff);
       O.rows = M.rows;
       O.cols = M.cols;
       O.o_transposed = M.transposed;
@@ -586,6 +616,7 @@ int launch_out_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGro
       const float ratio = static_cast<float>(M.rows) / static_cast<float>(M.cols);
       const float scale = ratio > 1.0f ? sqrtf(ratio) : 1.0f;
       O.ls = lr * scale;
+      O.vec = (M.cols % 8 == 0) && (G.ldn % 8 == 0) && aligned16(ys[i]);
       tiles += ((M.rows + ew::kTile - 1) / ew::kTile) * O.tiles_c;
     }
     op.nmat = i1 - i0;
@@ -658,6 +689,14 @@ extern "C" {
 
 int muon_version(void) { return kVersion; }
 
+#ifdef MUON_TRACE
+// Trace builds only: device buffer that tensor-core launches stamp into.
+int muon_debug_trace(void* dev_buffer) {
+  g_trace = static_cast<unsigned long long*>(dev_buffer);
+  return MUON_OK;
+}
+#endif
+
 const char* muon_last_error(void) { return t_err.c_str(); }
 
 int muon_set_wait_timeout_ms(int ms) {
@@ -710,15 +749,21 @@ int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a,
   const int kind = fp32 ? ew::kFromF32 : ew::kFromBf16;
   MUON_TRY(launch_flat_chunked(src, {}, numels, kind, 0.f, 0, partials, pb, pc, s));
   MUON_TRY(launch_cast_chunked(mats, groups, src, {}, kind, 0.f, 0, partials, pb, pc, !fp32, s));
-  std::vector<float*> final_xf;
+  std::vector<Result> res;
   if (fp32) {
+    std::vector<float*> final_xf;
     MUON_TRY(run_ns_fp32(groups, steps, a, b, c, s, final_xf));
+    for (float* f : final_xf) {
+      Result r;
+      r.f = f;
+      res.push_back(r);
+    }
   } else {
     MUON_TRY(run_ns_bf16(groups, steps, a, b, c, ws->status, dev.sms, s));
-    for (NsGroup& g : groups) final_xf.push_back(g.xf);
+    for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
   }
   std::vector<void*> ys(X_ptrs, X_ptrs + batch);
-  MUON_TRY(launch_out_chunked(mats, groups, final_xf, ys, fp32 ? 2 : 1, 0.f, 0.f, s));
+  MUON_TRY(launch_out_chunked(mats, groups, res, ys, fp32 ? 2 : 1, 0.f, 0.f, s));
   return MUON_OK;
 }
 
@@ -769,10 +814,10 @@ int muon_ns_orthogonalize_static(int batch, int m, int n, void* const* X_ptrs, f
   MUON_TRY(launch_flat_chunked(src, {}, numels, ew::kFromBf16, 0.f, 0, partials, pb, pc, s));
   MUON_TRY(launch_cast_chunked(mats, groups, src, {}, ew::kFromBf16, 0.f, 0, partials, pb, pc, true, s));
   MUON_TRY(run_ns_bf16(groups, steps, a, b, c, status, dev.sms, s));
-  std::vector<float*> final_xf;
-  for (NsGroup& g : groups) final_xf.push_back(g.xf);
+  std::vector<Result> res;
+  for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
   std::vector<void*> ys(X_ptrs, X_ptrs + batch);
-  MUON_TRY(launch_out_chunked(mats, groups, final_xf, ys, 1, 0.f, 0.f, s));
+  MUON_TRY(launch_out_chunked(mats, groups, res, ys, 1, 0.f, 0.f, s));
   return MUON_OK;
 }
 
@@ -823,10 +868,10 @@ int muon_step(int count, float* const* params, const void* const* grads,
   MUON_TRY(launch_cast_chunked(mats, groups, gsrc, cbufs, ew::kFromMomentum, beta, nesterov,
                                partials, pb, pc, true, s));
   MUON_TRY(run_ns_bf16(groups, steps, kCoefA, kCoefB, kCoefC, ws->status, dev.sms, s));
-  std::vector<float*> final_xf;
-  for (NsGroup& g : groups) final_xf.push_back(g.xf);
+  std::vector<Result> res;
+  for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
   std::vector<void*> ys(params, params + count);
-  MUON_TRY(launch_out_chunked(mats, groups, final_xf, ys, 0, lr, wd, s));
+  MUON_TRY(launch_out_chunked(mats, groups, res, ys, 0, lr, wd, s));
   return MUON_OK;
 }
 
@@ -910,6 +955,7 @@ int muon_apply(int count, float* const* params, const float* const* updates, con
       const float ratio = static_cast<float>(r) / static_cast<float>(c);
       const float scale = ratio > 1.0f ? sqrtf(ratio) : 1.0f;
       O.ls = lr * scale;
+      O.vec = (c % 8 == 0) && aligned16(params[i]) && aligned16(updates[i]);
       tiles += ((r + ew::kTile - 1) / ew::kTile) * O.tiles_c;
     }
     op.nmat = i1 - i0;
@@ -967,13 +1013,14 @@ int muon_poly_bf16(int batch, int m, const void* A, void* B, float b, float c, v
   return launch_tc(tc::kPoly, P, dev.sms, s);
 }
 
-int muon_bx_bf16(int batch, int m, int n, const void* B, const void* Xb, float* Xf, void* Xb_out,
+int muon_bx_bf16(int batch, int m, int n, const void* B, const void* Xhi, void* Xlo, void* Xhi_out,
                  float a, void* stream) {
   t_err.clear();
   if (batch == 0) return MUON_OK;
-  if (!B || !Xb || !Xf || !Xb_out || !aligned16(B) || !aligned16(Xb) || !aligned16(Xf) || !aligned16(Xb_out))
-    return set_err(MUON_ERR_ARG, "B, Xb, Xf and Xb_out must be non-NULL and 16-byte aligned");
-  if (Xb == Xb_out) return set_err(MUON_ERR_ARG, "Xb_out must not alias Xb");
+  if (!B || !Xhi || !Xlo || !Xhi_out || !aligned16(B) || !aligned16(Xhi) || !aligned16(Xlo) ||
+      !aligned16(Xhi_out))
+    return set_err(MUON_ERR_ARG, "B, Xhi, Xlo and Xhi_out must be non-NULL and 16-byte aligned");
+  if (Xhi == Xhi_out) return set_err(MUON_ERR_ARG, "Xhi_out must not alias Xhi");
   if (m > n) return set_err(MUON_ERR_SHAPE, "muon_bx_bf16 expects m <= n (got %dx%d)", m, n);
   cudaStream_t s = as_stream(stream);
   DevInfo dev;
@@ -983,7 +1030,7 @@ int muon_bx_bf16(int batch, int m, int n, const void* B, const void* Xb, float* 
   init_tc_params(P, ws->status, a, 0.f, 0.f);
   const long long xs = static_cast<long long>(m) * n, as = static_cast<long long>(m) * m;
   P.grp[0] = tc_group(batch, m, n, m, false, 0);
-  MUON_TRY(bx_maps(P.map[0], B, m, as, Xb, Xf, Xb_out, m, n, n, xs, batch));
+  MUON_TRY(bx_maps(P.map[0], B, m, as, Xhi, Xlo, Xhi_out, m, n, n, xs, batch));
   P.ngroups = 1;
   P.total_tiles = batch * P.grp[0].tiles_per_mat;
   return launch_tc(tc::kBx, P, dev.sms, s);

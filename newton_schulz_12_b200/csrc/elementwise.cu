@@ -5,8 +5,8 @@
 //                 orthogonalisation entry, the partial of sum(x^2) only.
 //                 128-bit loads/stores, fixed-order block reduction.
 //   cast_kernel   X0 = u / (||u||_F + eps), transposed to rows <= cols when the
-//                 matrix is tall, written as the fp32 master X and its bf16
-//                 operand copy.  64x64 tiles staged through shared memory so
+//                 matrix is tall, written as the bf16 pair hi = bf16(X),
+//                 lo = bf16(X - hi) (fp32 for the verification path).  64x64 tiles staged through shared memory so
 //                 both the read and the (possibly transposed) write coalesce.
 //   out_kernel    W' = (W - lw W) - ls O (the apply), or the write-back of the
 //                 result into the caller's bf16 / fp32 buffer, with O read
@@ -157,6 +157,113 @@ __device__ __forceinline__ int find_tile_mat(const Mats& mats, int nmat, int t) 
   return lo;
 }
 
+// ---------------------------------------------------------------- tile kernels
+// One 64x64 tile per block; thread t owns two runs of 8 consecutive elements
+// (rows t/8 and t/8 + 32, columns 8*(t%8) .. +7) and moves them with 128-bit
+// accesses when the rows are 16-byte aligned (`vec`), else element by element.
+// A tall matrix's tile is transposed through shared memory so that both the
+// read and the write run along rows.
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4 w, float (&x)[8]) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    x[2 * h] = bf16_bits_to_f32(static_cast<uint16_t>(ws[h] & 0xFFFFu));
+    x[2 * h + 1] = bf16_bits_to_f32(static_cast<uint16_t>(ws[h] >> 16));
+  }
+}
+
+// u[k] = U[r][c + k] for k < 8 (0 outside the matrix); U is the momentum
+// update (recomputed from g and the updated buffer with flat_kernel's
+// rounding) or the caller's X.
+__device__ __forceinline__ void load_u8(const CastParams& p, const CastMat& M, int r, int c,
+                                        float (&u)[8]) {
+  const int cnt = r < M.rows ? min(8, M.cols - c) : 0;
+  const long long idx = static_cast<long long>(r) * M.cols + c;
+  if (cnt == 8 && M.vec) {
+    if (p.src_kind == kFromF32) {
+      const float4* s4 = reinterpret_cast<const float4*>(static_cast<const float*>(M.src0) + idx);
+      const float4 a = s4[0], b = s4[1];
+      u[0] = a.x; u[1] = a.y; u[2] = a.z; u[3] = a.w;
+      u[4] = b.x; u[5] = b.y; u[6] = b.z; u[7] = b.w;
+      return;
+    }
+    float g[8];
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const bf16*>(M.src0) + idx), g);
+    if (p.src_kind == kFromMomentum) {
+      const float4* b4 = reinterpret_cast<const float4*>(M.src1 + idx);
+      const float4 a = b4[0], b = b4[1];
+      const float nb[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        u[k] = p.nesterov ? __fadd_rn(__fmul_rn(p.omb, g[k]), __fmul_rn(p.beta, nb[k])) : nb[k];
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) u[k] = g[k];
+    }
+    return;
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float v = 0.f;
+    if (k < cnt) {
+      if (p.src_kind == kFromF32) {
+        v = static_cast<const float*>(M.src0)[idx + k];
+      } else {
+        const float g = bf16_bits_to_f32(static_cast<const uint16_t*>(M.src0)[idx + k]);
+        if (p.src_kind == kFromMomentum) {
+          const float nb = M.src1[idx + k];
+          v = p.nesterov ? __fadd_rn(__fmul_rn(p.omb, g), __fmul_rn(p.beta, nb)) : nb;
+        } else {
+          v = g;
+        }
+      }
+    }
+    u[k] = v;
+  }
+}
+
+// X[i][j + k] = u[k] / den, written as fp32 (verification path) or as the
+// bf16 pair hi = bf16(x), lo = bf16(x - hi) that carries X between steps.
+__device__ __forceinline__ void store_x8(const CastMat& M, int i, int j, int m, int n, float den,
+                                         const float (&u)[8]) {
+  if (i >= m || j >= n) return;
+  const long long o = static_cast<long long>(i) * M.ld + j;
+  float x[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) x[k] = __fdiv_rn(u[k], den);
+  uint32_t hi[4], lo[4];
+  if (!M.xf) {
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      hi[h] = pack_bf16x2(x[2 * h], x[2 * h + 1]);
+      lo[h] = pack_bf16x2(x[2 * h] - bf16_bits_to_f32(static_cast<uint16_t>(hi[h] & 0xFFFFu)),
+                          x[2 * h + 1] - bf16_bits_to_f32(static_cast<uint16_t>(hi[h] >> 16)));
+    }
+  }
+  if (j + 8 <= n) {  // the workspace row stride is a multiple of 8: always aligned
+    if (M.xf) {
+      float4* f4 = reinterpret_cast<float4*>(M.xf + o);
+      f4[0] = make_float4(x[0], x[1], x[2], x[3]);
+      f4[1] = make_float4(x[4], x[5], x[6], x[7]);
+    } else {
+      *reinterpret_cast<uint4*>(static_cast<bf16*>(M.xb) + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(static_cast<bf16*>(M.xlo) + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+  } else {
+    for (int k = 0; k < n - j; ++k) {
+      if (M.xf) {
+        M.xf[o + k] = x[k];
+      } else {
+        const uint32_t w = (k & 1) ? (hi[k >> 1] >> 16) : (hi[k >> 1] & 0xFFFFu);
+        const uint32_t l = (k & 1) ? (lo[k >> 1] >> 16) : (lo[k >> 1] & 0xFFFFu);
+        static_cast<uint16_t*>(M.xb)[o + k] = static_cast<uint16_t>(w);
+        static_cast<uint16_t*>(M.xlo)[o + k] = static_cast<uint16_t>(l);
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kTileThreads) cast_kernel(const __grid_constant__ CastParams p) {
   __shared__ float tile[kTile][kTile + 1];
   __shared__ float s_den;
@@ -167,47 +274,111 @@ __global__ void __launch_bounds__(kTileThreads) cast_kernel(const __grid_constan
   const int m = M.transposed ? M.cols : M.rows;  // X is m x n
   const int n = M.transposed ? M.rows : M.cols;
   const int i0 = ti * kTile, j0 = tj * kTile;
-
   if (threadIdx.x < 32) {
     const float ss = warp_sum_partials(p.partials, M.part_begin, M.part_count);
     if (threadIdx.x == 0) s_den = __fadd_rn(__fsqrt_rn(ss), p.eps);
   }
-  // source region: U rows [sr0, sr0+64), cols [sc0, sc0+64)
-  const int sr0 = M.transposed ? j0 : i0;
-  const int sc0 = M.transposed ? i0 : j0;
-  const int tx = threadIdx.x & (kTile - 1), ty = threadIdx.x >> 6;
-#pragma unroll 4
-  for (int y = ty; y < kTile; y += kTileThreads / kTile) {
-    const int r = sr0 + y, c = sc0 + tx;
-    float u = 0.f;
-    if (r < M.rows && c < M.cols) {
-      const long long idx = static_cast<long long>(r) * M.cols + c;
-      if (p.src_kind == kFromF32) {
-        u = static_cast<const float*>(M.src0)[idx];
-      } else {
-        const float g = bf16_bits_to_f32(static_cast<const uint16_t*>(M.src0)[idx]);
-        if (p.src_kind == kFromMomentum) {
-          // recompute u from g and the already updated buffer (same rounding as flat_kernel)
-          const float nb = M.src1[idx];
-          u = p.nesterov ? __fadd_rn(__fmul_rn(p.omb, g), __fmul_rn(p.beta, nb)) : nb;
-        } else {
-          u = g;
-        }
-      }
+  const int y = threadIdx.x >> 3, xg = (threadIdx.x & 7) * 8;
+  float u[2][8];
+  if (!M.transposed) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) load_u8(p, M, i0 + y + 32 * h, j0 + xg, u[h]);
+    __syncthreads();
+    const float den = s_den;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) store_x8(M, i0 + y + 32 * h, j0 + xg, m, n, den, u[h]);
+  } else {
+    // X[i0 + a][j0 + b] = U[j0 + b][i0 + a]: read U rows j0.., columns i0..
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      load_u8(p, M, j0 + y + 32 * h, i0 + xg, u[h]);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) tile[y + 32 * h][xg + k] = u[h][k];
     }
-    tile[y][tx] = u;
+    __syncthreads();
+    const float den = s_den;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float t[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) t[k] = tile[xg + k][y + 32 * h];
+      store_x8(M, i0 + y + 32 * h, j0 + xg, m, n, den, t);
+    }
   }
-  __syncthreads();
-  const float den = s_den;
-#pragma unroll 4
-  for (int y = ty; y < kTile; y += kTileThreads / kTile) {
-    const int i = i0 + y, j = j0 + tx;
-    if (i < m && j < n) {
-      const float u = M.transposed ? tile[tx][y] : tile[y][tx];
-      const float x = __fdiv_rn(u, den);
-      const long long o = static_cast<long long>(i) * M.ld + j;
-      M.xf[o] = x;
-      if (M.xb) static_cast<bf16*>(M.xb)[o] = __float2bfloat16_rn(x);
+}
+
+// o[k] = O[r][c + k] read from the m x n result buffer (row stride ld) as laid
+// out there: rows r of that buffer, columns c.. (0 outside it).  The buffer is
+// fp32, or the bf16 pair hi + lo.
+__device__ __forceinline__ void load_o8(const OutMat& M, int r, int c, int orows, int ocols,
+                                        float (&o)[8]) {
+  const int cnt = r < orows ? min(8, ocols - c) : 0;
+  const long long idx = static_cast<long long>(r) * M.ld + c;
+  if (M.o_hi) {
+    if (cnt == 8 && M.vec) {
+      float h[8], l[8];
+      unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const bf16*>(M.o_hi) + idx), h);
+      unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const bf16*>(M.o_lo) + idx), l);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) o[k] = h[k] + l[k];
+      return;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      o[k] = k < cnt ? bf16_bits_to_f32(static_cast<const uint16_t*>(M.o_hi)[idx + k]) +
+                           bf16_bits_to_f32(static_cast<const uint16_t*>(M.o_lo)[idx + k])
+                     : 0.f;
+    return;
+  }
+  if (cnt == 8 && M.vec) {
+    const float4* s4 = reinterpret_cast<const float4*>(M.o + idx);
+    const float4 a = s4[0], b = s4[1];
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+    o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+    return;
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) o[k] = k < cnt ? M.o[idx + k] : 0.f;
+}
+
+// Y[r][c + k] op= o[k]: the apply W' = (W - lw W) - ls O, or a write-back.
+__device__ __forceinline__ void update_y8(const OutParams& p, const OutMat& M, int r, int c,
+                                          const float (&o)[8]) {
+  if (r >= M.rows || c >= M.cols) return;
+  const long long idx = static_cast<long long>(r) * M.cols + c;
+  const int cnt = min(8, M.cols - c);
+  if (cnt == 8 && M.vec) {
+    if (p.mode == 0) {
+      float4* w4 = reinterpret_cast<float4*>(static_cast<float*>(M.y) + idx);
+      const float4 a = w4[0], b = w4[1];
+      float w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w[k] = __fsub_rn(__fsub_rn(w[k], __fmul_rn(p.lw, w[k])), __fmul_rn(M.ls, o[k]));
+      w4[0] = make_float4(w[0], w[1], w[2], w[3]);
+      w4[1] = make_float4(w[4], w[5], w[6], w[7]);
+    } else if (p.mode == 1) {
+      uint4 v;
+      v.x = pack_bf16x2(o[0], o[1]);
+      v.y = pack_bf16x2(o[2], o[3]);
+      v.z = pack_bf16x2(o[4], o[5]);
+      v.w = pack_bf16x2(o[6], o[7]);
+      *reinterpret_cast<uint4*>(static_cast<bf16*>(M.y) + idx) = v;
+    } else {
+      float4* y4 = reinterpret_cast<float4*>(static_cast<float*>(M.y) + idx);
+      y4[0] = make_float4(o[0], o[1], o[2], o[3]);
+      y4[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+    return;
+  }
+  for (int k = 0; k < cnt; ++k) {
+    if (p.mode == 0) {
+      float* W = static_cast<float*>(M.y);
+      const float w = W[idx + k];
+      W[idx + k] = __fsub_rn(__fsub_rn(w, __fmul_rn(p.lw, w)), __fmul_rn(M.ls, o[k]));
+    } else if (p.mode == 1) {
+      static_cast<bf16*>(M.y)[idx + k] = __float2bfloat16_rn(o[k]);
+    } else {
+      static_cast<float*>(M.y)[idx + k] = o[k];
     }
   }
 }
@@ -219,34 +390,30 @@ __global__ void __launch_bounds__(kTileThreads) out_kernel(const __grid_constant
   const int local = blockIdx.x - M.tile_begin;
   const int tr = local / M.tiles_c, tcn = local - tr * M.tiles_c;
   const int r0 = tr * kTile, c0 = tcn * kTile;
-  const int tx = threadIdx.x & (kTile - 1), ty = threadIdx.x >> 6;
-
-  // stage O's tile: O[r][c] = o[c*ld + r] when transposed, else o[r*ld + c]
-  const int orow0 = M.o_transposed ? c0 : r0;
-  const int ocol0 = M.o_transposed ? r0 : c0;
-  const int orows = M.o_transposed ? M.cols : M.rows;
-  const int ocols = M.o_transposed ? M.rows : M.cols;
-#pragma unroll 4
-  for (int y = ty; y < kTile; y += kTileThreads / kTile) {
-    const int r = orow0 + y, c = ocol0 + tx;
-    tile[y][tx] = (r < orows && c < ocols) ? M.o[static_cast<long long>(r) * M.ld + c] : 0.f;
-  }
-  __syncthreads();
-#pragma unroll 4
-  for (int y = ty; y < kTile; y += kTileThreads / kTile) {
-    const int r = r0 + y, c = c0 + tx;
-    if (r < M.rows && c < M.cols) {
-      const float o = M.o_transposed ? tile[tx][y] : tile[y][tx];
-      const long long idx = static_cast<long long>(r) * M.cols + c;
-      if (p.mode == 0) {
-        float* W = static_cast<float*>(M.y);
-        const float w = W[idx];
-        W[idx] = __fsub_rn(__fsub_rn(w, __fmul_rn(p.lw, w)), __fmul_rn(M.ls, o));
-      } else if (p.mode == 1) {
-        static_cast<bf16*>(M.y)[idx] = __float2bfloat16_rn(o);
-      } else {
-        static_cast<float*>(M.y)[idx] = o;
-      }
+  const int y = threadIdx.x >> 3, xg = (threadIdx.x & 7) * 8;
+  if (!M.o_transposed) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float o[8];
+      load_o8(M, r0 + y + 32 * h, c0 + xg, M.rows, M.cols, o);
+      update_y8(p, M, r0 + y + 32 * h, c0 + xg, o);
+    }
+  } else {
+    // O[r0 + a][c0 + b] = buffer[c0 + b][r0 + a]
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float o[8];
+      load_o8(M, c0 + y + 32 * h, r0 + xg, M.cols, M.rows, o);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) tile[y + 32 * h][xg + k] = o[k];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float o[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) o[k] = tile[xg + k][y + 32 * h];
+      update_y8(p, M, r0 + y + 32 * h, c0 + xg, o);
     }
   }
 }

@@ -7,9 +7,11 @@
 //
 //   kGram  A  = X X^T            tiles touching the upper triangle, mirrored
 //   kPoly  B  = b A + c A A      A symmetric, so A A = A A^T: same tiling
-//   kBx    X' = a X + B X        fp32 master X updated in place, bf16 copy out
+//   kBx    X' = a X + B X        X carried as a pair of bf16 matrices, X = hi + lo
 //
 // One CTA per SM, persistent over a static tile stride; 128 x 256 output tiles.
+// (Roles below; the epilogue runs on warps 2-9, two warps per TMEM lane
+// quarter, each on half of every 32-column chunk.)
 //   warp 0      one thread issues bulk tensor copies of the operand tiles
 //               (128x64 and 256x64 bf16, 128-byte swizzle) into a ring of
 //               STAGES shared-memory stages;
@@ -40,17 +42,17 @@ constexpr uint32_t kTileBytesQ = BN * BK * 2;               // 32 KiB
 constexpr uint32_t kStageBytes = kTileBytesP + kTileBytesQ;  // 48 KiB
 constexpr uint32_t kTmemCols = 2 * BN;                      // two accumulators
 constexpr uint32_t kChunkBf16 = BM * kChunk * 2;            // 8 KiB
-constexpr uint32_t kChunkF32 = BM * kChunk * 4;             // 16 KiB
 
 template <int EPI>
 struct Cfg {
   static constexpr int kStages = (EPI == kGram) ? 4 : 3;
   // epilogue operand ring
-  static constexpr uint32_t kSlotBytes = (EPI == kBx) ? kChunkF32 : (EPI == kPoly ? kChunkBf16 : 0);
+  // kBx slot: the hi and lo bf16 chunks of X (8 KiB each); kPoly slot: A's chunk
+  static constexpr uint32_t kSlotBytes = (EPI == kBx) ? 2 * kChunkBf16 : (EPI == kPoly ? kChunkBf16 : 0);
   static constexpr uint32_t kSlotsBytes = kSlotBytes * kEpiSlots;
   // staging: kBx two bf16 output chunks; kGram / kPoly 2 direct + 2 mirror chunks,
   // aliased by the 128 x 128 diagonal block (2 x [128 rows][64 cols] bf16)
-  static constexpr uint32_t kStagingBytes = (EPI == kBx) ? 2 * kChunkBf16 : 4 * kChunkBf16;
+  static constexpr uint32_t kStagingBytes = (EPI == kBx) ? 0 : 4 * kChunkBf16;
   static constexpr uint32_t kRingBytes = kStages * kStageBytes;
   static constexpr int kNumBars = 2 * kStages + 5 + kEpiSlots;
   static constexpr size_t kSmem =
@@ -146,7 +148,7 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 
-// AND of `v` over the 128 epilogue threads (hardware barrier 3).  Every
+// AND of `v` over the 256 epilogue threads (hardware barrier 3).  Every
 // possibly-failing wait of the epilogue is followed by this, so the four
 // epilogue warps always take the same branch and never strand one another at
 // a later barrier.
@@ -155,13 +157,25 @@ __device__ __forceinline__ bool epi_all(bool v) {
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 3, 128, p;\n\t"
+      "bar.red.and.pred q, 3, 256, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(out)
       : "r"(static_cast<uint32_t>(v))
       : "memory");
   return out != 0;
 }
+
+#ifdef MUON_TRACE
+__device__ __forceinline__ void trace_stamp(const Params& p, int tile, int slot) {
+  if (p.trace && blockIdx.x < kTraceCtas && tile < kTraceTiles)
+    p.trace[(blockIdx.x * kTraceTiles + tile) * kTraceSlots + slot] = global_ns();
+}
+#define TRACE(tile, slot) trace_stamp(p, tile, slot)
+#else
+#define TRACE(tile, slot) \
+  do {                    \
+  } while (0)
+#endif
 
 // ---------------------------------------------------------------------- kernel
 template <int EPI>
@@ -195,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 4 * 32);
+      mbar_init(tempty_bar(a), 8 * 32);
     }
     mbar_init(drain_bar, 1);
     for (int s = 0; s < kEpiSlots; ++s) mbar_init(efull_bar(s), 1);
@@ -251,6 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const int left = G.n - tc.tn * BN;
             qboxes = left >= BN ? BN / 64 : (left + 63) / 64;
           }
+          if (kb == 0) TRACE(k, 0);
+          if (kb == kblocks - 1) TRACE(k, 1);
           mbar_arrive_expect_tx(full_bar(stage), kTileBytesP + qboxes * 8192u);
           issued_mask |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -293,6 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         const int kblocks = (p.grp[tc.g].k + BK - 1) / BK;
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, ctl)) break;
         tc_fence_after();
+        TRACE(k, 2);
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, ctl)) {
@@ -316,6 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           }
         }
         if (!ok) break;
+        TRACE(k, 3);
         tc_commit(tfull_bar(acc));
         if (++acc == 2) {
           acc = 0;
@@ -327,13 +345,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (warps 2-9)
+    // Two warps per TMEM lane quarter: warp w reads lanes 32*(w%4).. and the
+    // half `hf` of each 32-column chunk (16 columns), so a chunk's element
+    // work is spread over all four SM sub-partitions twice.
     const int lane_base = 32 * (warp & 3);
+    const int hf = (warp - 2) >> 2;  // column half of the chunk
     const int r = lane_base + lane;  // tile row owned by this thread
     const bool leader = (warp == 2 && lane == 0);
     const int total_chunks = my_tiles * kChunks;
     const uint32_t slots_u32 = smem_u32(slots);
     const uint32_t stage_u32 = smem_u32(staging);
+    constexpr int kEpiThreads = 256;
 
     // Epilogue operand prefetch of chunk s into slot s % kEpiSlots (leader only).
     int pend[kEpiSlots] = {-1, -1, -1, -1};  // last chunk issued per slot
@@ -348,11 +371,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       if (kind == kSkip) {
         mbar_arrive(efull_bar(slot));
       } else {
+        const uint32_t dst = slots_u32 + slot * C::kSlotBytes;
         mbar_arrive_expect_tx(efull_bar(slot), C::kSlotBytes);
-        tma_load_3d(slots_u32 + slot * C::kSlotBytes, &p.map[tc.g].e, efull_bar(slot), col0,
-                    tc.tm * BM, tc.b);
+        tma_load_3d(dst, &p.map[tc.g].e, efull_bar(slot), col0, tc.tm * BM, tc.b);
+        if (EPI == kBx)  // lo half of X next to its hi half
+          tma_load_3d(dst + kChunkBf16, &p.map[tc.g].mt, efull_bar(slot), col0, tc.tm * BM, tc.b);
       }
     };
+    // kBx refills a slot one chunk late (its store drains meanwhile): chunks
+    // 0..kEpiSlots-1 are loaded up front, then chunk s+kEpiSlots-1 into chunk
+    // s-1's slot once chunk s (s >= 1) is handed to its stores.
+    constexpr int kAhead = (EPI == kBx) ? kEpiSlots - 1 : kEpiSlots;
     if (leader) {
       for (int g = 0; g < p.ngroups; ++g) {
         tma_prefetch_map(&p.map[g].e);
@@ -378,29 +407,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         break;
       }
       tc_fence_after();
+      if (leader) TRACE(k, 4);
       for (int c = 0; c < kChunks; ++c) {
+        if (leader && c > 0) TRACE(k, 4 + c);
         const int s = k * kChunks + c;
         const int col0 = tc.tn * BN + c * kChunk;
         const int kind = chunk_kind<EPI>(G, tc.tm, col0);
-        float v[32];
+        float v[16];
         if (kind != kSkip) {
-          uint32_t rr[32];
+          uint32_t rr[16];
           __syncwarp();
-          tmem_ld_32x32(tmem_base + (static_cast<uint32_t>(lane_base) << 16) +
-                            static_cast<uint32_t>(acc * BN + c * kChunk),
-                        rr);
+          tmem_ld_32x32_x16(tmem_base + (static_cast<uint32_t>(lane_base) << 16) +
+                                static_cast<uint32_t>(acc * BN + c * kChunk + hf * 16),
+                            rr);
           tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(rr[q]);
+          for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(rr[q]);
         }
+        if (leader && c == 2) TRACE(k, 13);
         if (c == kChunks - 1) {
           // accumulator fully read: hand it back to the MMA warp
           tc_fence_before();
           mbar_arrive(tempty_bar(acc));
         }
         if (kind == kSkip) {
-          // nothing loaded for this chunk; its slot goes to chunk s + kEpiSlots
-          if (leader) issue_eload(s + kEpiSlots);
+          if (leader) {
+            if (EPI == kBx) {
+              bulk_wait_read_all();
+              if (s >= 1) issue_eload(s + kAhead);  // chunk s-1's slot is free
+            } else {
+              issue_eload(s + kAhead);
+            }
+          }
           continue;
         }
         const int slot = s % kEpiSlots;
@@ -410,40 +448,49 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             ok = false;
             break;
           }
+          if (leader && c == 2) TRACE(k, 14);
         }
         if (EPI == kBx) {
-          // X' = a X + acc, in place in the slot; bf16 copy to staging[s % 2]
-          const uint32_t es = slots_u32 + slot * C::kSlotBytes;
-          const uint32_t os = stage_u32 + (s & 1) * kChunkBf16;
+          // X = hi + lo from the slot; X' = a X + acc; hi' = bf16(X'),
+          // lo' = bf16(X' - hi'), written back in place and stored from there
+          const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
+          const uint32_t ls = hs + kChunkBf16;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            uint32_t x0, x1, x2, x3;
-            const uint32_t addr = es + sw128(r, u);
-            ld_shared_v4(addr, x0, x1, x2, x3);
-            const float y0 = fmaf(p.a, __uint_as_float(x0), v[4 * u + 0]);
-            const float y1 = fmaf(p.a, __uint_as_float(x1), v[4 * u + 1]);
-            const float y2 = fmaf(p.a, __uint_as_float(x2), v[4 * u + 2]);
-            const float y3 = fmaf(p.a, __uint_as_float(x3), v[4 * u + 3]);
-            st_shared_v4(addr, __float_as_uint(y0), __float_as_uint(y1), __float_as_uint(y2),
-                         __float_as_uint(y3));
-            v[4 * u + 0] = y0;
-            v[4 * u + 1] = y1;
-            v[4 * u + 2] = y2;
-            v[4 * u + 3] = y3;
+          for (int uu = 0; uu < 2; ++uu) {
+            const int u = 2 * hf + uu;  // 16-byte unit of the 64-byte row
+            uint32_t h4[4], l4[4];
+            ld_shared_v4(hs + sw64(r, u), h4[0], h4[1], h4[2], h4[3]);
+            ld_shared_v4(ls + sw64(r, u), l4[0], l4[1], l4[2], l4[3]);
+            uint32_t ho[4], lo[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              float y[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const float xh = bf16_bits_to_f32(static_cast<uint16_t>(h4[h] >> (16 * e)));
+                const float xl = bf16_bits_to_f32(static_cast<uint16_t>(l4[h] >> (16 * e)));
+                y[e] = fmaf(p.a, xh + xl, v[8 * uu + 2 * h + e]);
+              }
+              ho[h] = pack_bf16x2(y[0], y[1]);
+              const float r0 = y[0] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] & 0xFFFFu));
+              const float r1 = y[1] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] >> 16));
+              lo[h] = pack_bf16x2(r0, r1);
+            }
+            st_shared_v4(hs + sw64(r, u), ho[0], ho[1], ho[2], ho[3]);
+            st_shared_v4(ls + sw64(r, u), lo[0], lo[1], lo[2], lo[3]);
           }
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            st_shared_v4(os + sw64(r, u), pack_bf16x2(v[8 * u + 0], v[8 * u + 1]),
-                         pack_bf16x2(v[8 * u + 2], v[8 * u + 3]), pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
-                         pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+          if (leader && c == 2) TRACE(k, 15);
           fence_async_smem();
-          named_bar(1, 128);
+          named_bar(1, kEpiThreads);
+          if (leader && c == 2) TRACE(k, 16);
           if (leader) {
-            tma_store_3d(&M.e, es, col0, row0, tc.b);
-            tma_store_3d(&M.d, os, col0, row0, tc.b);
+            tma_store_3d(&M.d, hs, col0, row0, tc.b);   // hi' -> the other hi buffer
+            tma_store_3d(&M.mt, ls, col0, row0, tc.b);  // lo' -> lo, in place
             bulk_commit();
-            bulk_wait_read_all();
-            issue_eload(s + kEpiSlots);
+            // the store of chunk s-1 has read its slot: refill that slot
+            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+            if (c == 2) TRACE(k, 17);
+            if (s >= 1) issue_eload(s + kAhead);
           }
           prev_kind = kind;
           continue;
@@ -453,32 +500,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           // B = b A + c acc with A's chunk from the slot (bf16, 64-byte swizzle)
           const uint32_t es = slots_u32 + slot * C::kSlotBytes;
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int uu = 0; uu < 2; ++uu) {
             uint32_t a4[4];
-            ld_shared_v4(es + sw64(r, u), a4[0], a4[1], a4[2], a4[3]);
+            ld_shared_v4(es + sw64(r, 2 * hf + uu), a4[0], a4[1], a4[2], a4[3]);
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
               const float lo = bf16_bits_to_f32(static_cast<uint16_t>(a4[h] & 0xFFFFu));
               const float hi = bf16_bits_to_f32(static_cast<uint16_t>(a4[h] >> 16));
-              v[8 * u + 2 * h] = fmaf(p.c, v[8 * u + 2 * h], p.b * lo);
-              v[8 * u + 2 * h + 1] = fmaf(p.c, v[8 * u + 2 * h + 1], p.b * hi);
+              v[8 * uu + 2 * h] = fmaf(p.c, v[8 * uu + 2 * h], p.b * lo);
+              v[8 * uu + 2 * h + 1] = fmaf(p.c, v[8 * uu + 2 * h + 1], p.b * hi);
             }
           }
         }
 
         if (kind == kUpper) {
-          if (prev_kind == kDiag) named_bar(2, 128);  // staging is aliased by the diagonal block
-          const uint32_t ds = stage_u32 + (s & 1) * kChunkBf16;      // direct [128][32]
+          if (prev_kind == kDiag) named_bar(2, kEpiThreads);  // staging is aliased by the diagonal block
+          const uint32_t ds = stage_u32 + (s & 1) * kChunkBf16;        // direct [128][32]
           const uint32_t ms = stage_u32 + (2 + (s & 1)) * kChunkBf16;  // mirror [32][128]
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            st_shared_v4(ds + sw64(r, u), pack_bf16x2(v[8 * u + 0], v[8 * u + 1]),
-                         pack_bf16x2(v[8 * u + 2], v[8 * u + 3]), pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
-                         pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+          for (int uu = 0; uu < 2; ++uu)
+            st_shared_v4(ds + sw64(r, 2 * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
+                         pack_bf16x2(v[8 * uu + 2], v[8 * uu + 3]), pack_bf16x2(v[8 * uu + 4], v[8 * uu + 5]),
+                         pack_bf16x2(v[8 * uu + 6], v[8 * uu + 7]));
 #pragma unroll
-          for (int q = 0; q < 32; ++q) st_shared_u16(ms + q * 256 + r * 2, bf16_bits(v[q]));
+          for (int q = 0; q < 16; ++q) st_shared_u16(ms + (16 * hf + q) * 256 + r * 2, bf16_bits(v[q]));
           fence_async_smem();
-          named_bar(1, 128);
+          named_bar(1, kEpiThreads);
           if (leader) {
             tma_store_3d(&M.d, ds, col0, row0, tc.b);
             tma_store_3d(&M.mt, ms, row0, col0, tc.b);
@@ -488,29 +535,39 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           }
         } else {  // kDiag: chunk dq of the 128 x 128 diagonal block
           const int dq = (col0 - row0) / kChunk;
-          if (dq == 0) named_bar(2, 128);  // previous stores done reading the staging
+          if (dq == 0) named_bar(2, kEpiThreads);  // previous stores done reading the staging
           const uint32_t sb = stage_u32 + (dq >> 1) * (2 * kChunkBf16);  // [128][64] half
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            st_shared_v4(sb + sw128(r, (dq & 1) * 4 + u), pack_bf16x2(v[8 * u + 0], v[8 * u + 1]),
-                         pack_bf16x2(v[8 * u + 2], v[8 * u + 3]), pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
-                         pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+          for (int uu = 0; uu < 2; ++uu)
+            st_shared_v4(sb + sw128(r, (dq & 1) * 4 + 2 * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
+                         pack_bf16x2(v[8 * uu + 2], v[8 * uu + 3]), pack_bf16x2(v[8 * uu + 4], v[8 * uu + 5]),
+                         pack_bf16x2(v[8 * uu + 6], v[8 * uu + 7]));
           if (EPI == kPoly) {
-            named_bar(1, 128);  // every thread has read its slot
+            named_bar(1, kEpiThreads);  // every thread has read its slot
             if (leader) issue_eload(s + kEpiSlots);
           }
           if (dq == 3 || col0 + kChunk >= G.m) {
-            // block complete: lower half := transpose of the upper half
-            named_bar(1, 128);
-            for (int j = 0; j < r; ++j) {
-              const uint32_t src = stage_u32 + (r >> 6) * (2 * kChunkBf16) +
-                                   static_cast<uint32_t>(j * 128 + ((((r & 63) >> 3) ^ (j & 7)) << 4) + (r & 7) * 2);
-              const uint32_t dst = stage_u32 + (j >> 6) * (2 * kChunkBf16) +
-                                   static_cast<uint32_t>(r * 128 + ((((j & 63) >> 3) ^ (r & 7)) << 4) + (j & 7) * 2);
-              st_shared_u16(dst, ld_shared_u16(src));
+            // block complete: lower half := transpose of the upper half.
+            // Row r takes S[r][j] = S[j][r] for j < r, eight columns per
+            // 16-byte write; the two warps of a lane quarter split the groups.
+            named_bar(1, kEpiThreads);
+            auto s_addr = [&](int row, int col) {
+              return stage_u32 + (col >> 6) * (2 * kChunkBf16) +
+                     static_cast<uint32_t>(row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2);
+            };
+            for (int j0 = 8 * hf; j0 < r; j0 += 16) {
+              uint16_t t[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q) t[q] = (j0 + q < r) ? ld_shared_u16(s_addr(j0 + q, r)) : uint16_t(0);
+              if (j0 + 8 <= r) {
+                st_shared_v4(s_addr(r, j0), t[0] | (uint32_t(t[1]) << 16), t[2] | (uint32_t(t[3]) << 16),
+                             t[4] | (uint32_t(t[5]) << 16), t[6] | (uint32_t(t[7]) << 16));
+              } else {
+                for (int q = 0; q < r - j0; ++q) st_shared_u16(s_addr(r, j0 + q), t[q]);
+              }
             }
             fence_async_smem();
-            named_bar(1, 128);
+            named_bar(1, kEpiThreads);
             if (leader) {
               tma_store_3d(&M.s, stage_u32, row0, row0, tc.b);
               if (row0 + 64 < G.m)  // never start a store wholly outside the matrix
@@ -522,6 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         }
         prev_kind = kind;
       }
+      if (leader) TRACE(k, 12);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -531,8 +589,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       bulk_wait_all();
       if (!ok) {
         // prefetched epilogue operands still in flight land before exit
-        for (int s = 0; s < kEpiSlots; ++s)
-          if (pend[s] >= 0) mbar_wait_drain(efull_bar(s), (pend[s] / kEpiSlots) & 1, drain_ns);
+        for (int q = 0; q < kEpiSlots; ++q)
+          if (pend[q] >= 0) mbar_wait_drain(efull_bar(q), (pend[q] / kEpiSlots) & 1, drain_ns);
       }
     }
   }

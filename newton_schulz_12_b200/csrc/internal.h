@@ -17,7 +17,7 @@ constexpr int BK = 64;               // K per stage: one 128-byte swizzle row of
 constexpr int kChunk = 32;           // epilogue columns handled per step
 constexpr int kChunks = BN / kChunk;
 constexpr int kEpiSlots = 4;         // ring of prefetched epilogue operand chunks
-constexpr int kThreads = 192;        // warp 0 copies, warp 1 issues MMAs, warps 2-5 epilogue
+constexpr int kThreads = 320;        // warp 0 copies, warp 1 issues MMAs, warps 2-9 epilogue
 
 enum Epi : int { kGram = 0, kPoly = 1, kBx = 2 };
 
@@ -30,12 +30,14 @@ struct Group {
 };
 
 // Tensor maps of one group (3-D: {inner, rows, batch}).
+// kBx uses e = hi chunk of X (read), mt = lo chunk of X (read and written in
+// place), d = hi chunk of X' (written); all bf16 32 x 128, 64-byte swizzle.
 struct Maps {
   CUtensorMap p;   // rows of D: X (kGram), A (kPoly), B (kBx); K-major, box 64 x 128
   CUtensorMap q;   // columns of D: X / A K-major box 64 x 256; X MN-major box 64 x 64 (kBx)
-  CUtensorMap e;   // epilogue input chunk: A bf16 32 x 128 (kPoly); fp32 X 32 x 128 (kBx, also stored)
-  CUtensorMap d;   // direct output chunk, bf16 32 x 128: A (kGram), B (kPoly), bf16 X' (kBx)
-  CUtensorMap mt;  // mirrored output chunk, bf16 128 x 32 (kGram / kPoly)
+  CUtensorMap e;   // epilogue input chunk, bf16 32 x 128: A (kPoly); hi of X (kBx)
+  CUtensorMap d;   // direct output chunk, bf16 32 x 128: A (kGram), B (kPoly), hi of X' (kBx)
+  CUtensorMap mt;  // mirrored output chunk, bf16 128 x 32 (kGram / kPoly); lo of X, 32 x 128 (kBx)
   CUtensorMap s;   // symmetrised diagonal block, bf16 64 x 128 (kGram / kPoly)
 };
 
@@ -48,7 +50,15 @@ struct Params {
   int* status;
   unsigned long long timeout_ns;
   int inject;  // 1: withhold one operand copy in CTA 0 (timeout-path test)
+  unsigned long long* trace;  // timestamps (only recorded in builds with MUON_TRACE)
 };
+
+// Trace layout (MUON_TRACE builds): per CTA < kTraceCtas, per tile < kTraceTiles,
+// kTraceSlots %globaltimer stamps: 0 copier first issue, 1 copier last issue,
+// 2 MMA start, 3 MMA last commit, 4 epilogue start, 5..11 chunk ends, 12 end,
+// and within chunk 2: 13 TMEM loaded, 14 operand slot ready, 15 computed,
+// 16 after the epilogue barrier, 17 (leader) stores drained from the staging.
+constexpr int kTraceCtas = 16, kTraceTiles = 24, kTraceSlots = 18;
 
 // Symmetric-output tiles per m x m matrix (128 x 256 tiles touching the upper triangle).
 inline int sym_tiles(int m) {
@@ -118,9 +128,11 @@ struct CastMat {
   int tiles_n;        // 64-wide tiles along X's columns
   int tile_begin;
   int part_begin, part_count;
-  float* xf;          // fp32 X (m x n, row stride ld)
-  void* xb;           // bf16 X or null
+  float* xf;          // fp32 X (m x n, row stride ld), fp32 path; else null
+  void* xb;           // bf16 path: hi = bf16(X)
+  void* xlo;          // bf16 path: lo = bf16(X - hi)
   long long ld;
+  int vec;            // source rows are 16-byte aligned (cols % 8 == 0): 128-bit loads
 };
 
 struct CastParams {
@@ -137,13 +149,16 @@ struct CastParams {
 // caller's matrix; O is read from an m x n buffer, transposed when needed.
 struct OutMat {
   void* y;            // W (fp32, in/out) or destination X (bf16 / f32)
-  const float* o;     // update / result in X layout (or in W layout if !o_transposed)
+  const float* o;     // fp32 update / result (X layout, or W layout if !o_transposed); or null
+  const void* o_hi;   // else the result as a bf16 pair: O = hi + lo (X layout)
+  const void* o_lo;
   int rows, cols;     // caller layout of y
   int o_transposed;   // O[r][s] = o[s * ld + r]
   long long ld;
   int tiles_c;        // 64-wide tiles along y's columns
   int tile_begin;
   float ls;           // fl(lr * scale)
+  int vec;            // cols % 8 == 0 and ld % 8 == 0: 128-bit accesses
 };
 
 struct OutParams {

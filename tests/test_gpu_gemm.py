@@ -63,18 +63,25 @@ def test_poly(batch, m):
                                        (2, 384, 384), (1, 136, 520), (1, 1024, 4096),
                                        (80, 256, 520), (6, 768, 3072)])
 def test_bx(batch, m, n):
+    """X' = aX + BX with X = hi + lo; the pair must hold X' to about 2^-17."""
     B = rnd_bf16((batch, m, m), seed=m, scale=m ** -0.5)
-    Xf = torch.randn(batch, m, n, generator=torch.Generator().manual_seed(n)) / n ** 0.5
-    Xb = Xf.to(torch.bfloat16)
+    X = torch.randn(batch, m, n, generator=torch.Generator().manual_seed(n)) / n ** 0.5
+    hi = X.to(torch.bfloat16)
+    lo = (X - hi.float()).to(torch.bfloat16)
+    Xd = hi.double() + lo.double()          # the X the kernel sees
     a = 3.4445
     a32 = float(torch.tensor(a, dtype=torch.float32))
-    Xf_dev = Xf.to(DEV)
-    out_b = nsb.muon_bx_bf16(B.to(DEV), Xb.to(DEV), Xf_dev, a).cpu()
-    got = Xf_dev.cpu()
-    ref = a32 * Xf.double() + B.double() @ Xb.double()
-    absref = abs(a32) * Xf.double().abs() + B.double().abs() @ Xb.double().abs()
-    check_close(got, ref, absref, rel=2.0 ** -23, acc=2.0 ** -16)
-    assert torch.equal(out_b, got.to(torch.bfloat16)), "bf16 copy must be RNE of the fp32 result"
+    lo_dev = lo.cuda()
+    hi_out = nsb.muon_bx_bf16(B.cuda(), hi.cuda(), lo_dev, a).cpu()
+    lo_out = lo_dev.cpu()
+    assert nsb.muon_get_status() == 0
+    got = hi_out.double() + lo_out.double()
+    ref = a32 * Xd + B.double() @ hi.double()
+    absref = abs(a32) * Xd.abs() + B.double().abs() @ hi.double().abs()
+    check_close(got, ref, absref, rel=2.0 ** -16, acc=2.0 ** -16)
+    # hi' is the round-to-nearest bf16 of X', lo' the rounded remainder
+    xh = hi_out.float()
+    assert torch.all((got - xh.double()).abs() <= 2.0 ** -8 * xh.double().abs() + 1e-30)
 
 
 def test_stage_kernels_are_deterministic():
