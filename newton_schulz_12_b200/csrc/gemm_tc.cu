@@ -54,7 +54,8 @@ struct Cfg {
   // aliased by the 128 x 128 diagonal block (2 x [128 rows][64 cols] bf16)
   static constexpr uint32_t kStagingBytes = (EPI == kBx) ? 0 : 4 * kChunkBf16;
   static constexpr uint32_t kRingBytes = kStages * kStageBytes;
-  static constexpr int kNumBars = 2 * kStages + 5 + kEpiSlots;
+  // full, empty, tfull x2, tempty x2, drain, efull x4, ready x4, sfree x2, econs x4
+  static constexpr int kNumBars = 2 * kStages + 5 + 3 * kEpiSlots + 2;
   static constexpr size_t kSmem =
       1024 + kRingBytes + kSlotsBytes + kStagingBytes + kNumBars * 8 + 16;
 };
@@ -148,23 +149,6 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 
-// AND of `v` over the 256 epilogue threads (hardware barrier 3).  Every
-// possibly-failing wait of the epilogue is followed by this, so the four
-// epilogue warps always take the same branch and never strand one another at
-// a later barrier.
-__device__ __forceinline__ bool epi_all(bool v) {
-  uint32_t out;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 3, 256, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(out)
-      : "r"(static_cast<uint32_t>(v))
-      : "memory");
-  return out != 0;
-}
-
 #ifdef MUON_TRACE
 __device__ __forceinline__ void trace_stamp(const Params& p, int tile, int slot) {
   if (p.trace && blockIdx.x < kTraceCtas && tile < kTraceTiles)
@@ -201,6 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * S + 2 + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * S + 4);
   auto efull_bar = [&](int s) { return bar0 + 8u * (2 * S + 5 + s); };
+  auto ready_bar = [&](int s) { return bar0 + 8u * (2 * S + 5 + kEpiSlots + s); };
+  auto sfree_bar = [&](int b) { return bar0 + 8u * (2 * S + 5 + 2 * kEpiSlots + b); };
+  auto econs_bar = [&](int s) { return bar0 + 8u * (2 * S + 7 + 2 * kEpiSlots + s); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -209,10 +196,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 8 * 32);
+      mbar_init(tempty_bar(a), kEpiThreads);
     }
     mbar_init(drain_bar, 1);
-    for (int s = 0; s < kEpiSlots; ++s) mbar_init(efull_bar(s), 1);
+    for (int s = 0; s < kEpiSlots; ++s) {
+      mbar_init(efull_bar(s), 1);
+      mbar_init(ready_bar(s), kEpiThreads);
+      mbar_init(econs_bar(s), kEpiThreads);
+    }
+    for (int b = 0; b < 2; ++b) mbar_init(sfree_bar(b), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -345,252 +337,267 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-9)
-    // Two warps per TMEM lane quarter: warp w reads lanes 32*(w%4).. and the
-    // half `hf` of each 32-column chunk (16 columns), so a chunk's element
-    // work is spread over all four SM sub-partitions twice.
-    const int lane_base = 32 * (warp & 3);
-    const int hf = (warp - 2) >> 2;  // column half of the chunk
-    const int r = lane_base + lane;  // tile row owned by this thread
-    const bool leader = (warp == 2 && lane == 0);
+    // ------------------------------------------------------------ epilogue (warps 2-9) and IO (warp 10)
     const int total_chunks = my_tiles * kChunks;
     const uint32_t slots_u32 = smem_u32(slots);
     const uint32_t stage_u32 = smem_u32(staging);
-    constexpr int kEpiThreads = 256;
 
-    // Epilogue operand prefetch of chunk s into slot s % kEpiSlots (leader only).
-    int pend[kEpiSlots] = {-1, -1, -1, -1};  // last chunk issued per slot
-    auto issue_eload = [&](int s) {
-      if (EPI == kGram || s >= total_chunks) return;
-      const int slot = s % kEpiSlots;
-      pend[slot] = s;
-      const TileCoord tc = decode_tile<EPI>(p, blockIdx.x + (s / kChunks) * gridDim.x);
-      const Group& G = p.grp[tc.g];
-      const int col0 = tc.tn * BN + (s % kChunks) * kChunk;
-      const int kind = chunk_kind<EPI>(G, tc.tm, col0);
-      if (kind == kSkip) {
-        mbar_arrive(efull_bar(slot));
-      } else {
-        const uint32_t dst = slots_u32 + slot * C::kSlotBytes;
-        mbar_arrive_expect_tx(efull_bar(slot), C::kSlotBytes);
-        tma_load_3d(dst, &p.map[tc.g].e, efull_bar(slot), col0, tc.tm * BM, tc.b);
-        if (EPI == kBx)  // lo half of X next to its hi half
-          tma_load_3d(dst + kChunkBf16, &p.map[tc.g].mt, efull_bar(slot), col0, tc.tm * BM, tc.b);
-      }
-    };
-    // kBx refills a slot one chunk late (its store drains meanwhile): chunks
-    // 0..kEpiSlots-1 are loaded up front, then chunk s+kEpiSlots-1 into chunk
-    // s-1's slot once chunk s (s >= 1) is handed to its stores.
-    constexpr int kAhead = (EPI == kBx) ? kEpiSlots - 1 : kEpiSlots;
-    if (leader) {
-      for (int g = 0; g < p.ngroups; ++g) {
-        tma_prefetch_map(&p.map[g].e);
-        tma_prefetch_map(&p.map[g].d);
-        tma_prefetch_map(&p.map[g].mt);
-        tma_prefetch_map(&p.map[g].s);
-      }
-      for (int s = 0; s < kEpiSlots; ++s) issue_eload(s);
-    }
-
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    int prev_kind = kSkip;
-    bool ok = true;
-    for (int k = 0; k < my_tiles && ok; ++k) {
-      const TileCoord tc = decode_tile<EPI>(p, blockIdx.x + k * gridDim.x);
-      const Group& G = p.grp[tc.g];
-      const Maps& M = p.map[tc.g];
-      const int row0 = tc.tm * BM;
-      const bool w = epi_all(mbar_wait(tfull_bar(acc), acc_phase, ctl));
-      if (!w) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (leader) TRACE(k, 4);
-      for (int c = 0; c < kChunks; ++c) {
-        if (leader && c > 0) TRACE(k, 4 + c);
-        const int s = k * kChunks + c;
-        const int col0 = tc.tn * BN + c * kChunk;
-        const int kind = chunk_kind<EPI>(G, tc.tm, col0);
-        float v[16];
-        if (kind != kSkip) {
-          uint32_t rr[16];
-          __syncwarp();
-          tmem_ld_32x32_x16(tmem_base + (static_cast<uint32_t>(lane_base) << 16) +
-                                static_cast<uint32_t>(acc * BN + c * kChunk + hf * 16),
-                            rr);
-          tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(rr[q]);
+    if (warp == 10) {
+      // ---------------------------------------------------------- IO thread
+      // Issues every epilogue bulk copy: operand chunks into the slot ring
+      // ahead of use, and the stores of what the compute warps finished,
+      // draining each store before the buffer it read is handed back.
+      if (lane == 0) {
+        for (int g = 0; g < p.ngroups; ++g) {
+          tma_prefetch_map(&p.map[g].e);
+          tma_prefetch_map(&p.map[g].d);
+          tma_prefetch_map(&p.map[g].mt);
+          tma_prefetch_map(&p.map[g].s);
         }
-        if (leader && c == 2) TRACE(k, 13);
-        if (c == kChunks - 1) {
-          // accumulator fully read: hand it back to the MMA warp
-          tc_fence_before();
-          mbar_arrive(tempty_bar(acc));
-        }
-        if (kind == kSkip) {
-          if (leader) {
-            if (EPI == kBx) {
-              bulk_wait_read_all();
-              if (s >= 1) issue_eload(s + kAhead);  // chunk s-1's slot is free
+        int pend[kEpiSlots] = {-1, -1, -1, -1};
+        auto issue_eload = [&](int s) {
+          if (EPI == kGram || s >= total_chunks) return;
+          const int slot = s % kEpiSlots;
+          pend[slot] = s;
+          const TileCoord tc = decode_tile<EPI>(p, blockIdx.x + (s / kChunks) * gridDim.x);
+          const int col0 = tc.tn * BN + (s % kChunks) * kChunk;
+          if (chunk_kind<EPI>(p.grp[tc.g], tc.tm, col0) == kSkip) {
+            mbar_arrive(efull_bar(slot));
+          } else {
+            const uint32_t dst = slots_u32 + slot * C::kSlotBytes;
+            mbar_arrive_expect_tx(efull_bar(slot), C::kSlotBytes);
+            tma_load_3d(dst, &p.map[tc.g].e, efull_bar(slot), col0, tc.tm * BM, tc.b);
+            if (EPI == kBx)  // lo half of X next to its hi half
+              tma_load_3d(dst + kChunkBf16, &p.map[tc.g].mt, efull_bar(slot), col0, tc.tm * BM, tc.b);
+          }
+        };
+        for (int s = 0; s < kEpiSlots; ++s) issue_eload(s);
+        int njob[3] = {0, 0, 0};  // kGram / kPoly: jobs seen per ready barrier (0, 1: staging; 2: block)
+        int nup = 0;              // strictly-upper chunks so far (staging buffer = nup & 1)
+        for (int s = 0; s < total_chunks; ++s) {
+          const int k = s / kChunks, c = s % kChunks;
+          const TileCoord tc = decode_tile<EPI>(p, blockIdx.x + k * gridDim.x);
+          const Group& G = p.grp[tc.g];
+          const Maps& M = p.map[tc.g];
+          const int row0 = tc.tm * BM;
+          const int col0 = tc.tn * BN + c * kChunk;
+          const int kind = chunk_kind<EPI>(G, tc.tm, col0);
+          if (EPI == kBx) {
+            const int slot = s % kEpiSlots;
+            mbar_wait(ready_bar(slot), (s / kEpiSlots) & 1, ctl);
+            if (kind != kSkip) {
+              const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
+              tma_store_3d(&M.d, hs, col0, row0, tc.b);                // hi' -> the other hi buffer
+              tma_store_3d(&M.mt, hs + kChunkBf16, col0, row0, tc.b);  // lo' -> lo, in place
+              bulk_commit();
+              asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");  // chunk s-1 drained
             } else {
-              issue_eload(s + kAhead);
+              bulk_wait_read_all();
             }
+            if (s >= 1) issue_eload(s + kEpiSlots - 1);  // into chunk s-1's slot
+            continue;
           }
-          continue;
-        }
-        const int slot = s % kEpiSlots;
-        if (EPI != kGram) {
-          const bool e = epi_all(mbar_wait(efull_bar(slot), (s / kEpiSlots) & 1, ctl));
-          if (!e) {
-            ok = false;
-            break;
+          if (EPI == kPoly) {
+            // every compute thread has read chunk s's A operand: refill its slot
+            mbar_wait(econs_bar(s % kEpiSlots), (s / kEpiSlots) & 1, ctl);
+            issue_eload(s + kEpiSlots);
           }
-          if (leader && c == 2) TRACE(k, 14);
-        }
-        if (EPI == kBx) {
-          // X = hi + lo from the slot; X' = a X + acc; hi' = bf16(X'),
-          // lo' = bf16(X' - hi'), written back in place and stored from there
-          const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
-          const uint32_t ls = hs + kChunkBf16;
-#pragma unroll
-          for (int uu = 0; uu < 2; ++uu) {
-            const int u = 2 * hf + uu;  // 16-byte unit of the 64-byte row
-            uint32_t h4[4], l4[4];
-            ld_shared_v4(hs + sw64(r, u), h4[0], h4[1], h4[2], h4[3]);
-            ld_shared_v4(ls + sw64(r, u), l4[0], l4[1], l4[2], l4[3]);
-            uint32_t ho[4], lo[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              float y[2];
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const float xh = bf16_bits_to_f32(static_cast<uint16_t>(h4[h] >> (16 * e)));
-                const float xl = bf16_bits_to_f32(static_cast<uint16_t>(l4[h] >> (16 * e)));
-                y[e] = fmaf(p.a, xh + xl, v[8 * uu + 2 * h + e]);
-              }
-              ho[h] = pack_bf16x2(y[0], y[1]);
-              const float r0 = y[0] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] & 0xFFFFu));
-              const float r1 = y[1] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] >> 16));
-              lo[h] = pack_bf16x2(r0, r1);
-            }
-            st_shared_v4(hs + sw64(r, u), ho[0], ho[1], ho[2], ho[3]);
-            st_shared_v4(ls + sw64(r, u), lo[0], lo[1], lo[2], lo[3]);
-          }
-          if (leader && c == 2) TRACE(k, 15);
-          fence_async_smem();
-          named_bar(1, kEpiThreads);
-          if (leader && c == 2) TRACE(k, 16);
-          if (leader) {
-            tma_store_3d(&M.d, hs, col0, row0, tc.b);   // hi' -> the other hi buffer
-            tma_store_3d(&M.mt, ls, col0, row0, tc.b);  // lo' -> lo, in place
-            bulk_commit();
-            // the store of chunk s-1 has read its slot: refill that slot
-            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-            if (c == 2) TRACE(k, 17);
-            if (s >= 1) issue_eload(s + kAhead);
-          }
-          prev_kind = kind;
-          continue;
-        }
-
-        if (EPI == kPoly) {
-          // B = b A + c acc with A's chunk from the slot (bf16, 64-byte swizzle)
-          const uint32_t es = slots_u32 + slot * C::kSlotBytes;
-#pragma unroll
-          for (int uu = 0; uu < 2; ++uu) {
-            uint32_t a4[4];
-            ld_shared_v4(es + sw64(r, 2 * hf + uu), a4[0], a4[1], a4[2], a4[3]);
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const float lo = bf16_bits_to_f32(static_cast<uint16_t>(a4[h] & 0xFFFFu));
-              const float hi = bf16_bits_to_f32(static_cast<uint16_t>(a4[h] >> 16));
-              v[8 * uu + 2 * h] = fmaf(p.c, v[8 * uu + 2 * h], p.b * lo);
-              v[8 * uu + 2 * h + 1] = fmaf(p.c, v[8 * uu + 2 * h + 1], p.b * hi);
-            }
-          }
-        }
-
-        if (kind == kUpper) {
-          if (prev_kind == kDiag) named_bar(2, kEpiThreads);  // staging is aliased by the diagonal block
-          const uint32_t ds = stage_u32 + (s & 1) * kChunkBf16;        // direct [128][32]
-          const uint32_t ms = stage_u32 + (2 + (s & 1)) * kChunkBf16;  // mirror [32][128]
-#pragma unroll
-          for (int uu = 0; uu < 2; ++uu)
-            st_shared_v4(ds + sw64(r, 2 * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
-                         pack_bf16x2(v[8 * uu + 2], v[8 * uu + 3]), pack_bf16x2(v[8 * uu + 4], v[8 * uu + 5]),
-                         pack_bf16x2(v[8 * uu + 6], v[8 * uu + 7]));
-#pragma unroll
-          for (int q = 0; q < 16; ++q) st_shared_u16(ms + (16 * hf + q) * 256 + r * 2, bf16_bits(v[q]));
-          fence_async_smem();
-          named_bar(1, kEpiThreads);
-          if (leader) {
+          if (kind == kUpper) {
+            const int b = nup & 1;
+            ++nup;
+            mbar_wait(ready_bar(b), njob[b] & 1, ctl);
+            ++njob[b];
+            const uint32_t ds = stage_u32 + b * kChunkBf16;        // direct [128][32]
+            const uint32_t ms = stage_u32 + (2 + b) * kChunkBf16;  // mirror [32][128]
             tma_store_3d(&M.d, ds, col0, row0, tc.b);
             tma_store_3d(&M.mt, ms, row0, col0, tc.b);
             bulk_commit();
             bulk_wait_read_all();
-            if (EPI == kPoly) issue_eload(s + kEpiSlots);
+            mbar_arrive(sfree_bar(b));
+          } else if (kind == kDiag && ((col0 - row0) / kChunk == 3 || col0 + kChunk >= G.m)) {
+            mbar_wait(ready_bar(2), njob[2] & 1, ctl);
+            ++njob[2];
+            tma_store_3d(&M.s, stage_u32, row0, row0, tc.b);
+            if (row0 + 64 < G.m)  // never start a store wholly outside the matrix
+              tma_store_3d(&M.s, stage_u32 + 2 * kChunkBf16, row0 + 64, row0, tc.b);
+            bulk_commit();
+            bulk_wait_read_all();
+            mbar_arrive(sfree_bar(0));  // the block used both staging buffers
+            mbar_arrive(sfree_bar(1));
           }
-        } else {  // kDiag: chunk dq of the 128 x 128 diagonal block
-          const int dq = (col0 - row0) / kChunk;
-          if (dq == 0) named_bar(2, kEpiThreads);  // previous stores done reading the staging
-          const uint32_t sb = stage_u32 + (dq >> 1) * (2 * kChunkBf16);  // [128][64] half
+        }
+        bulk_wait_all();
+        for (int q = 0; q < kEpiSlots; ++q)  // operand copies still in flight land before exit
+          if (pend[q] >= 0) mbar_wait_drain(efull_bar(q), (pend[q] / kEpiSlots) & 1, drain_ns);
+      }
+      __syncwarp();
+    } else {
+      // ---------------------------------------------------------- compute (warps 2-9)
+      // Two warps per TMEM lane quarter: warp w reads lanes 32*(w%4).. and
+      // the half `hf` of each 32-column chunk.  A failed (timed-out) wait is
+      // recorded and the schedule continues -- every later wait then returns
+      // at once -- so the compute warps always meet at the same barriers.
+      const int lane_base = 32 * (warp & 3);
+      const int hf = (warp - 2) >> 2;
+      const int r = lane_base + lane;  // tile row owned by this thread
+      const bool leader = (warp == 2 && lane == 0);
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      int nuse[2] = {0, 0};  // kGram / kPoly: jobs that used staging buffer b so far
+      int nup = 0;
+      for (int k = 0; k < my_tiles; ++k) {
+        const TileCoord tc = decode_tile<EPI>(p, blockIdx.x + k * gridDim.x);
+        const Group& G = p.grp[tc.g];
+        const int row0 = tc.tm * BM;
+        mbar_wait(tfull_bar(acc), acc_phase, ctl);
+        tc_fence_after();
+        if (leader) TRACE(k, 4);
+        for (int c = 0; c < kChunks; ++c) {
+          if (leader && c > 0) TRACE(k, 4 + c);
+          const int s = k * kChunks + c;
+          const int col0 = tc.tn * BN + c * kChunk;
+          const int kind = chunk_kind<EPI>(G, tc.tm, col0);
+          float v[16];
+          if (kind != kSkip) {
+            uint32_t rr[16];
+            __syncwarp();
+            tmem_ld_32x32_x16(tmem_base + (static_cast<uint32_t>(lane_base) << 16) +
+                                  static_cast<uint32_t>(acc * BN + c * kChunk + hf * 16),
+                              rr);
+            tmem_ld_wait();
 #pragma unroll
-          for (int uu = 0; uu < 2; ++uu)
-            st_shared_v4(sb + sw128(r, (dq & 1) * 4 + 2 * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
-                         pack_bf16x2(v[8 * uu + 2], v[8 * uu + 3]), pack_bf16x2(v[8 * uu + 4], v[8 * uu + 5]),
-                         pack_bf16x2(v[8 * uu + 6], v[8 * uu + 7]));
+            for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(rr[q]);
+          }
+          if (c == kChunks - 1) {
+            // accumulator fully read: hand it back to the MMA warp
+            tc_fence_before();
+            mbar_arrive(tempty_bar(acc));
+          }
+          const int slot = s % kEpiSlots;
+          if (EPI != kGram) mbar_wait(efull_bar(slot), (s / kEpiSlots) & 1, ctl);
+
+          if (EPI == kBx) {
+            // X = hi + lo from the slot; X' = a X + acc; hi' = bf16(X'),
+            // lo' = bf16(X' - hi'), written back in place for the IO thread to store
+            if (kind != kSkip) {
+              const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
+              const uint32_t ls = hs + kChunkBf16;
+#pragma unroll
+              for (int uu = 0; uu < 2; ++uu) {
+                const int u = 2 * hf + uu;  // 16-byte unit of the 64-byte row
+                uint32_t h4[4], l4[4];
+                ld_shared_v4(hs + sw64(r, u), h4[0], h4[1], h4[2], h4[3]);
+                ld_shared_v4(ls + sw64(r, u), l4[0], l4[1], l4[2], l4[3]);
+                uint32_t ho[4], lo[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  float y[2];
+#pragma unroll
+                  for (int e = 0; e < 2; ++e) {
+                    const float xh = bf16_bits_to_f32(static_cast<uint16_t>(h4[h] >> (16 * e)));
+                    const float xl = bf16_bits_to_f32(static_cast<uint16_t>(l4[h] >> (16 * e)));
+                    y[e] = fmaf(p.a, xh + xl, v[8 * uu + 2 * h + e]);
+                  }
+                  ho[h] = pack_bf16x2(y[0], y[1]);
+                  const float r0 = y[0] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] & 0xFFFFu));
+                  const float r1 = y[1] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] >> 16));
+                  lo[h] = pack_bf16x2(r0, r1);
+                }
+                st_shared_v4(hs + sw64(r, u), ho[0], ho[1], ho[2], ho[3]);
+                st_shared_v4(ls + sw64(r, u), lo[0], lo[1], lo[2], lo[3]);
+              }
+              fence_async_smem();
+            }
+            mbar_arrive(ready_bar(slot));
+            continue;
+          }
+
+          // ------------------------------------------------ kGram / kPoly
           if (EPI == kPoly) {
-            named_bar(1, kEpiThreads);  // every thread has read its slot
-            if (leader) issue_eload(s + kEpiSlots);
-          }
-          if (dq == 3 || col0 + kChunk >= G.m) {
-            // block complete: lower half := transpose of the upper half.
-            // Row r takes S[r][j] = S[j][r] for j < r, eight columns per
-            // 16-byte write; the two warps of a lane quarter split the groups.
-            named_bar(1, kEpiThreads);
-            auto s_addr = [&](int row, int col) {
-              return stage_u32 + (col >> 6) * (2 * kChunkBf16) +
-                     static_cast<uint32_t>(row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2);
-            };
-            for (int j0 = 8 * hf; j0 < r; j0 += 16) {
-              uint16_t t[8];
+            if (kind != kSkip) {
+              // B = b A + c acc with A's chunk from the slot (bf16, 64-byte swizzle)
+              const uint32_t es = slots_u32 + slot * C::kSlotBytes;
 #pragma unroll
-              for (int q = 0; q < 8; ++q) t[q] = (j0 + q < r) ? ld_shared_u16(s_addr(j0 + q, r)) : uint16_t(0);
-              if (j0 + 8 <= r) {
-                st_shared_v4(s_addr(r, j0), t[0] | (uint32_t(t[1]) << 16), t[2] | (uint32_t(t[3]) << 16),
-                             t[4] | (uint32_t(t[5]) << 16), t[6] | (uint32_t(t[7]) << 16));
-              } else {
-                for (int q = 0; q < r - j0; ++q) st_shared_u16(s_addr(r, j0 + q), t[q]);
+              for (int uu = 0; uu < 2; ++uu) {
+                uint32_t a4[4];
+                ld_shared_v4(es + sw64(r, 2 * hf + uu), a4[0], a4[1], a4[2], a4[3]);
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  const float lo = bf16_bits_to_f32(static_cast<uint16_t>(a4[h] & 0xFFFFu));
+                  const float hi = bf16_bits_to_f32(static_cast<uint16_t>(a4[h] >> 16));
+                  v[8 * uu + 2 * h] = fmaf(p.c, v[8 * uu + 2 * h], p.b * lo);
+                  v[8 * uu + 2 * h + 1] = fmaf(p.c, v[8 * uu + 2 * h + 1], p.b * hi);
+                }
               }
             }
+            mbar_arrive(econs_bar(slot));  // slot read (or unused): the IO thread may refill it
+          }
+          if (kind == kUpper) {
+            const int b = nup & 1;
+            ++nup;
+            if (nuse[b] > 0) mbar_wait(sfree_bar(b), (nuse[b] - 1) & 1, ctl);
+            ++nuse[b];
+            const uint32_t ds = stage_u32 + b * kChunkBf16;        // direct [128][32]
+            const uint32_t ms = stage_u32 + (2 + b) * kChunkBf16;  // mirror [32][128]
+#pragma unroll
+            for (int uu = 0; uu < 2; ++uu)
+              st_shared_v4(ds + sw64(r, 2 * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
+                           pack_bf16x2(v[8 * uu + 2], v[8 * uu + 3]), pack_bf16x2(v[8 * uu + 4], v[8 * uu + 5]),
+                           pack_bf16x2(v[8 * uu + 6], v[8 * uu + 7]));
+#pragma unroll
+            for (int q = 0; q < 16; ++q) st_shared_u16(ms + (16 * hf + q) * 256 + r * 2, bf16_bits(v[q]));
             fence_async_smem();
-            named_bar(1, kEpiThreads);
-            if (leader) {
-              tma_store_3d(&M.s, stage_u32, row0, row0, tc.b);
-              if (row0 + 64 < G.m)  // never start a store wholly outside the matrix
-                tma_store_3d(&M.s, stage_u32 + 2 * kChunkBf16, row0 + 64, row0, tc.b);
-              bulk_commit();
-              bulk_wait_read_all();
+            mbar_arrive(ready_bar(b));
+          } else if (kind == kDiag) {  // chunk dq of the 128 x 128 diagonal block
+            const int dq = (col0 - row0) / kChunk;
+            if (dq == 0) {
+              // the block occupies both staging buffers: wait for their last stores
+              for (int b = 0; b < 2; ++b) {
+                if (nuse[b] > 0) mbar_wait(sfree_bar(b), (nuse[b] - 1) & 1, ctl);
+                ++nuse[b];
+              }
+            }
+            const uint32_t sb = stage_u32 + (dq >> 1) * (2 * kChunkBf16);  // [128][64] half
+#pragma unroll
+            for (int uu = 0; uu < 2; ++uu)
+              st_shared_v4(sb + sw128(r, (dq & 1) * 4 + 2 * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
+                           pack_bf16x2(v[8 * uu + 2], v[8 * uu + 3]), pack_bf16x2(v[8 * uu + 4], v[8 * uu + 5]),
+                           pack_bf16x2(v[8 * uu + 6], v[8 * uu + 7]));
+            if (dq == 3 || col0 + kChunk >= G.m) {
+              // block complete: lower half := transpose of the upper half.
+              // Row r takes S[r][j] = S[j][r] for j < r, eight columns per
+              // 16-byte write; the two warps of a lane quarter split the groups.
+              named_bar(1, kEpiThreads);
+              auto s_addr = [&](int row, int col) {
+                return stage_u32 + (col >> 6) * (2 * kChunkBf16) +
+                       static_cast<uint32_t>(row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2);
+              };
+              for (int j0 = 8 * hf; j0 < r; j0 += 16) {
+                uint32_t t[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  const uint32_t lo = (j0 + 2 * q < r) ? ld_shared_u16(s_addr(j0 + 2 * q, r)) : 0u;
+                  const uint32_t hi = (j0 + 2 * q + 1 < r) ? ld_shared_u16(s_addr(j0 + 2 * q + 1, r)) : 0u;
+                  t[q] = lo | (hi << 16);
+                }
+                if (j0 + 8 <= r) {
+                  st_shared_v4(s_addr(r, j0), t[0], t[1], t[2], t[3]);
+                } else {
+#pragma unroll
+                  for (int q = 0; q < 8; ++q)
+                    if (j0 + q < r) st_shared_u16(s_addr(r, j0 + q), static_cast<uint16_t>(t[q >> 1] >> (16 * (q & 1))));
+                }
+              }
+              fence_async_smem();
+              mbar_arrive(ready_bar(2));
             }
           }
         }
-        prev_kind = kind;
-      }
-      if (leader) TRACE(k, 12);
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
-    }
-    if (leader) {
-      bulk_wait_all();
-      if (!ok) {
-        // prefetched epilogue operands still in flight land before exit
-        for (int q = 0; q < kEpiSlots; ++q)
-          if (pend[q] >= 0) mbar_wait_drain(efull_bar(q), (pend[q] / kEpiSlots) & 1, drain_ns);
+        if (leader) TRACE(k, 12);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
     }
   }

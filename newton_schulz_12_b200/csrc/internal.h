@@ -17,7 +17,9 @@ constexpr int BK = 64;               // K per stage: one 128-byte swizzle row of
 constexpr int kChunk = 32;           // epilogue columns handled per step
 constexpr int kChunks = BN / kChunk;
 constexpr int kEpiSlots = 4;         // ring of prefetched epilogue operand chunks
-constexpr int kThreads = 320;        // warp 0 copies, warp 1 issues MMAs, warps 2-9 epilogue
+constexpr int kThreads = 352;        // warp 0 copies, warp 1 MMAs, warps 2-9 epilogue math,
+                                     // warp 10 epilogue loads and stores
+constexpr int kEpiThreads = 256;     // warps 2-9
 
 enum Epi : int { kGram = 0, kPoly = 1, kBx = 2 };
 
