@@ -193,7 +193,7 @@ def cpu_baseline(shapes, budget_s=12.0):
 
 def run_reference(args):
     """`--impl reference`: the fp64 oracle as it stands, on host cores, rank 0 only."""
-    rank = int(os.environ.get("RANK", "0"))
+    rank = rank_env()[1]
     if rank != 0:
         return
     shapes = gpt2_shapes()
@@ -218,6 +218,29 @@ def run_reference(args):
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ ranks
+def rank_env():
+    """(world, rank, local_rank) from the torch.distributed launcher's environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value, device):
+    """Maximum of a per-rank float over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, steps, ms):
+    """Whole-job throughput: units processed by all ranks over the slowest rank's time."""
+    return units_per_rank * world * steps / (ms / 1000.0)
 
 
 # ------------------------------------------------------------------ our arm
@@ -245,9 +268,7 @@ def run_ours(args):
     import newton_schulz_12_b200 as nsb
     from newton_schulz_12_b200 import workloads
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -302,11 +323,7 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
     prof = nsb.muon_profile_end()
     barrier()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), dev)
     if nsb.muon_get_status(stream) != 0:
         raise RuntimeError("device status after timed region: " + nsb.muon_last_error())
     launches = sum(n for _, n in prof.values())
@@ -326,14 +343,10 @@ def run_ours(args):
     e_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e_ms = e_start.elapsed_time(e_end)
-    if world > 1:
-        t = torch.tensor([e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
+    e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
 
     nmat = len(shapes) * world
-    value = nmat * args.steps / (ms / 1000.0)
+    value = job_throughput(len(shapes), world, args.steps, ms)
     flops_step = nominal_flops(shapes)
     tflops = flops_step * world * args.steps / (ms / 1000.0) / 1e12
 
@@ -381,7 +394,7 @@ def run_ours(args):
             "roofline": roofline,
             "kernels": kernels,
             "gpu_launches": launches,
-            "e2e": {"value": nmat * e2e_steps / (e_ms / 1000.0), "unit": UNIT,
+            "e2e": {"value": job_throughput(len(shapes), world, e2e_steps, e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": G_host.numel() * G_host.element_size(),
                     "d2h_bytes_per_step": W_host.numel() * W_host.element_size()},
             "clocks": clocks.summary(),
