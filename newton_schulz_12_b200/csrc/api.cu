@@ -231,7 +231,7 @@ int make_map(CUtensorMap* map, const void* base, int esize, uint64_t inner, uint
 int sym_maps(tc::Maps& M, const void* S, int m, int k, long long lds, long long ss, void* D,
              long long ldd, long long sd, int batch, bool with_e) {
   MUON_TRY(make_map(&M.p, S, 2, k, m, batch, lds, ss, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
-  MUON_TRY(make_map(&M.q, S, 2, k, m, batch, lds, ss, 64, tc::BN, CU_TENSOR_MAP_SWIZZLE_128B));
+  MUON_TRY(make_map(&M.q, S, 2, k, m, batch, lds, ss, 64, tc::BNH, CU_TENSOR_MAP_SWIZZLE_128B));
   if (with_e)
     MUON_TRY(make_map(&M.e, S, 2, m, m, batch, lds, ss, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
   else
@@ -305,7 +305,7 @@ tc::Group tc_group(int batch, int m, int n, int k, bool sym, int tile_begin) {
   G.m = m;
   G.n = n;
   G.k = k;
-  G.tiles_m = (m + tc::BM - 1) / tc::BM;
+  G.tiles_m = (m + tc::PM - 1) / tc::PM;
   G.tiles_n = sym ? (m + tc::BN - 1) / tc::BN : (n + tc::BN - 1) / tc::BN;
   G.tiles_per_mat = sym ? tc::sym_tiles(m) : G.tiles_m * G.tiles_n;
   G.tile_begin = tile_begin;
@@ -339,9 +339,8 @@ int launch_tc(int epi, tc::Params& P, int sms, cudaStream_t s) {
       g_inject = 0;
     }
   }
-  const int grid = std::min(P.total_tiles, sms);
   ProfScope prof(MUON_KERNEL_GRAM + epi, s);
-  CUDA_TRY(tc::launch(epi, P, grid, s));
+  CUDA_TRY(tc::launch(epi, P, sms / 2, s));  // one CTA pair per two SMs
   P.inject = 0;
   return MUON_OK;
 }

@@ -25,6 +25,7 @@ struct WaitCtl {
   int* status;               // global status word
   unsigned long long timeout_ns;
   int where;                 // tag recorded with the failure (which wait)
+  uint32_t peer_abort;       // shared::cluster address of the partner CTA's flag, or 0
 };
 
 __device__ __forceinline__ unsigned long long global_ns() {
@@ -82,6 +83,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     if (*ctl.abort_flag) return false;
     if (global_ns() - t0 > ctl.timeout_ns) {
       *ctl.abort_flag = 1;
+      if (ctl.peer_abort)  // the partner CTA of a pair leaves its loops too
+        asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(ctl.peer_abort), "r"(1) : "memory");
       atomicCAS(ctl.status, kStatusOk, kStatusTimeout);
       return false;
     }
@@ -99,6 +102,31 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------
+// Clusters of two CTAs (an SM pair sharing one tcgen05 MMA)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address in the shared::cluster window of the same offset in CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t smem_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+  return r;
+}
+// All threads of both CTAs; orders prior shared-memory writes (barrier
+// initialisation included) before the partner's later accesses.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// Arrive once on an mbarrier given by its shared::cluster address (any CTA of the cluster).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cbar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cbar) : "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Bulk tensor copies (global -> shared), completing on an mbarrier.
 // The innermost coordinate is always a multiple of 64 bf16 elements here.
 // ---------------------------------------------------------------------------
@@ -112,6 +140,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, uint3
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// Pair form: the box lands in this CTA's shared memory, and the byte count is
+// credited to the mbarrier at shared::cluster address `cbar` (the pair
+// leader's), so one barrier tracks the operands of both CTAs.
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void* map, uint32_t cbar,
+                                                 int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(cbar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
 
@@ -159,6 +199,21 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
                : "memory");
 }
+// Pair forms: one warp of EACH CTA of the pair executes them; the two CTAs
+// receive the same tensor-memory address.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t holder_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   holder_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -175,6 +230,26 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, ui
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// Pair MMA (M = 256 over two CTAs): each CTA supplies 128 rows of A and half
+// of B's N rows from the same shared-memory offsets, and receives its 128
+// rows of D, all N columns, in its own tensor memory.  Issued by the leader.
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the mbarrier at shared::cluster address `cbar` (either CTA
+// of the pair) when every pair MMA issued so far by this thread completes.
+__device__ __forceinline__ void tc_commit_pair(uint32_t cbar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   cbar)
+               : "memory");
 }
 
 // Arrive once on `bar` when every MMA issued so far by this thread completes.
@@ -234,13 +309,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
-// Instruction descriptor of kind::f16 with bf16 A/B, fp32 D, M = 128.
-__host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major) {
+// Instruction descriptor of kind::f16 with bf16 A/B, fp32 D, M x N
+// (M = 128 for one CTA, 256 for a pair).
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool b_mn_major) {
   return (1u << 4)                        // D format: f32
          | (1u << 7)                      // A format: bf16
          | (1u << 10)                     // B format: bf16
          | ((b_mn_major ? 1u : 0u) << 16) // B major-ness
-         | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+         | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
 }
 
 // ---------------------------------------------------------------------------

@@ -5,60 +5,94 @@
 // its nearest semi-orthogonal matrix).  It is three dense contractions, each a
 // grouped, persistent launch over every matrix of every shape group:
 //
-//   kGram  A  = X X^T            tiles touching the upper triangle, mirrored
+//   kGram  A  = X X^T            tiles on or above the diagonal, mirrored
 //   kPoly  B  = b A + c A A      A symmetric, so A A = A A^T: same tiling
 //   kBx    X' = a X + B X        X carried as a pair of bf16 matrices, X = hi + lo
 //
-// One CTA per SM, persistent over a static tile stride; 128 x 256 output tiles.
-// (Roles below; the epilogue runs on warps 2-9, two warps per TMEM lane
-// quarter, each on half of every 32-column chunk.)
-//   warp 0      one thread issues bulk tensor copies of the operand tiles
-//               (128x64 and 256x64 bf16, 128-byte swizzle) into a ring of
-//               STAGES shared-memory stages;
+// CTAs run in clusters of two on an SM pair, one cluster per pair tile of
+// 256 x 256 outputs at a time, persistent over a static tile stride.  One
+// tcgen05.mma (cta_group::2, M = 256, N = 256, K = 16), issued by the leader
+// CTA, reads 128 rows of the row operand and 128 of the 256 column-operand
+// rows from EACH CTA's shared memory and writes each CTA's 128 x 256 half of
+// the tile into that CTA's tensor memory: per CTA a 64-deep K stage is 32 KiB
+// (16 KiB of its own rows + its half of the shared columns) instead of 48 KiB,
+// so more stages fit and fewer bytes cross from L2 per MMA.
+// Roles, in both CTAs:
+//   warp 0      one thread issues bulk tensor copies of this CTA's operand
+//               tiles (128x64 bf16, 128-byte swizzle) into a ring of stages;
+//               the bytes of both CTAs complete on the leader's barrier;
 //   warp 1      allocates 512 tensor-memory columns (two 128x256 fp32
-//               accumulators); one thread issues tcgen05.mma (M=128, N=256,
-//               K=16), commits each stage back to the copier and each finished
-//               accumulator to the epilogue;
-//   warps 2-5   the epilogue: per 32-column chunk, tcgen05.ld (one row per
-//               thread), combine with the chunk's epilogue operand (prefetched
-//               by bulk copy into a 4-slot ring), write swizzled staging in
-//               shared memory, and hand it to bulk tensor stores -- no
+//               accumulators) for the pair; in the leader one thread issues
+//               the pair MMAs and commits each stage back to both copiers and
+//               each finished accumulator to both epilogues;
+//   warps 2-9   the epilogue: per 32-column chunk, tcgen05.ld (one row per
+//               thread, two warps per lane quarter), combine with the chunk's
+//               epilogue operand (prefetched by bulk copy into a 4-slot
+//               ring), write swizzled staging in shared memory -- no
 //               row-strided global accesses; the other accumulator fills
-//               meanwhile.
+//               meanwhile;
+//   warp 10     one thread issues the epilogue's bulk loads and stores.
 // Symmetric outputs: a chunk strictly above the diagonal 128x128 block is
 // stored twice (direct, and transposed through a second staging buffer); the
 // diagonal block is assembled in shared memory, its lower half overwritten
 // from its upper half, and stored once; chunks strictly below it are skipped.
 // So A and B are bit-exactly symmetric.
-// Every wait is bounded (WaitCtl); on expiry the CTA drains and exits.
+// Every wait is bounded (WaitCtl); on expiry both CTAs of the pair drain and exit.
 #include "common.cuh"
 #include "internal.h"
 
 namespace muon {
 namespace tc {
 
-constexpr uint32_t kTileBytesP = BM * BK * 2;               // 16 KiB
-constexpr uint32_t kTileBytesQ = BN * BK * 2;               // 32 KiB
-constexpr uint32_t kStageBytes = kTileBytesP + kTileBytesQ;  // 48 KiB
+constexpr uint32_t kTileBytesP = BM * BK * 2;               // 16 KiB: this CTA's rows
+constexpr uint32_t kTileBytesQ = BNH * BK * 2;              // 16 KiB: its half of the columns
+constexpr uint32_t kStageBytes = kTileBytesP + kTileBytesQ;  // 32 KiB
 constexpr uint32_t kTmemCols = 2 * BN;                      // two accumulators
 constexpr uint32_t kChunkBf16 = BM * kChunk * 2;            // 8 KiB
+constexpr size_t kMaxSmem = 232448;                         // 227 KiB per CTA on sm_100
+
+// Shared memory per CTA is split between the operand ring (K stages) and the
+// epilogue (operand slots, output staging); the split is a compile-time
+// choice per kernel.
+#ifndef MUON_GRAM_STAGES
+#define MUON_GRAM_STAGES 6
+#endif
+#ifndef MUON_POLY_STAGES
+#define MUON_POLY_STAGES 5
+#endif
+#ifndef MUON_POLY_SLOTS
+#define MUON_POLY_SLOTS 4
+#endif
+#ifndef MUON_BX_STAGES
+#define MUON_BX_STAGES 4
+#endif
+#ifndef MUON_BX_SLOTS
+#define MUON_BX_SLOTS 6
+#endif
 
 template <int EPI>
 struct Cfg {
-  static constexpr int kStages = (EPI == kGram) ? 4 : 3;
-  // epilogue operand ring
+  static constexpr int kStages =
+      (EPI == kGram) ? MUON_GRAM_STAGES : (EPI == kPoly ? MUON_POLY_STAGES : MUON_BX_STAGES);
+  // epilogue operand ring of kSlots chunks (kGram: none, the count only sizes barriers)
   // kBx slot: the hi and lo bf16 chunks of X (8 KiB each); kPoly slot: A's chunk
+  static constexpr int kSlots = (EPI == kBx) ? MUON_BX_SLOTS : MUON_POLY_SLOTS;
+  static_assert(kSlots >= 3, "ready barriers 0-2 double as staging barriers");
   static constexpr uint32_t kSlotBytes = (EPI == kBx) ? 2 * kChunkBf16 : (EPI == kPoly ? kChunkBf16 : 0);
-  static constexpr uint32_t kSlotsBytes = kSlotBytes * kEpiSlots;
+  static constexpr uint32_t kSlotsBytes = kSlotBytes * kSlots;
   // staging: kBx two bf16 output chunks; kGram / kPoly 2 direct + 2 mirror chunks,
   // aliased by the 128 x 128 diagonal block (2 x [128 rows][64 cols] bf16)
   static constexpr uint32_t kStagingBytes = (EPI == kBx) ? 0 : 4 * kChunkBf16;
   static constexpr uint32_t kRingBytes = kStages * kStageBytes;
   // full, empty, tfull x2, tempty x2, drain, efull x4, ready x4, sfree x2, econs x4
-  static constexpr int kNumBars = 2 * kStages + 5 + 3 * kEpiSlots + 2;
+  static constexpr int kNumBars = 2 * kStages + 5 + 3 * kSlots + 2;
   static constexpr size_t kSmem =
       1024 + kRingBytes + kSlotsBytes + kStagingBytes + kNumBars * 8 + 16;
 };
+
+static_assert(Cfg<kGram>::kSmem <= kMaxSmem, "kGram shared memory");
+static_assert(Cfg<kPoly>::kSmem <= kMaxSmem, "kPoly shared memory");
+static_assert(Cfg<kBx>::kSmem <= kMaxSmem, "kBx shared memory");
 
 size_t smem_bytes(int epi) {
   switch (epi) {
@@ -72,8 +106,10 @@ struct TileCoord {
   int g, b, tm, tn;
 };
 
+// Pair tile t of the launch, seen from CTA `rank` of the pair: tm is the
+// CTA's own 128-row tile, tn the pair's 256-column tile.
 template <int EPI>
-__device__ __forceinline__ TileCoord decode_tile(const Params& p, int t) {
+__device__ __forceinline__ TileCoord decode_tile(const Params& p, int t, int rank) {
   TileCoord c;
   int g = 0;
   while (g + 1 < p.ngroups && t >= p.grp[g + 1].tile_begin) ++g;
@@ -82,22 +118,21 @@ __device__ __forceinline__ TileCoord decode_tile(const Params& p, int t) {
   c.g = g;
   c.b = local / G.tiles_per_mat;
   int r = local - c.b * G.tiles_per_mat;
+  int tm2;
   if (EPI == kBx) {
-    // column panel outer, row panel inner: neighbouring CTAs share X's panel
+    // column panel outer, row panel inner: neighbouring pairs share X's panel
     c.tn = r / G.tiles_m;
-    c.tm = r - c.tn * G.tiles_m;
+    tm2 = r - c.tn * G.tiles_m;
   } else {
-    // row tile tm holds column tiles (tm / 2) .. tiles_n - 1
-    int tm = 0;
-    while (true) {
-      const int len = G.tiles_n - (tm >> 1);
-      if (r < len) break;
-      r -= len;
-      ++tm;
+    // pair row tm2 holds column tiles tm2 .. tiles_n - 1
+    tm2 = 0;
+    while (r >= G.tiles_n - tm2) {
+      r -= G.tiles_n - tm2;
+      ++tm2;
     }
-    c.tm = tm;
-    c.tn = (tm >> 1) + r;
+    c.tn = tm2 + r;
   }
+  c.tm = 2 * tm2 + rank;
   return c;
 }
 
@@ -106,7 +141,8 @@ enum ChunkKind : int { kSkip = 0, kUpper = 1, kDiag = 2, kPlain = 3 };
 
 template <int EPI>
 __device__ __forceinline__ int chunk_kind(const Group& G, int tm, int col0) {
-  if (EPI == kBx) return col0 < G.n ? kPlain : kSkip;
+  // a CTA whose rows lie wholly below the matrix stores nothing
+  if (EPI == kBx) return (col0 < G.n && tm * BM < G.m) ? kPlain : kSkip;
   if (col0 >= G.m) return kSkip;
   const int d0 = tm * BM;
   if (col0 + kChunk <= d0) return kSkip;  // strictly below the diagonal block
@@ -149,6 +185,16 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 
+// Bytes of one K stage over BOTH CTAs of the pair (armed on the leader's barrier).
+template <int EPI>
+__device__ __forceinline__ uint32_t pair_stage_bytes(const Group& G, int tn) {
+  if (EPI != kBx) return 2 * kStageBytes;  // out-of-range rows are zero-filled, still counted
+  // kBx: 64-column boxes of X wholly beyond n are not copied
+  const int left = G.n - tn * BN;
+  const int boxes = left >= BN ? BN / 64 : (left + 63) / 64;
+  return 2 * kTileBytesP + static_cast<uint32_t>(boxes) * 8192u;
+}
+
 #ifdef MUON_TRACE
 __device__ __forceinline__ void trace_stamp(const Params& p, int tile, int slot) {
   if (p.trace && blockIdx.x < kTraceCtas && tile < kTraceTiles)
@@ -163,10 +209,14 @@ __device__ __forceinline__ void trace_stamp(const Params& p, int tile, int slot)
 
 // ---------------------------------------------------------------------- kernel
 template <int EPI>
-__global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ Params p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ Params p) {
   using C = Cfg<EPI>;
   constexpr int S = C::kStages;
+  constexpr int K = C::kSlots;
   extern __shared__ uint8_t smem_raw[];
+  // identical layout in both CTAs: the pair MMA addresses the partner's
+  // operands at this CTA's offsets
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* ring = smem;
@@ -178,6 +228,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int rank = static_cast<int>(cluster_ctarank());  // 0 = leader
+  const uint32_t peer = static_cast<uint32_t>(rank ^ 1);
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
@@ -185,21 +239,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * S + 2 + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * S + 4);
   auto efull_bar = [&](int s) { return bar0 + 8u * (2 * S + 5 + s); };
-  auto ready_bar = [&](int s) { return bar0 + 8u * (2 * S + 5 + kEpiSlots + s); };
-  auto sfree_bar = [&](int b) { return bar0 + 8u * (2 * S + 5 + 2 * kEpiSlots + b); };
-  auto econs_bar = [&](int s) { return bar0 + 8u * (2 * S + 7 + 2 * kEpiSlots + s); };
+  auto ready_bar = [&](int s) { return bar0 + 8u * (2 * S + 5 + K + s); };
+  auto sfree_bar = [&](int b) { return bar0 + 8u * (2 * S + 5 + 2 * K + b); };
+  auto econs_bar = [&](int s) { return bar0 + 8u * (2 * S + 7 + 2 * K + s); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(full_bar(s), 1);   // leader's: its arrive + both CTAs' bytes
+      mbar_init(empty_bar(s), 1);  // one commit from the leader's MMA thread
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), kEpiThreads);
+      // one arrival per epilogue warp; the leader's also takes the partner's relayed one
+      mbar_init(tempty_bar(a), kEpiThreads / 32 + (rank == 0 ? 1 : 0));
     }
     mbar_init(drain_bar, 1);
-    for (int s = 0; s < kEpiSlots; ++s) {
+    for (int s = 0; s < K; ++s) {
       mbar_init(efull_bar(s), 1);
       mbar_init(ready_bar(s), kEpiThreads);
       mbar_init(econs_bar(s), kEpiThreads);
@@ -209,8 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish_pair();
   }
   if (warp == 0 && lane == 0) {
     for (int g = 0; g < p.ngroups; ++g) {
@@ -219,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before either touches the other's
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
@@ -228,12 +283,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   ctl.status = p.status;
   ctl.timeout_ns = p.timeout_ns;
   ctl.where = 0;
+  ctl.peer_abort = cluster_addr(smem_u32(const_cast<int*>(abort_flag)), peer);
   const unsigned long long drain_ns = p.timeout_ns < 50000000ull ? p.timeout_ns : 50000000ull;
-  const int my_tiles =
-      blockIdx.x < p.total_tiles ? (p.total_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int my_tiles = pair < p.total_tiles ? (p.total_tiles - 1 - pair) / npairs + 1 : 0;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ copier
+    // ------------------------------------------------------------ copier (both CTAs)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -241,38 +296,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       bool inject = (p.inject == 1 && blockIdx.x == 0);
       bool ok = true;
       for (int k = 0; k < my_tiles && ok; ++k) {
-        const TileCoord tc = decode_tile<EPI>(p, blockIdx.x + k * gridDim.x);
+        const TileCoord tc = decode_tile<EPI>(p, pair + k * npairs, rank);
         const Group& G = p.grp[tc.g];
         const Maps& M = p.map[tc.g];
         const int kblocks = (G.k + BK - 1) / BK;
+        const uint32_t bytes = pair_stage_bytes<EPI>(G, tc.tn);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, ctl)) {
             ok = false;
             break;
           }
-          // kBx: 64-column boxes wholly beyond n are not copied (their
-          // accumulator columns are never stored)
-          int qboxes = BN / 64;
-          if (EPI == kBx) {
-            const int left = G.n - tc.tn * BN;
-            qboxes = left >= BN ? BN / 64 : (left + 63) / 64;
-          }
           if (kb == 0) TRACE(k, 0);
           if (kb == kblocks - 1) TRACE(k, 1);
-          mbar_arrive_expect_tx(full_bar(stage), kTileBytesP + qboxes * 8192u);
-          issued_mask |= 1u << stage;
-          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          const uint32_t fbar = cluster_addr(full_bar(stage), 0);  // the leader's barrier
+          if (rank == 0) {
+            mbar_arrive_expect_tx(full_bar(stage), bytes);
+            issued_mask |= 1u << stage;
+            issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          }
           if (inject) {
             inject = false;  // withhold this stage's copies: its consumer's wait runs out
           } else {
             const uint32_t dP = smem_u32(ring + stage * kStageBytes);
             const uint32_t dQ = dP + kTileBytesP;
-            tma_load_3d(dP, &M.p, full_bar(stage), kb * BK, tc.tm * BM, tc.b);
+            const int qcol = tc.tn * BN + rank * BNH;  // this CTA's half of the columns
+            tma_load_3d_pair(dP, &M.p, fbar, kb * BK, tc.tm * BM, tc.b);
             if (EPI == kBx) {
-              for (int c = 0; c < qboxes; ++c)
-                tma_load_3d(dQ + c * 8192, &M.q, full_bar(stage), tc.tn * BN + c * 64, kb * BK, tc.b);
+              for (int c = 0; c < BNH / 64; ++c)
+                if (qcol + c * 64 < G.n)
+                  tma_load_3d_pair(dQ + c * 8192, &M.q, fbar, qcol + c * 64, kb * BK, tc.b);
             } else {
-              tma_load_3d(dQ, &M.q, full_bar(stage), kb * BK, tc.tn * BN, tc.b);
+              tma_load_3d_pair(dQ, &M.q, fbar, kb * BK, qcol, tc.b);
             }
           }
           if (++stage == S) {
@@ -282,22 +336,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         }
       }
       if (!ok) {
+        // the leader's barriers count both CTAs' copies: once they complete,
+        // nothing is still landing in either CTA's ring
         for (int s = 0; s < S; ++s)
           if (issued_mask & (1u << s)) mbar_wait_drain(full_bar(s), (issued_parity >> s) & 1u, drain_ns);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(BN, EPI == kBx);
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16(PM, BN, EPI == kBx);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int k = 0; k < my_tiles && ok; ++k) {
-        const TileCoord tc = decode_tile<EPI>(p, blockIdx.x + k * gridDim.x);
+        const TileCoord tc = decode_tile<EPI>(p, pair + k * npairs, rank);
         const int kblocks = (p.grp[tc.g].k + BK - 1) / BK;
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, ctl)) break;
         tc_fence_after();
@@ -316,9 +372,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const uint64_t adesc = sdesc_sw128(aP + kk * 32, 16, 1024);
             const uint64_t bdesc = (EPI == kBx) ? sdesc_sw128(aQ + kk * 2048, 8192, 1024)
                                                 : sdesc_sw128(aQ + kk * 32, 16, 1024);
-            tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
-          tc_commit(empty_bar(stage));
+          // stage consumed in both CTAs
+          tc_commit_pair(empty_bar(stage));
+          tc_commit_pair(cluster_addr(empty_bar(stage), peer));
           if (++stage == S) {
             stage = 0;
             phase ^= 1u;
@@ -326,14 +384,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         }
         if (!ok) break;
         TRACE(k, 3);
-        tc_commit(tfull_bar(acc));
+        tc_commit_pair(tfull_bar(acc));
+        tc_commit_pair(cluster_addr(tfull_bar(acc), peer));
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
-      tc_commit(drain_bar);
+      tc_commit_pair(drain_bar);
       mbar_wait_drain(drain_bar, 0, drain_ns > 1000000ull ? drain_ns : 1000000ull);
+    } else if (lane == 0) {
+      // partner CTA: relay "accumulator drained" to the leader's MMA thread,
+      // one remote arrival per tile instead of one per epilogue warp
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int k = 0; k < my_tiles; ++k) {
+        if (!mbar_wait(tempty_bar(acc), acc_phase, ctl)) break;
+        mbar_arrive_remote(cluster_addr(tempty_bar(acc), 0));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
     }
     __syncwarp();
   } else {
@@ -354,12 +426,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           tma_prefetch_map(&p.map[g].mt);
           tma_prefetch_map(&p.map[g].s);
         }
-        int pend[kEpiSlots] = {-1, -1, -1, -1};
+        int pend[K];
+        for (int q = 0; q < K; ++q) pend[q] = -1;
         auto issue_eload = [&](int s) {
           if (EPI == kGram || s >= total_chunks) return;
-          const int slot = s % kEpiSlots;
+          const int slot = s % K;
           pend[slot] = s;
-          const TileCoord tc = decode_tile<EPI>(p, blockIdx.x + (s / kChunks) * gridDim.x);
+          const TileCoord tc = decode_tile<EPI>(p, pair + (s / kChunks) * npairs, rank);
           const int col0 = tc.tn * BN + (s % kChunks) * kChunk;
           if (chunk_kind<EPI>(p.grp[tc.g], tc.tm, col0) == kSkip) {
             mbar_arrive(efull_bar(slot));
@@ -371,20 +444,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
               tma_load_3d(dst + kChunkBf16, &p.map[tc.g].mt, efull_bar(slot), col0, tc.tm * BM, tc.b);
           }
         };
-        for (int s = 0; s < kEpiSlots; ++s) issue_eload(s);
+        for (int s = 0; s < K; ++s) issue_eload(s);
         int njob[3] = {0, 0, 0};  // kGram / kPoly: jobs seen per ready barrier (0, 1: staging; 2: block)
         int nup = 0;              // strictly-upper chunks so far (staging buffer = nup & 1)
+        int held = -1;            // staging buffer whose stores may still be reading it
         for (int s = 0; s < total_chunks; ++s) {
           const int k = s / kChunks, c = s % kChunks;
-          const TileCoord tc = decode_tile<EPI>(p, blockIdx.x + k * gridDim.x);
+          const TileCoord tc = decode_tile<EPI>(p, pair + k * npairs, rank);
           const Group& G = p.grp[tc.g];
           const Maps& M = p.map[tc.g];
           const int row0 = tc.tm * BM;
           const int col0 = tc.tn * BN + c * kChunk;
           const int kind = chunk_kind<EPI>(G, tc.tm, col0);
           if (EPI == kBx) {
-            const int slot = s % kEpiSlots;
-            mbar_wait(ready_bar(slot), (s / kEpiSlots) & 1, ctl);
+            const int slot = s % K;
+            mbar_wait(ready_bar(slot), (s / K) & 1, ctl);
             if (kind != kSkip) {
               const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
               tma_store_3d(&M.d, hs, col0, row0, tc.b);                // hi' -> the other hi buffer
@@ -394,13 +468,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             } else {
               bulk_wait_read_all();
             }
-            if (s >= 1) issue_eload(s + kEpiSlots - 1);  // into chunk s-1's slot
+            if (s >= 1) issue_eload(s + K - 1);  // into chunk s-1's slot
             continue;
           }
           if (EPI == kPoly) {
             // every compute thread has read chunk s's A operand: refill its slot
-            mbar_wait(econs_bar(s % kEpiSlots), (s / kEpiSlots) & 1, ctl);
-            issue_eload(s + kEpiSlots);
+            mbar_wait(econs_bar(s % K), (s / K) & 1, ctl);
+            issue_eload(s + K);
           }
           if (kind == kUpper) {
             const int b = nup & 1;
@@ -412,9 +486,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             tma_store_3d(&M.d, ds, col0, row0, tc.b);
             tma_store_3d(&M.mt, ms, row0, col0, tc.b);
             bulk_commit();
+            // two chunks' stores in flight: release the previous buffer once
+            // its stores have read it, keep this one until the next chunk
+            if (held >= 0) {
+              asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+              mbar_arrive(sfree_bar(held));
+            }
+            held = b;
+            continue;
+          }
+          if (kind == kDiag && col0 == row0 && held >= 0) {
+            // a diagonal block starts: it takes both staging buffers
             bulk_wait_read_all();
-            mbar_arrive(sfree_bar(b));
-          } else if (kind == kDiag && ((col0 - row0) / kChunk == 3 || col0 + kChunk >= G.m)) {
+            mbar_arrive(sfree_bar(held));
+            held = -1;
+          }
+          if (kind == kDiag && ((col0 - row0) / kChunk == 3 || col0 + kChunk >= G.m)) {
             mbar_wait(ready_bar(2), njob[2] & 1, ctl);
             ++njob[2];
             tma_store_3d(&M.s, stage_u32, row0, row0, tc.b);
@@ -427,8 +514,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           }
         }
         bulk_wait_all();
-        for (int q = 0; q < kEpiSlots; ++q)  // operand copies still in flight land before exit
-          if (pend[q] >= 0) mbar_wait_drain(efull_bar(q), (pend[q] / kEpiSlots) & 1, drain_ns);
+        if (held >= 0) mbar_arrive(sfree_bar(held));
+        for (int q = 0; q < K; ++q)  // operand copies still in flight land before exit
+          if (pend[q] >= 0) mbar_wait_drain(efull_bar(q), (pend[q] / K) & 1, drain_ns);
       }
       __syncwarp();
     } else {
@@ -446,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       int nuse[2] = {0, 0};  // kGram / kPoly: jobs that used staging buffer b so far
       int nup = 0;
       for (int k = 0; k < my_tiles; ++k) {
-        const TileCoord tc = decode_tile<EPI>(p, blockIdx.x + k * gridDim.x);
+        const TileCoord tc = decode_tile<EPI>(p, pair + k * npairs, rank);
         const Group& G = p.grp[tc.g];
         const int row0 = tc.tm * BM;
         mbar_wait(tfull_bar(acc), acc_phase, ctl);
@@ -469,12 +557,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(rr[q]);
           }
           if (c == kChunks - 1) {
-            // accumulator fully read: hand it back to the MMA warp
+            // accumulator fully read: one arrival per warp hands it back (in
+            // the partner CTA through the relay thread of warp 1)
             tc_fence_before();
-            mbar_arrive(tempty_bar(acc));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(acc));
           }
-          const int slot = s % kEpiSlots;
-          if (EPI != kGram) mbar_wait(efull_bar(slot), (s / kEpiSlots) & 1, ctl);
+          const int slot = s % K;
+          if (EPI != kGram) mbar_wait(efull_bar(slot), (s / K) & 1, ctl);
 
           if (EPI == kBx) {
             // X = hi + lo from the slot; X' = a X + acc; hi' = bf16(X'),
@@ -602,17 +692,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
   }
 
+  // Every role above ends after bounded waits; the pair meets here so that no
+  // MMA, copy or remote arrival still targets a CTA that frees its memory.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
 template <int EPI>
-static cudaError_t launch_one(const Params& p, int grid, cudaStream_t stream) {
+static cudaError_t launch_one(const Params& p, int max_pairs, cudaStream_t stream) {
   static thread_local int configured_device = -1;
+  static thread_local int resident_pairs = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   const size_t smem = Cfg<EPI>::kSmem;
@@ -621,18 +714,30 @@ static cudaError_t launch_one(const Params& p, int grid, cudaStream_t stream) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
+    // clusters of two that fit at once: the persistent grid never waits for a second wave
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * max_pairs, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel<EPI>, &cfg);
+    if (e != cudaSuccess) return e;
+    resident_pairs = n;
     configured_device = dev;
   }
-  gemm_kernel<EPI><<<grid, kThreads, smem, stream>>>(p);
+  int pairs = p.total_tiles < max_pairs ? p.total_tiles : max_pairs;
+  if (resident_pairs > 0 && pairs > resident_pairs) pairs = resident_pairs;
+  gemm_kernel<EPI><<<2 * pairs, kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch(int epi, const Params& p, int grid, cudaStream_t stream) {
+cudaError_t launch(int epi, const Params& p, int max_pairs, cudaStream_t stream) {
   if (p.total_tiles <= 0) return cudaSuccess;
+  if (max_pairs < 1) max_pairs = 1;
   switch (epi) {
-    case kGram: return launch_one<kGram>(p, grid, stream);
-    case kPoly: return launch_one<kPoly>(p, grid, stream);
-    case kBx: return launch_one<kBx>(p, grid, stream);
+    case kGram: return launch_one<kGram>(p, max_pairs, stream);
+    case kPoly: return launch_one<kPoly>(p, max_pairs, stream);
+    case kBx: return launch_one<kBx>(p, max_pairs, stream);
   }
   return cudaErrorInvalidValue;
 }

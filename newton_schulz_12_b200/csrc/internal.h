@@ -11,24 +11,30 @@ namespace muon {
 namespace tc {
 
 constexpr int kMaxGroups = 4;        // shape groups per launch
-constexpr int BM = 128;              // tile rows (TMEM lanes)
+constexpr int BM = 128;              // tile rows per CTA (TMEM lanes)
+constexpr int PM = 2 * BM;           // tile rows per CTA pair (one M = 256 pair MMA)
 constexpr int BN = 256;              // tile columns (fp32 TMEM columns per accumulator)
+constexpr int BNH = BN / 2;          // rows of the column operand each CTA of a pair stages
 constexpr int BK = 64;               // K per stage: one 128-byte swizzle row of bf16
 constexpr int kChunk = 32;           // epilogue columns handled per step
 constexpr int kChunks = BN / kChunk;
-constexpr int kEpiSlots = 4;         // ring of prefetched epilogue operand chunks
 constexpr int kThreads = 352;        // warp 0 copies, warp 1 MMAs, warps 2-9 epilogue math,
                                      // warp 10 epilogue loads and stores
 constexpr int kEpiThreads = 256;     // warps 2-9
 
 enum Epi : int { kGram = 0, kPoly = 1, kBx = 2 };
 
+// Work unit: a PM x BN pair tile of D, rows split between the two CTAs of a
+// cluster (CTA rank r owns rows [PM*tm2 + BM*r, +BM)).
 struct Group {
   int batch;  // matrices in the group
   int m;      // rows of D
   int n;      // columns of D (= m for kGram / kPoly)
   int k;      // reduction length
-  int tiles_m, tiles_n, tiles_per_mat, tile_begin;
+  int tiles_m;        // pair-tile rows: ceil(m / PM)
+  int tiles_n;        // tile columns: ceil(n / BN)
+  int tiles_per_mat;  // pair tiles per matrix
+  int tile_begin;     // first pair tile of the group in the launch
 };
 
 // Tensor maps of one group (3-D: {inner, rows, batch}).
@@ -36,7 +42,7 @@ struct Group {
 // place), d = hi chunk of X' (written); all bf16 32 x 128, 64-byte swizzle.
 struct Maps {
   CUtensorMap p;   // rows of D: X (kGram), A (kPoly), B (kBx); K-major, box 64 x 128
-  CUtensorMap q;   // columns of D: X / A K-major box 64 x 256; X MN-major box 64 x 64 (kBx)
+  CUtensorMap q;   // columns of D: X / A K-major box 64 x 128; X MN-major box 64 x 64 (kBx)
   CUtensorMap e;   // epilogue input chunk, bf16 32 x 128: A (kPoly); hi of X (kBx)
   CUtensorMap d;   // direct output chunk, bf16 32 x 128: A (kGram), B (kPoly), hi of X' (kBx)
   CUtensorMap mt;  // mirrored output chunk, bf16 128 x 32 (kGram / kPoly); lo of X, 32 x 128 (kBx)
@@ -47,7 +53,7 @@ struct Params {
   Maps map[kMaxGroups];
   Group grp[kMaxGroups];
   int ngroups;
-  int total_tiles;
+  int total_tiles;  // pair tiles
   float a, b, c;
   int* status;
   unsigned long long timeout_ns;
@@ -62,16 +68,16 @@ struct Params {
 // 16 after the epilogue barrier, 17 (leader) stores drained from the staging.
 constexpr int kTraceCtas = 16, kTraceTiles = 24, kTraceSlots = 18;
 
-// Symmetric-output tiles per m x m matrix (128 x 256 tiles touching the upper triangle).
+// Symmetric-output pair tiles per m x m matrix: the 256 x 256 tiles on or
+// above the diagonal.
 inline int sym_tiles(int m) {
-  const int tm = (m + BM - 1) / BM, tn = (m + BN - 1) / BN;
-  int t = 0;
-  for (int r = 0; r < tm; ++r) t += tn - (r >> 1);
-  return t;
+  const int t = (m + PM - 1) / PM;
+  return t * (t + 1) / 2;
 }
 
 size_t smem_bytes(int epi);
-cudaError_t launch(int epi, const Params& p, int grid, cudaStream_t stream);
+// `max_pairs` bounds the number of CTA pairs (clusters) of the persistent grid.
+cudaError_t launch(int epi, const Params& p, int max_pairs, cudaStream_t stream);
 
 }  // namespace tc
 
