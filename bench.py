@@ -83,16 +83,19 @@ def stage_work(shapes):
     """Algorithmic work of one launch of each kernel kind over the whole set.
 
     GEMMs: nominal FLOPs (X X^T: 2 m^2 n, A A: 2 m^3, B X: 2 m^2 n).
-    Memory-bound kernels: bytes that must cross HBM per element -- momentum
-    g(2)+buf(4) read, buf(4) written = 10 B; cast g(2)+buf(4) read, the bf16
-    pair hi(2)+lo(2) of X written = 10 B; apply W(4) + O as hi(2)+lo(2) read,
-    W(4) written = 12 B.
+    Memory-bound kernels: bytes that must cross HBM per element -- prep
+    g(2)+buf(4) read, buf(4) and the bf16 pair hi(2)+lo(2) of u written =
+    14 B; apply W(4) + O as hi(2)+lo(2) read, W(4) written = 12 B; (fp32 and
+    stand-alone paths) momentum 10 B, cast 10 B.  The per-matrix scale reads
+    one partial per prep block.
     """
     elems = sum(r * c for r, c in shapes)
     g = sum(2 * min(r, c) ** 2 * max(r, c) for r, c in shapes)
     p = sum(2 * min(r, c) ** 3 for r, c in shapes)
+    prep_blocks = sum(-(-r // 64) * -(-c // 128) for r, c in shapes)
     return {
         "gram": ("tensor", g), "poly": ("tensor", p), "bx": ("tensor", g),
+        "prep": ("hbm", 14 * elems), "scale": ("hbm", 4 * prep_blocks + 4 * len(shapes)),
         "flat": ("hbm", 10 * elems), "cast": ("hbm", 10 * elems), "out": ("hbm", 12 * elems),
     }
 

@@ -53,7 +53,7 @@ SIGNATURES = {
 }
 
 #: muon_kernel_kind names, in enum order.
-KERNEL_KINDS = ["flat", "cast", "gram", "poly", "bx", "out", "simt", "sums"]
+KERNEL_KINDS = ["flat", "cast", "gram", "poly", "bx", "out", "simt", "sums", "prep", "scale"]
 
 _lock = threading.Lock()
 _lib = None

@@ -269,6 +269,7 @@ struct NsGroup {
   bf16* B = nullptr;
   float* Af = nullptr;
   float* Bf = nullptr;
+  int mat_base = 0;             // bf16 path: index of the group's first matrix in the scale array
 };
 
 // Bytes of workspace a group needs; assigns its offsets from `base` (or counts
@@ -322,6 +323,7 @@ void init_tc_params(tc::Params& P, int* status, float a, float b, float c) {
   P.a = a;
   P.b = b;
   P.c = c;
+  P.xscale = nullptr;
   P.status = status;
   P.timeout_ns = g_timeout_ns;
   P.inject = 0;
@@ -346,9 +348,11 @@ int launch_tc(int epi, tc::Params& P, int sms, cudaStream_t s) {
 }
 
 // T steps of X <- aX + (bA + cA^2)X on bf16 operands, X carried as hi + lo.
-// On entry each group's xb[0] / xlo hold X0; on exit xb[T % 2] / xlo hold X_T.
+// On entry each group's xb[0] / xlo hold X0 / s with s = xscale[mat_base + i]
+// per matrix (s = 1 when xscale is null); on exit xb[T % 2] / xlo hold X_T
+// (for T >= 1; X0 / s itself for T = 0).
 int run_ns_bf16(std::vector<NsGroup>& gs, int steps, float a, float b, float c, int* status,
-                int sms, cudaStream_t s) {
+                int sms, cudaStream_t s, const float* xscale) {
   if (steps <= 0 || gs.empty()) return MUON_OK;
   MUON_TRY(get_encoder());
   for (size_t g0 = 0; g0 < gs.size(); g0 += tc::kMaxGroups) {
@@ -382,11 +386,22 @@ int run_ns_bf16(std::vector<NsGroup>& gs, int steps, float a, float b, float c, 
       poly.total_tiles += G.batch * poly.grp[k].tiles_per_mat;
       poly.ngroups = k + 1;
     }
+    for (size_t gi = g0; gi < g1; ++gi) {
+      const int k = static_cast<int>(gi - g0);
+      for (int par = 0; par < 2; ++par) {
+        gram[par].grp[k].mat_base = gs[gi].mat_base;
+        bx[par].grp[k].mat_base = gs[gi].mat_base;
+      }
+    }
+    // the first step folds the per-matrix scale into its Gram and BX epilogues
+    tc::Params gram0 = gram[0], bx0 = bx[0];
+    gram0.xscale = xscale;
+    bx0.xscale = xscale;
     int cur = 0;
     for (int t = 0; t < steps; ++t) {
-      MUON_TRY(launch_tc(tc::kGram, gram[cur], sms, s));
+      MUON_TRY(launch_tc(tc::kGram, t == 0 ? gram0 : gram[cur], sms, s));
       MUON_TRY(launch_tc(tc::kPoly, poly, sms, s));
-      MUON_TRY(launch_tc(tc::kBx, bx[cur], sms, s));
+      MUON_TRY(launch_tc(tc::kBx, t == 0 ? bx0 : bx[cur], sms, s));
       cur ^= 1;
     }
   }
@@ -584,11 +599,142 @@ int launch_cast_chunked(const std::vector<MatInfo>& mats, std::vector<NsGroup>& 
   return MUON_OK;
 }
 
+// Blocks of the prep pass of one matrix.
+int prep_tiles(const MatInfo& M) {
+  return ((M.rows + ew::kPrepRows - 1) / ew::kPrepRows) * ((M.cols + ew::kPrepCols - 1) / ew::kPrepCols);
+}
+
+int count_prep_blocks(const std::vector<MatInfo>& mats) {
+  long long nb = 0;
+  for (const MatInfo& M : mats) nb += prep_tiles(M);
+  return static_cast<int>(nb);
+}
+
+// Index of every group's first matrix in the per-matrix scale array.
+void assign_mat_base(std::vector<NsGroup>& groups) {
+  int base = 0;
+  for (NsGroup& g : groups) {
+    g.mat_base = base;
+    base += g.batch;
+  }
+}
+
+// Momentum (src_kind kFromMomentum) or a plain read of bf16 X (kFromBf16), u
+// written as hi + lo into the group workspaces, partial sums of u^2 per block.
+int launch_prep_chunked(const std::vector<MatInfo>& mats, std::vector<NsGroup>& groups,
+                        const std::vector<const void*>& src, const std::vector<float*>& bufs,
+                        int src_kind, float beta, int nesterov, double* partials,
+                        std::vector<int>& part_begin, std::vector<int>& part_count,
+                        cudaStream_t s) {
+  const int count = static_cast<int>(mats.size());
+  part_begin.assign(count, 0);
+  part_count.assign(count, 0);
+  int global_blk = 0;
+  for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
+    const int i1 = std::min(count, i0 + ew::kMaxMats);
+    ew::PrepParams pp{};
+    pp.src_kind = src_kind;
+    pp.beta = beta;
+    pp.omb = 1.0f - beta;
+    pp.nesterov = nesterov;
+    pp.partials = partials + global_blk;
+    int tiles = 0;
+    for (int i = i0; i < i1; ++i) {
+      const MatInfo& M = mats[i];
+      const NsGroup& G = groups[M.group];
+      ew::PrepMat& P = pp.mat[i - i0];
+      P.src = src[i];
+      P.buf = bufs.empty() ? nullptr : bufs[i];
+      P.rows = M.rows;
+      P.cols = M.cols;
+      P.transposed = M.transposed;
+      P.tiles_c = (M.cols + ew::kPrepCols - 1) / ew::kPrepCols;
+      P.tile_begin = tiles;
+      const long long off = static_cast<long long>(M.index) * G.m * G.ldn;
+      P.xhi = G.xb[0] + off;
+      P.xlo = G.xlo + off;
+      P.ld = G.ldn;
+      P.vec = (M.cols % 8 == 0);  // every pointer is 16-byte aligned (checked on entry)
+      part_begin[i] = global_blk + tiles;
+      part_count[i] = prep_tiles(M);
+      tiles += part_count[i];
+    }
+    pp.nmat = i1 - i0;
+    pp.ntiles = tiles;
+    ProfScope prof(MUON_KERNEL_PREP, s);
+    CUDA_TRY(ew::launch_prep(pp, s));
+    global_blk += tiles;
+  }
+  return MUON_OK;
+}
+
+// s = 1 / (||u|| + eps) of every matrix into xscale[mat_base + index].
+int launch_scale_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGroup>& groups,
+                         const double* partials, const std::vector<int>& part_begin,
+                         const std::vector<int>& part_count, float* xscale, cudaStream_t s) {
+  const int count = static_cast<int>(mats.size());
+  for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
+    const int i1 = std::min(count, i0 + ew::kMaxMats);
+    ew::ScaleParams sp{};
+    sp.partials = partials;
+    sp.eps = 1e-7;  // the same epsilon as kNormEps, in fp64
+    for (int i = i0; i < i1; ++i) {
+      const MatInfo& M = mats[i];
+      const NsGroup& G = groups[M.group];
+      ew::ScaleMat& S = sp.mat[i - i0];
+      S.part_begin = part_begin[i];
+      S.part_count = part_count[i];
+      const long long off = static_cast<long long>(M.index) * G.m * G.ldn;
+      S.xhi = G.xb[0] + off;
+      S.xlo = G.xlo + off;
+      S.m = G.m;
+      S.n = G.n;
+      S.ld = G.ldn;
+      S.scale = xscale + G.mat_base + M.index;
+    }
+    sp.nmat = i1 - i0;
+    ProfScope prof(MUON_KERNEL_SCALE, s);
+    CUDA_TRY(ew::launch_scale(sp, s));
+  }
+  return MUON_OK;
+}
+
+// Workspace of the bf16 path: prep partials, per-matrix scales, then the
+// groups' buffers.  With base null only the size is computed.
+struct BfLayout {
+  double* partials = nullptr;
+  float* xscale = nullptr;
+};
+
+size_t bf16_layout(const std::vector<MatInfo>& mats, std::vector<NsGroup>& groups, char* base,
+                   BfLayout& L) {
+  const size_t nblk = static_cast<size_t>(count_prep_blocks(mats));
+  size_t off = 0;
+  L.partials = base ? reinterpret_cast<double*>(base + off) : nullptr;
+  off = align_up(off + nblk * 8, 1024);
+  L.xscale = base ? reinterpret_cast<float*>(base + off) : nullptr;
+  off = align_up(off + mats.size() * 4, 1024);
+  for (NsGroup& g : groups) off = layout_group(g, base, off, false);
+  return off;
+}
+
+// prep (momentum or plain read) -> per-matrix scale -> T Newton-Schulz steps.
+int run_bf16_path(const std::vector<MatInfo>& mats, std::vector<NsGroup>& groups,
+                  const BfLayout& L, const std::vector<const void*>& src,
+                  const std::vector<float*>& bufs, int src_kind, float beta, int nesterov,
+                  float a, float b, float c, int steps, int* status, int sms, cudaStream_t s) {
+  std::vector<int> pb, pc;
+  MUON_TRY(launch_prep_chunked(mats, groups, src, bufs, src_kind, beta, nesterov, L.partials, pb,
+                               pc, s));
+  MUON_TRY(launch_scale_chunked(mats, groups, L.partials, pb, pc, L.xscale, s));
+  return run_ns_bf16(groups, steps, a, b, c, status, sms, s, L.xscale);
+}
+
 // mode 0: apply into W; 1: bf16 write-back; 2: fp32 write-back.  O of matrix i
 // is read from its group's result (X layout, transposed back).
 int launch_out_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGroup>& groups,
                        const std::vector<Result>& res, const std::vector<void*>& ys, int mode,
-                       float lr, float wd, cudaStream_t s) {
+                       float lr, float wd, cudaStream_t s, const float* oscale = nullptr) {
   const int count = static_cast<int>(mats.size());
   for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
     const int i1 = std::min(count, i0 + ew::kMaxMats);
@@ -615,6 +761,7 @@ int launch_out_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGro
       const float ratio = static_cast<float>(M.rows) / static_cast<float>(M.cols);
       const float scale = ratio > 1.0f ? sqrtf(ratio) : 1.0f;
       O.ls = lr * scale;
+      O.oscale = oscale ? oscale + G.mat_base + M.index : nullptr;
       O.vec = (M.cols % 8 == 0) && (G.ldn % 8 == 0) && aligned16(ys[i]);
       tiles += ((M.rows + ew::kTile - 1) / ew::kTile) * O.tiles_c;
     }
@@ -732,37 +879,44 @@ int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a,
   std::vector<MatInfo> mats;
   std::vector<NsGroup> groups;
   group_shapes(shapes, mats, groups);
+  std::vector<const void*> src(X_ptrs, X_ptrs + batch);
+  std::vector<void*> ys(X_ptrs, X_ptrs + batch);
+  std::vector<Result> res;
+  if (!fp32) {
+    assign_mat_base(groups);
+    BfLayout L;
+    size_t off = bf16_layout(mats, groups, nullptr, L);
+    Workspace* ws = nullptr;
+    MUON_TRY(get_workspace(s, off, &ws));
+    bf16_layout(mats, groups, static_cast<char*>(ws->ptr), L);
+    MUON_TRY(run_bf16_path(mats, groups, L, src, {}, ew::kFromBf16, 0.f, 0, a, b, c, steps,
+                           ws->status, dev.sms, s));
+    for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
+    MUON_TRY(launch_out_chunked(mats, groups, res, ys, 1, 0.f, 0.f, s, steps == 0 ? L.xscale : nullptr));
+    return MUON_OK;
+  }
+  // fp32 verification path: normalised fp32 X, SIMT GEMMs
   std::vector<long long> numels(batch, static_cast<long long>(m) * n);
   const int nblk = count_flat_blocks(numels);
   size_t off = align_up(static_cast<size_t>(nblk) * 4, 1024);
-  for (NsGroup& g : groups) off = layout_group(g, nullptr, off, fp32);
+  for (NsGroup& g : groups) off = layout_group(g, nullptr, off, true);
   Workspace* ws = nullptr;
   MUON_TRY(get_workspace(s, off, &ws));
   char* base = static_cast<char*>(ws->ptr);
   float* partials = reinterpret_cast<float*>(base);
   off = align_up(static_cast<size_t>(nblk) * 4, 1024);
-  for (NsGroup& g : groups) off = layout_group(g, base, off, fp32);
-
-  std::vector<const void*> src(X_ptrs, X_ptrs + batch);
+  for (NsGroup& g : groups) off = layout_group(g, base, off, true);
   std::vector<int> pb, pc;
-  const int kind = fp32 ? ew::kFromF32 : ew::kFromBf16;
-  MUON_TRY(launch_flat_chunked(src, {}, numels, kind, 0.f, 0, partials, pb, pc, s));
-  MUON_TRY(launch_cast_chunked(mats, groups, src, {}, kind, 0.f, 0, partials, pb, pc, !fp32, s));
-  std::vector<Result> res;
-  if (fp32) {
-    std::vector<float*> final_xf;
-    MUON_TRY(run_ns_fp32(groups, steps, a, b, c, s, final_xf));
-    for (float* f : final_xf) {
-      Result r;
-      r.f = f;
-      res.push_back(r);
-    }
-  } else {
-    MUON_TRY(run_ns_bf16(groups, steps, a, b, c, ws->status, dev.sms, s));
-    for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
+  MUON_TRY(launch_flat_chunked(src, {}, numels, ew::kFromF32, 0.f, 0, partials, pb, pc, s));
+  MUON_TRY(launch_cast_chunked(mats, groups, src, {}, ew::kFromF32, 0.f, 0, partials, pb, pc, false, s));
+  std::vector<float*> final_xf;
+  MUON_TRY(run_ns_fp32(groups, steps, a, b, c, s, final_xf));
+  for (float* f : final_xf) {
+    Result r;
+    r.f = f;
+    res.push_back(r);
   }
-  std::vector<void*> ys(X_ptrs, X_ptrs + batch);
-  MUON_TRY(launch_out_chunked(mats, groups, res, ys, fp32 ? 2 : 1, 0.f, 0.f, s));
+  MUON_TRY(launch_out_chunked(mats, groups, res, ys, 2, 0.f, 0.f, s));
   return MUON_OK;
 }
 
@@ -783,10 +937,9 @@ int muon_ns_orthogonalize_static(int batch, int m, int n, void* const* X_ptrs, f
   std::vector<MatInfo> mats;
   std::vector<NsGroup> groups;
   group_shapes(shapes, mats, groups);
-  std::vector<long long> numels(batch, static_cast<long long>(m) * n);
-  const int nblk = count_flat_blocks(numels);
-  size_t need = align_up(static_cast<size_t>(nblk) * 4, 1024);
-  for (NsGroup& g : groups) need = layout_group(g, nullptr, need, false);
+  assign_mat_base(groups);
+  BfLayout L;
+  const size_t need = bf16_layout(mats, groups, nullptr, L);
   if (need + kStaticStatusBytes > kStaticScratchBytes)
     return set_err(MUON_ERR_SHAPE,
                    "batch %d of %dx%d needs %zu bytes of scratch; the static scratch holds %zu "
@@ -803,20 +956,15 @@ int muon_ns_orthogonalize_static(int batch, int m, int n, void* const* X_ptrs, f
     CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
   }
   HooksOff no_hooks;
-  char* base = scratch + kStaticStatusBytes;
-  float* partials = reinterpret_cast<float*>(base);
-  size_t off = align_up(static_cast<size_t>(nblk) * 4, 1024);
-  for (NsGroup& g : groups) off = layout_group(g, base, off, false);
+  bf16_layout(mats, groups, scratch + kStaticStatusBytes, L);
 
   std::vector<const void*> src(X_ptrs, X_ptrs + batch);
-  std::vector<int> pb, pc;
-  MUON_TRY(launch_flat_chunked(src, {}, numels, ew::kFromBf16, 0.f, 0, partials, pb, pc, s));
-  MUON_TRY(launch_cast_chunked(mats, groups, src, {}, ew::kFromBf16, 0.f, 0, partials, pb, pc, true, s));
-  MUON_TRY(run_ns_bf16(groups, steps, a, b, c, status, dev.sms, s));
+  MUON_TRY(run_bf16_path(mats, groups, L, src, {}, ew::kFromBf16, 0.f, 0, a, b, c, steps, status,
+                         dev.sms, s));
   std::vector<Result> res;
   for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
   std::vector<void*> ys(X_ptrs, X_ptrs + batch);
-  MUON_TRY(launch_out_chunked(mats, groups, res, ys, 1, 0.f, 0.f, s));
+  MUON_TRY(launch_out_chunked(mats, groups, res, ys, 1, 0.f, 0.f, s, steps == 0 ? L.xscale : nullptr));
   return MUON_OK;
 }
 
@@ -846,31 +994,21 @@ int muon_step(int count, float* const* params, const void* const* grads,
   std::vector<MatInfo> mats;
   std::vector<NsGroup> groups;
   group_shapes(shp, mats, groups);
-  std::vector<long long> numels(count);
-  for (int i = 0; i < count; ++i) numels[i] = static_cast<long long>(shp[i].first) * shp[i].second;
-  const int nblk = count_flat_blocks(numels);
-  size_t off = align_up(static_cast<size_t>(nblk) * 4, 1024);
-  for (NsGroup& g : groups) off = layout_group(g, nullptr, off, false);
+  assign_mat_base(groups);
+  BfLayout L;
+  size_t off = bf16_layout(mats, groups, nullptr, L);
   Workspace* ws = nullptr;
   MUON_TRY(get_workspace(s, off, &ws));
-  char* base = static_cast<char*>(ws->ptr);
-  float* partials = reinterpret_cast<float*>(base);
-  off = align_up(static_cast<size_t>(nblk) * 4, 1024);
-  for (NsGroup& g : groups) off = layout_group(g, base, off, false);
+  bf16_layout(mats, groups, static_cast<char*>(ws->ptr), L);
 
   std::vector<const void*> gsrc(grads, grads + count);
   std::vector<float*> bufs(momentum_bufs, momentum_bufs + count);
-  std::vector<const float*> cbufs(momentum_bufs, momentum_bufs + count);
-  std::vector<int> pb, pc;
-  MUON_TRY(launch_flat_chunked(gsrc, bufs, numels, ew::kFromMomentum, beta, nesterov, partials, pb,
-                               pc, s));
-  MUON_TRY(launch_cast_chunked(mats, groups, gsrc, cbufs, ew::kFromMomentum, beta, nesterov,
-                               partials, pb, pc, true, s));
-  MUON_TRY(run_ns_bf16(groups, steps, kCoefA, kCoefB, kCoefC, ws->status, dev.sms, s));
+  MUON_TRY(run_bf16_path(mats, groups, L, gsrc, bufs, ew::kFromMomentum, beta, nesterov,
+                         kCoefA, kCoefB, kCoefC, steps, ws->status, dev.sms, s));
   std::vector<Result> res;
   for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
   std::vector<void*> ys(params, params + count);
-  MUON_TRY(launch_out_chunked(mats, groups, res, ys, 0, lr, wd, s));
+  MUON_TRY(launch_out_chunked(mats, groups, res, ys, 0, lr, wd, s, steps == 0 ? L.xscale : nullptr));
   return MUON_OK;
 }
 

@@ -315,18 +315,19 @@ __device__ __forceinline__ void load_o8(const OutMat& M, int r, int c, int orows
   const int cnt = r < orows ? min(8, ocols - c) : 0;
   const long long idx = static_cast<long long>(r) * M.ld + c;
   if (M.o_hi) {
+    const float f = M.oscale ? *M.oscale : 1.0f;
     if (cnt == 8 && M.vec) {
       float h[8], l[8];
       unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const bf16*>(M.o_hi) + idx), h);
       unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const bf16*>(M.o_lo) + idx), l);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) o[k] = h[k] + l[k];
+      for (int k = 0; k < 8; ++k) o[k] = (h[k] + l[k]) * f;
       return;
     }
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-      o[k] = k < cnt ? bf16_bits_to_f32(static_cast<const uint16_t*>(M.o_hi)[idx + k]) +
-                           bf16_bits_to_f32(static_cast<const uint16_t*>(M.o_lo)[idx + k])
+      o[k] = k < cnt ? (bf16_bits_to_f32(static_cast<const uint16_t*>(M.o_hi)[idx + k]) +
+                        bf16_bits_to_f32(static_cast<const uint16_t*>(M.o_lo)[idx + k])) * f
                      : 0.f;
     return;
   }
@@ -416,6 +417,240 @@ __global__ void __launch_bounds__(kTileThreads) out_kernel(const __grid_constant
       update_y8(p, M, r0 + y + 32 * h, c0 + xg, o);
     }
   }
+}
+
+// ------------------------------------------------------------------ prep kernel
+// One kPrepRows x kPrepCols tile of the caller's matrix per block (8192
+// elements, as a flat_kernel block).  Thread t owns column group t % 16
+// (eight consecutive columns) of rows t / 16 + 16 h, h = 0..3, and issues all
+// of its loads before any arithmetic.  A wide matrix's hi / lo are written
+// straight from registers (X = U); a tall one's go through a shared-memory
+// transpose (X = U^T) so that the writes also run along X's rows.
+constexpr int kPrepThreads = 256;
+#ifndef MUON_PREP_MIN_BLOCKS
+#define MUON_PREP_MIN_BLOCKS 3  // resident blocks per SM the register budget aims for
+#endif
+constexpr int kPrepUnits = kPrepRows * kPrepCols / (kPrepThreads * 8);  // 4 runs of 8 per thread
+
+__device__ __forceinline__ void store_pair8(void* hi_base, void* lo_base, long long off, int cnt,
+                                            const float (&v)[8]) {
+  uint32_t hi[4], lo[4];
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    hi[h] = pack_bf16x2(v[2 * h], v[2 * h + 1]);
+    lo[h] = pack_bf16x2(v[2 * h] - bf16_bits_to_f32(static_cast<uint16_t>(hi[h] & 0xFFFFu)),
+                        v[2 * h + 1] - bf16_bits_to_f32(static_cast<uint16_t>(hi[h] >> 16)));
+  }
+  if (cnt == 8) {  // the workspace row stride is a multiple of 8: aligned
+    *reinterpret_cast<uint4*>(static_cast<bf16*>(hi_base) + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(static_cast<bf16*>(lo_base) + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    return;
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    if (k < cnt) {
+      const uint32_t w = (k & 1) ? (hi[k >> 1] >> 16) : (hi[k >> 1] & 0xFFFFu);
+      const uint32_t l = (k & 1) ? (lo[k >> 1] >> 16) : (lo[k >> 1] & 0xFFFFu);
+      static_cast<uint16_t*>(hi_base)[off + k] = static_cast<uint16_t>(w);
+      static_cast<uint16_t*>(lo_base)[off + k] = static_cast<uint16_t>(l);
+    }
+  }
+}
+
+// Fixed-order fp64 block sum (result in thread 0); contains a block barrier.
+__device__ __forceinline__ double block_sum_f64(double v, double* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  double s = 0.0;
+  if (threadIdx.x == 0) {
+    for (int w = 0; w < kPrepThreads / 32; ++w) s += red[w];
+  }
+  return s;
+}
+
+__global__ void __launch_bounds__(kPrepThreads, MUON_PREP_MIN_BLOCKS) prep_kernel(const __grid_constant__ PrepParams p) {
+  __shared__ float tile[kPrepRows][kPrepCols + 1];
+  __shared__ double red[kPrepThreads / 32];
+  const int mi = find_tile_mat(p.mat, p.nmat, blockIdx.x);
+  const PrepMat& M = p.mat[mi];
+  const int local = blockIdx.x - M.tile_begin;
+  const int tr = local / M.tiles_c, tcn = local - tr * M.tiles_c;
+  const int r0 = tr * kPrepRows, c0 = tcn * kPrepCols;
+  const int cg = threadIdx.x & 15, ry = threadIdx.x >> 4;
+  const int c = c0 + 8 * cg;
+  const MomentumOp op{p.beta, p.omb, p.nesterov};
+  const bool mom = (p.src_kind == kFromMomentum);
+  float u[kPrepUnits][8];
+
+  if (M.vec) {
+    // cols % 8 == 0: a run is either wholly inside the row or wholly outside
+    uint4 g4[kPrepUnits];
+    float4 b4[kPrepUnits][2];
+#pragma unroll
+    for (int h = 0; h < kPrepUnits; ++h) {
+      const int r = r0 + ry + 16 * h;
+      if (r < M.rows && c < M.cols) {
+        const long long idx = static_cast<long long>(r) * M.cols + c;
+        g4[h] = *reinterpret_cast<const uint4*>(static_cast<const bf16*>(M.src) + idx);
+        if (mom) {
+          const float4* q = reinterpret_cast<const float4*>(M.buf + idx);
+          b4[h][0] = q[0];
+          b4[h][1] = q[1];
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < kPrepUnits; ++h) {
+      const int r = r0 + ry + 16 * h;
+      if (r < M.rows && c < M.cols) {
+        float x[8];
+        unpack_bf16x8(g4[h], x);
+        if (mom) {
+          float mb[8] = {b4[h][0].x, b4[h][0].y, b4[h][0].z, b4[h][0].w,
+                         b4[h][1].x, b4[h][1].y, b4[h][1].z, b4[h][1].w};
+#pragma unroll
+          for (int k = 0; k < 8; ++k) u[h][k] = op(x[k], mb[k]);
+          float4* q = reinterpret_cast<float4*>(M.buf + static_cast<long long>(r) * M.cols + c);
+          q[0] = make_float4(mb[0], mb[1], mb[2], mb[3]);
+          q[1] = make_float4(mb[4], mb[5], mb[6], mb[7]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) u[h][k] = x[k];
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) u[h][k] = 0.f;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int h = 0; h < kPrepUnits; ++h) {
+      const int r = r0 + ry + 16 * h;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        float v = 0.f;
+        if (r < M.rows && c + k < M.cols) {
+          const long long idx = static_cast<long long>(r) * M.cols + c + k;
+          const float x = bf16_bits_to_f32(static_cast<const uint16_t*>(M.src)[idx]);
+          if (mom) {
+            float mb = M.buf[idx];
+            v = op(x, mb);
+            M.buf[idx] = mb;
+          } else {
+            v = x;
+          }
+        }
+        u[h][k] = v;
+      }
+    }
+  }
+
+  double acc = 0.0;
+#pragma unroll
+  for (int h = 0; h < kPrepUnits; ++h)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const double w = u[h][k];
+      acc = fma(w, w, acc);
+    }
+
+  if (!M.transposed) {
+#pragma unroll
+    for (int h = 0; h < kPrepUnits; ++h) {
+      const int r = r0 + ry + 16 * h;
+      if (r < M.rows && c < M.cols)
+        store_pair8(M.xhi, M.xlo, static_cast<long long>(r) * M.ld + c, min(8, M.cols - c), u[h]);
+    }
+  } else {
+#pragma unroll
+    for (int h = 0; h < kPrepUnits; ++h)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) tile[ry + 16 * h][8 * cg + k] = u[h][k];
+  }
+  const double s = block_sum_f64(acc, red);  // its barrier also publishes the tile
+  if (threadIdx.x == 0) p.partials[blockIdx.x] = s;
+  if (M.transposed) {
+    // X rows c0 + xr (caller columns), X columns r0 + 8 xg .. +7 (caller rows)
+    const int xg = threadIdx.x & 7;
+#pragma unroll
+    for (int q = 0; q < kPrepUnits; ++q) {
+      const int xr = (threadIdx.x >> 3) + 32 * q;
+      const int xrow = c0 + xr, xcol = r0 + 8 * xg;
+      if (xrow < M.cols && xcol < M.rows) {
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = tile[8 * xg + k][xr];
+        store_pair8(M.xhi, M.xlo, static_cast<long long>(xrow) * M.ld + xcol, min(8, M.rows - xcol), v);
+      }
+    }
+  }
+}
+
+// One block per matrix: s = 1 / (||u||_F + eps) from the matrix's partials in
+// a fixed order.  Outside [2^-40, 2^40] the norm is first brought to [1, 2)
+// by scaling the workspace pair with an exact power of two (both factors at
+// least 2^-64), so that the first Gram product of the unnormalised pair
+// neither overflows nor loses its leading terms to underflow.
+constexpr int kScaleThreads = 256;
+
+__global__ void __launch_bounds__(kScaleThreads) scale_kernel(const __grid_constant__ ScaleParams p) {
+  __shared__ float s_f[2];
+  const ScaleMat& M = p.mat[blockIdx.x];
+  if (threadIdx.x < 32) {
+    // lane l adds partials l, l+32, ... then a fixed xor tree
+    const int lane = threadIdx.x;
+    double ss = 0.0;
+    for (int q = lane; q < M.part_count; q += 32) ss += p.partials[M.part_begin + q];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) {
+      double den = sqrt(ss) + p.eps;
+      float f1 = 1.0f, f2 = 1.0f;
+      if (isfinite(den) && (den > 0x1p40 || den < 0x1p-40)) {
+        const int e = ilogb(den);  // |e| <= 1100: each factor stays a normal fp32
+        f1 = ldexpf(1.0f, -(e / 2));
+        f2 = ldexpf(1.0f, -(e - e / 2));
+        den = (den * f1) * f2;
+      }
+      s_f[0] = f1;
+      s_f[1] = f2;
+      *M.scale = static_cast<float>(1.0 / den);
+    }
+  }
+  __syncthreads();
+  const float f1 = s_f[0], f2 = s_f[1];
+  if (f1 == 1.0f && f2 == 1.0f) return;
+  const long long units = static_cast<long long>(M.m) * M.ld / 8;
+  for (long long i = threadIdx.x; i < units; i += kScaleThreads) {
+    uint4* ph = reinterpret_cast<uint4*>(static_cast<bf16*>(M.xhi)) + i;
+    uint4* pl = reinterpret_cast<uint4*>(static_cast<bf16*>(M.xlo)) + i;
+    float h[8], l[8];
+    unpack_bf16x8(*ph, h);
+    unpack_bf16x8(*pl, l);
+    uint32_t oh[4], ol[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      oh[k] = pack_bf16x2((h[2 * k] * f1) * f2, (h[2 * k + 1] * f1) * f2);
+      ol[k] = pack_bf16x2((l[2 * k] * f1) * f2, (l[2 * k + 1] * f1) * f2);
+    }
+    *ph = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+    *pl = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+  }
+}
+
+cudaError_t launch_prep(const PrepParams& p, cudaStream_t s) {
+  if (p.ntiles <= 0) return cudaSuccess;
+  prep_kernel<<<p.ntiles, kPrepThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scale(const ScaleParams& p, cudaStream_t s) {
+  if (p.nmat <= 0) return cudaSuccess;
+  scale_kernel<<<p.nmat, kScaleThreads, 0, s>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_flat(const FlatParams& p, cudaStream_t s) {

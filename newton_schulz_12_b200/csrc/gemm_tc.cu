@@ -537,6 +537,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const TileCoord tc = decode_tile<EPI>(p, pair + k * npairs, rank);
         const Group& G = p.grp[tc.g];
         const int row0 = tc.tm * BM;
+        // X = s (hi + lo) on the first step: A = s^2 acc, X' = s (a (hi + lo) + acc)
+        float xs = 1.0f;
+        if (EPI != kPoly && p.xscale) {
+          xs = p.xscale[G.mat_base + tc.b];
+          if (EPI == kGram) xs = xs * xs;
+        }
         mbar_wait(tfull_bar(acc), acc_phase, ctl);
         tc_fence_after();
         if (leader) TRACE(k, 4);
@@ -586,7 +592,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                   for (int e = 0; e < 2; ++e) {
                     const float xh = bf16_bits_to_f32(static_cast<uint16_t>(h4[h] >> (16 * e)));
                     const float xl = bf16_bits_to_f32(static_cast<uint16_t>(l4[h] >> (16 * e)));
-                    y[e] = fmaf(p.a, xh + xl, v[8 * uu + 2 * h + e]);
+                    y[e] = fmaf(p.a, xh + xl, v[8 * uu + 2 * h + e]) * xs;
                   }
                   ho[h] = pack_bf16x2(y[0], y[1]);
                   const float r0 = y[0] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] & 0xFFFFu));
@@ -603,6 +609,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
 
           // ------------------------------------------------ kGram / kPoly
+          if (EPI == kGram && kind != kSkip) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v[q] *= xs;
+          }
           if (EPI == kPoly) {
             if (kind != kSkip) {
               // B = b A + c acc with A's chunk from the slot (bf16, 64-byte swizzle)

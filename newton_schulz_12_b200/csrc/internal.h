@@ -35,6 +35,7 @@ struct Group {
   int tiles_n;        // tile columns: ceil(n / BN)
   int tiles_per_mat;  // pair tiles per matrix
   int tile_begin;     // first pair tile of the group in the launch
+  int mat_base;       // index of the group's first matrix in Params::xscale
 };
 
 // Tensor maps of one group (3-D: {inner, rows, batch}).
@@ -55,6 +56,9 @@ struct Params {
   int ngroups;
   int total_tiles;  // pair tiles
   float a, b, c;
+  // Per-matrix factor s of X = s * (hi + lo), or null (s = 1): kGram scales
+  // A by s^2, kBx scales X' by s.
+  const float* xscale;
   int* status;
   unsigned long long timeout_ns;
   int inject;  // 1: withhold one operand copy in CTA 0 (timeout-path test)
@@ -166,6 +170,7 @@ struct OutMat {
   int tiles_c;        // 64-wide tiles along y's columns
   int tile_begin;
   float ls;           // fl(lr * scale)
+  const float* oscale;  // O = oscale[0] * (hi + lo) when set (result of zero steps)
   int vec;            // cols % 8 == 0 and ld % 8 == 0: 128-bit accesses
 };
 
@@ -174,6 +179,53 @@ struct OutParams {
   int nmat, ntiles;
   int mode;           // 0: apply, 1: write bf16, 2: write f32
   float lw;           // fl(lr * wd)
+};
+
+// One pass over the caller's matrices: momentum (or a plain read of X), the
+// Nesterov blend u, and u written to the workspace as the bf16 pair hi + lo
+// (transposed when tall), plus a partial sum of u^2 per block.  Blocks cover
+// kPrepRows x kPrepCols tiles of the caller's layout.
+constexpr int kPrepRows = 64, kPrepCols = 128;
+
+struct PrepMat {
+  const void* src;    // grad (bf16) or X (bf16)
+  float* buf;         // momentum buffer (in/out), or null
+  int rows, cols;     // caller layout
+  int transposed;     // rows > cols: X = U^T
+  int tiles_c;        // tiles along the caller's columns
+  int tile_begin;
+  void* xhi;          // workspace X (m x n, row stride ld): hi and lo of u
+  void* xlo;
+  long long ld;
+  int vec;            // cols % 8 == 0: 128-bit accesses of the caller's rows
+};
+
+struct PrepParams {
+  PrepMat mat[kMaxMats];
+  int nmat, ntiles;
+  int src_kind;       // kFromMomentum or kFromBf16
+  float beta, omb;
+  int nesterov;
+  double* partials;   // sum of u^2 per block (fp64: no overflow for any bf16 / fp32 u)
+};
+
+// Per-matrix scale of the first Newton-Schulz step: s = 1 / (||u||_F + eps)
+// from the partials; matrices with ||u|| outside [2^-40, 2^40] have their
+// workspace pair rescaled by an exact power of two first.
+struct ScaleMat {
+  int part_begin, part_count;
+  void* xhi;          // workspace pair of the matrix (m rows, row stride ld)
+  void* xlo;
+  int m, n;
+  long long ld;
+  float* scale;       // destination of s
+};
+
+struct ScaleParams {
+  ScaleMat mat[kMaxMats];
+  int nmat;
+  const double* partials;
+  double eps;
 };
 
 struct SumParams {
@@ -188,6 +240,8 @@ cudaError_t launch_flat(const FlatParams& p, cudaStream_t s);
 cudaError_t launch_cast(const CastParams& p, cudaStream_t s);
 cudaError_t launch_out(const OutParams& p, cudaStream_t s);
 cudaError_t launch_sums(const SumParams& p, cudaStream_t s);
+cudaError_t launch_prep(const PrepParams& p, cudaStream_t s);
+cudaError_t launch_scale(const ScaleParams& p, cudaStream_t s);
 
 }  // namespace ew
 

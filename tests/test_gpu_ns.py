@@ -78,6 +78,18 @@ def test_other_coefficients():
     assert rel_fro(run_ns([X], steps=5, coeffs=coeffs)[0], ref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("scale", [2.0 ** 60, 2.0 ** 45, 2.0 ** -45, 2.0 ** -100])
+def test_bf16_extreme_magnitudes(scale):
+    """Norms far from 1: the first Gram product runs on the unnormalised pair,
+    so norms beyond 2^40 are rescaled by a power of two first and tiny inputs
+    reduce to X_k ~ a^k X0 (A underflows), as in the oracle."""
+    X = (workloads.gaussian((256, 640), 1.0, seed=11) * scale).to(torch.bfloat16)
+    ref = oracle.newton_schulz(X.double().numpy())
+    got = run_ns([X])[0]
+    assert np.all(np.isfinite(got))
+    assert rel_fro(got, ref) <= TOL_BF16
+
+
 def test_zero_matrix_gives_zero():
     for dt in (torch.bfloat16, torch.float32):
         got = run_ns([torch.zeros(64, 96, dtype=dt)])[0]
