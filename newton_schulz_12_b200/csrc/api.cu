@@ -249,9 +249,10 @@ int bx_maps(tc::Maps& M, const void* B, long long ldb, long long sb, const void*
             void* Xlo, void* Xhi_out, int m, int n, long long ldx, long long sx, int batch) {
   MUON_TRY(make_map(&M.p, B, 2, m, m, batch, ldb, sb, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
   MUON_TRY(make_map(&M.q, Xhi, 2, n, m, batch, ldx, sx, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
-  MUON_TRY(make_map(&M.e, Xhi, 2, n, m, batch, ldx, sx, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
-  MUON_TRY(make_map(&M.mt, Xlo, 2, n, m, batch, ldx, sx, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
-  MUON_TRY(make_map(&M.d, Xhi_out, 2, n, m, batch, ldx, sx, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
+  // epilogue chunks of 64 columns: 128-byte rows
+  MUON_TRY(make_map(&M.e, Xhi, 2, n, m, batch, ldx, sx, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
+  MUON_TRY(make_map(&M.mt, Xlo, 2, n, m, batch, ldx, sx, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
+  MUON_TRY(make_map(&M.d, Xhi_out, 2, n, m, batch, ldx, sx, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
   M.s = M.d;  // unused
   return MUON_OK;
 }

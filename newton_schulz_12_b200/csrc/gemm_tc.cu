@@ -67,7 +67,7 @@ constexpr size_t kMaxSmem = 232448;                         // 227 KiB per CTA o
 #define MUON_BX_STAGES 4
 #endif
 #ifndef MUON_BX_SLOTS
-#define MUON_BX_SLOTS 6
+#define MUON_BX_SLOTS 3
 #endif
 
 template <int EPI>
@@ -78,7 +78,12 @@ struct Cfg {
   // kBx slot: the hi and lo bf16 chunks of X (8 KiB each); kPoly slot: A's chunk
   static constexpr int kSlots = (EPI == kBx) ? MUON_BX_SLOTS : MUON_POLY_SLOTS;
   static_assert(kSlots >= 3, "ready barriers 0-2 double as staging barriers");
-  static constexpr uint32_t kSlotBytes = (EPI == kBx) ? 2 * kChunkBf16 : (EPI == kPoly ? kChunkBf16 : 0);
+  static_assert(BN % (2 * kChunk) == 0, "whole chunks per tile");
+  // kBx works on 64-column chunks (128-byte rows in global memory), the
+  // symmetric kernels on 32-column chunks (their mirrored stores are 32 rows)
+  static constexpr int kCW = (EPI == kBx) ? 2 * kChunk : kChunk;
+  static constexpr int kNCh = BN / kCW;  // per tile
+  static constexpr uint32_t kSlotBytes = (EPI == kBx) ? 4 * kChunkBf16 : (EPI == kPoly ? kChunkBf16 : 0);
   static constexpr uint32_t kSlotsBytes = kSlotBytes * kSlots;
   // staging: kBx two bf16 output chunks; kGram / kPoly 2 direct + 2 mirror chunks,
   // aliased by the 128 x 128 diagonal block (2 x [128 rows][64 cols] bf16)
@@ -410,7 +415,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-9) and IO (warp 10)
-    const int total_chunks = my_tiles * kChunks;
+    constexpr int NCH = C::kNCh, CW = C::kCW;
+    const int total_chunks = my_tiles * NCH;
     const uint32_t slots_u32 = smem_u32(slots);
     const uint32_t stage_u32 = smem_u32(staging);
 
@@ -432,16 +438,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (EPI == kGram || s >= total_chunks) return;
           const int slot = s % K;
           pend[slot] = s;
-          const TileCoord tc = decode_tile<EPI>(p, pair + (s / kChunks) * npairs, rank);
-          const int col0 = tc.tn * BN + (s % kChunks) * kChunk;
-          if (chunk_kind<EPI>(p.grp[tc.g], tc.tm, col0) == kSkip) {
+          const TileCoord tc = decode_tile<EPI>(p, pair + (s / NCH) * npairs, rank);
+          const int col0 = tc.tn * BN + (s % NCH) * CW;
+          const int row0 = tc.tm * BM;
+          const Group& G = p.grp[tc.g];
+          const bool skip = (EPI == kBx) ? !(col0 < G.n && row0 < G.m)
+                                         : chunk_kind<EPI>(G, tc.tm, col0) == kSkip;
+          if (skip) {
             mbar_arrive(efull_bar(slot));
           } else {
             const uint32_t dst = slots_u32 + slot * C::kSlotBytes;
             mbar_arrive_expect_tx(efull_bar(slot), C::kSlotBytes);
-            tma_load_3d(dst, &p.map[tc.g].e, efull_bar(slot), col0, tc.tm * BM, tc.b);
+            tma_load_3d(dst, &p.map[tc.g].e, efull_bar(slot), col0, row0, tc.b);
             if (EPI == kBx)  // lo half of X next to its hi half
-              tma_load_3d(dst + kChunkBf16, &p.map[tc.g].mt, efull_bar(slot), col0, tc.tm * BM, tc.b);
+              tma_load_3d(dst + C::kSlotBytes / 2, &p.map[tc.g].mt, efull_bar(slot), col0, row0, tc.b);
           }
         };
         for (int s = 0; s < K; ++s) issue_eload(s);
@@ -449,20 +459,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int nup = 0;              // strictly-upper chunks so far (staging buffer = nup & 1)
         int held = -1;            // staging buffer whose stores may still be reading it
         for (int s = 0; s < total_chunks; ++s) {
-          const int k = s / kChunks, c = s % kChunks;
+          const int k = s / NCH, c = s % NCH;
           const TileCoord tc = decode_tile<EPI>(p, pair + k * npairs, rank);
           const Group& G = p.grp[tc.g];
           const Maps& M = p.map[tc.g];
           const int row0 = tc.tm * BM;
-          const int col0 = tc.tn * BN + c * kChunk;
+          const int col0 = tc.tn * BN + c * CW;
           const int kind = chunk_kind<EPI>(G, tc.tm, col0);
           if (EPI == kBx) {
             const int slot = s % K;
             mbar_wait(ready_bar(slot), (s / K) & 1, ctl);
-            if (kind != kSkip) {
+            if (kind != kSkip) {  // never start a store wholly outside the matrix
               const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
-              tma_store_3d(&M.d, hs, col0, row0, tc.b);                // hi' -> the other hi buffer
-              tma_store_3d(&M.mt, hs + kChunkBf16, col0, row0, tc.b);  // lo' -> lo, in place
+              tma_store_3d(&M.d, hs, col0, row0, tc.b);                       // hi' -> the other hi buffer
+              tma_store_3d(&M.mt, hs + C::kSlotBytes / 2, col0, row0, tc.b);  // lo' -> lo, in place
               bulk_commit();
               asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");  // chunk s-1 drained
             } else {
@@ -546,6 +556,71 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_wait(tfull_bar(acc), acc_phase, ctl);
         tc_fence_after();
         if (leader) TRACE(k, 4);
+        if (EPI == kBx) {
+          // 64-column chunks c: thread (r, hf) takes accumulator columns
+          // 32 hf .. +31 of the chunk, i.e. 16-byte units 4 hf .. 4 hf + 3 of
+          // its 128-byte row in the slot's hi and lo tiles (128-byte swizzle)
+          const int sr = r;
+          for (int c = 0; c < C::kNCh; ++c) {
+            if (leader && c > 0) TRACE(k, 4 + c);
+            const int s = k * C::kNCh + c;
+            const int col0 = tc.tn * BN + c * C::kCW;
+            const bool live = chunk_kind<EPI>(G, tc.tm, col0) != kSkip;
+            float v[32];
+            if (live) {
+              uint32_t rr[32];
+              __syncwarp();
+              tmem_ld_32x32(tmem_base + (static_cast<uint32_t>(lane_base) << 16) +
+                                static_cast<uint32_t>(acc * BN + c * C::kCW + hf * 32),
+                            rr);
+              tmem_ld_wait();
+#pragma unroll
+              for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(rr[q]);
+            }
+            if (c == C::kNCh - 1) {
+              // accumulator fully read: one arrival per warp hands it back (in
+              // the partner CTA through the relay thread of warp 1)
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(tempty_bar(acc));
+            }
+            const int slot = s % K;
+            mbar_wait(efull_bar(slot), (s / K) & 1, ctl);
+            // X = hi + lo from the slot; X' = a X + acc (times s on the first
+            // step); hi' = bf16(X'), lo' = bf16(X' - hi'), written back in
+            // place for the IO thread to store
+            if (live) {
+              const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
+              const uint32_t ls = hs + C::kSlotBytes / 2;
+#pragma unroll
+              for (int uu = 0; uu < 4; ++uu) {
+                const int u = 4 * hf + uu;
+                uint32_t h4[4], l4[4];
+                ld_shared_v4(hs + sw128(sr, u), h4[0], h4[1], h4[2], h4[3]);
+                ld_shared_v4(ls + sw128(sr, u), l4[0], l4[1], l4[2], l4[3]);
+                uint32_t ho[4], lo[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  float y[2];
+#pragma unroll
+                  for (int e = 0; e < 2; ++e) {
+                    const float xh = bf16_bits_to_f32(static_cast<uint16_t>(h4[h] >> (16 * e)));
+                    const float xl = bf16_bits_to_f32(static_cast<uint16_t>(l4[h] >> (16 * e)));
+                    y[e] = fmaf(p.a, xh + xl, v[8 * uu + 2 * h + e]) * xs;
+                  }
+                  ho[h] = pack_bf16x2(y[0], y[1]);
+                  const float r0 = y[0] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] & 0xFFFFu));
+                  const float r1 = y[1] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] >> 16));
+                  lo[h] = pack_bf16x2(r0, r1);
+                }
+                st_shared_v4(hs + sw128(sr, u), ho[0], ho[1], ho[2], ho[3]);
+                st_shared_v4(ls + sw128(sr, u), lo[0], lo[1], lo[2], lo[3]);
+              }
+              fence_async_smem();
+            }
+            mbar_arrive(ready_bar(slot));
+          }
+        } else {
         for (int c = 0; c < kChunks; ++c) {
           if (leader && c > 0) TRACE(k, 4 + c);
           const int s = k * kChunks + c;
@@ -570,43 +645,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(tempty_bar(acc));
           }
           const int slot = s % K;
-          if (EPI != kGram) mbar_wait(efull_bar(slot), (s / K) & 1, ctl);
-
-          if (EPI == kBx) {
-            // X = hi + lo from the slot; X' = a X + acc; hi' = bf16(X'),
-            // lo' = bf16(X' - hi'), written back in place for the IO thread to store
-            if (kind != kSkip) {
-              const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
-              const uint32_t ls = hs + kChunkBf16;
-#pragma unroll
-              for (int uu = 0; uu < 2; ++uu) {
-                const int u = 2 * hf + uu;  // 16-byte unit of the 64-byte row
-                uint32_t h4[4], l4[4];
-                ld_shared_v4(hs + sw64(r, u), h4[0], h4[1], h4[2], h4[3]);
-                ld_shared_v4(ls + sw64(r, u), l4[0], l4[1], l4[2], l4[3]);
-                uint32_t ho[4], lo[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                  float y[2];
-#pragma unroll
-                  for (int e = 0; e < 2; ++e) {
-                    const float xh = bf16_bits_to_f32(static_cast<uint16_t>(h4[h] >> (16 * e)));
-                    const float xl = bf16_bits_to_f32(static_cast<uint16_t>(l4[h] >> (16 * e)));
-                    y[e] = fmaf(p.a, xh + xl, v[8 * uu + 2 * h + e]) * xs;
-                  }
-                  ho[h] = pack_bf16x2(y[0], y[1]);
-                  const float r0 = y[0] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] & 0xFFFFu));
-                  const float r1 = y[1] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] >> 16));
-                  lo[h] = pack_bf16x2(r0, r1);
-                }
-                st_shared_v4(hs + sw64(r, u), ho[0], ho[1], ho[2], ho[3]);
-                st_shared_v4(ls + sw64(r, u), lo[0], lo[1], lo[2], lo[3]);
-              }
-              fence_async_smem();
-            }
-            mbar_arrive(ready_bar(slot));
-            continue;
-          }
+          if (EPI == kPoly) mbar_wait(efull_bar(slot), (s / K) & 1, ctl);
 
           // ------------------------------------------------ kGram / kPoly
           if (EPI == kGram && kind != kSkip) {
@@ -692,6 +731,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               mbar_arrive(ready_bar(2));
             }
           }
+        }
         }
         if (leader) TRACE(k, 12);
         if (++acc == 2) {

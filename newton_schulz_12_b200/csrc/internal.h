@@ -40,7 +40,7 @@ struct Group {
 
 // Tensor maps of one group (3-D: {inner, rows, batch}).
 // kBx uses e = hi chunk of X (read), mt = lo chunk of X (read and written in
-// place), d = hi chunk of X' (written); all bf16 32 x 128, 64-byte swizzle.
+// place), d = hi chunk of X' (written); all bf16 64 x 128, 128-byte swizzle.
 struct Maps {
   CUtensorMap p;   // rows of D: X (kGram), A (kPoly), B (kBx); K-major, box 64 x 128
   CUtensorMap q;   // columns of D: X / A K-major box 64 x 128; X MN-major box 64 x 64 (kBx)
