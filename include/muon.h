@@ -100,11 +100,12 @@ int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a,
  *             library never clears it).  With NULL the code goes to a slot of
  *             the static array, which each call clears first, and is not
  *             reported.
- * Limits: the workspace of the batch -- 6*batch*m*n + 4*batch*min(m,n)^2
- * bytes with the row strides rounded up to 8 elements, plus ~1 KiB -- must fit
- * in the 24 MiB; larger requests return MUON_ERR_SHAPE with the byte counts
- * and do nothing.  One 768 x 3072 matrix (about 15.8 MiB) fits; so do four
- * 768 x 768 matrices.
+ * Limits: the workspace of the batch -- 5*batch*m*n + 4*batch*min(m,n)^2
+ * bytes with the row strides of the m x n buffers rounded up to 16 elements
+ * and those of the square ones to 8, plus a few KiB -- must fit in the
+ * 24 MiB; larger requests return MUON_ERR_SHAPE with the byte counts and do
+ * nothing.  One 768 x 3072 matrix (about 13.5 MiB) fits; so do four 768 x 768
+ * matrices.
  * Sharing: every call on every stream of a device uses the same array and
  * leaves its last contents there.  No byte of it needs to start at zero (each
  * call writes everything it later reads).  Calls whose work overlaps on the
@@ -178,14 +179,21 @@ int muon_apply(int count, float* const* params, const float* const* updates,
  * tensor copies).
  *
  * muon_gram_bf16:  A = X X^T          X: batch x m x k bf16, A: batch x m x m bf16.
- *                  Only 128x256 tiles touching the upper triangle are computed;
- *                  A is exactly symmetric.
+ *                  Only the 256x256 tiles on or above the diagonal are
+ *                  computed; A is exactly symmetric.
  * muon_poly_bf16:  B = b*A + c*(A A)   A, B: batch x m x m bf16, A symmetric.
- * muon_bx_bf16:    X' = a*X + B X, with X carried as the bf16 pair hi + lo (the
- *                  representation the iteration keeps between steps, about 16
- *                  significant bits): B m x m bf16; Xhi: bf16(X), the operand;
- *                  Xlo: bf16(X - Xhi), read then overwritten by bf16(X' - bf16(X'));
- *                  Xhi_out: bf16(X') (must not alias Xhi).
+ * muon_bx_bf16:    X' = a*X + B X, with X carried as the pair the iteration
+ *                  keeps between steps (about 16 significant bits):
+ *                    X = hi + q * 2^(E - 15),  hi = bf16(X) (nearest even),
+ *                    E the exponent of hi (hi = 1.f * 2^E), q an int8 with
+ *                    q = round-to-nearest-even((X - hi) / 2^(E-15)) clamped
+ *                    to [-128, 127]; where hi is 0, subnormal or below
+ *                    2^-111, q is ignored (X = hi).  |X - value| <= 2^(E-16)
+ *                    (2^(E-15) when X lies exactly halfway above hi).
+ *                  B: m x m bf16; Xhi: hi of X (bf16), the operand; Xlo: q of
+ *                  X (int8, batch x m x n, n a multiple of 16), read then
+ *                  overwritten by q of X'; Xhi_out: hi of X' (must not alias
+ *                  Xhi).  m <= n.
  */
 int muon_gram_bf16(int batch, int m, int k, const void* X, void* A, void* stream);
 int muon_poly_bf16(int batch, int m, const void* A, void* B, float b, float c, void* stream);

@@ -219,13 +219,13 @@ def muon_poly_bf16(A, b=NS_COEFFS[1], c=NS_COEFFS[2], B=None, stream=None):
 
 
 def muon_bx_bf16(B, Xhi, Xlo, a=NS_COEFFS[0], Xhi_out=None, stream=None):
-    """X' = a X + B X with X = Xhi + Xlo (bf16 pair).
+    """X' = a X + B X with X = Xhi + Xlo * 2^(E(Xhi) - 15) (bf16 hi, int8 lo).
 
-    Xlo is overwritten by bf16(X' - bf16(X')); returns Xhi_out = bf16(X').
+    Xlo is overwritten by the int8 part of X'; returns Xhi_out = bf16(X').
     """
     _check_cuda(B, "B", torch.bfloat16)
     _check_cuda(Xhi, "Xhi", torch.bfloat16)
-    _check_cuda(Xlo, "Xlo", torch.bfloat16)
+    _check_cuda(Xlo, "Xlo", torch.int8)
     bsz, m, n = Xhi.shape
     if Xhi_out is None:
         Xhi_out = torch.empty_like(Xhi)

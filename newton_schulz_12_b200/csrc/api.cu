@@ -201,11 +201,13 @@ int get_workspace(cudaStream_t s, size_t need, Workspace** out) {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline long long round8(long long x) { return (x + 7) / 8 * 8; }
+inline long long round16(long long x) { return (x + 15) / 16 * 16; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 // 3-D tensor map {inner, rows, batch} over a contiguous batch with row stride
-// `ld` and matrix stride `mat_stride` (elements); `esize` 2 = bf16, 4 = fp32.
+// `ld` and matrix stride `mat_stride` (elements); `esize` 1 = int8, 2 = bf16,
+// 4 = fp32.
 int make_map(CUtensorMap* map, const void* base, int esize, uint64_t inner, uint64_t rows,
              uint64_t batch, uint64_t ld, uint64_t mat_stride, uint32_t box_inner, uint32_t box_rows,
              CUtensorMapSwizzle swz) {
@@ -213,8 +215,9 @@ int make_map(CUtensorMap* map, const void* base, int esize, uint64_t inner, uint
   cuuint64_t strides[2] = {ld * esize, mat_stride * esize};
   cuuint32_t box[3] = {box_inner, box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
-  const CUtensorMapDataType dt =
-      esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const CUtensorMapDataType dt = esize == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   CUresult r = g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box, es,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -242,16 +245,16 @@ int sym_maps(tc::Maps& M, const void* S, int m, int k, long long lds, long long 
   return MUON_OK;
 }
 
-// Maps of X' = a X + B X with X carried as the bf16 pair hi + lo: B (m x m),
-// hi of X (m x n: MN-major operand and epilogue chunks), lo of X (read and
-// written in place), hi of X' (written).
+// Maps of X' = a X + B X with X carried as the pair bf16 hi + int8 lo: B
+// (m x m), hi of X (m x n: MN-major operand and epilogue chunks), lo of X
+// (read and written in place), hi of X' (written).
 int bx_maps(tc::Maps& M, const void* B, long long ldb, long long sb, const void* Xhi,
             void* Xlo, void* Xhi_out, int m, int n, long long ldx, long long sx, int batch) {
   MUON_TRY(make_map(&M.p, B, 2, m, m, batch, ldb, sb, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
   MUON_TRY(make_map(&M.q, Xhi, 2, n, m, batch, ldx, sx, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
   // epilogue chunks of 64 columns: 128-byte rows
   MUON_TRY(make_map(&M.e, Xhi, 2, n, m, batch, ldx, sx, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
-  MUON_TRY(make_map(&M.mt, Xlo, 2, n, m, batch, ldx, sx, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
+  MUON_TRY(make_map(&M.mt, Xlo, 1, n, m, batch, ldx, sx, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
   MUON_TRY(make_map(&M.d, Xhi_out, 2, n, m, batch, ldx, sx, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
   M.s = M.d;  // unused
   return MUON_OK;
@@ -265,7 +268,7 @@ struct NsGroup {
   float* xf = nullptr;          // fp32 path: ping buffer of X
   float* xf1 = nullptr;         // fp32 path: pong buffer of X
   bf16* xb[2] = {nullptr, nullptr};  // bf16 path: hi of X (ping-pong; the GEMM operand)
-  bf16* xlo = nullptr;               // bf16 path: lo of X, X = hi + lo
+  int8_t* xlo = nullptr;             // bf16 path: lo of X, X = hi + q 2^(E(hi) - 15)
   bf16* A = nullptr;
   bf16* B = nullptr;
   float* Af = nullptr;
@@ -276,7 +279,7 @@ struct NsGroup {
 // Bytes of workspace a group needs; assigns its offsets from `base` (or counts
 // only, when base is null).
 size_t layout_group(NsGroup& g, char* base, size_t off, bool fp32) {
-  g.ldn = round8(g.n);
+  g.ldn = round16(g.n);  // 16-byte rows for the int8 lo as well
   g.ldm = round8(g.m);
   const size_t xe = static_cast<size_t>(g.batch) * g.m * g.ldn;
   const size_t ae = static_cast<size_t>(g.batch) * g.m * g.ldm;
@@ -289,7 +292,7 @@ size_t layout_group(NsGroup& g, char* base, size_t off, bool fp32) {
   if (!fp32) {
     g.xb[0] = reinterpret_cast<bf16*>(take(xe * 2));
     g.xb[1] = reinterpret_cast<bf16*>(take(xe * 2));
-    g.xlo = reinterpret_cast<bf16*>(take(xe * 2));
+    g.xlo = reinterpret_cast<int8_t*>(take(xe));
     g.A = reinterpret_cast<bf16*>(take(ae * 2));
     g.B = reinterpret_cast<bf16*>(take(ae * 2));
   } else {
@@ -413,7 +416,7 @@ int run_ns_bf16(std::vector<NsGroup>& gs, int steps, float a, float b, float c, 
 struct Result {
   const float* f = nullptr;
   const bf16* hi = nullptr;
-  const bf16* lo = nullptr;
+  const int8_t* lo = nullptr;
 };
 
 Result bf16_result(const NsGroup& g, int steps) {
@@ -559,7 +562,7 @@ int launch_cast_chunked(const std::vector<MatInfo>& mats, std::vector<NsGroup>& 
                         const std::vector<const void*>& src0, const std::vector<const float*>& src1,
                         int src_kind, float beta, int nesterov, const float* partials,
                         const std::vector<int>& part_begin, const std::vector<int>& part_count,
-                        bool with_bf16, cudaStream_t s) {
+                        cudaStream_t s) {
   const int count = static_cast<int>(mats.size());
   for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
     const int i1 = std::min(count, i0 + ew::kMaxMats);
@@ -585,9 +588,7 @@ int launch_cast_chunked(const std::vector<MatInfo>& mats, std::vector<NsGroup>& 
       C.part_begin = part_begin[i];
       C.part_count = part_count[i];
       const long long off = static_cast<long long>(M.index) * G.m * G.ldn;
-      C.xf = with_bf16 ? nullptr : G.xf + off;
-      C.xb = with_bf16 ? static_cast<void*>(G.xb[0] + off) : nullptr;
-      C.xlo = with_bf16 ? static_cast<void*>(G.xlo + off) : nullptr;
+      C.xf = G.xf + off;
       C.ld = G.ldn;
       C.vec = (M.cols % 8 == 0) && aligned16(src0[i]) && (src1.empty() || aligned16(src1[i]));
       tiles += ((M.m + ew::kTile - 1) / ew::kTile) * C.tiles_n;
@@ -909,7 +910,7 @@ int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a,
   for (NsGroup& g : groups) off = layout_group(g, base, off, true);
   std::vector<int> pb, pc;
   MUON_TRY(launch_flat_chunked(src, {}, numels, ew::kFromF32, 0.f, 0, partials, pb, pc, s));
-  MUON_TRY(launch_cast_chunked(mats, groups, src, {}, ew::kFromF32, 0.f, 0, partials, pb, pc, false, s));
+  MUON_TRY(launch_cast_chunked(mats, groups, src, {}, ew::kFromF32, 0.f, 0, partials, pb, pc, s));
   std::vector<float*> final_xf;
   MUON_TRY(run_ns_fp32(groups, steps, a, b, c, s, final_xf));
   for (float* f : final_xf) {
@@ -1160,6 +1161,8 @@ int muon_bx_bf16(int batch, int m, int n, const void* B, const void* Xhi, void* 
     return set_err(MUON_ERR_ARG, "B, Xhi, Xlo and Xhi_out must be non-NULL and 16-byte aligned");
   if (Xhi == Xhi_out) return set_err(MUON_ERR_ARG, "Xhi_out must not alias Xhi");
   if (m > n) return set_err(MUON_ERR_SHAPE, "muon_bx_bf16 expects m <= n (got %dx%d)", m, n);
+  if (n % 16)
+    return set_err(MUON_ERR_SHAPE, "muon_bx_bf16 needs n (%d) a multiple of 16 (16-byte rows of the int8 Xlo)", n);
   cudaStream_t s = as_stream(stream);
   DevInfo dev;
   Workspace* ws = nullptr;

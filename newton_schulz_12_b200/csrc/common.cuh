@@ -331,4 +331,66 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// ---------------------------------------------------------------------------
+// The pair X = hi + lo that carries X between Newton-Schulz steps: hi =
+// bf16(X) (round to nearest even), lo an int8 q with X ~ hi + q * 2^(E - 15),
+// E the exponent of hi.  |X - hi| <= 2^(E - 8), so (X - hi) / 2^(E-15) lies in
+// [-128, 128]; q is its nearest-even rounding clamped to [-128, 127], and
+// |X - (hi + q 2^(E-15))| <= 2^(E - 16) (2^(E - 15) in the one clamped case,
+// X exactly halfway above hi): about 16 significant bits.  Where hi is 0,
+// subnormal or below 2^-111, q is ignored (the value is hi).
+// ---------------------------------------------------------------------------
+// Branch-free: the exponent comes from hi's bits with masks, and E < -111 is
+// handled by integer max on those bits (the decoder's unit is then 0, so q
+// there carries nothing; the encoder writes 0 or any small value).
+//
+// fb: fp32 bits of a bf16 (the bf16 in the upper half).  2^(E - 15), or 0
+// when E < -111.
+__device__ __forceinline__ float lo8_unit(uint32_t fb) {
+  const int eb = static_cast<int>(fb & 0x7F800000u) - (15 << 23);
+  return __int_as_float(max(eb, 0));
+}
+
+// 2^(15 - E) with E clamped below at -111 (exact power of two).
+__device__ __forceinline__ float lo8_inv_unit(uint32_t fb) {
+  return __uint_as_float(0x86800000u - max(fb & 0x7F800000u, 16u << 23));
+}
+
+// fp32 bits of element k (0 = low half) of a bf16x2 word.
+__device__ __forceinline__ uint32_t bf16_word_bits(uint32_t w, int k) {
+  return k ? (w & 0xFFFF0000u) : (w << 16);
+}
+
+// Eight values -> eight bf16 (uint4) and eight int8 (uint2) of the pair.
+// d = x - hi is exact in fp32 and scaling by 2^(15 - E) is exact, so q is
+// the nearest-even rounding of d / 2^(E - 15), clamped to [-128, 127].
+__device__ __forceinline__ void pair_encode8(const float (&v)[8], uint4& hi, uint2& lo) {
+  uint32_t h[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) h[k] = pack_bf16x2(v[2 * k], v[2 * k + 1]);
+  uint32_t qb[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t fb = bf16_word_bits(h[k >> 1], k & 1);
+    const float t = (v[k] - __uint_as_float(fb)) * lo8_inv_unit(fb);
+    const int q = min(max(__float2int_rn(t), -128), 127);
+    qb[k] = static_cast<uint32_t>(q) & 0xFFu;
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint2(qb[0] | (qb[1] << 8) | (qb[2] << 16) | (qb[3] << 24),
+                  qb[4] | (qb[5] << 8) | (qb[6] << 16) | (qb[7] << 24));
+}
+
+// Eight values of the pair back to fp32: hi + q * 2^(E - 15).
+__device__ __forceinline__ void pair_decode8(const uint4 hi, const uint2 lo, float (&v)[8]) {
+  const uint32_t h[4] = {hi.x, hi.y, hi.z, hi.w};
+  const uint32_t l[2] = {lo.x, lo.y};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t fb = bf16_word_bits(h[k >> 1], k & 1);
+    const int q = static_cast<int>(l[k >> 2] << (24 - 8 * (k & 3))) >> 24;  // sign-extended byte
+    v[k] = fmaf(static_cast<float>(q), lo8_unit(fb), __uint_as_float(fb));
+  }
+}
+
 }  // namespace muon

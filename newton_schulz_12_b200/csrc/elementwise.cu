@@ -1,17 +1,22 @@
 // Memory-bound steps of the Muon update on sm_100a.
 //
-//   flat_kernel   momentum lerp + Nesterov blend (buf written in place) and a
-//                 per-block partial of sum(u^2); or, for the plain
-//                 orthogonalisation entry, the partial of sum(x^2) only.
-//                 128-bit loads/stores, fixed-order block reduction.
-//   cast_kernel   X0 = u / (||u||_F + eps), transposed to rows <= cols when the
-//                 matrix is tall, written as the bf16 pair hi = bf16(X),
-//                 lo = bf16(X - hi) (fp32 for the verification path).  64x64 tiles staged through shared memory so
+//   prep_kernel   the bf16 path's first pass: momentum lerp + Nesterov blend
+//                 (buf written in place), u written to the iteration layout
+//                 (transposed to rows <= cols when the matrix is tall) as the
+//                 pair bf16 hi + int8 lo, and an fp64 partial of sum(u^2) per
+//                 block.  The 1 / ||u|| factor is applied later, inside the
+//                 first Newton-Schulz step.
+//   scale_kernel  per-matrix s = 1 / (||u||_F + eps) from those partials.
+//   flat_kernel   momentum on its own (muon_momentum) or the partial of
+//                 sum(x^2) of the fp32 verification path; 128-bit accesses,
+//                 fixed-order block reduction.
+//   cast_kernel   fp32 verification path: X0 = x / (||x||_F + eps) in fp32,
+//                 transposed when tall; 64x64 tiles through shared memory so
 //                 both the read and the (possibly transposed) write coalesce.
 //   out_kernel    W' = (W - lw W) - ls O (the apply), or the write-back of the
 //                 result into the caller's bf16 / fp32 buffer, with O read
-//                 through the same transposing tile.
-//   sums_kernel   per-matrix sum of the partials (same order as cast_kernel).
+//                 (from fp32 or from the pair) through the same transposing tile.
+//   sums_kernel   per-matrix sum of flat_kernel's partials.
 //
 // Operation order of momentum and apply is fixed with explicit round-to-nearest
 // intrinsics (no contraction into FMA) so that they are bit-exact against an
@@ -223,8 +228,7 @@ __device__ __forceinline__ void load_u8(const CastParams& p, const CastMat& M, i
   }
 }
 
-// X[i][j + k] = u[k] / den, written as fp32 (verification path) or as the
-// bf16 pair hi = bf16(x), lo = bf16(x - hi) that carries X between steps.
+// X[i][j + k] = u[k] / den in fp32 (the verification path).
 __device__ __forceinline__ void store_x8(const CastMat& M, int i, int j, int m, int n, float den,
                                          const float (&u)[8]) {
   if (i >= m || j >= n) return;
@@ -232,35 +236,14 @@ __device__ __forceinline__ void store_x8(const CastMat& M, int i, int j, int m, 
   float x[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) x[k] = __fdiv_rn(u[k], den);
-  uint32_t hi[4], lo[4];
-  if (!M.xf) {
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      hi[h] = pack_bf16x2(x[2 * h], x[2 * h + 1]);
-      lo[h] = pack_bf16x2(x[2 * h] - bf16_bits_to_f32(static_cast<uint16_t>(hi[h] & 0xFFFFu)),
-                          x[2 * h + 1] - bf16_bits_to_f32(static_cast<uint16_t>(hi[h] >> 16)));
-    }
-  }
   if (j + 8 <= n) {  // the workspace row stride is a multiple of 8: always aligned
-    if (M.xf) {
-      float4* f4 = reinterpret_cast<float4*>(M.xf + o);
-      f4[0] = make_float4(x[0], x[1], x[2], x[3]);
-      f4[1] = make_float4(x[4], x[5], x[6], x[7]);
-    } else {
-      *reinterpret_cast<uint4*>(static_cast<bf16*>(M.xb) + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(static_cast<bf16*>(M.xlo) + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    }
+    float4* f4 = reinterpret_cast<float4*>(M.xf + o);
+    f4[0] = make_float4(x[0], x[1], x[2], x[3]);
+    f4[1] = make_float4(x[4], x[5], x[6], x[7]);
   } else {
-    for (int k = 0; k < n - j; ++k) {
-      if (M.xf) {
-        M.xf[o + k] = x[k];
-      } else {
-        const uint32_t w = (k & 1) ? (hi[k >> 1] >> 16) : (hi[k >> 1] & 0xFFFFu);
-        const uint32_t l = (k & 1) ? (lo[k >> 1] >> 16) : (lo[k >> 1] & 0xFFFFu);
-        static_cast<uint16_t*>(M.xb)[o + k] = static_cast<uint16_t>(w);
-        static_cast<uint16_t*>(M.xlo)[o + k] = static_cast<uint16_t>(l);
-      }
-    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k < n - j) M.xf[o + k] = x[k];
   }
 }
 
@@ -317,18 +300,22 @@ __device__ __forceinline__ void load_o8(const OutMat& M, int r, int c, int orows
   if (M.o_hi) {
     const float f = M.oscale ? *M.oscale : 1.0f;
     if (cnt == 8 && M.vec) {
-      float h[8], l[8];
-      unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const bf16*>(M.o_hi) + idx), h);
-      unpack_bf16x8(*reinterpret_cast<const uint4*>(static_cast<const bf16*>(M.o_lo) + idx), l);
+      pair_decode8(*reinterpret_cast<const uint4*>(static_cast<const bf16*>(M.o_hi) + idx),
+                   *reinterpret_cast<const uint2*>(static_cast<const int8_t*>(M.o_lo) + idx), o);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) o[k] = (h[k] + l[k]) * f;
+      for (int k = 0; k < 8; ++k) o[k] *= f;
       return;
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-      o[k] = k < cnt ? (bf16_bits_to_f32(static_cast<const uint16_t*>(M.o_hi)[idx + k]) +
-                        bf16_bits_to_f32(static_cast<const uint16_t*>(M.o_lo)[idx + k])) * f
-                     : 0.f;
+    for (int k = 0; k < 8; ++k) {
+      float v = 0.f;
+      if (k < cnt) {
+        const uint32_t fb = static_cast<uint32_t>(static_cast<const uint16_t*>(M.o_hi)[idx + k]) << 16;
+        const int q = static_cast<const int8_t*>(M.o_lo)[idx + k];
+        v = fmaf(static_cast<float>(q), lo8_unit(fb), __uint_as_float(fb)) * f;
+      }
+      o[k] = v;
+    }
     return;
   }
   if (cnt == 8 && M.vec) {
@@ -432,27 +419,24 @@ constexpr int kPrepThreads = 256;
 #endif
 constexpr int kPrepUnits = kPrepRows * kPrepCols / (kPrepThreads * 8);  // 4 runs of 8 per thread
 
+// Eight values of u as the pair: bf16 hi (16 bytes) and int8 lo (8 bytes).
 __device__ __forceinline__ void store_pair8(void* hi_base, void* lo_base, long long off, int cnt,
                                             const float (&v)[8]) {
-  uint32_t hi[4], lo[4];
-#pragma unroll
-  for (int h = 0; h < 4; ++h) {
-    hi[h] = pack_bf16x2(v[2 * h], v[2 * h + 1]);
-    lo[h] = pack_bf16x2(v[2 * h] - bf16_bits_to_f32(static_cast<uint16_t>(hi[h] & 0xFFFFu)),
-                        v[2 * h + 1] - bf16_bits_to_f32(static_cast<uint16_t>(hi[h] >> 16)));
-  }
-  if (cnt == 8) {  // the workspace row stride is a multiple of 8: aligned
-    *reinterpret_cast<uint4*>(static_cast<bf16*>(hi_base) + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4*>(static_cast<bf16*>(lo_base) + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  uint4 hi;
+  uint2 lo;
+  pair_encode8(v, hi, lo);
+  if (cnt == 8) {  // the workspace row stride is a multiple of 16: aligned
+    *reinterpret_cast<uint4*>(static_cast<bf16*>(hi_base) + off) = hi;
+    *reinterpret_cast<uint2*>(static_cast<int8_t*>(lo_base) + off) = lo;
     return;
   }
+  const uint32_t h[4] = {hi.x, hi.y, hi.z, hi.w};
+  const uint32_t l[2] = {lo.x, lo.y};
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     if (k < cnt) {
-      const uint32_t w = (k & 1) ? (hi[k >> 1] >> 16) : (hi[k >> 1] & 0xFFFFu);
-      const uint32_t l = (k & 1) ? (lo[k >> 1] >> 16) : (lo[k >> 1] & 0xFFFFu);
-      static_cast<uint16_t*>(hi_base)[off + k] = static_cast<uint16_t>(w);
-      static_cast<uint16_t*>(lo_base)[off + k] = static_cast<uint16_t>(l);
+      static_cast<uint16_t*>(hi_base)[off + k] = static_cast<uint16_t>(h[k >> 1] >> (16 * (k & 1)));
+      static_cast<uint8_t*>(lo_base)[off + k] = static_cast<uint8_t>(l[k >> 2] >> (8 * (k & 3)));
     }
   }
 }
@@ -623,21 +607,16 @@ __global__ void __launch_bounds__(kScaleThreads) scale_kernel(const __grid_const
   __syncthreads();
   const float f1 = s_f[0], f2 = s_f[1];
   if (f1 == 1.0f && f2 == 1.0f) return;
+  // lo counts in units of hi's exponent, so only hi changes
   const long long units = static_cast<long long>(M.m) * M.ld / 8;
   for (long long i = threadIdx.x; i < units; i += kScaleThreads) {
     uint4* ph = reinterpret_cast<uint4*>(static_cast<bf16*>(M.xhi)) + i;
-    uint4* pl = reinterpret_cast<uint4*>(static_cast<bf16*>(M.xlo)) + i;
-    float h[8], l[8];
+    float h[8];
     unpack_bf16x8(*ph, h);
-    unpack_bf16x8(*pl, l);
-    uint32_t oh[4], ol[4];
+    uint32_t oh[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      oh[k] = pack_bf16x2((h[2 * k] * f1) * f2, (h[2 * k + 1] * f1) * f2);
-      ol[k] = pack_bf16x2((l[2 * k] * f1) * f2, (l[2 * k + 1] * f1) * f2);
-    }
+    for (int k = 0; k < 4; ++k) oh[k] = pack_bf16x2((h[2 * k] * f1) * f2, (h[2 * k + 1] * f1) * f2);
     *ph = make_uint4(oh[0], oh[1], oh[2], oh[3]);
-    *pl = make_uint4(ol[0], ol[1], ol[2], ol[3]);
   }
 }
 

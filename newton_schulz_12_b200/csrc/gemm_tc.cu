@@ -67,7 +67,7 @@ constexpr size_t kMaxSmem = 232448;                         // 227 KiB per CTA o
 #define MUON_BX_STAGES 4
 #endif
 #ifndef MUON_BX_SLOTS
-#define MUON_BX_SLOTS 3
+#define MUON_BX_SLOTS 4
 #endif
 
 template <int EPI>
@@ -83,7 +83,9 @@ struct Cfg {
   // symmetric kernels on 32-column chunks (their mirrored stores are 32 rows)
   static constexpr int kCW = (EPI == kBx) ? 2 * kChunk : kChunk;
   static constexpr int kNCh = BN / kCW;  // per tile
-  static constexpr uint32_t kSlotBytes = (EPI == kBx) ? 4 * kChunkBf16 : (EPI == kPoly ? kChunkBf16 : 0);
+  // kBx slot: hi (bf16, 128 rows x 128 B) then lo (int8, 128 rows x 64 B)
+  static constexpr uint32_t kSlotBytes = (EPI == kBx) ? 3 * kChunkBf16 : (EPI == kPoly ? kChunkBf16 : 0);
+  static constexpr uint32_t kLoOff = 2 * kChunkBf16;
   static constexpr uint32_t kSlotsBytes = kSlotBytes * kSlots;
   // staging: kBx two bf16 output chunks; kGram / kPoly 2 direct + 2 mirror chunks,
   // aliased by the 128 x 128 diagonal block (2 x [128 rows][64 cols] bf16)
@@ -451,7 +453,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(efull_bar(slot), C::kSlotBytes);
             tma_load_3d(dst, &p.map[tc.g].e, efull_bar(slot), col0, row0, tc.b);
             if (EPI == kBx)  // lo half of X next to its hi half
-              tma_load_3d(dst + C::kSlotBytes / 2, &p.map[tc.g].mt, efull_bar(slot), col0, row0, tc.b);
+              tma_load_3d(dst + C::kLoOff, &p.map[tc.g].mt, efull_bar(slot), col0, row0, tc.b);
           }
         };
         for (int s = 0; s < K; ++s) issue_eload(s);
@@ -472,7 +474,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (kind != kSkip) {  // never start a store wholly outside the matrix
               const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
               tma_store_3d(&M.d, hs, col0, row0, tc.b);                       // hi' -> the other hi buffer
-              tma_store_3d(&M.mt, hs + C::kSlotBytes / 2, col0, row0, tc.b);  // lo' -> lo, in place
+              tma_store_3d(&M.mt, hs + C::kLoOff, col0, row0, tc.b);          // lo' -> lo, in place
               bulk_commit();
               asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");  // chunk s-1 drained
             } else {
@@ -587,34 +589,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int slot = s % K;
             mbar_wait(efull_bar(slot), (s / K) & 1, ctl);
             // X = hi + lo from the slot; X' = a X + acc (times s on the first
-            // step); hi' = bf16(X'), lo' = bf16(X' - hi'), written back in
-            // place for the IO thread to store
+            // step) written back in place as the pair (hi', lo') for the IO
+            // thread to store.  Columns 32 hf + 8 uu .. +7: 16-byte unit
+            // 4 hf + uu of the hi row (128-byte swizzle), bytes 8 (uu & 1)..
+            // of unit 2 hf + uu / 2 of the lo row (64-byte swizzle).
             if (live) {
               const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
-              const uint32_t ls = hs + C::kSlotBytes / 2;
+              const uint32_t ls = hs + C::kLoOff;
 #pragma unroll
               for (int uu = 0; uu < 4; ++uu) {
-                const int u = 4 * hf + uu;
-                uint32_t h4[4], l4[4];
-                ld_shared_v4(hs + sw128(sr, u), h4[0], h4[1], h4[2], h4[3]);
-                ld_shared_v4(ls + sw128(sr, u), l4[0], l4[1], l4[2], l4[3]);
-                uint32_t ho[4], lo[4];
+                const uint32_t ha = hs + sw128(sr, 4 * hf + uu);
+                const uint32_t la = ls + sw64(sr, 2 * hf + (uu >> 1)) + 8 * (uu & 1);
+                uint4 h4;
+                uint2 l2;
+                ld_shared_v4(ha, h4.x, h4.y, h4.z, h4.w);
+                asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(l2.x), "=r"(l2.y) : "r"(la) : "memory");
+                float x[8];
+                pair_decode8(h4, l2, x);
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                  float y[2];
-#pragma unroll
-                  for (int e = 0; e < 2; ++e) {
-                    const float xh = bf16_bits_to_f32(static_cast<uint16_t>(h4[h] >> (16 * e)));
-                    const float xl = bf16_bits_to_f32(static_cast<uint16_t>(l4[h] >> (16 * e)));
-                    y[e] = fmaf(p.a, xh + xl, v[8 * uu + 2 * h + e]) * xs;
-                  }
-                  ho[h] = pack_bf16x2(y[0], y[1]);
-                  const float r0 = y[0] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] & 0xFFFFu));
-                  const float r1 = y[1] - bf16_bits_to_f32(static_cast<uint16_t>(ho[h] >> 16));
-                  lo[h] = pack_bf16x2(r0, r1);
-                }
-                st_shared_v4(hs + sw128(sr, u), ho[0], ho[1], ho[2], ho[3]);
-                st_shared_v4(ls + sw128(sr, u), lo[0], lo[1], lo[2], lo[3]);
+                for (int e = 0; e < 8; ++e) x[e] = fmaf(p.a, x[e], v[8 * uu + e]) * xs;
+                pair_encode8(x, h4, l2);
+                st_shared_v4(ha, h4.x, h4.y, h4.z, h4.w);
+                asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(la), "r"(l2.x), "r"(l2.y) : "memory");
               }
               fence_async_smem();
             }

@@ -39,8 +39,9 @@ struct Group {
 };
 
 // Tensor maps of one group (3-D: {inner, rows, batch}).
-// kBx uses e = hi chunk of X (read), mt = lo chunk of X (read and written in
-// place), d = hi chunk of X' (written); all bf16 64 x 128, 128-byte swizzle.
+// kBx uses e = hi chunk of X (read), mt = lo chunk of X (int8, read and
+// written in place), d = hi chunk of X' (written); 64 x 128 boxes, hi with
+// 128-byte swizzle, lo with 64-byte swizzle.
 struct Maps {
   CUtensorMap p;   // rows of D: X (kGram), A (kPoly), B (kBx); K-major, box 64 x 128
   CUtensorMap q;   // columns of D: X / A K-major box 64 x 128; X MN-major box 64 x 64 (kBx)
@@ -140,9 +141,7 @@ struct CastMat {
   int tiles_n;        // 64-wide tiles along X's columns
   int tile_begin;
   int part_begin, part_count;
-  float* xf;          // fp32 X (m x n, row stride ld), fp32 path; else null
-  void* xb;           // bf16 path: hi = bf16(X)
-  void* xlo;          // bf16 path: lo = bf16(X - hi)
+  float* xf;          // fp32 X (m x n, row stride ld)
   long long ld;
   int vec;            // source rows are 16-byte aligned (cols % 8 == 0): 128-bit loads
 };
@@ -162,7 +161,7 @@ struct CastParams {
 struct OutMat {
   void* y;            // W (fp32, in/out) or destination X (bf16 / f32)
   const float* o;     // fp32 update / result (X layout, or W layout if !o_transposed); or null
-  const void* o_hi;   // else the result as a bf16 pair: O = hi + lo (X layout)
+  const void* o_hi;   // else the result as the pair bf16 hi + int8 lo (X layout)
   const void* o_lo;
   int rows, cols;     // caller layout of y
   int o_transposed;   // O[r][s] = o[s * ld + r]
@@ -194,7 +193,7 @@ struct PrepMat {
   int transposed;     // rows > cols: X = U^T
   int tiles_c;        // tiles along the caller's columns
   int tile_begin;
-  void* xhi;          // workspace X (m x n, row stride ld): hi and lo of u
+  void* xhi;          // workspace X (m x n, row stride ld): hi (bf16) and lo (int8) of u
   void* xlo;
   long long ld;
   int vec;            // cols % 8 == 0: 128-bit accesses of the caller's rows

@@ -8,7 +8,7 @@ entry point `reps` times and synchronises, so a profiler can skip the first
 exceed the 126 MB L2, so DRAM counters are meaningful, while staying far
 below the device's memory:
 
-  bx    X' = aX + BX over 24 matrices 768x3072 (B 768x768)      ~370 MB
+  bx    X' = aX + BX over 24 matrices 768x3072 (B 768x768)      ~310 MB
   gram  A = X X^T over 24 matrices 768x3072                      ~140 MB
   poly  B = bA + cA^2 over 72 matrices 768x768                   ~170 MB
   step  one full muon_step over the 72-matrix GPT-2-small set    ~1.7 GB
@@ -34,7 +34,7 @@ def main():
         B = (torch.randn(24, 768, 768, generator=g) / 768 ** 0.5).to(torch.bfloat16).to(dev)
         X = (torch.randn(24, 768, 3072, generator=g) / 3072 ** 0.5).to(dev)
         hi = X.to(torch.bfloat16)
-        lo = (X - hi.float()).to(torch.bfloat16)
+        lo = torch.zeros(X.shape, dtype=torch.int8, device=dev)  # the int8 part of the pair
         out = torch.empty_like(hi)
         for _ in range(args.reps):
             nsb.muon_bx_bf16(B, hi, lo, Xhi_out=out)

@@ -97,6 +97,9 @@ def test_stage_argument_errors(lib):
     assert lib.muon_gram_bf16(1, 8, 8, None, None, null) == -1
     assert lib.muon_poly_bf16(1, 8, 0x1000, 0x1000, 1.0, 1.0, null) == -1  # aliasing
     assert lib.muon_bx_bf16(1, 8, 8, 0x1000, 0x2000, 0x3000, 0x2000, 1.0, null) == -1
+    # the int8 low part needs 16-byte rows: n a multiple of 16
+    assert lib.muon_bx_bf16(1, 8, 24, 0x1000, 0x2000, 0x3000, 0x4000, 1.0, null) == -2
+    assert "multiple of 16" in _err(lib)
     assert lib.muon_gram_bf16(0, 8, 8, None, None, null) == 0
 
 

@@ -59,29 +59,65 @@ def test_poly(batch, m):
     assert torch.equal(B, B.transpose(1, 2)), "B must be exactly symmetric"
 
 
-@pytest.mark.parametrize("batch,m,n", [(1, 128, 128), (2, 200, 328), (1, 768, 3072), (3, 8, 72),
-                                       (2, 384, 384), (1, 136, 520), (1, 1024, 4096),
-                                       (80, 256, 520), (6, 768, 3072)])
+def pair_unit(hi):
+    """2^(E - 15) for hi = 1.f * 2^E (0 where the low part is unused: hi = 0,
+    subnormal or below 2^-111), in fp64."""
+    h = hi.double()
+    _, e = torch.frexp(hi.float())
+    E = (e - 1).double()
+    ok = (h != 0) & (E >= -111)
+    return torch.where(ok, torch.exp2(E - 15), torch.zeros_like(h))
+
+
+def pair_split(X):
+    """The pair format of the iteration: hi = bf16(X), q = nearest-even of
+    (X - hi) / 2^(E-15), clamped to [-128, 127] (X fp32, so X - hi is exact)."""
+    hi = X.to(torch.bfloat16)
+    unit = pair_unit(hi)
+    d = X.double() - hi.double()
+    q = torch.where(unit > 0, torch.round(d / torch.where(unit > 0, unit, torch.ones_like(unit))),
+                    torch.zeros_like(d)).clamp(-128, 127)
+    return hi, q.to(torch.int8)
+
+
+def pair_value(hi, q):
+    return hi.double() + q.double() * pair_unit(hi)
+
+
+def test_pair_format_resolution():
+    """The pair holds fp32 values to 2^-16 of |hi|, 2^-15 in the clamped tie
+    (CPU check of the test's own encoder)."""
+    X = torch.randn(4096, generator=torch.Generator().manual_seed(0)) * torch.exp2(
+        torch.randint(-60, 60, (4096,), generator=torch.Generator().manual_seed(1)).float())
+    hi, q = pair_split(X)
+    err = (pair_value(hi, q) - X.double()).abs()
+    assert torch.all(err <= 2.0 ** -15 * hi.double().abs())
+
+
+# n a multiple of 16 (16-byte rows of the int8 part); 336, 528, 80 leave a ragged 64-column chunk
+@pytest.mark.parametrize("batch,m,n", [(1, 128, 128), (2, 200, 336), (1, 768, 3072), (3, 8, 80),
+                                       (2, 384, 384), (1, 136, 528), (1, 1024, 4096),
+                                       (80, 256, 528), (6, 768, 3072)])
 def test_bx(batch, m, n):
-    """X' = aX + BX with X = hi + lo; the pair must hold X' to about 2^-17."""
+    """X' = aX + BX with X carried as the pair (bf16 hi, int8 lo): the output
+    pair must hold X' to about 2^-16 and hi' must be bf16(X')."""
     B = rnd_bf16((batch, m, m), seed=m, scale=m ** -0.5)
     X = torch.randn(batch, m, n, generator=torch.Generator().manual_seed(n)) / n ** 0.5
-    hi = X.to(torch.bfloat16)
-    lo = (X - hi.float()).to(torch.bfloat16)
-    Xd = hi.double() + lo.double()          # the X the kernel sees
+    hi, lo = pair_split(X)
+    Xd = pair_value(hi, lo)                  # the X the kernel sees
     a = 3.4445
     a32 = float(torch.tensor(a, dtype=torch.float32))
     lo_dev = lo.cuda()
     hi_out = nsb.muon_bx_bf16(B.cuda(), hi.cuda(), lo_dev, a).cpu()
     lo_out = lo_dev.cpu()
     assert nsb.muon_get_status() == 0
-    got = hi_out.double() + lo_out.double()
+    got = pair_value(hi_out, lo_out)
     ref = a32 * Xd + B.double() @ hi.double()
     absref = abs(a32) * Xd.abs() + B.double().abs() @ hi.double().abs()
-    check_close(got, ref, absref, rel=2.0 ** -16, acc=2.0 ** -16)
-    # hi' is the round-to-nearest bf16 of X', lo' the rounded remainder
-    xh = hi_out.float()
-    assert torch.all((got - xh.double()).abs() <= 2.0 ** -8 * xh.double().abs() + 1e-30)
+    check_close(got, ref, absref, rel=2.0 ** -15, acc=2.0 ** -16)
+    # hi' is the round-to-nearest bf16 of X'
+    xh = hi_out.double()
+    assert torch.all((got - xh).abs() <= 2.0 ** -8 * xh.abs() + 1e-30)
 
 
 def test_stage_kernels_are_deterministic():

@@ -59,9 +59,9 @@ def test_static_matches_allocating_call_twice(rows, cols, batch):
 
 
 def test_static_rejects_oversized_batch():
-    x = [torch.zeros(1024, 4096, dtype=torch.bfloat16, device="cuda")]
+    x = [torch.zeros(1024, 8192, dtype=torch.bfloat16, device="cuda")]
     arr = _lib.ptr_array([x[0].data_ptr()])
-    rc = _lib.lib().muon_ns_orthogonalize_static(1, 1024, 4096, arr, 3.4445, -4.7750, 2.0315, 5,
+    rc = _lib.lib().muon_ns_orthogonalize_static(1, 1024, 8192, arr, 3.4445, -4.7750, 2.0315, 5,
                                                  None, ctypes.c_void_p(0))
     assert rc == -2
     assert "static scratch" in nsb.muon_last_error()
