@@ -7,6 +7,7 @@ small (12 layers x [4 x 768x768, 768x3072, 3072x768]); bf16 gradients drawn
 iid N(0, 0.01^2), fp32 momentum (beta 0.95, Nesterov), lr 0.05, wd 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --ns-cases      # NS-only: batched 768x3072 and the width sweep
 
 Prints one JSON line (rank 0).  `value` is matrices/s over all ranks with
 inputs resident in HBM; `e2e` repeats the measurement with the gradients
@@ -51,6 +52,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ns-cases", action="store_true",
+                    help="instead of the step benchmark: muon_ns_orthogonalize (bf16) on the "
+                         "batched 768x3072 case and the square width sweep, one JSON line each")
     return ap.parse_args()
 
 
@@ -409,11 +413,67 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------- NS-only case sweep
+NS_CASES = [  # (label, m, n, batch): the batched 768x3072 case, then m in {256..4096} with
+              # batch 64 (768/m)^2 rounded, at least 1
+    ("768x3072 x64", 768, 3072, 64),
+    ("256^2 x576", 256, 256, 576), ("512^2 x144", 512, 512, 144), ("768^2 x64", 768, 768, 64),
+    ("1024^2 x36", 1024, 1024, 36), ("2048^2 x9", 2048, 2048, 9), ("4096^2 x2", 4096, 4096, 2),
+]
+
+
+def run_ns_cases(args):
+    """Per case: the whole muon_ns_orthogonalize call and its three GEMM kernels
+    (device time from the library's timing hooks) against the bf16 peak."""
+    import torch
+    import newton_schulz_12_b200 as nsb
+    peaks, peak_src = load_peaks()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    for label, m, n, batch in NS_CASES:
+        g = torch.Generator(device="cpu").manual_seed(3000 + m)
+        xs = [torch.randn(m, n, generator=g).to(torch.bfloat16).to(dev) for _ in range(batch)]
+        flops = nominal_flops([(m, n)] * batch)
+        for _ in range(args.warmup):
+            nsb.muon_ns_orthogonalize(xs)
+        torch.cuda.synchronize()
+        reps = max(3, min(args.steps, 50))
+        nsb.muon_profile_begin()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(reps):
+            nsb.muon_ns_orthogonalize(xs)
+        t1.record()
+        torch.cuda.synchronize()
+        prof = nsb.muon_profile_end()
+        if nsb.muon_get_status() != 0:
+            raise SystemExit(f"device status error in case {label}")
+        call_ms = t0.elapsed_time(t1) / reps
+        gemm_ms = sum(prof[k][0] for k in ("gram", "poly", "bx")) / reps
+        x_bytes = batch * m * n * 2
+        print(json.dumps({
+            "case": label, "m": m, "n": n, "batch": batch, "reps": reps,
+            "nominal_gflop": flops / 1e9,
+            "call_ms": call_ms, "tflops_call": flops / call_ms / 1e9,
+            "gemm_ms": gemm_ms, "tflops_gemm": flops / gemm_ms / 1e9,
+            "gemm_frac_of_peak": flops / gemm_ms / 1e9 / peaks["bf16_tflops"],
+            "peak": peaks["bf16_tflops"], "peak_source": f"{peak_src} (bf16 burst)",
+            "per_kernel_us": {k: v[0] / v[1] * 1e3 for k, v in prof.items() if v[1]},
+            "l2": "X %.0f MB (%s the 126 MB L2), workspace larger; no flush" % (
+                x_bytes / 1e6, "above" if x_bytes > 126e6 else "below"),
+        }), flush=True)
+        del xs
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.ns_cases:
+        run_ns_cases(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -314,6 +314,7 @@ tc::Group tc_group(int batch, int m, int n, int k, bool sym, int tile_begin) {
   G.tiles_n = sym ? (m + tc::BN - 1) / tc::BN : (n + tc::BN - 1) / tc::BN;
   G.tiles_per_mat = sym ? tc::sym_tiles(m) : G.tiles_m * G.tiles_n;
   G.tile_begin = tile_begin;
+  G.mat_base = 0;
   return G;
 }
 

@@ -582,19 +582,24 @@ constexpr int kScaleThreads = 256;
 
 __global__ void __launch_bounds__(kScaleThreads) scale_kernel(const __grid_constant__ ScaleParams p) {
   __shared__ float s_f[2];
+  __shared__ double s_red[kScaleThreads / 32];
   const ScaleMat& M = p.mat[blockIdx.x];
-  if (threadIdx.x < 32) {
-    // lane l adds partials l, l+32, ... then a fixed xor tree
-    const int lane = threadIdx.x;
+  {
+    // thread t adds partials t, t+256, ...; then a fixed xor tree per warp
+    // and the eight warp sums in order: a fixed summation order
     double ss = 0.0;
-    for (int q = lane; q < M.part_count; q += 32) ss += p.partials[M.part_begin + q];
+    for (int q = threadIdx.x; q < M.part_count; q += kScaleThreads) ss += p.partials[M.part_begin + q];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) {
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      ss = 0.0;
+      for (int w = 0; w < kScaleThreads / 32; ++w) ss += s_red[w];
       double den = sqrt(ss) + p.eps;
       float f1 = 1.0f, f2 = 1.0f;
       if (isfinite(den) && (den > 0x1p40 || den < 0x1p-40)) {
-        const int e = ilogb(den);  // |e| <= 1100: each factor stays a normal fp32
+        const int e = ilogb(den);  // e <= 150 for any fp32 / bf16 u: both factors are normal fp32
         f1 = ldexpf(1.0f, -(e / 2));
         f2 = ldexpf(1.0f, -(e - e / 2));
         den = (den * f1) * f2;

@@ -63,6 +63,12 @@ constexpr size_t kMaxSmem = 232448;                         // 227 KiB per CTA o
 #ifndef MUON_POLY_SLOTS
 #define MUON_POLY_SLOTS 4
 #endif
+#ifndef MUON_GRAM_SBUF
+#define MUON_GRAM_SBUF 2
+#endif
+#ifndef MUON_POLY_SBUF
+#define MUON_POLY_SBUF 2
+#endif
 #ifndef MUON_BX_STAGES
 #define MUON_BX_STAGES 4
 #endif
@@ -77,7 +83,6 @@ struct Cfg {
   // epilogue operand ring of kSlots chunks (kGram: none, the count only sizes barriers)
   // kBx slot: the hi and lo bf16 chunks of X (8 KiB each); kPoly slot: A's chunk
   static constexpr int kSlots = (EPI == kBx) ? MUON_BX_SLOTS : MUON_POLY_SLOTS;
-  static_assert(kSlots >= 3, "ready barriers 0-2 double as staging barriers");
   static_assert(BN % (2 * kChunk) == 0, "whole chunks per tile");
   // kBx works on 64-column chunks (128-byte rows in global memory), the
   // symmetric kernels on 32-column chunks (their mirrored stores are 32 rows)
@@ -89,10 +94,18 @@ struct Cfg {
   static constexpr uint32_t kSlotsBytes = kSlotBytes * kSlots;
   // staging: kBx two bf16 output chunks; kGram / kPoly 2 direct + 2 mirror chunks,
   // aliased by the 128 x 128 diagonal block (2 x [128 rows][64 cols] bf16)
-  static constexpr uint32_t kStagingBytes = (EPI == kBx) ? 0 : 4 * kChunkBf16;
+  // kGram / kPoly output staging: kSBuf pairs of a direct [128][32] and a
+  // mirrored [32][128] chunk, laid out as d0 .. d(kSBuf-1), m0 .. m(kSBuf-1);
+  // a diagonal 128 x 128 block aliases d0 d1 (its first [128][64] half) and
+  // m0 m1 (its second half)
+  static constexpr int kSBuf = (EPI == kGram) ? MUON_GRAM_SBUF : (EPI == kPoly ? MUON_POLY_SBUF : 2);
+  static_assert(kSBuf >= 2, "the diagonal block takes staging pairs 0 and 1");
+  static constexpr uint32_t kStagingBytes = (EPI == kBx) ? 0 : 2 * kSBuf * kChunkBf16;
+  // ready barriers: kBx one per slot; kGram / kPoly one per staging pair + the block
+  static constexpr int kReady = (EPI == kBx) ? kSlots : kSBuf + 1;
   static constexpr uint32_t kRingBytes = kStages * kStageBytes;
-  // full, empty, tfull x2, tempty x2, drain, efull x4, ready x4, sfree x2, econs x4
-  static constexpr int kNumBars = 2 * kStages + 5 + 3 * kSlots + 2;
+  // full, empty, tfull x2, tempty x2, drain, efull, ready, sfree, econs
+  static constexpr int kNumBars = 2 * kStages + 5 + 2 * kSlots + kReady + kSBuf;
   static constexpr size_t kSmem =
       1024 + kRingBytes + kSlotsBytes + kStagingBytes + kNumBars * 8 + 16;
 };
@@ -246,9 +259,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * S + 2 + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * S + 4);
   auto efull_bar = [&](int s) { return bar0 + 8u * (2 * S + 5 + s); };
+  constexpr int NB = C::kSBuf;
   auto ready_bar = [&](int s) { return bar0 + 8u * (2 * S + 5 + K + s); };
-  auto sfree_bar = [&](int b) { return bar0 + 8u * (2 * S + 5 + 2 * K + b); };
-  auto econs_bar = [&](int s) { return bar0 + 8u * (2 * S + 7 + 2 * K + s); };
+  auto sfree_bar = [&](int b) { return bar0 + 8u * (2 * S + 5 + K + C::kReady + b); };
+  // staging addresses (kGram / kPoly): direct and mirror chunk of pair b, and
+  // the two [128][64] halves of a diagonal block
+  auto econs_bar = [&](int s) { return bar0 + 8u * (2 * S + 5 + K + C::kReady + NB + s); };
+  auto stg_direct = [&](uint32_t base, int b) { return base + static_cast<uint32_t>(b) * kChunkBf16; };
+  auto stg_mirror = [&](uint32_t base, int b) { return base + static_cast<uint32_t>(NB + b) * kChunkBf16; };
+  auto stg_half = [&](uint32_t base, int h) { return base + static_cast<uint32_t>(h ? NB : 0) * kChunkBf16; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -263,10 +282,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(drain_bar, 1);
     for (int s = 0; s < K; ++s) {
       mbar_init(efull_bar(s), 1);
-      mbar_init(ready_bar(s), kEpiThreads);
       mbar_init(econs_bar(s), kEpiThreads);
     }
-    for (int b = 0; b < 2; ++b) mbar_init(sfree_bar(b), 1);
+    for (int s = 0; s < C::kReady; ++s) mbar_init(ready_bar(s), kEpiThreads);
+    for (int b = 0; b < NB; ++b) mbar_init(sfree_bar(b), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -457,9 +476,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         };
         for (int s = 0; s < K; ++s) issue_eload(s);
-        int njob[3] = {0, 0, 0};  // kGram / kPoly: jobs seen per ready barrier (0, 1: staging; 2: block)
-        int nup = 0;              // strictly-upper chunks so far (staging buffer = nup & 1)
-        int held = -1;            // staging buffer whose stores may still be reading it
+        int njob[NB + 1];  // kGram / kPoly: jobs seen per ready barrier (staging pairs, then the block)
+        for (int q = 0; q <= NB; ++q) njob[q] = 0;
+        int nup = 0;       // strictly-upper chunks so far (staging pair = nup % NB)
+        int hq[NB];        // FIFO of staging pairs whose stores may still be reading them
+        int hq_head = 0, hq_n = 0;
         for (int s = 0; s < total_chunks; ++s) {
           const int k = s / NCH, c = s % NCH;
           const TileCoord tc = decode_tile<EPI>(p, pair + k * npairs, rank);
@@ -486,47 +507,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (EPI == kPoly) {
             // every compute thread has read chunk s's A operand: refill its slot
             mbar_wait(econs_bar(s % K), (s / K) & 1, ctl);
+            if (c == 5) TRACE(k, 17);
             issue_eload(s + K);
           }
           if (kind == kUpper) {
-            const int b = nup & 1;
+            const int b = nup % NB;
             ++nup;
             mbar_wait(ready_bar(b), njob[b] & 1, ctl);
             ++njob[b];
-            const uint32_t ds = stage_u32 + b * kChunkBf16;        // direct [128][32]
-            const uint32_t ms = stage_u32 + (2 + b) * kChunkBf16;  // mirror [32][128]
-            tma_store_3d(&M.d, ds, col0, row0, tc.b);
-            tma_store_3d(&M.mt, ms, row0, col0, tc.b);
+            if (c == 5) TRACE(k, 18);
+            tma_store_3d(&M.d, stg_direct(stage_u32, b), col0, row0, tc.b);
+            tma_store_3d(&M.mt, stg_mirror(stage_u32, b), row0, col0, tc.b);
             bulk_commit();
-            // two chunks' stores in flight: release the previous buffer once
-            // its stores have read it, keep this one until the next chunk
-            if (held >= 0) {
-              asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-              mbar_arrive(sfree_bar(held));
+            hq[(hq_head + hq_n) % NB] = b;
+            ++hq_n;
+            // up to NB chunks' stores in flight: once all pairs are taken,
+            // release the oldest as soon as its stores have read it (the
+            // compute warps need it for the next chunk)
+            if (hq_n == NB) {
+              asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(NB - 1) : "memory");
+              mbar_arrive(sfree_bar(hq[hq_head]));
+              hq_head = (hq_head + 1) % NB;
+              --hq_n;
             }
-            held = b;
+            if (c == 5) TRACE(k, 19);
             continue;
           }
-          if (kind == kDiag && col0 == row0 && held >= 0) {
-            // a diagonal block starts: it takes both staging buffers
+          if (kind == kDiag && col0 == row0 && hq_n > 0) {
+            // a diagonal block starts: it takes staging pairs 0 and 1
             bulk_wait_read_all();
-            mbar_arrive(sfree_bar(held));
-            held = -1;
+            for (; hq_n > 0; --hq_n, hq_head = (hq_head + 1) % NB) mbar_arrive(sfree_bar(hq[hq_head]));
           }
           if (kind == kDiag && ((col0 - row0) / kChunk == 3 || col0 + kChunk >= G.m)) {
-            mbar_wait(ready_bar(2), njob[2] & 1, ctl);
-            ++njob[2];
-            tma_store_3d(&M.s, stage_u32, row0, row0, tc.b);
+            mbar_wait(ready_bar(NB), njob[NB] & 1, ctl);
+            ++njob[NB];
+            tma_store_3d(&M.s, stg_half(stage_u32, 0), row0, row0, tc.b);
             if (row0 + 64 < G.m)  // never start a store wholly outside the matrix
-              tma_store_3d(&M.s, stage_u32 + 2 * kChunkBf16, row0 + 64, row0, tc.b);
+              tma_store_3d(&M.s, stg_half(stage_u32, 1), row0 + 64, row0, tc.b);
             bulk_commit();
             bulk_wait_read_all();
-            mbar_arrive(sfree_bar(0));  // the block used both staging buffers
+            mbar_arrive(sfree_bar(0));  // the block used staging pairs 0 and 1
             mbar_arrive(sfree_bar(1));
           }
         }
         bulk_wait_all();
-        if (held >= 0) mbar_arrive(sfree_bar(held));
+        for (; hq_n > 0; --hq_n, hq_head = (hq_head + 1) % NB) mbar_arrive(sfree_bar(hq[hq_head]));
         for (int q = 0; q < K; ++q)  // operand copies still in flight land before exit
           if (pend[q] >= 0) mbar_wait_drain(efull_bar(q), (pend[q] / K) & 1, drain_ns);
       }
@@ -543,7 +568,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool leader = (warp == 2 && lane == 0);
       int acc = 0;
       uint32_t acc_phase = 0;
-      int nuse[2] = {0, 0};  // kGram / kPoly: jobs that used staging buffer b so far
+      int nuse[NB];  // kGram / kPoly: jobs that used staging pair b so far
+      for (int q = 0; q < NB; ++q) nuse[q] = 0;
+
       int nup = 0;
       for (int k = 0; k < my_tiles; ++k) {
         const TileCoord tc = decode_tile<EPI>(p, pair + k * npairs, rank);
@@ -633,6 +660,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(rr[q]);
           }
+          if (leader && c == 5) TRACE(k, 13);
           if (c == kChunks - 1) {
             // accumulator fully read: one arrival per warp hands it back (in
             // the partner CTA through the relay thread of warp 1)
@@ -642,6 +670,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           const int slot = s % K;
           if (EPI == kPoly) mbar_wait(efull_bar(slot), (s / K) & 1, ctl);
+          if (leader && c == 5) TRACE(k, 14);
 
           // ------------------------------------------------ kGram / kPoly
           if (EPI == kGram && kind != kSkip) {
@@ -668,12 +697,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_arrive(econs_bar(slot));  // slot read (or unused): the IO thread may refill it
           }
           if (kind == kUpper) {
-            const int b = nup & 1;
+            const int b = nup % NB;
             ++nup;
             if (nuse[b] > 0) mbar_wait(sfree_bar(b), (nuse[b] - 1) & 1, ctl);
             ++nuse[b];
-            const uint32_t ds = stage_u32 + b * kChunkBf16;        // direct [128][32]
-            const uint32_t ms = stage_u32 + (2 + b) * kChunkBf16;  // mirror [32][128]
+            if (leader && c == 5) TRACE(k, 15);
+            const uint32_t ds = stg_direct(stage_u32, b);  // direct [128][32]
+            const uint32_t ms = stg_mirror(stage_u32, b);  // mirror [32][128]
 #pragma unroll
             for (int uu = 0; uu < 2; ++uu)
               st_shared_v4(ds + sw64(r, 2 * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
@@ -683,6 +713,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int q = 0; q < 16; ++q) st_shared_u16(ms + (16 * hf + q) * 256 + r * 2, bf16_bits(v[q]));
             fence_async_smem();
             mbar_arrive(ready_bar(b));
+            if (leader && c == 5) TRACE(k, 16);
           } else if (kind == kDiag) {  // chunk dq of the 128 x 128 diagonal block
             const int dq = (col0 - row0) / kChunk;
             if (dq == 0) {
@@ -692,7 +723,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 ++nuse[b];
               }
             }
-            const uint32_t sb = stage_u32 + (dq >> 1) * (2 * kChunkBf16);  // [128][64] half
+            const uint32_t sb = stg_half(stage_u32, dq >> 1);  // [128][64] half
 #pragma unroll
             for (int uu = 0; uu < 2; ++uu)
               st_shared_v4(sb + sw128(r, (dq & 1) * 4 + 2 * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
@@ -704,7 +735,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               // 16-byte write; the two warps of a lane quarter split the groups.
               named_bar(1, kEpiThreads);
               auto s_addr = [&](int row, int col) {
-                return stage_u32 + (col >> 6) * (2 * kChunkBf16) +
+                return stg_half(stage_u32, col >> 6) +
                        static_cast<uint32_t>(row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2);
               };
               for (int j0 = 8 * hf; j0 < r; j0 += 16) {
@@ -724,7 +755,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
               }
               fence_async_smem();
-              mbar_arrive(ready_bar(2));
+              mbar_arrive(ready_bar(NB));
             }
           }
         }

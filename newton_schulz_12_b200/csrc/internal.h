@@ -68,10 +68,12 @@ struct Params {
 
 // Trace layout (MUON_TRACE builds): per CTA < kTraceCtas, per tile < kTraceTiles,
 // kTraceSlots %globaltimer stamps: 0 copier first issue, 1 copier last issue,
-// 2 MMA start, 3 MMA last commit, 4 epilogue start, 5..11 chunk ends, 12 end,
-// and within chunk 2: 13 TMEM loaded, 14 operand slot ready, 15 computed,
-// 16 after the epilogue barrier, 17 (leader) stores drained from the staging.
-constexpr int kTraceCtas = 16, kTraceTiles = 24, kTraceSlots = 18;
+// 2 MMA start, 3 MMA last commit, 4 epilogue start, 5..11 chunk starts, 12
+// end; kGram / kPoly chunk 5, compute leader: 13 accumulator loaded, 14
+// operand chunk landed, 15 staging pair free, 16 chunk handed to the IO
+// thread; IO thread: 17 operand chunk consumed, 18 chunk ready, 19 stores
+// issued and the oldest pair released.
+constexpr int kTraceCtas = 16, kTraceTiles = 24, kTraceSlots = 20;
 
 // Symmetric-output pair tiles per m x m matrix: the 256 x 256 tiles on or
 // above the diagonal.
