@@ -41,7 +41,8 @@ extern "C" {
 /* Storage / arithmetic type of muon_ns_orthogonalize's matrices. */
 typedef enum {
   MUON_BF16 = 0, /* bf16 storage; bf16 tensor-core operands, fp32 accumulate,
-                    X kept between steps as a pair of bf16 matrices hi + lo */
+                    X kept between steps as the pair bf16 hi + int8 residual
+                    (see muon_bx_bf16), about 16 significant bits */
   MUON_FP32 = 1  /* fp32 storage; fp32 SIMT FMA verification path */
 } muon_dtype;
 
@@ -77,6 +78,28 @@ typedef enum {
  */
 int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a, float b,
                           float c, int steps, int dtype, void* stream);
+
+/*
+ * muon_ns_orthogonalize_schedule -- muon_ns_orthogonalize with its own
+ * coefficient triple for every step.
+ *
+ * Source: "The NanoGPT speedrun", paragraph "Reading guide", names Polar
+ * Express polynomials among the later refinements of the same update: the
+ * iteration keeps its form, X <- a_t X + (b_t A + c_t A^2) X, but the
+ * polynomial changes from step to step.  The pages give no coefficients;
+ * the caller supplies them.
+ *
+ * coeffs  HOST array of 3 * steps floats, read during the call: step t
+ *         (t = 0 .. steps-1, in that order) uses a_t = coeffs[3t],
+ *         b_t = coeffs[3t+1], c_t = coeffs[3t+2].  May be NULL only when
+ *         steps == 0.  Every value must be finite.
+ * All other arguments, the layout, the in-place result and the errors are
+ * those of muon_ns_orthogonalize (a NULL table with steps > 0 or a
+ * non-finite value returns MUON_ERR_ARG before any work).  A table that
+ * repeats one triple gives exactly muon_ns_orthogonalize's result.
+ */
+int muon_ns_orthogonalize_schedule(int batch, int m, int n, void* const* X_ptrs,
+                                   const float* coeffs, int steps, int dtype, void* stream);
 
 /*
  * muon_ns_orthogonalize_static -- muon_ns_orthogonalize (bf16 storage, the

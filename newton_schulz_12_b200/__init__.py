@@ -21,6 +21,7 @@ from ._lib import MUON_BF16, MUON_FP32, MuonError, check, ptr_array, shape_array
 
 __all__ = [
     "NS_COEFFS", "MuonError", "MuonStepPlan", "muon_ns_orthogonalize",
+    "muon_ns_orthogonalize_schedule",
     "muon_ns_orthogonalize_static", "muon_step", "muon_momentum",
     "muon_apply", "muon_gram_bf16", "muon_poly_bf16", "muon_bx_bf16", "muon_get_status",
     "muon_last_error", "muon_release", "muon_set_wait_timeout_ms", "muon_set_fault_injection",
@@ -48,16 +49,8 @@ def _check_cuda(t, name, dtype=None):
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
 
 
-def muon_ns_orthogonalize(xs, a=NS_COEFFS[0], b=NS_COEFFS[1], c=NS_COEFFS[2], steps=5,
-                          stream=None):
-    """Orthogonalise every matrix of ``xs`` in place (list of equal-shape CUDA tensors).
-
-    bf16 tensors take the tensor-core path; fp32 tensors take the fp32 SIMT
-    verification path.  Returns ``xs``.
-    """
-    xs = list(xs)
-    if not xs:
-        return xs
+def _ns_batch(xs):
+    """Checks a list of equal-shape bf16 / fp32 CUDA matrices; returns (shape, mode, ptrs)."""
     shape, dtype = tuple(xs[0].shape), xs[0].dtype
     if len(shape) != 2:
         raise ValueError("matrices must be 2-D")
@@ -68,9 +61,37 @@ def muon_ns_orthogonalize(xs, a=NS_COEFFS[0], b=NS_COEFFS[1], c=NS_COEFFS[2], st
         if tuple(x.shape) != shape:
             raise ValueError("all matrices must have the same shape")
     mode = MUON_BF16 if dtype == torch.bfloat16 else MUON_FP32
-    arr = ptr_array([x.data_ptr() for x in xs])
+    return shape, mode, ptr_array([x.data_ptr() for x in xs])
+
+
+def muon_ns_orthogonalize(xs, a=NS_COEFFS[0], b=NS_COEFFS[1], c=NS_COEFFS[2], steps=5,
+                          stream=None):
+    """Orthogonalise every matrix of ``xs`` in place (list of equal-shape CUDA tensors).
+
+    bf16 tensors take the tensor-core path; fp32 tensors take the fp32 SIMT
+    verification path.  Returns ``xs``.
+    """
+    xs = list(xs)
+    if not xs:
+        return xs
+    shape, mode, arr = _ns_batch(xs)
     check(_lib.lib().muon_ns_orthogonalize(len(xs), shape[0], shape[1], arr, a, b, c, steps, mode,
                                            _stream(stream)))
+    return xs
+
+
+def muon_ns_orthogonalize_schedule(xs, schedule, stream=None):
+    """``muon_ns_orthogonalize`` with one (a, b, c) triple per step, applied in order."""
+    xs = list(xs)
+    flat = [float(v) for triple in schedule for v in triple]
+    if len(flat) != 3 * len(schedule):
+        raise ValueError("schedule must be a sequence of (a, b, c) triples")
+    if not xs:
+        return xs
+    shape, mode, arr = _ns_batch(xs)
+    table = (ctypes.c_float * max(1, len(flat)))(*flat)
+    check(_lib.lib().muon_ns_orthogonalize_schedule(len(xs), shape[0], shape[1], arr, table,
+                                                    len(schedule), mode, _stream(stream)))
     return xs
 
 

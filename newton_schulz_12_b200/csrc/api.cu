@@ -352,14 +352,16 @@ int launch_tc(int epi, tc::Params& P, int sms, cudaStream_t s) {
   return MUON_OK;
 }
 
-// T steps of X <- aX + (bA + cA^2)X on bf16 operands, X carried as hi + lo.
-// On entry each group's xb[0] / xlo hold X0 / s with s = xscale[mat_base + i]
-// per matrix (s = 1 when xscale is null); on exit xb[T % 2] / xlo hold X_T
-// (for T >= 1; X0 / s itself for T = 0).
-int run_ns_bf16(std::vector<NsGroup>& gs, int steps, float a, float b, float c, int* status,
-                int sms, cudaStream_t s, const float* xscale) {
+// T steps of X <- a_t X + (b_t A + c_t A^2) X on bf16 operands, X carried as
+// the pair hi + lo; step t uses abc[3t .. 3t+2].  On entry each group's xb[0]
+// / xlo hold X0 / s with s = xscale[mat_base + i] per matrix (s = 1 when
+// xscale is null); on exit xb[T % 2] / xlo hold X_T (for T >= 1; X0 / s
+// itself for T = 0).
+int run_ns_bf16(std::vector<NsGroup>& gs, int steps, const float* abc, int* status, int sms,
+                cudaStream_t s, const float* xscale) {
   if (steps <= 0 || gs.empty()) return MUON_OK;
   MUON_TRY(get_encoder());
+  const float a = abc[0], b = abc[1], c = abc[2];
   for (size_t g0 = 0; g0 < gs.size(); g0 += tc::kMaxGroups) {
     const size_t g1 = std::min(gs.size(), g0 + tc::kMaxGroups);
     tc::Params gram[2], poly, bx[2];
@@ -404,9 +406,14 @@ int run_ns_bf16(std::vector<NsGroup>& gs, int steps, float a, float b, float c, 
     bx0.xscale = xscale;
     int cur = 0;
     for (int t = 0; t < steps; ++t) {
+      // the step's own (a, b, c): B = b A + c A^2 in kPoly, a X in kBx
+      poly.b = abc[3 * t + 1];
+      poly.c = abc[3 * t + 2];
+      tc::Params& bxt = t == 0 ? bx0 : bx[cur];
+      bxt.a = abc[3 * t];
       MUON_TRY(launch_tc(tc::kGram, t == 0 ? gram0 : gram[cur], sms, s));
       MUON_TRY(launch_tc(tc::kPoly, poly, sms, s));
-      MUON_TRY(launch_tc(tc::kBx, t == 0 ? bx0 : bx[cur], sms, s));
+      MUON_TRY(launch_tc(tc::kBx, bxt, sms, s));
       cur ^= 1;
     }
   }
@@ -427,8 +434,9 @@ Result bf16_result(const NsGroup& g, int steps) {
   return r;
 }
 
-// fp32 SIMT verification path; on exit *final_xf of each group holds X_T.
-int run_ns_fp32(std::vector<NsGroup>& gs, int steps, float a, float b, float c, cudaStream_t s,
+// fp32 SIMT verification path (step t uses abc[3t .. 3t+2]); on exit
+// *final_xf of each group holds X_T.
+int run_ns_fp32(std::vector<NsGroup>& gs, int steps, const float* abc, cudaStream_t s,
                 std::vector<float*>& final_xf) {
   final_xf.clear();
   for (NsGroup& G : gs) {
@@ -439,9 +447,9 @@ int run_ns_fp32(std::vector<NsGroup>& gs, int steps, float a, float b, float c, 
     for (int t = 0; t < steps; ++t) {
       simt::Params p{};
       p.batch = G.batch;
-      p.a = a;
-      p.b = b;
-      p.c = c;
+      p.a = abc[3 * t];
+      p.b = abc[3 * t + 1];
+      p.c = abc[3 * t + 2];
       // A = X X^T
       p.m = G.m; p.n = G.m; p.k = G.n;
       p.P = x[cur]; p.ldp = G.ldn; p.sp = xs;
@@ -725,12 +733,12 @@ size_t bf16_layout(const std::vector<MatInfo>& mats, std::vector<NsGroup>& group
 int run_bf16_path(const std::vector<MatInfo>& mats, std::vector<NsGroup>& groups,
                   const BfLayout& L, const std::vector<const void*>& src,
                   const std::vector<float*>& bufs, int src_kind, float beta, int nesterov,
-                  float a, float b, float c, int steps, int* status, int sms, cudaStream_t s) {
+                  const float* abc, int steps, int* status, int sms, cudaStream_t s) {
   std::vector<int> pb, pc;
   MUON_TRY(launch_prep_chunked(mats, groups, src, bufs, src_kind, beta, nesterov, L.partials, pb,
                                pc, s));
   MUON_TRY(launch_scale_chunked(mats, groups, L.partials, pb, pc, L.xscale, s));
-  return run_ns_bf16(groups, steps, a, b, c, status, sms, s, L.xscale);
+  return run_ns_bf16(groups, steps, abc, status, sms, s, L.xscale);
 }
 
 // mode 0: apply into W; 1: bf16 write-back; 2: fp32 write-back.  O of matrix i
@@ -862,13 +870,19 @@ int muon_set_fault_injection(int mode) {
   return MUON_OK;
 }
 
-int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a, float b, float c,
-                          int steps, int dtype, void* stream) {
-  t_err.clear();
+}  // extern "C"
+
+namespace {
+
+// muon_ns_orthogonalize with a table of (a, b, c) per step (host, 3 * steps).
+int ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, const float* abc, int steps,
+                     int dtype, void* stream) {
   if (batch < 0 || batch > 65535) return set_err(MUON_ERR_ARG, "batch %d out of range 0..65535", batch);
   if (steps < 0 || steps > kMaxStepsArg) return set_err(MUON_ERR_ARG, "steps %d out of range 0..%d", steps, kMaxStepsArg);
   if (dtype != MUON_BF16 && dtype != MUON_FP32) return set_err(MUON_ERR_ARG, "dtype %d unknown", dtype);
-  if (!finite(a) || !finite(b) || !finite(c)) return set_err(MUON_ERR_ARG, "coefficients must be finite");
+  if (steps > 0 && !abc) return set_err(MUON_ERR_ARG, "coefficient table is NULL");
+  for (int i = 0; i < 3 * steps; ++i)
+    if (!finite(abc[i])) return set_err(MUON_ERR_ARG, "coefficient %d of step %d is not finite", i % 3, i / 3);
   MUON_TRY(check_shape(m, n, 0));
   if (batch == 0) return MUON_OK;
   if (!X_ptrs) return set_err(MUON_ERR_ARG, "X_ptrs is NULL");
@@ -892,7 +906,7 @@ int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a,
     Workspace* ws = nullptr;
     MUON_TRY(get_workspace(s, off, &ws));
     bf16_layout(mats, groups, static_cast<char*>(ws->ptr), L);
-    MUON_TRY(run_bf16_path(mats, groups, L, src, {}, ew::kFromBf16, 0.f, 0, a, b, c, steps,
+    MUON_TRY(run_bf16_path(mats, groups, L, src, {}, ew::kFromBf16, 0.f, 0, abc, steps,
                            ws->status, dev.sms, s));
     for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
     MUON_TRY(launch_out_chunked(mats, groups, res, ys, 1, 0.f, 0.f, s, steps == 0 ? L.xscale : nullptr));
@@ -913,7 +927,7 @@ int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a,
   MUON_TRY(launch_flat_chunked(src, {}, numels, ew::kFromF32, 0.f, 0, partials, pb, pc, s));
   MUON_TRY(launch_cast_chunked(mats, groups, src, {}, ew::kFromF32, 0.f, 0, partials, pb, pc, s));
   std::vector<float*> final_xf;
-  MUON_TRY(run_ns_fp32(groups, steps, a, b, c, s, final_xf));
+  MUON_TRY(run_ns_fp32(groups, steps, abc, s, final_xf));
   for (float* f : final_xf) {
     Result r;
     r.f = f;
@@ -921,6 +935,36 @@ int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a,
   }
   MUON_TRY(launch_out_chunked(mats, groups, res, ys, 2, 0.f, 0.f, s));
   return MUON_OK;
+}
+
+// The fixed triple as a table of `steps` rows.
+std::vector<float> constant_schedule(float a, float b, float c, int steps) {
+  std::vector<float> t;
+  for (int i = 0; i < steps; ++i) {
+    t.push_back(a);
+    t.push_back(b);
+    t.push_back(c);
+  }
+  return t;
+}
+
+}  // namespace
+
+extern "C" {
+
+int muon_ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, float a, float b, float c,
+                          int steps, int dtype, void* stream) {
+  t_err.clear();
+  if (steps < 0 || steps > kMaxStepsArg) return set_err(MUON_ERR_ARG, "steps %d out of range 0..%d", steps, kMaxStepsArg);
+  if (!finite(a) || !finite(b) || !finite(c)) return set_err(MUON_ERR_ARG, "coefficients must be finite");
+  const std::vector<float> abc = constant_schedule(a, b, c, steps);
+  return ns_orthogonalize(batch, m, n, X_ptrs, abc.data(), steps, dtype, stream);
+}
+
+int muon_ns_orthogonalize_schedule(int batch, int m, int n, void* const* X_ptrs, const float* coeffs,
+                                   int steps, int dtype, void* stream) {
+  t_err.clear();
+  return ns_orthogonalize(batch, m, n, X_ptrs, coeffs, steps, dtype, stream);
 }
 
 int muon_ns_orthogonalize_static(int batch, int m, int n, void* const* X_ptrs, float a, float b,
@@ -962,7 +1006,8 @@ int muon_ns_orthogonalize_static(int batch, int m, int n, void* const* X_ptrs, f
   bf16_layout(mats, groups, scratch + kStaticStatusBytes, L);
 
   std::vector<const void*> src(X_ptrs, X_ptrs + batch);
-  MUON_TRY(run_bf16_path(mats, groups, L, src, {}, ew::kFromBf16, 0.f, 0, a, b, c, steps, status,
+  const std::vector<float> abc = constant_schedule(a, b, c, steps);
+  MUON_TRY(run_bf16_path(mats, groups, L, src, {}, ew::kFromBf16, 0.f, 0, abc.data(), steps, status,
                          dev.sms, s));
   std::vector<Result> res;
   for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
@@ -1006,8 +1051,9 @@ int muon_step(int count, float* const* params, const void* const* grads,
 
   std::vector<const void*> gsrc(grads, grads + count);
   std::vector<float*> bufs(momentum_bufs, momentum_bufs + count);
+  const std::vector<float> abc = constant_schedule(kCoefA, kCoefB, kCoefC, steps);
   MUON_TRY(run_bf16_path(mats, groups, L, gsrc, bufs, ew::kFromMomentum, beta, nesterov,
-                         kCoefA, kCoefB, kCoefC, steps, ws->status, dev.sms, s));
+                         abc.data(), steps, ws->status, dev.sms, s));
   std::vector<Result> res;
   for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
   std::vector<void*> ys(params, params + count);

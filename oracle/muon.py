@@ -11,6 +11,9 @@ Citations name the page title and the passage:
   Tuning" (Muon paragraph).
 * [Overview ¶Six records] "The NanoGPT speedrun", paragraph "Six records
   account for most of the speedup" (record #3).
+* [Overview ¶Reading guide] the same page, paragraph "Reading guide": later
+  refinements tune the same update, among them Polar Express polynomials
+  (per-step coefficients; none are printed on the pages).
 """
 from __future__ import annotations
 
@@ -43,7 +46,7 @@ def frobenius_normalize(X, eps=NORM_EPS):
     return X / (np.sqrt(np.sum(X * X)) + eps)
 
 
-def newton_schulz(G, steps=NS_STEPS, coeffs=NS_COEFFS, eps=NORM_EPS):
+def newton_schulz(G, steps=NS_STEPS, coeffs=NS_COEFFS, eps=NORM_EPS, schedule=None):
     """Newton-Schulz orthogonalisation of one matrix, fp64.
 
     Follows, in order: transpose so that rows <= cols (a view choice; undone
@@ -51,8 +54,14 @@ def newton_schulz(G, steps=NS_STEPS, coeffs=NS_COEFFS, eps=NORM_EPS):
     A = X X^T, B = bA + c A A, X = aX + B X [Overview ¶Six records: "five
     Newton-Schulz steps"; Guide §Optimizer: orthogonalisation by
     Newton-Schulz iteration].  Square matrices are not transposed.
+
+    ``schedule``: optional list of (a, b, c) triples, one per step, in the
+    order applied (the per-step polynomials the Overview's ¶Reading guide
+    names as Polar Express; the pages give no coefficients).  When given it
+    replaces ``steps`` and ``coeffs``.
     """
-    a, b, c = (float(v) for v in coeffs)
+    if schedule is None:
+        schedule = [coeffs] * steps
     X = np.asarray(G, dtype=np.float64)
     if X.ndim != 2:
         raise ValueError("newton_schulz expects one 2-D matrix")
@@ -60,7 +69,8 @@ def newton_schulz(G, steps=NS_STEPS, coeffs=NS_COEFFS, eps=NORM_EPS):
     if transposed:
         X = X.T
     X = frobenius_normalize(X, eps)
-    for _ in range(steps):
+    for triple in schedule:
+        a, b, c = (float(v) for v in triple)
         A = X @ X.T
         B = b * A + c * (A @ A)
         X = a * X + B @ X

@@ -72,6 +72,22 @@ def test_argument_errors_need_no_device(lib):
     assert lib.muon_ns_orthogonalize(0, 4, 4, None, 1.0, 0.0, 0.0, 5, 0, null) == 0
 
 
+def test_schedule_argument_errors(lib):
+    null = ctypes.c_void_p(0)
+    table = (ctypes.c_float * 6)(3.4445, -4.775, 2.0315, 1.5, -0.5, 0.0)
+    bad = (ctypes.c_float * 6)(3.4445, -4.775, 2.0315, 1.5, float("inf"), 0.0)
+    arr = _lib.ptr_array([0x1000])
+    assert lib.muon_ns_orthogonalize_schedule(1, 4, 4, arr, None, 2, 0, null) == -1
+    assert "table" in _err(lib)
+    assert lib.muon_ns_orthogonalize_schedule(1, 4, 4, arr, bad, 2, 0, null) == -1
+    assert "step 1" in _err(lib)
+    assert lib.muon_ns_orthogonalize_schedule(1, 4, 4, arr, table, 101, 0, null) == -1
+    assert lib.muon_ns_orthogonalize_schedule(1, 4, 4, arr, table, 2, 9, null) == -1
+    # no steps: the table may be NULL; batch 0 is a no-op without a device
+    assert lib.muon_ns_orthogonalize_schedule(0, 4, 4, None, None, 0, 0, null) == 0
+    assert lib.muon_ns_orthogonalize_schedule(0, 4, 4, None, table, 2, 0, null) == 0
+
+
 def test_step_argument_errors(lib):
     null = ctypes.c_void_p(0)
     p = _lib.ptr_array([0x1000])
