@@ -228,8 +228,14 @@ __device__ __forceinline__ void trace_stamp(const Params& p, int tile, int slot)
 #endif
 
 // ---------------------------------------------------------------------- kernel
+// kPoly adds warp 11, its operand loader.
 template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+constexpr int threads_of() {
+  return EPI == kPoly ? kThreads + 32 : kThreads;
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1)
     gemm_kernel(const __grid_constant__ Params p) {
   using C = Cfg<EPI>;
   constexpr int S = C::kStages;
@@ -441,11 +447,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t slots_u32 = smem_u32(slots);
     const uint32_t stage_u32 = smem_u32(staging);
 
-    if (warp == 10) {
-      // ---------------------------------------------------------- IO thread
-      // Issues every epilogue bulk copy: operand chunks into the slot ring
-      // ahead of use, and the stores of what the compute warps finished,
-      // draining each store before the buffer it read is handed back.
+    if (warp >= 10) {
+      // ---------------------------------------------------------- IO threads
+      // Warp 10 issues the epilogue's bulk stores of what the compute warps
+      // finished, draining each store before the buffer it read is handed
+      // back, and (kBx) the operand chunk copies into the slot ring ahead of
+      // use.  kPoly's operand copies come from warp 11, so that a stalled
+      // copy issue never delays a store.
+      constexpr bool kLoaderWarp = (EPI == kPoly);
+      const bool loads_here = (EPI != kGram) && (kLoaderWarp ? warp == 11 : warp == 10);
       if (lane == 0) {
         for (int g = 0; g < p.ngroups; ++g) {
           tma_prefetch_map(&p.map[g].e);
@@ -475,13 +485,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               tma_load_3d(dst + C::kLoOff, &p.map[tc.g].mt, efull_bar(slot), col0, row0, tc.b);
           }
         };
-        for (int s = 0; s < K; ++s) issue_eload(s);
+        if (loads_here)
+          for (int s = 0; s < K; ++s) issue_eload(s);
+        if (kLoaderWarp && warp == 11) {
+          // kPoly loader: refill each slot as soon as every compute thread has read it
+          for (int s = 0; s < total_chunks; ++s) {
+            mbar_wait(econs_bar(s % K), (s / K) & 1, ctl);
+            if (s % NCH == 5) TRACE(s / NCH, 17);
+            issue_eload(s + K);
+          }
+        }
+        const int io_chunks = (kLoaderWarp && warp == 11) ? 0 : total_chunks;
         int njob[NB + 1];  // kGram / kPoly: jobs seen per ready barrier (staging pairs, then the block)
         for (int q = 0; q <= NB; ++q) njob[q] = 0;
         int nup = 0;       // strictly-upper chunks so far (staging pair = nup % NB)
         int hq[NB];        // FIFO of staging pairs whose stores may still be reading them
         int hq_head = 0, hq_n = 0;
-        for (int s = 0; s < total_chunks; ++s) {
+        for (int s = 0; s < io_chunks; ++s) {
           const int k = s / NCH, c = s % NCH;
           const TileCoord tc = decode_tile<EPI>(p, pair + k * npairs, rank);
           const Group& G = p.grp[tc.g];
@@ -503,12 +523,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             if (s >= 1) issue_eload(s + K - 1);  // into chunk s-1's slot
             continue;
-          }
-          if (EPI == kPoly) {
-            // every compute thread has read chunk s's A operand: refill its slot
-            mbar_wait(econs_bar(s % K), (s / K) & 1, ctl);
-            if (c == 5) TRACE(k, 17);
-            issue_eload(s + K);
           }
           if (kind == kUpper) {
             const int b = nup % NB;
@@ -552,8 +566,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         bulk_wait_all();
         for (; hq_n > 0; --hq_n, hq_head = (hq_head + 1) % NB) mbar_arrive(sfree_bar(hq[hq_head]));
-        for (int q = 0; q < K; ++q)  // operand copies still in flight land before exit
-          if (pend[q] >= 0) mbar_wait_drain(efull_bar(q), (pend[q] / K) & 1, drain_ns);
+        if (loads_here)
+          for (int q = 0; q < K; ++q)  // operand copies still in flight land before exit
+            if (pend[q] >= 0) mbar_wait_drain(efull_bar(q), (pend[q] / K) & 1, drain_ns);
       }
       __syncwarp();
     } else {
@@ -794,7 +809,7 @@ static cudaError_t launch_one(const Params& p, int max_pairs, cudaStream_t strea
     // clusters of two that fit at once: the persistent grid never waits for a second wave
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * max_pairs, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(threads_of<EPI>(), 1, 1);
     cfg.dynamicSmemBytes = smem;
     int n = 0;
     e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel<EPI>, &cfg);
@@ -804,7 +819,7 @@ static cudaError_t launch_one(const Params& p, int max_pairs, cudaStream_t strea
   }
   int pairs = p.total_tiles < max_pairs ? p.total_tiles : max_pairs;
   if (resident_pairs > 0 && pairs > resident_pairs) pairs = resident_pairs;
-  gemm_kernel<EPI><<<2 * pairs, kThreads, smem, stream>>>(p);
+  gemm_kernel<EPI><<<2 * pairs, threads_of<EPI>(), smem, stream>>>(p);
   return cudaGetLastError();
 }
 
