@@ -228,10 +228,10 @@ __device__ __forceinline__ void trace_stamp(const Params& p, int tile, int slot)
 #endif
 
 // ---------------------------------------------------------------------- kernel
-// kPoly adds warp 11, its operand loader.
+// kPoly and kBx add warp 11, their operand loader.
 template <int EPI>
 constexpr int threads_of() {
-  return EPI == kPoly ? kThreads + 32 : kThreads;
+  return EPI == kGram ? kThreads : kThreads + 32;
 }
 
 template <int EPI>
@@ -288,7 +288,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
     mbar_init(drain_bar, 1);
     for (int s = 0; s < K; ++s) {
       mbar_init(efull_bar(s), 1);
-      mbar_init(econs_bar(s), kEpiThreads);
+      // kPoly: every compute thread has read the slot; kBx: the slot's stores
+      // have read it (one arrival from the store thread)
+      mbar_init(econs_bar(s), EPI == kBx ? 1 : kEpiThreads);
     }
     for (int s = 0; s < C::kReady; ++s) mbar_init(ready_bar(s), kEpiThreads);
     for (int b = 0; b < NB; ++b) mbar_init(sfree_bar(b), 1);
@@ -451,10 +453,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
       // ---------------------------------------------------------- IO threads
       // Warp 10 issues the epilogue's bulk stores of what the compute warps
       // finished, draining each store before the buffer it read is handed
-      // back, and (kBx) the operand chunk copies into the slot ring ahead of
-      // use.  kPoly's operand copies come from warp 11, so that a stalled
-      // copy issue never delays a store.
-      constexpr bool kLoaderWarp = (EPI == kPoly);
+      // back.  The operand chunk copies into the slot ring come from warp 11,
+      // so that a copy issue stalled on the tensor-copy unit never delays a
+      // store: kPoly refills a slot once the compute warps have read it, kBx
+      // (whose results are stored from the slot itself) once its stores have.
+      constexpr bool kLoaderWarp = (EPI != kGram);
       const bool loads_here = (EPI != kGram) && (kLoaderWarp ? warp == 11 : warp == 10);
       if (lane == 0) {
         for (int g = 0; g < p.ngroups; ++g) {
@@ -488,11 +491,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
         if (loads_here)
           for (int s = 0; s < K; ++s) issue_eload(s);
         if (kLoaderWarp && warp == 11) {
-          // kPoly loader: refill each slot as soon as every compute thread has read it
-          for (int s = 0; s < total_chunks; ++s) {
-            mbar_wait(econs_bar(s % K), (s / K) & 1, ctl);
-            if (s % NCH == 5) TRACE(s / NCH, 17);
-            issue_eload(s + K);
+          if (EPI == kPoly) {
+            // refill each slot as soon as every compute thread has read it
+            for (int s = 0; s < total_chunks; ++s) {
+              mbar_wait(econs_bar(s % K), (s / K) & 1, ctl);
+              if (s % NCH == 5) TRACE(s / NCH, 17);
+              issue_eload(s + K);
+            }
+          } else {
+            // kBx: chunk s + K - 1 goes into chunk s - 1's slot once its stores have read it
+            for (int s = 1; s + K - 1 < total_chunks; ++s) {
+              mbar_wait(econs_bar((s - 1) % K), ((s - 1) / K) & 1, ctl);
+              issue_eload(s + K - 1);
+            }
           }
         }
         const int io_chunks = (kLoaderWarp && warp == 11) ? 0 : total_chunks;
@@ -521,7 +532,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             } else {
               bulk_wait_read_all();
             }
-            if (s >= 1) issue_eload(s + K - 1);  // into chunk s-1's slot
+            if (s >= 1) mbar_arrive(econs_bar((s - 1) % K));  // the loader may refill chunk s-1's slot
             continue;
           }
           if (kind == kUpper) {
