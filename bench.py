@@ -88,10 +88,10 @@ def stage_work(shapes):
 
     GEMMs: nominal FLOPs (X X^T: 2 m^2 n, A A: 2 m^3, B X: 2 m^2 n).
     Memory-bound kernels: bytes that must cross HBM per element -- prep
-    g(2)+buf(4) read, buf(4) and the bf16 pair hi(2)+lo(2) of u written =
-    14 B; apply W(4) + O as hi(2)+lo(2) read, W(4) written = 12 B; (fp32 and
-    stand-alone paths) momentum 10 B, cast 10 B.  The per-matrix scale reads
-    one partial per prep block.
+    g(2)+buf(4) read, buf(4) and the pair bf16 hi(2) + int8 lo(1) of u
+    written = 13 B; apply W(4) + O as hi(2)+lo(1) read, W(4) written = 11 B;
+    (fp32 and stand-alone paths) momentum 10 B, cast 10 B.  The per-matrix
+    scale reads one fp64 partial per prep block.
     """
     elems = sum(r * c for r, c in shapes)
     g = sum(2 * min(r, c) ** 2 * max(r, c) for r, c in shapes)
@@ -99,8 +99,8 @@ def stage_work(shapes):
     prep_blocks = sum(-(-r // 64) * -(-c // 128) for r, c in shapes)
     return {
         "gram": ("tensor", g), "poly": ("tensor", p), "bx": ("tensor", g),
-        "prep": ("hbm", 14 * elems), "scale": ("hbm", 4 * prep_blocks + 4 * len(shapes)),
-        "flat": ("hbm", 10 * elems), "cast": ("hbm", 10 * elems), "out": ("hbm", 12 * elems),
+        "prep": ("hbm", 13 * elems), "scale": ("hbm", 8 * prep_blocks + 4 * len(shapes)),
+        "flat": ("hbm", 10 * elems), "cast": ("hbm", 10 * elems), "out": ("hbm", 11 * elems),
     }
 
 
@@ -394,7 +394,7 @@ def run_ours(args):
             "config": {"workload": WORKLOAD, "matrices_per_step": len(shapes) * world,
                        "parallelism": f"replicas x{world} (one independent 72-matrix set per GPU)",
                        "l2": "inputs larger than L2 (W 340 MB + momentum 340 MB + grads 170 MB "
-                             "per GPU, plus a 680 MB workspace); no flush"},
+                             "per GPU, plus a 600 MB workspace); no flush"},
             "tflops": tflops,
             "pct_of_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
             "pct_of_bf16_peak_sustained": 100.0 * tflops / peaks["bf16_tflops_sustained"],
