@@ -235,12 +235,15 @@ int sym_maps(tc::Maps& M, const void* S, int m, int k, long long lds, long long 
              long long ldd, long long sd, int batch, bool with_e) {
   MUON_TRY(make_map(&M.p, S, 2, k, m, batch, lds, ss, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
   MUON_TRY(make_map(&M.q, S, 2, k, m, batch, lds, ss, 64, tc::BNH, CU_TENSOR_MAP_SWIZZLE_128B));
+  // epilogue chunks of kSymChunk columns: rows of 64 or 128 bytes
+  const CUtensorMapSwizzle cswz =
+      tc::kSymChunk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   if (with_e)
-    MUON_TRY(make_map(&M.e, S, 2, m, m, batch, lds, ss, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
+    MUON_TRY(make_map(&M.e, S, 2, m, m, batch, lds, ss, tc::kSymChunk, tc::BM, cswz));
   else
     M.e = M.p;
-  MUON_TRY(make_map(&M.d, D, 2, m, m, batch, ldd, sd, tc::kChunk, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
-  MUON_TRY(make_map(&M.mt, D, 2, m, m, batch, ldd, sd, tc::BM, tc::kChunk, CU_TENSOR_MAP_SWIZZLE_NONE));
+  MUON_TRY(make_map(&M.d, D, 2, m, m, batch, ldd, sd, tc::kSymChunk, tc::BM, cswz));
+  MUON_TRY(make_map(&M.mt, D, 2, m, m, batch, ldd, sd, tc::BM, tc::kSymChunk, CU_TENSOR_MAP_SWIZZLE_NONE));
   MUON_TRY(make_map(&M.s, D, 2, m, m, batch, ldd, sd, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
   return MUON_OK;
 }

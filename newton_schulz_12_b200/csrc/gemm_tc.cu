@@ -54,14 +54,16 @@ constexpr size_t kMaxSmem = 232448;                         // 227 KiB per CTA o
 // Shared memory per CTA is split between the operand ring (K stages) and the
 // epilogue (operand slots, output staging); the split is a compile-time
 // choice per kernel.
+// Defaults for 64-column symmetric chunks (their staging pairs are 32 KiB);
+// with 32-column chunks the staging halves and one more stage fits.
 #ifndef MUON_GRAM_STAGES
-#define MUON_GRAM_STAGES 6
+#define MUON_GRAM_STAGES (MUON_SYM_CHUNK == 64 ? 5 : 6)
 #endif
 #ifndef MUON_POLY_STAGES
-#define MUON_POLY_STAGES 5
+#define MUON_POLY_STAGES (MUON_SYM_CHUNK == 64 ? 4 : 5)
 #endif
 #ifndef MUON_POLY_SLOTS
-#define MUON_POLY_SLOTS 4
+#define MUON_POLY_SLOTS (MUON_SYM_CHUNK == 64 ? 2 : 4)
 #endif
 #ifndef MUON_GRAM_SBUF
 #define MUON_GRAM_SBUF 2
@@ -83,24 +85,24 @@ struct Cfg {
   // epilogue operand ring of kSlots chunks (kGram: none, the count only sizes barriers)
   // kBx slot: the hi and lo bf16 chunks of X (8 KiB each); kPoly slot: A's chunk
   static constexpr int kSlots = (EPI == kBx) ? MUON_BX_SLOTS : MUON_POLY_SLOTS;
-  static_assert(BN % (2 * kChunk) == 0, "whole chunks per tile");
   // kBx works on 64-column chunks (128-byte rows in global memory), the
-  // symmetric kernels on 32-column chunks (their mirrored stores are 32 rows)
-  static constexpr int kCW = (EPI == kBx) ? 2 * kChunk : kChunk;
+  // symmetric kernels on kSymChunk-column chunks
+  static constexpr int kCW = (EPI == kBx) ? 2 * kChunk : kSymChunk;
   static constexpr int kNCh = BN / kCW;  // per tile
-  // kBx slot: hi (bf16, 128 rows x 128 B) then lo (int8, 128 rows x 64 B)
-  static constexpr uint32_t kSlotBytes = (EPI == kBx) ? 3 * kChunkBf16 : (EPI == kPoly ? kChunkBf16 : 0);
+  // bytes of one bf16 chunk, 128 rows x kCW columns
+  static constexpr uint32_t kChunkBytes = BM * kCW * 2;
+  // kBx slot: hi (bf16, 128 rows x 128 B) then lo (int8, 128 rows x 64 B);
+  // kPoly slot: A's chunk
+  static constexpr uint32_t kSlotBytes = (EPI == kBx) ? 3 * kChunkBf16 : (EPI == kPoly ? kChunkBytes : 0);
   static constexpr uint32_t kLoOff = 2 * kChunkBf16;
   static constexpr uint32_t kSlotsBytes = kSlotBytes * kSlots;
-  // staging: kBx two bf16 output chunks; kGram / kPoly 2 direct + 2 mirror chunks,
-  // aliased by the 128 x 128 diagonal block (2 x [128 rows][64 cols] bf16)
-  // kGram / kPoly output staging: kSBuf pairs of a direct [128][32] and a
-  // mirrored [32][128] chunk, laid out as d0 .. d(kSBuf-1), m0 .. m(kSBuf-1);
-  // a diagonal 128 x 128 block aliases d0 d1 (its first [128][64] half) and
-  // m0 m1 (its second half)
+  // kGram / kPoly output staging: kSBuf pairs of a direct [128][kCW] and a
+  // mirrored [kCW][128] chunk, laid out as d0 .. d(kSBuf-1), m0 .. m(kSBuf-1).
+  // A diagonal 128 x 128 block (two [128][64] halves, 128-byte swizzle)
+  // aliases d0 d1 and m0 m1 (32-column chunks) or d0 and d1 (64-column).
   static constexpr int kSBuf = (EPI == kGram) ? MUON_GRAM_SBUF : (EPI == kPoly ? MUON_POLY_SBUF : 2);
   static_assert(kSBuf >= 2, "the diagonal block takes staging pairs 0 and 1");
-  static constexpr uint32_t kStagingBytes = (EPI == kBx) ? 0 : 2 * kSBuf * kChunkBf16;
+  static constexpr uint32_t kStagingBytes = (EPI == kBx) ? 0 : 2 * kSBuf * kChunkBytes;
   // ready barriers: kBx one per slot; kGram / kPoly one per staging pair + the block
   static constexpr int kReady = (EPI == kBx) ? kSlots : kSBuf + 1;
   static constexpr uint32_t kRingBytes = kStages * kStageBytes;
@@ -161,11 +163,12 @@ enum ChunkKind : int { kSkip = 0, kUpper = 1, kDiag = 2, kPlain = 3 };
 
 template <int EPI>
 __device__ __forceinline__ int chunk_kind(const Group& G, int tm, int col0) {
+  constexpr int W = (EPI == kBx) ? 2 * kChunk : kSymChunk;
   // a CTA whose rows lie wholly below the matrix stores nothing
   if (EPI == kBx) return (col0 < G.n && tm * BM < G.m) ? kPlain : kSkip;
   if (col0 >= G.m) return kSkip;
   const int d0 = tm * BM;
-  if (col0 + kChunk <= d0) return kSkip;  // strictly below the diagonal block
+  if (col0 + W <= d0) return kSkip;  // strictly below the diagonal block
   if (col0 >= d0 + BM) return kUpper;     // strictly above it
   return kDiag;
 }
@@ -271,9 +274,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
   // staging addresses (kGram / kPoly): direct and mirror chunk of pair b, and
   // the two [128][64] halves of a diagonal block
   auto econs_bar = [&](int s) { return bar0 + 8u * (2 * S + 5 + K + C::kReady + NB + s); };
-  auto stg_direct = [&](uint32_t base, int b) { return base + static_cast<uint32_t>(b) * kChunkBf16; };
-  auto stg_mirror = [&](uint32_t base, int b) { return base + static_cast<uint32_t>(NB + b) * kChunkBf16; };
-  auto stg_half = [&](uint32_t base, int h) { return base + static_cast<uint32_t>(h ? NB : 0) * kChunkBf16; };
+  auto stg_direct = [&](uint32_t base, int b) { return base + static_cast<uint32_t>(b) * C::kChunkBytes; };
+  auto stg_mirror = [&](uint32_t base, int b) {
+    return base + static_cast<uint32_t>(NB + b) * C::kChunkBytes;
+  };
+  auto stg_half = [&](uint32_t base, int h) {
+    return C::kCW == 64 ? stg_direct(base, h) : base + static_cast<uint32_t>(h ? NB : 0) * kChunkBf16;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -495,7 +502,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             // refill each slot as soon as every compute thread has read it
             for (int s = 0; s < total_chunks; ++s) {
               mbar_wait(econs_bar(s % K), (s / K) & 1, ctl);
-              if (s % NCH == 5) TRACE(s / NCH, 17);
+              if (s % NCH == NCH - 3) TRACE(s / NCH, 17);
               issue_eload(s + K);
             }
           } else {
@@ -540,7 +547,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             ++nup;
             mbar_wait(ready_bar(b), njob[b] & 1, ctl);
             ++njob[b];
-            if (c == 5) TRACE(k, 18);
+            if (c == NCH - 3) TRACE(k, 18);
             tma_store_3d(&M.d, stg_direct(stage_u32, b), col0, row0, tc.b);
             tma_store_3d(&M.mt, stg_mirror(stage_u32, b), row0, col0, tc.b);
             bulk_commit();
@@ -555,7 +562,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
               hq_head = (hq_head + 1) % NB;
               --hq_n;
             }
-            if (c == 5) TRACE(k, 19);
+            if (c == NCH - 3) TRACE(k, 19);
             continue;
           }
           if (kind == kDiag && col0 == row0 && hq_n > 0) {
@@ -563,7 +570,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             bulk_wait_read_all();
             for (; hq_n > 0; --hq_n, hq_head = (hq_head + 1) % NB) mbar_arrive(sfree_bar(hq[hq_head]));
           }
-          if (kind == kDiag && ((col0 - row0) / kChunk == 3 || col0 + kChunk >= G.m)) {
+          if (kind == kDiag && ((col0 - row0) / CW == BM / CW - 1 || col0 + CW >= G.m)) {
             mbar_wait(ready_bar(NB), njob[NB] & 1, ctl);
             ++njob[NB];
             tma_store_3d(&M.s, stg_half(stage_u32, 0), row0, row0, tc.b);
@@ -670,24 +677,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             mbar_arrive(ready_bar(slot));
           }
         } else {
-        for (int c = 0; c < kChunks; ++c) {
+        // kCW-column chunks: thread (r, hf) takes accumulator columns
+        // VPT hf .. VPT hf + VPT-1 of the chunk, i.e. 16-byte units
+        // UPT hf .. UPT hf + UPT-1 of the chunk's swizzled row (64-byte
+        // swizzle for 32-column chunks, 128-byte for 64-column ones)
+        constexpr int SCW = C::kCW, VPT = SCW / 2, UPT = VPT / 8;
+        auto swz = [](int row, int u) { return SCW == 64 ? sw128(row, u) : sw64(row, u); };
+        for (int c = 0; c < C::kNCh; ++c) {
           if (leader && c > 0) TRACE(k, 4 + c);
-          const int s = k * kChunks + c;
-          const int col0 = tc.tn * BN + c * kChunk;
+          const int s = k * C::kNCh + c;
+          const int col0 = tc.tn * BN + c * SCW;
           const int kind = chunk_kind<EPI>(G, tc.tm, col0);
-          float v[16];
+          float v[VPT];
           if (kind != kSkip) {
-            uint32_t rr[16];
+            uint32_t rr[VPT];
             __syncwarp();
-            tmem_ld_32x32_x16(tmem_base + (static_cast<uint32_t>(lane_base) << 16) +
-                                  static_cast<uint32_t>(acc * BN + c * kChunk + hf * 16),
-                              rr);
+            const uint32_t ta = tmem_base + (static_cast<uint32_t>(lane_base) << 16) +
+                                static_cast<uint32_t>(acc * BN + c * SCW + hf * VPT);
+            if constexpr (VPT == 32)
+              tmem_ld_32x32(ta, rr);
+            else
+              tmem_ld_32x32_x16(ta, rr);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(rr[q]);
+            for (int q = 0; q < VPT; ++q) v[q] = __uint_as_float(rr[q]);
           }
-          if (leader && c == 5) TRACE(k, 13);
-          if (c == kChunks - 1) {
+          if (leader && c == C::kNCh - 3) TRACE(k, 13);
+          if (c == C::kNCh - 1) {
             // accumulator fully read: one arrival per warp hands it back (in
             // the partner CTA through the relay thread of warp 1)
             tc_fence_before();
@@ -696,21 +712,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
           }
           const int slot = s % K;
           if (EPI == kPoly) mbar_wait(efull_bar(slot), (s / K) & 1, ctl);
-          if (leader && c == 5) TRACE(k, 14);
+          if (leader && c == C::kNCh - 3) TRACE(k, 14);
 
           // ------------------------------------------------ kGram / kPoly
           if (EPI == kGram && kind != kSkip) {
 #pragma unroll
-            for (int q = 0; q < 16; ++q) v[q] *= xs;
+            for (int q = 0; q < VPT; ++q) v[q] *= xs;
           }
           if (EPI == kPoly) {
             if (kind != kSkip) {
-              // B = b A + c acc with A's chunk from the slot (bf16, 64-byte swizzle)
+              // B = b A + c acc with A's chunk from the slot (bf16, swizzled like the staging)
               const uint32_t es = slots_u32 + slot * C::kSlotBytes;
 #pragma unroll
-              for (int uu = 0; uu < 2; ++uu) {
+              for (int uu = 0; uu < UPT; ++uu) {
                 uint32_t a4[4];
-                ld_shared_v4(es + sw64(r, 2 * hf + uu), a4[0], a4[1], a4[2], a4[3]);
+                ld_shared_v4(es + swz(r, UPT * hf + uu), a4[0], a4[1], a4[2], a4[3]);
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                   const float lo = bf16_bits_to_f32(static_cast<uint16_t>(a4[h] & 0xFFFFu));
@@ -720,42 +736,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                 }
               }
             }
-            mbar_arrive(econs_bar(slot));  // slot read (or unused): the IO thread may refill it
+            mbar_arrive(econs_bar(slot));  // slot read (or unused): the loader may refill it
           }
           if (kind == kUpper) {
             const int b = nup % NB;
             ++nup;
             if (nuse[b] > 0) mbar_wait(sfree_bar(b), (nuse[b] - 1) & 1, ctl);
             ++nuse[b];
-            if (leader && c == 5) TRACE(k, 15);
-            const uint32_t ds = stg_direct(stage_u32, b);  // direct [128][32]
-            const uint32_t ms = stg_mirror(stage_u32, b);  // mirror [32][128]
+            if (leader && c == C::kNCh - 3) TRACE(k, 15);
+            const uint32_t ds = stg_direct(stage_u32, b);  // direct [128][SCW]
+            const uint32_t ms = stg_mirror(stage_u32, b);  // mirror [SCW][128]
 #pragma unroll
-            for (int uu = 0; uu < 2; ++uu)
-              st_shared_v4(ds + sw64(r, 2 * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
+            for (int uu = 0; uu < UPT; ++uu)
+              st_shared_v4(ds + swz(r, UPT * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
                            pack_bf16x2(v[8 * uu + 2], v[8 * uu + 3]), pack_bf16x2(v[8 * uu + 4], v[8 * uu + 5]),
                            pack_bf16x2(v[8 * uu + 6], v[8 * uu + 7]));
 #pragma unroll
-            for (int q = 0; q < 16; ++q) st_shared_u16(ms + (16 * hf + q) * 256 + r * 2, bf16_bits(v[q]));
+            for (int q = 0; q < VPT; ++q) st_shared_u16(ms + (VPT * hf + q) * 256 + r * 2, bf16_bits(v[q]));
             fence_async_smem();
             mbar_arrive(ready_bar(b));
-            if (leader && c == 5) TRACE(k, 16);
+            if (leader && c == C::kNCh - 3) TRACE(k, 16);
           } else if (kind == kDiag) {  // chunk dq of the 128 x 128 diagonal block
-            const int dq = (col0 - row0) / kChunk;
+            const int dq = (col0 - row0) / SCW;
             if (dq == 0) {
-              // the block occupies both staging buffers: wait for their last stores
+              // the block occupies staging pairs 0 and 1: wait for their last stores
               for (int b = 0; b < 2; ++b) {
                 if (nuse[b] > 0) mbar_wait(sfree_bar(b), (nuse[b] - 1) & 1, ctl);
                 ++nuse[b];
               }
             }
-            const uint32_t sb = stg_half(stage_u32, dq >> 1);  // [128][64] half
+            // columns dq SCW .. of the block: half (dq SCW) / 64, first unit ((dq SCW) % 64) / 8
+            const uint32_t sb = stg_half(stage_u32, (dq * SCW) >> 6);  // [128][64] half
+            const int u0 = ((dq * SCW) & 63) >> 3;
 #pragma unroll
-            for (int uu = 0; uu < 2; ++uu)
-              st_shared_v4(sb + sw128(r, (dq & 1) * 4 + 2 * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
+            for (int uu = 0; uu < UPT; ++uu)
+              st_shared_v4(sb + sw128(r, u0 + UPT * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
                            pack_bf16x2(v[8 * uu + 2], v[8 * uu + 3]), pack_bf16x2(v[8 * uu + 4], v[8 * uu + 5]),
                            pack_bf16x2(v[8 * uu + 6], v[8 * uu + 7]));
-            if (dq == 3 || col0 + kChunk >= G.m) {
+            if (dq == BM / SCW - 1 || col0 + SCW >= G.m) {
               // block complete: lower half := transpose of the upper half.
               // Row r takes S[r][j] = S[j][r] for j < r, eight columns per
               // 16-byte write; the two warps of a lane quarter split the groups.

@@ -16,8 +16,14 @@ constexpr int PM = 2 * BM;           // tile rows per CTA pair (one M = 256 pair
 constexpr int BN = 256;              // tile columns (fp32 TMEM columns per accumulator)
 constexpr int BNH = BN / 2;          // rows of the column operand each CTA of a pair stages
 constexpr int BK = 64;               // K per stage: one 128-byte swizzle row of bf16
-constexpr int kChunk = 32;           // epilogue columns handled per step
+constexpr int kChunk = 32;           // base epilogue chunk width (columns)
 constexpr int kChunks = BN / kChunk;
+#ifndef MUON_SYM_CHUNK
+#define MUON_SYM_CHUNK 64
+#endif
+// Epilogue chunk width of the symmetric-output kernels (kGram / kPoly): 32 or 64.
+constexpr int kSymChunk = MUON_SYM_CHUNK;
+static_assert(kSymChunk == 32 || kSymChunk == 64, "symmetric chunk width");
 constexpr int kThreads = 352;        // warp 0 copies, warp 1 MMAs, warps 2-9 epilogue math,
                                      // warp 10 epilogue loads and stores
 constexpr int kEpiThreads = 256;     // warps 2-9
@@ -45,10 +51,10 @@ struct Group {
 struct Maps {
   CUtensorMap p;   // rows of D: X (kGram), A (kPoly), B (kBx); K-major, box 64 x 128
   CUtensorMap q;   // columns of D: X / A K-major box 64 x 128; X MN-major box 64 x 64 (kBx)
-  CUtensorMap e;   // epilogue input chunk, bf16 32 x 128: A (kPoly); hi of X (kBx)
-  CUtensorMap d;   // direct output chunk, bf16 32 x 128: A (kGram), B (kPoly), hi of X' (kBx)
-  CUtensorMap mt;  // mirrored output chunk, bf16 128 x 32 (kGram / kPoly); lo of X, 32 x 128 (kBx)
-  CUtensorMap s;   // symmetrised diagonal block, bf16 64 x 128 (kGram / kPoly)
+  CUtensorMap e;   // epilogue input chunk, bf16 kSymChunk x 128: A (kPoly); hi of X (kBx)
+  CUtensorMap d;   // direct output chunk, bf16 kSymChunk x 128: A (kGram), B (kPoly); hi of X' (kBx)
+  CUtensorMap mt;  // mirrored output chunk, bf16 128 x kSymChunk (kGram / kPoly); lo of X (kBx)
+  CUtensorMap s;   // symmetrised diagonal block half, bf16 64 x 128 (kGram / kPoly)
 };
 
 struct Params {
@@ -69,7 +75,7 @@ struct Params {
 // Trace layout (MUON_TRACE builds): per CTA < kTraceCtas, per tile < kTraceTiles,
 // kTraceSlots %globaltimer stamps: 0 copier first issue, 1 copier last issue,
 // 2 MMA start, 3 MMA last commit, 4 epilogue start, 5..11 chunk starts, 12
-// end; kGram / kPoly chunk 5, compute leader: 13 accumulator loaded, 14
+// end; kGram / kPoly chunk kNCh-3, compute leader: 13 accumulator loaded, 14
 // operand chunk landed, 15 staging pair free, 16 chunk handed to the IO
 // thread; IO thread: 17 operand chunk consumed, 18 chunk ready, 19 stores
 // issued and the oldest pair released.
