@@ -11,7 +11,10 @@ import ctypes
 import os
 import threading
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmuon_b200.so")
+#: The in-tree build; MUON_B200_LIB may name another build of the same
+#: sources (e.g. a variant compiled with different tile parameters).
+LIB_PATH = os.environ.get("MUON_B200_LIB") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libmuon_b200.so")
 
 MUON_BF16 = 0
 MUON_FP32 = 1
