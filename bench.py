@@ -12,9 +12,10 @@ iid N(0, 0.01^2), fp32 momentum (beta 0.95, Nesterov), lr 0.05, wd 0.
 Prints one JSON line (rank 0).  `value` is matrices/s over all ranks with
 inputs resident in HBM; `e2e` repeats the measurement with the gradients
 copied in from pinned host memory and the updated weights copied back every
-step.  Per-kernel device times are taken live with CUDA events on the
-launching stream (the library's timing hooks); `roofline` reports the
-dominant kernel against the measured peaks in MEASURED_PEAKS.json.
+step (the copies of one step overlap the compute of its neighbours).
+Per-kernel device times are taken live with CUDA events on the launching
+stream (the library's timing hooks); `roofline` reports the dominant kernel
+against the measured peaks in MEASURED_PEAKS.json.
 `--impl reference` times the fp64 CPU oracle on a bounded sample instead.
 """
 from __future__ import annotations
@@ -335,22 +336,56 @@ def run_ours(args):
         raise RuntimeError("device status after timed region: " + nsb.muon_last_error())
     launches = sum(n for _, n in prof.values())
 
-    # ---- end to end: pinned host grads in, updated weights out, every step
+    # ---- end to end: pinned host grads in, updated weights out, every step.
+    # The copies overlap the neighbouring steps' compute, as a training loop
+    # would: step k's grads go into one of two device buffers on a copy-in
+    # stream while step k-1 runs; after step k the weights are copied to a
+    # device staging buffer (step k+1 then updates W in place) and read back
+    # to the host on a copy-out stream while step k+1 runs.
     G_host = G_flat.cpu().pin_memory()
     W_host = torch.empty(total, dtype=torch.float32).pin_memory()
+    G_dev = [G_flat, torch.empty_like(G_flat)]
+    plans = []
+    for g in G_dev:
+        views = [g[offs[i]:offs[i + 1]].view(shapes[i]) for i in range(len(shapes))]
+        plans.append(nsb.MuonStepPlan(W, views, M, beta=0.95, nesterov=True, lr=0.05, wd=0.0, steps=5))
+    W_stage = torch.empty_like(W_flat)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    g_ready = [torch.cuda.Event(), torch.cuda.Event()]
+    g_free = [torch.cuda.Event(), torch.cuda.Event()]
+    staged, out_done = torch.cuda.Event(), torch.cuda.Event()
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_steps = args.steps
     barrier()
     torch.cuda.synchronize(dev)
     e_start.record(stream)
-    for _ in range(e2e_steps):
-        G_flat.copy_(G_host, non_blocking=True)
-        step()
-        W_host.copy_(W_flat, non_blocking=True)
+    s_in.wait_event(e_start)
+    s_out.wait_event(e_start)
+    for k in range(e2e_steps):
+        j = k % 2
+        with torch.cuda.stream(s_in):
+            if k >= 2:
+                s_in.wait_event(g_free[j])  # step k-2 is done with this buffer
+            G_dev[j].copy_(G_host, non_blocking=True)
+            g_ready[j].record(s_in)
+        stream.wait_event(g_ready[j])
+        plans[j](stream)
+        g_free[j].record(stream)
+        if k >= 1:
+            stream.wait_event(out_done)  # step k-1's read-back is done with the staging buffer
+        W_stage.copy_(W_flat, non_blocking=True)
+        staged.record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(staged)
+            W_host.copy_(W_stage, non_blocking=True)
+            out_done.record(s_out)
+    stream.wait_event(out_done)
     e_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
+    if nsb.muon_get_status(stream) != 0:
+        raise RuntimeError("device status after the end-to-end run: " + nsb.muon_last_error())
 
     nmat = len(shapes) * world
     value = job_throughput(len(shapes), world, args.steps, ms)
