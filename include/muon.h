@@ -276,7 +276,7 @@ typedef enum {
   MUON_KERNEL_OUT = 5,  /* apply / write-back */
   MUON_KERNEL_SIMT = 6, /* fp32 verification GEMMs */
   MUON_KERNEL_SUMS = 7, /* per-matrix sums of partials */
-  MUON_KERNEL_PREP = 8, /* momentum + Nesterov blend written as the bf16 pair (transposing) */
+  MUON_KERNEL_PREP = 8, /* momentum + Nesterov blend written as the bf16 + int8 pair (transposing) */
   MUON_KERNEL_SCALE = 9, /* per-matrix 1 / (||u||_F + eps) */
   MUON_KERNEL_KINDS = 10
 } muon_kernel_kind;

@@ -423,7 +423,7 @@ int run_ns_bf16(std::vector<NsGroup>& gs, int steps, const float* abc, int* stat
   return MUON_OK;
 }
 
-// Where a group's result X_T lives: fp32, or the bf16 pair hi + lo.
+// Where a group's result X_T lives: fp32, or the pair bf16 hi + int8 residual.
 struct Result {
   const float* f = nullptr;
   const bf16* hi = nullptr;

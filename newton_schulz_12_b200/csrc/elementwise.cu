@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kTileThreads) cast_kernel(const __grid_constan
 
 // o[k] = O[r][c + k] read from the m x n result buffer (row stride ld) as laid
 // out there: rows r of that buffer, columns c.. (0 outside it).  The buffer is
-// fp32, or the bf16 pair hi + lo.
+// fp32, or the pair bf16 hi + int8 residual.
 __device__ __forceinline__ void load_o8(const OutMat& M, int r, int c, int orows, int ocols,
                                         float (&o)[8]) {
   const int cnt = r < orows ? min(8, ocols - c) : 0;

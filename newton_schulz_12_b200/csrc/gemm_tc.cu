@@ -7,7 +7,7 @@
 //
 //   kGram  A  = X X^T            tiles on or above the diagonal, mirrored
 //   kPoly  B  = b A + c A A      A symmetric, so A A = A A^T: same tiling
-//   kBx    X' = a X + B X        X carried as a pair of bf16 matrices, X = hi + lo
+//   kBx    X' = a X + B X        X carried as the pair bf16 hi + int8 residual
 //
 // CTAs run in clusters of two on an SM pair, one cluster per pair tile of
 // 256 x 256 outputs at a time, persistent over a static tile stride.  One
@@ -25,13 +25,14 @@
 //               accumulators) for the pair; in the leader one thread issues
 //               the pair MMAs and commits each stage back to both copiers and
 //               each finished accumulator to both epilogues;
-//   warps 2-9   the epilogue: per 32-column chunk, tcgen05.ld (one row per
+//   warps 2-9   the epilogue: per 64-column chunk, tcgen05.ld (one row per
 //               thread, two warps per lane quarter), combine with the chunk's
-//               epilogue operand (prefetched by bulk copy into a 4-slot
-//               ring), write swizzled staging in shared memory -- no
+//               epilogue operand (prefetched by bulk copy into a ring of
+//               slots), write swizzled staging in shared memory -- no
 //               row-strided global accesses; the other accumulator fills
 //               meanwhile;
-//   warp 10     one thread issues the epilogue's bulk loads and stores.
+//   warp 10     one thread issues the epilogue's bulk stores;
+//   warp 11     (kPoly, kBx) one thread issues the epilogue operand copies.
 // Symmetric outputs: a chunk strictly above the diagonal 128x128 block is
 // stored twice (direct, and transposed through a second staging buffer); the
 // diagonal block is assembled in shared memory, its lower half overwritten
@@ -158,7 +159,7 @@ __device__ __forceinline__ TileCoord decode_tile(const Params& p, int t, int ran
   return c;
 }
 
-// Role of one 32-column epilogue chunk of a symmetric-output tile.
+// Role of one epilogue chunk (kCW columns) of an output tile.
 enum ChunkKind : int { kSkip = 0, kUpper = 1, kDiag = 2, kPlain = 3 };
 
 template <int EPI>
@@ -592,7 +593,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
     } else {
       // ---------------------------------------------------------- compute (warps 2-9)
       // Two warps per TMEM lane quarter: warp w reads lanes 32*(w%4).. and
-      // the half `hf` of each 32-column chunk.  A failed (timed-out) wait is
+      // the half `hf` of each chunk's columns.  A failed (timed-out) wait is
       // recorded and the schedule continues -- every later wait then returns
       // at once -- so the compute warps always meet at the same barriers.
       const int lane_base = 32 * (warp & 3);

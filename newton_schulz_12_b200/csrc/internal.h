@@ -17,7 +17,6 @@ constexpr int BN = 256;              // tile columns (fp32 TMEM columns per accu
 constexpr int BNH = BN / 2;          // rows of the column operand each CTA of a pair stages
 constexpr int BK = 64;               // K per stage: one 128-byte swizzle row of bf16
 constexpr int kChunk = 32;           // base epilogue chunk width (columns)
-constexpr int kChunks = BN / kChunk;
 #ifndef MUON_SYM_CHUNK
 #define MUON_SYM_CHUNK 64
 #endif
@@ -189,7 +188,7 @@ struct OutParams {
 };
 
 // One pass over the caller's matrices: momentum (or a plain read of X), the
-// Nesterov blend u, and u written to the workspace as the bf16 pair hi + lo
+// Nesterov blend u, and u written to the workspace as the pair bf16 hi + int8 lo
 // (transposed when tall), plus a partial sum of u^2 per block.  Blocks cover
 // kPrepRows x kPrepCols tiles of the caller's layout.
 constexpr int kPrepRows = 64, kPrepCols = 128;
