@@ -90,6 +90,28 @@ def test_bf16_extreme_magnitudes(scale):
     assert rel_fro(got, ref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("rows,cols,batch", [(1, 32768, 1), (32768, 1, 1), (8, 32768, 2)])
+def test_maximum_dimension(rows, cols, batch):
+    """The largest side the ABI accepts (32768): a single row / column is
+    normalised and stays a unit vector scaled by the chained scalar map."""
+    mats = [workloads.gaussian((rows, cols), 1.0, seed=900 + i, dtype=torch.bfloat16)
+            for i in range(batch)]
+    got = run_ns(mats)
+    for g, x in zip(got, mats):
+        assert rel_fro(g, oracle.newton_schulz(x.double().numpy())) <= TOL_BF16
+
+
+def test_rank_one_and_constant_matrices():
+    """All the mass in one singular value (sigma = 1 after normalisation):
+    rank-1 outer products and an all-equal matrix follow p(p(...p(1)))."""
+    g = torch.Generator().manual_seed(12)
+    u = torch.randn(384, 1, generator=g)
+    v = torch.randn(1, 640, generator=g)
+    for X in ((u @ v).to(torch.bfloat16), torch.full((256, 512), 0.5).to(torch.bfloat16)):
+        ref = oracle.newton_schulz(X.double().numpy())
+        assert rel_fro(run_ns([X])[0], ref) <= TOL_BF16
+
+
 def test_zero_matrix_gives_zero():
     for dt in (torch.bfloat16, torch.float32):
         got = run_ns([torch.zeros(64, 96, dtype=dt)])[0]

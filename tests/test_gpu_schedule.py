@@ -79,3 +79,12 @@ def test_empty_schedule_normalises():
     got = run([X], [])[0]
     ref = oracle.newton_schulz(X.double().numpy(), schedule=[])
     assert rel_fro(got, ref) <= 1e-2
+
+
+def test_schedule_on_a_tall_hard_spectrum():
+    """Transposed (tall) input with a log-uniform spectrum through a mixed schedule."""
+    schedule = [QUINTIC, QUINTIC, FLAT, QUINTIC, CUBIC]
+    X = workloads.hard_spectrum(1024, 384, seed=8, spike=True)
+    got = run([X], schedule)[0]
+    ref = oracle.newton_schulz(X.double().numpy(), schedule=[f32(t) for t in schedule])
+    assert rel_fro(got, ref) <= 3e-2
