@@ -92,7 +92,9 @@ def stage_work(shapes):
     g(2)+buf(4) read, buf(4) and the pair bf16 hi(2) + int8 lo(1) of u
     written = 13 B; apply W(4) + O as hi(2)+lo(1) read, W(4) written = 11 B;
     (fp32 and stand-alone paths) momentum 10 B, cast 10 B.  The per-matrix
-    scale reads one fp64 partial per prep block.
+    scale reads one fp64 partial per prep block.  The last step's fused
+    BX + apply reads X's pair (3 B) and W (4 B), writes W (4 B) per element
+    and reads B (2 B per element of the m x m matrix): HBM-bound.
     """
     elems = sum(r * c for r, c in shapes)
     g = sum(2 * min(r, c) ** 2 * max(r, c) for r, c in shapes)
@@ -100,6 +102,7 @@ def stage_work(shapes):
     prep_blocks = sum(-(-r // 64) * -(-c // 128) for r, c in shapes)
     return {
         "gram": ("tensor", g), "poly": ("tensor", p), "bx": ("tensor", g),
+        "bx_apply": ("hbm", 11 * elems + sum(2 * min(r, c) ** 2 for r, c in shapes)),
         "prep": ("hbm", 13 * elems), "scale": ("hbm", 8 * prep_blocks + 4 * len(shapes)),
         "flat": ("hbm", 10 * elems), "cast": ("hbm", 10 * elems), "out": ("hbm", 11 * elems),
     }

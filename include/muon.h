@@ -278,7 +278,8 @@ typedef enum {
   MUON_KERNEL_SUMS = 7, /* per-matrix sums of partials */
   MUON_KERNEL_PREP = 8, /* momentum + Nesterov blend written as the bf16 + int8 pair (transposing) */
   MUON_KERNEL_SCALE = 9, /* per-matrix 1 / (||u||_F + eps) */
-  MUON_KERNEL_KINDS = 10
+  MUON_KERNEL_BX_APPLY = 10, /* tensor cores: the last step's X' = aX + BX applied to W */
+  MUON_KERNEL_KINDS = 11
 } muon_kernel_kind;
 
 int muon_profile_begin(void);

@@ -57,7 +57,7 @@ SIGNATURES = {
 }
 
 #: muon_kernel_kind names, in enum order.
-KERNEL_KINDS = ["flat", "cast", "gram", "poly", "bx", "out", "simt", "sums", "prep", "scale"]
+KERNEL_KINDS = ["flat", "cast", "gram", "poly", "bx", "out", "simt", "sums", "prep", "scale", "bx_apply"]
 
 _lock = threading.Lock()
 _lib = None

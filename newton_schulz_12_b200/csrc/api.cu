@@ -341,7 +341,7 @@ void init_tc_params(tc::Params& P, int* status, float a, float b, float c) {
 #endif
 }
 
-int launch_tc(int epi, tc::Params& P, int sms, cudaStream_t s) {
+int launch_tc(int epi, tc::Params& P, int sms, cudaStream_t s, const tc::LaunchApply* apply = nullptr) {
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (g_inject) {
@@ -349,9 +349,61 @@ int launch_tc(int epi, tc::Params& P, int sms, cudaStream_t s) {
       g_inject = 0;
     }
   }
-  ProfScope prof(MUON_KERNEL_GRAM + epi, s);
-  CUDA_TRY(tc::launch(epi, P, sms / 2, s));  // one CTA pair per two SMs
+  ProfScope prof(epi == tc::kBxApply ? MUON_KERNEL_BX_APPLY : MUON_KERNEL_GRAM + epi, s);
+  CUDA_TRY(tc::launch(epi, P, sms / 2, s, apply));  // one CTA pair per two SMs
   P.inject = 0;
+  return MUON_OK;
+}
+
+// A caller's matrix: its layout (rows x cols), its iteration shape m x n
+// (m <= n, transposed when rows > cols), and its place in a shape group.
+struct MatInfo {
+  int rows, cols, m, n, transposed, group, index;
+};
+
+// The caller's weights, for the last step's fused apply (kBxApply).
+struct ApplySpec {
+  const std::vector<MatInfo>* mats = nullptr;
+  const std::vector<void*>* w = nullptr;  // fp32 W of matrix i, the caller's layout
+  float lr = 0.f, wd = 0.f;
+  std::vector<char> done;  // out: matrix i was applied by the GEMM epilogue
+};
+
+// fl(lr * scale) with scale = sqrt(max(1, rows / cols)), as the apply pass uses.
+float apply_ls(const MatInfo& M, float lr) {
+  const float ratio = static_cast<float>(M.rows) / static_cast<float>(M.cols);
+  const float scale = ratio > 1.0f ? sqrtf(ratio) : 1.0f;
+  return lr * scale;
+}
+
+// Table of the groups [g0, g1) of one kBxApply launch: every matrix whose W
+// rows are 16-byte strided (cols % 4 == 0) among the first kMaxApply gets a
+// tensor map over W and mode 1 (W = X) or 2 (W = X^T); the rest keep mode 0.
+int build_apply_table(const std::vector<NsGroup>& gs, size_t g0, size_t g1, ApplySpec& A,
+                      tc::LaunchApply& T) {
+  T.nmat = 0;
+  T.mat_base = gs[g0].mat_base;
+  T.lw = A.lr * A.wd;
+  int span = 0;
+  for (size_t gi = g0; gi < g1; ++gi) span += gs[gi].batch;
+  T.nmat = std::min(span, tc::kMaxApply);
+  for (int j = 0; j < T.nmat; ++j) T.mat[j] = tc::ApplyMat{0, 0.f};
+  const std::vector<MatInfo>& mats = *A.mats;
+  for (size_t i = 0; i < mats.size(); ++i) {
+    const MatInfo& M = mats[i];
+    if (M.group < static_cast<int>(g0) || M.group >= static_cast<int>(g1)) continue;
+    const int j = gs[M.group].mat_base + M.index - T.mat_base;
+    if (j >= T.nmat || M.cols % 4 != 0) continue;
+    const void* W = (*A.w)[i];
+    if (!M.transposed)
+      MUON_TRY(make_map(&T.w[j], W, 4, M.cols, M.rows, 1, M.cols, static_cast<uint64_t>(M.rows) * M.cols, 32,
+                        tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
+    else
+      MUON_TRY(make_map(&T.w[j], W, 4, M.cols, M.rows, 1, M.cols, static_cast<uint64_t>(M.rows) * M.cols, 32,
+                        64, CU_TENSOR_MAP_SWIZZLE_128B));
+    T.mat[j] = tc::ApplyMat{M.transposed ? 2 : 1, apply_ls(M, A.lr)};
+    A.done[i] = 1;
+  }
   return MUON_OK;
 }
 
@@ -359,9 +411,10 @@ int launch_tc(int epi, tc::Params& P, int sms, cudaStream_t s) {
 // the pair hi + lo; step t uses abc[3t .. 3t+2].  On entry each group's xb[0]
 // / xlo hold X0 / s with s = xscale[mat_base + i] per matrix (s = 1 when
 // xscale is null); on exit xb[T % 2] / xlo hold X_T (for T >= 1; X0 / s
-// itself for T = 0).
+// itself for T = 0) -- except for the matrices that `apply` (when given, and
+// T >= 1) marks done: their last step updated the caller's weights instead.
 int run_ns_bf16(std::vector<NsGroup>& gs, int steps, const float* abc, int* status, int sms,
-                cudaStream_t s, const float* xscale) {
+                cudaStream_t s, const float* xscale, ApplySpec* apply = nullptr) {
   if (steps <= 0 || gs.empty()) return MUON_OK;
   MUON_TRY(get_encoder());
   const float a = abc[0], b = abc[1], c = abc[2];
@@ -416,7 +469,13 @@ int run_ns_bf16(std::vector<NsGroup>& gs, int steps, const float* abc, int* stat
       bxt.a = abc[3 * t];
       MUON_TRY(launch_tc(tc::kGram, t == 0 ? gram0 : gram[cur], sms, s));
       MUON_TRY(launch_tc(tc::kPoly, poly, sms, s));
-      MUON_TRY(launch_tc(tc::kBx, bxt, sms, s));
+      if (apply && t == steps - 1) {
+        tc::LaunchApply table;
+        MUON_TRY(build_apply_table(gs, g0, g1, *apply, table));
+        MUON_TRY(launch_tc(tc::kBxApply, bxt, sms, s, &table));
+      } else {
+        MUON_TRY(launch_tc(tc::kBx, bxt, sms, s));
+      }
       cur ^= 1;
     }
   }
@@ -491,10 +550,6 @@ int run_ns_fp32(std::vector<NsGroup>& gs, int steps, const float* abc, cudaStrea
 }
 
 bool finite(float v) { return std::isfinite(v); }
-
-struct MatInfo {
-  int rows, cols, m, n, transposed, group, index;
-};
 
 // Group matrices by (m, n) = (min, max); larger n first (longer K in kGram).
 void group_shapes(const std::vector<std::pair<int, int>>& shapes, std::vector<MatInfo>& mats,
@@ -736,30 +791,37 @@ size_t bf16_layout(const std::vector<MatInfo>& mats, std::vector<NsGroup>& group
 int run_bf16_path(const std::vector<MatInfo>& mats, std::vector<NsGroup>& groups,
                   const BfLayout& L, const std::vector<const void*>& src,
                   const std::vector<float*>& bufs, int src_kind, float beta, int nesterov,
-                  const float* abc, int steps, int* status, int sms, cudaStream_t s) {
+                  const float* abc, int steps, int* status, int sms, cudaStream_t s,
+                  ApplySpec* apply = nullptr) {
   std::vector<int> pb, pc;
   MUON_TRY(launch_prep_chunked(mats, groups, src, bufs, src_kind, beta, nesterov, L.partials, pb,
                                pc, s));
   MUON_TRY(launch_scale_chunked(mats, groups, L.partials, pb, pc, L.xscale, s));
-  return run_ns_bf16(groups, steps, abc, status, sms, s, L.xscale);
+  return run_ns_bf16(groups, steps, abc, status, sms, s, L.xscale, apply);
 }
 
 // mode 0: apply into W; 1: bf16 write-back; 2: fp32 write-back.  O of matrix i
-// is read from its group's result (X layout, transposed back).
+// is read from its group's result (X layout, transposed back).  Matrices that
+// `done` marks (already applied by the last GEMM) are left out.
 int launch_out_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGroup>& groups,
                        const std::vector<Result>& res, const std::vector<void*>& ys, int mode,
-                       float lr, float wd, cudaStream_t s, const float* oscale = nullptr) {
-  const int count = static_cast<int>(mats.size());
+                       float lr, float wd, cudaStream_t s, const float* oscale = nullptr,
+                       const std::vector<char>* done = nullptr) {
+  std::vector<int> todo;
+  for (int i = 0; i < static_cast<int>(mats.size()); ++i)
+    if (!done || !(*done)[i]) todo.push_back(i);
+  const int count = static_cast<int>(todo.size());
   for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
     const int i1 = std::min(count, i0 + ew::kMaxMats);
     ew::OutParams op{};
     op.mode = mode;
     op.lw = lr * wd;
     int tiles = 0;
-    for (int i = i0; i < i1; ++i) {
+    for (int t = i0; t < i1; ++t) {
+      const int i = todo[t];
       const MatInfo& M = mats[i];
       const NsGroup& G = groups[M.group];
-      ew::OutMat& O = op.mat[i - i0];
+      ew::OutMat& O = op.mat[t - i0];
       O.y = ys[i];
       const long long roff = static_cast<long long>(M.index) * G.m * G.ldn;
       const Result& R = res[M.group];
@@ -772,9 +834,7 @@ int launch_out_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGro
       O.ld = G.ldn;
       O.tiles_c = (M.cols + ew::kTile - 1) / ew::kTile;
       O.tile_begin = tiles;
-      const float ratio = static_cast<float>(M.rows) / static_cast<float>(M.cols);
-      const float scale = ratio > 1.0f ? sqrtf(ratio) : 1.0f;
-      O.ls = lr * scale;
+      O.ls = apply_ls(M, lr);
       O.oscale = oscale ? oscale + G.mat_base + M.index : nullptr;
       O.vec = (M.cols % 8 == 0) && (G.ldn % 8 == 0) && aligned16(ys[i]);
       tiles += ((M.rows + ew::kTile - 1) / ew::kTile) * O.tiles_c;
@@ -1055,12 +1115,20 @@ int muon_step(int count, float* const* params, const void* const* grads,
   std::vector<const void*> gsrc(grads, grads + count);
   std::vector<float*> bufs(momentum_bufs, momentum_bufs + count);
   const std::vector<float> abc = constant_schedule(kCoefA, kCoefB, kCoefC, steps);
+  std::vector<void*> ys(params, params + count);
+  // the last step applies the update to W in its epilogue where it can
+  ApplySpec apply;
+  apply.mats = &mats;
+  apply.w = &ys;
+  apply.lr = lr;
+  apply.wd = wd;
+  apply.done.assign(count, 0);
   MUON_TRY(run_bf16_path(mats, groups, L, gsrc, bufs, ew::kFromMomentum, beta, nesterov,
-                         abc.data(), steps, ws->status, dev.sms, s));
+                         abc.data(), steps, ws->status, dev.sms, s, &apply));
   std::vector<Result> res;
   for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
-  std::vector<void*> ys(params, params + count);
-  MUON_TRY(launch_out_chunked(mats, groups, res, ys, 0, lr, wd, s, steps == 0 ? L.xscale : nullptr));
+  MUON_TRY(launch_out_chunked(mats, groups, res, ys, 0, lr, wd, s, steps == 0 ? L.xscale : nullptr,
+                              &apply.done));
   return MUON_OK;
 }
 

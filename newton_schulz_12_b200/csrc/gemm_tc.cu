@@ -8,6 +8,10 @@
 //   kGram  A  = X X^T            tiles on or above the diagonal, mirrored
 //   kPoly  B  = b A + c A A      A symmetric, so A A = A A^T: same tiling
 //   kBx    X' = a X + B X        X carried as the pair bf16 hi + int8 residual
+//   kBxApply  the last step's kBx: X_T goes straight into the caller's
+//          weights, W' = (W - lw W) - ls X_T, W read and written by bulk
+//          tensor copies next to X's epilogue chunk (the update is never
+//          stored as X_T and read back by a separate pass)
 //
 // CTAs run in clusters of two on an SM pair, one cluster per pair tile of
 // 256 x 256 outputs at a time, persistent over a static tile stride.  One
@@ -78,24 +82,44 @@ constexpr size_t kMaxSmem = 232448;                         // 227 KiB per CTA o
 #ifndef MUON_BX_SLOTS
 #define MUON_BX_SLOTS 4
 #endif
+// kBxApply slots also hold the chunk's 32 KiB of W: fewer stages and slots fit
+#ifndef MUON_BXA_STAGES
+#define MUON_BXA_STAGES 3
+#endif
+#ifndef MUON_BXA_SLOTS
+#define MUON_BXA_SLOTS 2
+#endif
+
+// kBx and kBxApply share the operands, the tiling and X's epilogue chunks.
+template <int EPI>
+__host__ __device__ constexpr bool is_bx() {
+  return EPI == kBx || EPI == kBxApply;
+}
 
 template <int EPI>
 struct Cfg {
   static constexpr int kStages =
-      (EPI == kGram) ? MUON_GRAM_STAGES : (EPI == kPoly ? MUON_POLY_STAGES : MUON_BX_STAGES);
+      (EPI == kGram) ? MUON_GRAM_STAGES
+                     : (EPI == kPoly ? MUON_POLY_STAGES : (EPI == kBx ? MUON_BX_STAGES : MUON_BXA_STAGES));
   // epilogue operand ring of kSlots chunks (kGram: none, the count only sizes barriers)
   // kBx slot: the hi and lo bf16 chunks of X (8 KiB each); kPoly slot: A's chunk
-  static constexpr int kSlots = (EPI == kBx) ? MUON_BX_SLOTS : MUON_POLY_SLOTS;
+  static constexpr int kSlots =
+      (EPI == kBx) ? MUON_BX_SLOTS : (EPI == kBxApply ? MUON_BXA_SLOTS : MUON_POLY_SLOTS);
   // kBx works on 64-column chunks (128-byte rows in global memory), the
   // symmetric kernels on kSymChunk-column chunks
-  static constexpr int kCW = (EPI == kBx) ? 2 * kChunk : kSymChunk;
+  static constexpr int kCW = is_bx<EPI>() ? 2 * kChunk : kSymChunk;
   static constexpr int kNCh = BN / kCW;  // per tile
   // bytes of one bf16 chunk, 128 rows x kCW columns
   static constexpr uint32_t kChunkBytes = BM * kCW * 2;
   // kBx slot: hi (bf16, 128 rows x 128 B) then lo (int8, 128 rows x 64 B);
-  // kPoly slot: A's chunk
-  static constexpr uint32_t kSlotBytes = (EPI == kBx) ? 3 * kChunkBf16 : (EPI == kPoly ? kChunkBytes : 0);
+  // kBxApply: then W's 128 x 64 fp32 chunk (32 KiB); kPoly slot: A's chunk
   static constexpr uint32_t kLoOff = 2 * kChunkBf16;
+  static constexpr uint32_t kWOff = 3 * kChunkBf16;
+  static constexpr uint32_t kWBytes = BM * 64 * 4;
+  static constexpr uint32_t kSlotBytes = (EPI == kBx)        ? 3 * kChunkBf16
+                                         : (EPI == kBxApply) ? 3 * kChunkBf16 + kWBytes
+                                         : (EPI == kPoly)    ? kChunkBytes
+                                                             : 0;
   static constexpr uint32_t kSlotsBytes = kSlotBytes * kSlots;
   // kGram / kPoly output staging: kSBuf pairs of a direct [128][kCW] and a
   // mirrored [kCW][128] chunk, laid out as d0 .. d(kSBuf-1), m0 .. m(kSBuf-1).
@@ -103,9 +127,9 @@ struct Cfg {
   // aliases d0 d1 and m0 m1 (32-column chunks) or d0 and d1 (64-column).
   static constexpr int kSBuf = (EPI == kGram) ? MUON_GRAM_SBUF : (EPI == kPoly ? MUON_POLY_SBUF : 2);
   static_assert(kSBuf >= 2, "the diagonal block takes staging pairs 0 and 1");
-  static constexpr uint32_t kStagingBytes = (EPI == kBx) ? 0 : 2 * kSBuf * kChunkBytes;
+  static constexpr uint32_t kStagingBytes = is_bx<EPI>() ? 0 : 2 * kSBuf * kChunkBytes;
   // ready barriers: kBx one per slot; kGram / kPoly one per staging pair + the block
-  static constexpr int kReady = (EPI == kBx) ? kSlots : kSBuf + 1;
+  static constexpr int kReady = is_bx<EPI>() ? kSlots : kSBuf + 1;
   static constexpr uint32_t kRingBytes = kStages * kStageBytes;
   // full, empty, tfull x2, tempty x2, drain, efull, ready, sfree, econs
   static constexpr int kNumBars = 2 * kStages + 5 + 2 * kSlots + kReady + kSBuf;
@@ -116,11 +140,15 @@ struct Cfg {
 static_assert(Cfg<kGram>::kSmem <= kMaxSmem, "kGram shared memory");
 static_assert(Cfg<kPoly>::kSmem <= kMaxSmem, "kPoly shared memory");
 static_assert(Cfg<kBx>::kSmem <= kMaxSmem, "kBx shared memory");
+static_assert(Cfg<kBxApply>::kSmem <= kMaxSmem, "kBxApply shared memory");
+static_assert(Cfg<kBxApply>::kWOff % 1024 == 0 && Cfg<kBxApply>::kSlotBytes % 1024 == 0,
+              "W chunks start on the 1 KiB boundary of the 128-byte swizzle");
 
 size_t smem_bytes(int epi) {
   switch (epi) {
     case kGram: return Cfg<kGram>::kSmem;
     case kPoly: return Cfg<kPoly>::kSmem;
+    case kBxApply: return Cfg<kBxApply>::kSmem;
     default: return Cfg<kBx>::kSmem;
   }
 }
@@ -142,7 +170,7 @@ __device__ __forceinline__ TileCoord decode_tile(const Params& p, int t, int ran
   c.b = local / G.tiles_per_mat;
   int r = local - c.b * G.tiles_per_mat;
   int tm2;
-  if (EPI == kBx) {
+  if (is_bx<EPI>()) {
     // column panel outer, row panel inner: neighbouring pairs share X's panel
     c.tn = r / G.tiles_m;
     tm2 = r - c.tn * G.tiles_m;
@@ -164,9 +192,9 @@ enum ChunkKind : int { kSkip = 0, kUpper = 1, kDiag = 2, kPlain = 3 };
 
 template <int EPI>
 __device__ __forceinline__ int chunk_kind(const Group& G, int tm, int col0) {
-  constexpr int W = (EPI == kBx) ? 2 * kChunk : kSymChunk;
+  constexpr int W = is_bx<EPI>() ? 2 * kChunk : kSymChunk;
   // a CTA whose rows lie wholly below the matrix stores nothing
-  if (EPI == kBx) return (col0 < G.n && tm * BM < G.m) ? kPlain : kSkip;
+  if (is_bx<EPI>()) return (col0 < G.n && tm * BM < G.m) ? kPlain : kSkip;
   if (col0 >= G.m) return kSkip;
   const int d0 = tm * BM;
   if (col0 + W <= d0) return kSkip;  // strictly below the diagonal block
@@ -212,11 +240,32 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
 // Bytes of one K stage over BOTH CTAs of the pair (armed on the leader's barrier).
 template <int EPI>
 __device__ __forceinline__ uint32_t pair_stage_bytes(const Group& G, int tn) {
-  if (EPI != kBx) return 2 * kStageBytes;  // out-of-range rows are zero-filled, still counted
+  if (!is_bx<EPI>()) return 2 * kStageBytes;  // out-of-range rows are zero-filled, still counted
   // kBx: 64-column boxes of X wholly beyond n are not copied
   const int left = G.n - tn * BN;
   const int boxes = left >= BN ? BN / 64 : (left + 63) / 64;
   return 2 * kTileBytesP + static_cast<uint32_t>(boxes) * 8192u;
+}
+
+// Table entry of matrix b of group G in a kBxApply launch, or -1 (mode 0).
+template <int N>
+__device__ __forceinline__ int apply_entry(const ApplyTable<N>& t, const Group& G, int b) {
+  const int j = G.mat_base + b - t.mat_base;
+  return (j >= 0 && j < t.nmat && t.mat[j].mode != 0) ? j : -1;
+}
+
+// Bytes of W's chunk at (row0, col0) of X that the loader copies (boxes
+// wholly outside W are neither copied nor stored).
+__device__ __forceinline__ uint32_t w_chunk_bytes(int mode, const Group& G, int row0, int col0) {
+  if (mode == 1) return (col0 + 32 < G.n ? 2u : 1u) * (BM * 32 * 4);
+  uint32_t q = 0;
+  for (int i = 0; i < 4; ++i) q += (row0 + 32 * i < G.m) ? 1u : 0u;
+  return q * (64 * 32 * 4);
+}
+
+// W' = (W - lw W) - ls O, each operation rounded to nearest in fp32.
+__device__ __forceinline__ float apply_w(float w, float o, float lw, float ls) {
+  return __fsub_rn(__fsub_rn(w, __fmul_rn(lw, w)), __fmul_rn(ls, o));
 }
 
 #ifdef MUON_TRACE
@@ -239,8 +288,11 @@ constexpr int threads_of() {
 }
 
 template <int EPI>
+using TableOf = ApplyTable<EPI == kBxApply ? kMaxApply : 1>;
+
+template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1)
-    gemm_kernel(const __grid_constant__ Params p) {
+    gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ TableOf<EPI> tab) {
   using C = Cfg<EPI>;
   constexpr int S = C::kStages;
   constexpr int K = C::kSlots;
@@ -298,7 +350,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
       mbar_init(efull_bar(s), 1);
       // kPoly: every compute thread has read the slot; kBx: the slot's stores
       // have read it (one arrival from the store thread)
-      mbar_init(econs_bar(s), EPI == kBx ? 1 : kEpiThreads);
+      mbar_init(econs_bar(s), is_bx<EPI>() ? 1 : kEpiThreads);
     }
     for (int s = 0; s < C::kReady; ++s) mbar_init(ready_bar(s), kEpiThreads);
     for (int b = 0; b < NB; ++b) mbar_init(sfree_bar(b), 1);
@@ -363,7 +415,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             const uint32_t dQ = dP + kTileBytesP;
             const int qcol = tc.tn * BN + rank * BNH;  // this CTA's half of the columns
             tma_load_3d_pair(dP, &M.p, fbar, kb * BK, tc.tm * BM, tc.b);
-            if (EPI == kBx) {
+            if (is_bx<EPI>()) {
               for (int c = 0; c < BNH / 64; ++c)
                 if (qcol + c * 64 < G.n)
                   tma_load_3d_pair(dQ + c * 8192, &M.q, fbar, qcol + c * 64, kb * BK, tc.b);
@@ -388,7 +440,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_bf16(PM, BN, EPI == kBx);
+      constexpr uint32_t idesc = idesc_bf16(PM, BN, is_bx<EPI>());
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -412,7 +464,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t adesc = sdesc_sw128(aP + kk * 32, 16, 1024);
-            const uint64_t bdesc = (EPI == kBx) ? sdesc_sw128(aQ + kk * 2048, 8192, 1024)
+            const uint64_t bdesc = is_bx<EPI>() ? sdesc_sw128(aQ + kk * 2048, 8192, 1024)
                                                 : sdesc_sw128(aQ + kk * 32, 16, 1024);
             tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
@@ -484,16 +536,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
           const int col0 = tc.tn * BN + (s % NCH) * CW;
           const int row0 = tc.tm * BM;
           const Group& G = p.grp[tc.g];
-          const bool skip = (EPI == kBx) ? !(col0 < G.n && row0 < G.m)
+          const bool skip = is_bx<EPI>() ? !(col0 < G.n && row0 < G.m)
                                          : chunk_kind<EPI>(G, tc.tm, col0) == kSkip;
           if (skip) {
             mbar_arrive(efull_bar(slot));
           } else {
             const uint32_t dst = slots_u32 + slot * C::kSlotBytes;
-            mbar_arrive_expect_tx(efull_bar(slot), C::kSlotBytes);
+            const int j = (EPI == kBxApply) ? apply_entry(tab, G, tc.b) : -1;
+            const int mode = j >= 0 ? tab.mat[j].mode : 0;
+            const uint32_t bytes = is_bx<EPI>() ? 3 * kChunkBf16 : C::kSlotBytes;
+            mbar_arrive_expect_tx(efull_bar(slot), bytes + (mode ? w_chunk_bytes(mode, G, row0, col0) : 0u));
             tma_load_3d(dst, &p.map[tc.g].e, efull_bar(slot), col0, row0, tc.b);
-            if (EPI == kBx)  // lo half of X next to its hi half
+            if (is_bx<EPI>())  // lo half of X next to its hi half
               tma_load_3d(dst + C::kLoOff, &p.map[tc.g].mt, efull_bar(slot), col0, row0, tc.b);
+            if (mode == 1) {  // W as X: two 32-column boxes of 128 rows
+              for (int h = 0; h < 2; ++h)
+                if (col0 + 32 * h < G.n)
+                  tma_load_3d(dst + C::kWOff + h * (BM * 32 * 4), &tab.w[j], efull_bar(slot), col0 + 32 * h,
+                              row0, 0);
+            } else if (mode == 2) {  // W = X^T: four 32-column boxes of 64 rows
+              for (int q = 0; q < 4; ++q)
+                if (row0 + 32 * q < G.m)
+                  tma_load_3d(dst + C::kWOff + q * (64 * 32 * 4), &tab.w[j], efull_bar(slot), row0 + 32 * q,
+                              col0, 0);
+            }
           }
         };
         if (loads_here)
@@ -528,13 +594,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
           const int row0 = tc.tm * BM;
           const int col0 = tc.tn * BN + c * CW;
           const int kind = chunk_kind<EPI>(G, tc.tm, col0);
-          if (EPI == kBx) {
+          if (is_bx<EPI>()) {
             const int slot = s % K;
             mbar_wait(ready_bar(slot), (s / K) & 1, ctl);
             if (kind != kSkip) {  // never start a store wholly outside the matrix
               const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
-              tma_store_3d(&M.d, hs, col0, row0, tc.b);                       // hi' -> the other hi buffer
-              tma_store_3d(&M.mt, hs + C::kLoOff, col0, row0, tc.b);          // lo' -> lo, in place
+              const int j = (EPI == kBxApply) ? apply_entry(tab, G, tc.b) : -1;
+              const int mode = j >= 0 ? tab.mat[j].mode : 0;
+              if (mode == 1) {
+                for (int h = 0; h < 2; ++h)
+                  if (col0 + 32 * h < G.n) tma_store_3d(&tab.w[j], hs + C::kWOff + h * (BM * 32 * 4), col0 + 32 * h, row0, 0);
+              } else if (mode == 2) {
+                for (int q = 0; q < 4; ++q)
+                  if (row0 + 32 * q < G.m) tma_store_3d(&tab.w[j], hs + C::kWOff + q * (64 * 32 * 4), row0 + 32 * q, col0, 0);
+              } else {
+                tma_store_3d(&M.d, hs, col0, row0, tc.b);               // hi' -> the other hi buffer
+                tma_store_3d(&M.mt, hs + C::kLoOff, col0, row0, tc.b);  // lo' -> lo, in place
+              }
               bulk_commit();
               asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");  // chunk s-1 drained
             } else {
@@ -619,7 +695,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
         mbar_wait(tfull_bar(acc), acc_phase, ctl);
         tc_fence_after();
         if (leader) TRACE(k, 4);
-        if (EPI == kBx) {
+        if (is_bx<EPI>()) {
+          const int j = (EPI == kBxApply) ? apply_entry(tab, G, tc.b) : -1;
+          const int mode = j >= 0 ? tab.mat[j].mode : 0;
+          const float lsc = j >= 0 ? tab.mat[j].ls : 0.f;  // fl(lr * scale)
           // 64-column chunks c: thread (r, hf) takes accumulator columns
           // 32 hf .. +31 of the chunk, i.e. 16-byte units 4 hf .. 4 hf + 3 of
           // its 128-byte row in the slot's hi and lo tiles (128-byte swizzle)
@@ -669,9 +748,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                 pair_decode8(h4, l2, x);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) x[e] = fmaf(p.a, x[e], v[8 * uu + e]) * xs;
-                pair_encode8(x, h4, l2);
-                st_shared_v4(ha, h4.x, h4.y, h4.z, h4.w);
-                asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(la), "r"(l2.x), "r"(l2.y) : "memory");
+                if (EPI == kBxApply && mode == 1) {
+                  // W's row sr, columns 32 hf + 8 uu ..: 16-byte units 2 uu, 2 uu + 1
+                  // of row sr of box hf (128-byte swizzle)
+                  const uint32_t wb = hs + C::kWOff + hf * (BM * 32 * 4);
+#pragma unroll
+                  for (int h = 0; h < 2; ++h) {
+                    const uint32_t wa = wb + sw128(sr, 2 * uu + h);
+                    uint32_t w[4];
+                    ld_shared_v4(wa, w[0], w[1], w[2], w[3]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                      w[e] = __float_as_uint(apply_w(__uint_as_float(w[e]), x[4 * h + e], tab.lw, lsc));
+                    st_shared_v4(wa, w[0], w[1], w[2], w[3]);
+                  }
+                } else if (EPI == kBxApply && mode == 2) {
+                  // W = X^T: X's column 32 hf + 8 uu + e is row 32 hf + 8 uu + e of
+                  // box (warp & 3), whose 32 columns are this lane quarter's rows
+                  const uint32_t wb = hs + C::kWOff + (warp & 3) * (64 * 32 * 4);
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) {
+                    const int row = 32 * hf + 8 * uu + e;
+                    const uint32_t wa =
+                        wb + static_cast<uint32_t>(row * 128 + ((((lane >> 2) ^ row) & 7) << 4) + (lane & 3) * 4);
+                    float w;
+                    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(w) : "r"(wa) : "memory");
+                    w = apply_w(w, x[e], tab.lw, lsc);
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(wa), "f"(w) : "memory");
+                  }
+                } else {
+                  pair_encode8(x, h4, l2);
+                  st_shared_v4(ha, h4.x, h4.y, h4.z, h4.w);
+                  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(la), "r"(l2.x), "r"(l2.y) : "memory");
+                }
               }
               fence_async_smem();
             }
@@ -825,7 +934,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
 }
 
 template <int EPI>
-static cudaError_t launch_one(const Params& p, int max_pairs, cudaStream_t stream) {
+static cudaError_t launch_one(const Params& p, const TableOf<EPI>& tab, int max_pairs, cudaStream_t stream) {
   static thread_local int configured_device = -1;
   static thread_local int resident_pairs = 0;
   int dev = 0;
@@ -849,17 +958,21 @@ static cudaError_t launch_one(const Params& p, int max_pairs, cudaStream_t strea
   }
   int pairs = p.total_tiles < max_pairs ? p.total_tiles : max_pairs;
   if (resident_pairs > 0 && pairs > resident_pairs) pairs = resident_pairs;
-  gemm_kernel<EPI><<<2 * pairs, threads_of<EPI>(), smem, stream>>>(p);
+  gemm_kernel<EPI><<<2 * pairs, threads_of<EPI>(), smem, stream>>>(p, tab);
   return cudaGetLastError();
 }
 
-cudaError_t launch(int epi, const Params& p, int max_pairs, cudaStream_t stream) {
+cudaError_t launch(int epi, const Params& p, int max_pairs, cudaStream_t stream, const LaunchApply* apply) {
   if (p.total_tiles <= 0) return cudaSuccess;
   if (max_pairs < 1) max_pairs = 1;
+  const ApplyTable<1> none{};
   switch (epi) {
-    case kGram: return launch_one<kGram>(p, max_pairs, stream);
-    case kPoly: return launch_one<kPoly>(p, max_pairs, stream);
-    case kBx: return launch_one<kBx>(p, max_pairs, stream);
+    case kGram: return launch_one<kGram>(p, none, max_pairs, stream);
+    case kPoly: return launch_one<kPoly>(p, none, max_pairs, stream);
+    case kBx: return launch_one<kBx>(p, none, max_pairs, stream);
+    case kBxApply:
+      if (!apply) return cudaErrorInvalidValue;
+      return launch_one<kBxApply>(p, *apply, max_pairs, stream);
   }
   return cudaErrorInvalidValue;
 }

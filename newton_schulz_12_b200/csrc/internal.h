@@ -27,7 +27,9 @@ constexpr int kThreads = 352;        // warp 0 copies, warp 1 MMAs, warps 2-9 ep
                                      // warp 10 epilogue loads and stores
 constexpr int kEpiThreads = 256;     // warps 2-9
 
-enum Epi : int { kGram = 0, kPoly = 1, kBx = 2 };
+// kBxApply: the last step's kBx, whose epilogue also applies the result to
+// the caller's weights (ApplyTable) instead of writing X_T.
+enum Epi : int { kGram = 0, kPoly = 1, kBx = 2, kBxApply = 3 };
 
 // Work unit: a PM x BN pair tile of D, rows split between the two CTAs of a
 // cluster (CTA rank r owns rows [PM*tm2 + BM*r, +BM)).
@@ -71,6 +73,29 @@ struct Params {
   unsigned long long* trace;  // timestamps (only recorded in builds with MUON_TRACE)
 };
 
+// Final-step apply (kBxApply): per matrix of the launch, either X_T is written
+// as the pair (mode 0; the apply runs as its own pass later), or the caller's
+// fp32 W is updated in place from O = X_T, W' = (W - lw W) - ls O, with W
+// read and written through its own tensor map: mode 1, W has X's layout
+// (box 32 x 128, two per 64-column chunk); mode 2, W = X^T (a tall matrix;
+// box 32 x 64, four per chunk).
+constexpr int kMaxApply = 96;  // matrices per launch with a table entry
+
+struct ApplyMat {
+  int mode;  // 0, 1 or 2 as above
+  float ls;  // fl(lr * scale)
+};
+
+template <int N>
+struct ApplyTable {
+  CUtensorMap w[N];
+  ApplyMat mat[N];
+  int nmat;      // entries in use; matrices past them take mode 0
+  int mat_base;  // Group::mat_base value of entry 0
+  float lw;      // fl(lr * wd)
+};
+using LaunchApply = ApplyTable<kMaxApply>;
+
 // Trace layout (MUON_TRACE builds): per CTA < kTraceCtas, per tile < kTraceTiles,
 // kTraceSlots %globaltimer stamps: 0 copier first issue, 1 copier last issue,
 // 2 MMA start, 3 MMA last commit, 4 epilogue start, 5..11 chunk starts, 12
@@ -88,8 +113,10 @@ inline int sym_tiles(int m) {
 }
 
 size_t smem_bytes(int epi);
-// `max_pairs` bounds the number of CTA pairs (clusters) of the persistent grid.
-cudaError_t launch(int epi, const Params& p, int max_pairs, cudaStream_t stream);
+// `max_pairs` bounds the number of CTA pairs (clusters) of the persistent grid;
+// `apply` is the table of a kBxApply launch (ignored by the other kinds).
+cudaError_t launch(int epi, const Params& p, int max_pairs, cudaStream_t stream,
+                   const LaunchApply* apply = nullptr);
 
 }  // namespace tc
 

@@ -101,6 +101,43 @@ def test_scaled_set_sampled():
     check_step(st, 0, wd=0.01, check=[0, 4, 5, 142, 143])
 
 
+# The last step's BX applies its result to W in the GEMM epilogue.  These
+# shapes cover W with X's layout (wide, square), W = X^T (tall), ragged edges
+# both ways, a one-row X, and W rows that are not 16-byte strided (cols % 4 !=
+# 0: written as X_T and applied by the separate pass) -- the same shape group
+# holding both kinds, and more shape groups than one launch takes.
+APPLY_MIX = [(300, 1000), (1000, 300), (256, 256), (130, 68), (68, 130), (77, 5), (5, 77),
+             (4, 12), (12, 4), (1, 40), (40, 1)]
+
+
+def test_fused_apply_layouts_and_edges():
+    st = State(APPLY_MIX)
+    for step in range(2):
+        check_step(st, step)
+
+
+def test_fused_apply_weight_decay_dominant():
+    """lr * wd = 0.2: the decay term dominates W' - W, so a missing or wrong
+    decay in the fused epilogue breaks the tolerance."""
+    st = State(APPLY_MIX)
+    check_step(st, 0, lr=0.01, wd=20.0)
+
+
+@pytest.mark.parametrize("steps", [1, 2])
+def test_fused_apply_few_steps(steps):
+    """With one step the fused launch is also the one that folds in 1 / ||u||."""
+    st = State(APPLY_MIX[:5])
+    check_step(st, 0, steps=steps)
+
+
+def test_fused_apply_table_overflow():
+    """104 matrices in one launch: the first 96 (wide and tall alternating)
+    are applied in the epilogue, the rest written as X_T and applied by the
+    separate pass."""
+    st = State([(64, 192), (192, 64)] * 52)
+    check_step(st, 0, wd=0.5)
+
+
 def test_momentum_stage_bit_exact_and_sumsq():
     shapes = [(768, 768), (333, 77), (5, 3), (1, 1)]
     _, Gs = workloads.muon_set(shapes, step=0)
