@@ -163,7 +163,12 @@ int muon_ns_orthogonalize_static(int batch, int m, int n, void* const* X_ptrs, f
  * momentum_bufs  host array of device pointers to fp32 buf (r x s).
  * shapes         host array of 2*count int64: rows, cols of each matrix.
  * Matrices of equal (min, max) dimensions are batched into one group; any mix
- * of shapes is accepted.  Returns MUON_OK or a negative muon_status.
+ * of shapes is accepted.  With steps >= 1 the update of a weight whose column
+ * count is a multiple of 4 (among the first 96 matrices of each launch of the
+ * last step) is applied inside the last Newton-Schulz GEMM, with O its fp32
+ * value; the others are applied by a separate pass from O carried as the
+ * bf16 + int8 pair.  Both stay within the same tolerance of the definition.
+ * Returns MUON_OK or a negative muon_status.
  */
 int muon_step(int count, float* const* params, const void* const* grads,
               float* const* momentum_bufs, const int64_t* shapes, float beta, int nesterov,
