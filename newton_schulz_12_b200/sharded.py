@@ -1,0 +1,167 @@
+"""Muon over a data-parallel group: one process per GPU, torch.distributed.
+
+Every rank holds the full set of hidden matrices W.  A step over the group is
+the single-GPU step applied to the group-averaged gradients, with the work
+split by matrix ("The NanoGPT speedrun", record #3: the Newton-Schulz
+orthogonalisation of one matrix is independent of every other):
+
+1. gradients are averaged and delivered to their owner only -- one
+   reduce-scatter per bucket over a flat buffer laid out by owner;
+2. each owner runs the Muon step (momentum, Newton-Schulz, apply) on the
+   matrices it owns and keeps their momentum buffers;
+3. the updated weights are all-gathered in place, so that every rank again
+   holds the full set.
+
+Bucket b's all-gather is issued asynchronously right after its local step,
+so it runs on the communication stream while bucket b+1 is orthogonalised.
+
+Ownership: the matrices are split into ``buckets`` contiguous runs in the
+caller's order; inside a bucket each matrix, longest first by Newton-Schulz
+FLOPs T(4 m^2 n + 2 m^3) (m <= n; ties by index), goes to the least-loaded
+rank (ties to the lower rank), so every bucket's all-gather is balanced too.
+
+Storage: per bucket one flat fp32 W buffer and one flat gradient buffer of
+``world`` equal slots, slot r holding the matrices rank r owns (each start
+padded to 64 elements, 16-byte aligned as the C ABI requires).  ``params``
+and ``grads`` are views into them: the caller writes its gradients into
+``grads`` and reads the weights from ``params``.
+"""
+from __future__ import annotations
+
+import torch
+
+_ALIGN = 64  # elements; every matrix view starts 256-byte aligned
+
+
+def ns_flops(shape, steps=5):
+    """Nominal Newton-Schulz FLOPs of one (r x c) matrix: T (4 m^2 n + 2 m^3), m <= n."""
+    m, n = sorted((int(shape[0]), int(shape[1])))
+    return steps * (4 * m * m * n + 2 * m ** 3)
+
+
+def plan_ownership(shapes, world, buckets=2, steps=5):
+    """Owner rank of every matrix and the [begin, end) index range of every bucket."""
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    k = len(shapes)
+    nb = max(1, min(int(buckets), k)) if k else 0
+    bounds = [round(b * k / nb) for b in range(nb + 1)] if nb else [0]
+    owner = [0] * k
+    for b in range(nb):
+        load = [0] * world
+        idx = range(bounds[b], bounds[b + 1])
+        for i in sorted(idx, key=lambda i: (-ns_flops(shapes[i], steps), i)):
+            r = min(range(world), key=lambda q: (load[q], q))
+            owner[i] = r
+            load[r] += ns_flops(shapes[i], steps)
+    return owner, [(bounds[b], bounds[b + 1]) for b in range(nb)]
+
+
+def _round_up(x, a):
+    return (x + a - 1) // a * a
+
+
+class ShardedMuon:
+    """Muon step over the ranks of ``group`` (the default group when None).
+
+    ``local_step(params, grads, momentum_bufs, beta, nesterov, lr, wd, steps)``
+    updates the owned matrices in place; by default it is this package's
+    ``muon_step`` (bf16 gradients on the CUDA device), prepared once per
+    bucket.  Without an initialised process group the object runs as a
+    single rank.
+    """
+
+    def __init__(self, shapes, *, device=None, group=None, buckets=2, beta=0.95, nesterov=True,
+                 lr=0.05, wd=0.0, steps=5, grad_dtype=torch.bfloat16, local_step=None):
+        import torch.distributed as dist
+        self.dist = dist if dist.is_available() and dist.is_initialized() else None
+        self.group = group
+        self.world = self.dist.get_world_size(group) if self.dist else 1
+        self.rank = self.dist.get_rank(group) if self.dist else 0
+        self.shapes = [(int(r), int(c)) for r, c in shapes]
+        self.hyper = (float(beta), bool(nesterov), float(lr), float(wd), int(steps))
+        self.device = torch.device(device) if device is not None else torch.device("cpu")
+        self.owner, self.bucket_ranges = plan_ownership(self.shapes, self.world, buckets, steps)
+        self._nccl = bool(self.dist) and self.dist.get_backend(group) == "nccl"
+
+        self.params = [None] * len(self.shapes)
+        self.grads = [None] * len(self.shapes)
+        self.momentum = [None] * len(self.shapes)
+        self._buckets = []
+        for lo, hi in self.bucket_ranges:
+            offs, used = {}, [0] * self.world
+            for i in range(lo, hi):
+                r = self.owner[i]
+                offs[i] = used[r]
+                used[r] = _round_up(used[r] + self.shapes[i][0] * self.shapes[i][1], _ALIGN)
+            slot = max(max(used), _ALIGN)
+            W = torch.zeros(self.world * slot, dtype=torch.float32, device=self.device)
+            G = torch.zeros(self.world * slot, dtype=grad_dtype, device=self.device)
+            owned = []
+            for i in range(lo, hi):
+                r, (rows, cols) = self.owner[i], self.shapes[i]
+                a = r * slot + offs[i]
+                self.params[i] = W[a:a + rows * cols].view(rows, cols)
+                self.grads[i] = G[a:a + rows * cols].view(rows, cols)
+                if r == self.rank:
+                    self.momentum[i] = torch.zeros(rows, cols, dtype=torch.float32, device=self.device)
+                    owned.append(i)
+            self._buckets.append({"W": W, "G": G, "slot": slot, "owned": owned, "plan": None})
+
+        self._local_step = local_step
+        if local_step is None:
+            from . import MuonStepPlan
+            beta_, nest_, lr_, wd_, steps_ = self.hyper
+            for bk in self._buckets:
+                if bk["owned"]:
+                    bk["plan"] = MuonStepPlan([self.params[i] for i in bk["owned"]],
+                                              [self.grads[i] for i in bk["owned"]],
+                                              [self.momentum[i] for i in bk["owned"]],
+                                              beta=beta_, nesterov=nest_, lr=lr_, wd=wd_, steps=steps_)
+
+    # ------------------------------------------------------------ collectives
+    def _mine(self, flat, slot):
+        return flat[self.rank * slot:(self.rank + 1) * slot]
+
+    def _reduce_scatter_avg(self, G, slot):
+        """This rank's slot of G := the group mean of every rank's slot."""
+        if self.dist is None:
+            return
+        if self._nccl:
+            self.dist.reduce_scatter_tensor(self._mine(G, slot), G, op=self.dist.ReduceOp.AVG,
+                                            group=self.group)
+        else:  # backends without reduce-scatter: the same result through an all-reduce
+            self.dist.all_reduce(G, op=self.dist.ReduceOp.SUM, group=self.group)
+            self._mine(G, slot).div_(self.world)
+
+    def _all_gather(self, W, slot):
+        """Every rank's slot of W := its owner's; returns the pending work or None."""
+        if self.dist is None:
+            return None
+        if self._nccl:
+            return self.dist.all_gather_into_tensor(W, self._mine(W, slot), group=self.group,
+                                                    async_op=True)
+        chunks = list(W.split(slot))
+        return self.dist.all_gather(chunks, self._mine(W, slot).clone(), group=self.group,
+                                    async_op=True)
+
+    # ------------------------------------------------------------------ step
+    def step(self):
+        """One optimizer step over the group (every rank calls it)."""
+        for bk in self._buckets:
+            self._reduce_scatter_avg(bk["G"], bk["slot"])
+        pending = []
+        beta, nest, lr, wd, steps = self.hyper
+        for bk in self._buckets:
+            if bk["owned"]:
+                if bk["plan"] is not None:
+                    bk["plan"]()
+                else:
+                    own = bk["owned"]
+                    self._local_step([self.params[i] for i in own], [self.grads[i] for i in own],
+                                     [self.momentum[i] for i in own], beta, nest, lr, wd, steps)
+            work = self._all_gather(bk["W"], bk["slot"])
+            if work is not None:
+                pending.append(work)
+        for work in pending:
+            work.wait()

@@ -1,0 +1,161 @@
+"""The sharded Muon step's host logic on CPU: ownership, and two gloo ranks.
+
+The step over a data-parallel group must equal the single-process step on the
+group-averaged gradients (each matrix's update is independent of the
+others), on every rank.  The local step here is the oracle's fp64 Muon step
+run on CPU tensors, so the comparison with a single process running the same
+oracle on the averaged gradients is exact.
+"""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+from newton_schulz_12_b200.sharded import ns_flops, plan_ownership  # noqa: E402
+from oracle import muon as oracle  # noqa: E402
+
+SHAPES = [(16, 24), (24, 16), (32, 32), (8, 40), (40, 8), (12, 12)] * 2 + [(20, 20)]
+HYPER = dict(beta=0.95, nesterov=True, lr=0.05, wd=0.01, steps=5)
+
+
+def oracle_local_step(params, grads, bufs, beta, nesterov, lr, wd, steps):
+    for W, G, M in zip(params, grads, bufs):
+        Wn, Mn, _ = oracle.muon_step(W.double().numpy(), G.double().numpy(), M.double().numpy(),
+                                     beta=beta, nesterov=nesterov, lr=lr, wd=wd, steps=steps)
+        W.copy_(torch.from_numpy(Wn).float())
+        M.copy_(torch.from_numpy(Mn).float())
+
+
+def initial_w(i, shape):
+    g = torch.Generator().manual_seed(2000 + i)
+    return torch.randn(shape, generator=g) * 0.02
+
+
+def rank_grad(i, shape, rank, step):
+    g = torch.Generator().manual_seed(1000 + 100 * step + 10 * rank + i)
+    return torch.randn(shape, generator=g) * 0.01
+
+
+# ----------------------------------------------------------------- ownership
+def test_flops_match_the_oracle_count():
+    for r, c in [(768, 768), (768, 3072), (3072, 768), (5, 77)]:
+        assert ns_flops((r, c)) == oracle.ns_flops(r, c)
+
+
+@pytest.mark.parametrize("world,buckets", [(1, 1), (2, 2), (3, 1), (8, 2), (5, 4)])
+def test_every_matrix_has_one_owner_and_buckets_are_balanced(world, buckets):
+    shapes = [(768, 768)] * 4 + [(768, 3072), (3072, 768)]
+    shapes = shapes * 12  # the GPT-2-small hidden set in layer order
+    owner, ranges = plan_ownership(shapes, world, buckets)
+    assert len(owner) == len(shapes) and all(0 <= r < world for r in owner)
+    assert ranges[0][0] == 0 and ranges[-1][1] == len(shapes)
+    assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
+    for lo, hi in ranges:
+        load = [0] * world
+        for i in range(lo, hi):
+            load[owner[i]] += ns_flops(shapes[i])
+        biggest = max(ns_flops(shapes[i]) for i in range(lo, hi))
+        # greedy longest-first: no rank exceeds the mean by more than one item
+        assert max(load) <= sum(load) / world + biggest
+    assert plan_ownership(shapes, world, buckets) == (owner, ranges)  # deterministic
+
+
+def test_longest_first_on_a_small_case():
+    """Squares of 64, 56, 48, 40 (costs proportional to 262144, 175616, 110592,
+    64000) on two ranks, listed out of order: 64 -> r0, 56 -> r1, 48 -> r1
+    (175616 < 262144), 40 -> r0 (262144 < 286208)."""
+    shapes = [(48, 48), (64, 64), (40, 40), (56, 56)]
+    owner, _ = plan_ownership(shapes, 2, 1)
+    assert owner == [1, 0, 0, 1]
+
+
+def test_single_rank_step_equals_oracle_step():
+    from newton_schulz_12_b200.sharded import ShardedMuon
+    sm = ShardedMuon(SHAPES, buckets=3, grad_dtype=torch.float32, local_step=oracle_local_step,
+                     **HYPER)
+    W0 = [initial_w(i, s) for i, s in enumerate(SHAPES)]
+    for i, w in enumerate(W0):
+        sm.params[i].copy_(w)
+        sm.grads[i].copy_(rank_grad(i, SHAPES[i], 0, 0))
+    sm.step()
+    for i, s in enumerate(SHAPES):
+        Wn, _, _ = oracle.muon_step(W0[i].double().numpy(), rank_grad(i, s, 0, 0).double().numpy(),
+                                    np.zeros(s), **HYPER)
+        np.testing.assert_array_equal(sm.params[i].numpy(), Wn.astype(np.float32))
+
+
+# ------------------------------------------------------------ two gloo ranks
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, buckets, out):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from newton_schulz_12_b200.sharded import ShardedMuon
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        sm = ShardedMuon(SHAPES, buckets=buckets, grad_dtype=torch.float32,
+                         local_step=oracle_local_step, **HYPER)
+        for i, s in enumerate(SHAPES):
+            sm.params[i].copy_(initial_w(i, s))
+        for step in range(2):
+            for i, s in enumerate(SHAPES):
+                sm.grads[i].copy_(rank_grad(i, s, rank, step))
+            sm.step()
+        out.put((rank, [p.clone().numpy() for p in sm.params],
+                 {i: m.clone().numpy() for i, m in enumerate(sm.momentum) if m is not None}))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run_two_ranks(buckets):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, buckets, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=300) for _ in range(2)), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    return res
+
+
+def _single_process_reference():
+    W = [initial_w(i, s).double().numpy() for i, s in enumerate(SHAPES)]
+    M = [np.zeros(s) for s in SHAPES]
+    for step in range(2):
+        for i, s in enumerate(SHAPES):
+            # the group mean, in the fp32 order the ranks use: (g0 + g1) / 2
+            g = (rank_grad(i, s, 0, step) + rank_grad(i, s, 1, step)) / 2
+            Wn, Mn, _ = oracle.muon_step(W[i], g.double().numpy(), M[i], **HYPER)
+            W[i] = Wn.astype(np.float32).astype(np.float64)
+            M[i] = Mn.astype(np.float32).astype(np.float64)
+    return W, M
+
+
+@pytest.mark.parametrize("buckets", [1, 3])
+def test_two_gloo_ranks_equal_the_single_process_step(buckets):
+    res = _run_two_ranks(buckets)
+    W_ref, M_ref = _single_process_reference()
+    owner, _ = plan_ownership(SHAPES, 2, buckets)
+    for rank, params, moms in res:
+        for i in range(len(SHAPES)):
+            np.testing.assert_array_equal(params[i], W_ref[i].astype(np.float32),
+                                          err_msg=f"rank {rank} matrix {i}")
+        # momentum lives with the owner only
+        assert sorted(moms) == [i for i in range(len(SHAPES)) if owner[i] == rank]
+        for i, m in moms.items():
+            np.testing.assert_array_equal(m, M_ref[i].astype(np.float32))
