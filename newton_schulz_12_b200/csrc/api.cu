@@ -361,12 +361,15 @@ struct MatInfo {
   int rows, cols, m, n, transposed, group, index;
 };
 
-// The caller's weights, for the last step's fused apply (kBxApply).
+// The caller's buffers that the last step's BX epilogue writes directly:
+// kind 0, fp32 weights W updated by the apply (kBxApply); kind 1, bf16
+// buffers receiving X_T itself (kBx, mode 3: matrices in X's layout only).
 struct ApplySpec {
   const std::vector<MatInfo>* mats = nullptr;
-  const std::vector<void*>* w = nullptr;  // fp32 W of matrix i, the caller's layout
+  const std::vector<void*>* w = nullptr;  // W (kind 0) or the output (kind 1) of matrix i, caller's layout
+  int kind = 0;
   float lr = 0.f, wd = 0.f;
-  std::vector<char> done;  // out: matrix i was applied by the GEMM epilogue
+  std::vector<char> done;  // out: matrix i was finished by the GEMM epilogue
 };
 
 // fl(lr * scale) with scale = sqrt(max(1, rows / cols)), as the apply pass uses.
@@ -376,9 +379,11 @@ float apply_ls(const MatInfo& M, float lr) {
   return lr * scale;
 }
 
-// Table of the groups [g0, g1) of one kBxApply launch: every matrix whose W
-// rows are 16-byte strided (cols % 4 == 0) among the first kMaxApply gets a
-// tensor map over W and mode 1 (W = X) or 2 (W = X^T); the rest keep mode 0.
+// Table of the groups [g0, g1) of the last BX launch.  Kind 0: every matrix
+// whose W rows are 16-byte strided (cols % 4 == 0) among the first kMaxApply
+// gets a tensor map over W and mode 1 (W = X) or 2 (W = X^T).  Kind 1: every
+// such matrix in X's layout (not transposed) with 16-byte bf16 rows (cols % 8
+// == 0) gets a map over its output and mode 3.  The rest keep mode 0.
 int build_apply_table(const std::vector<NsGroup>& gs, size_t g0, size_t g1, ApplySpec& A,
                       tc::LaunchApply& T) {
   T.nmat = 0;
@@ -393,8 +398,17 @@ int build_apply_table(const std::vector<NsGroup>& gs, size_t g0, size_t g1, Appl
     const MatInfo& M = mats[i];
     if (M.group < static_cast<int>(g0) || M.group >= static_cast<int>(g1)) continue;
     const int j = gs[M.group].mat_base + M.index - T.mat_base;
-    if (j >= T.nmat || M.cols % 4 != 0) continue;
+    if (j >= T.nmat) continue;
     const void* W = (*A.w)[i];
+    if (A.kind == 1) {
+      if (M.transposed || M.cols % 8 != 0) continue;
+      MUON_TRY(make_map(&T.w[j], W, 2, M.cols, M.rows, 1, M.cols, static_cast<uint64_t>(M.rows) * M.cols, 64,
+                        tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
+      T.mat[j] = tc::ApplyMat{3, 0.f};
+      A.done[i] = 1;
+      continue;
+    }
+    if (M.cols % 4 != 0) continue;
     if (!M.transposed)
       MUON_TRY(make_map(&T.w[j], W, 4, M.cols, M.rows, 1, M.cols, static_cast<uint64_t>(M.rows) * M.cols, 32,
                         tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
@@ -472,7 +486,7 @@ int run_ns_bf16(std::vector<NsGroup>& gs, int steps, const float* abc, int* stat
       if (apply && t == steps - 1) {
         tc::LaunchApply table;
         MUON_TRY(build_apply_table(gs, g0, g1, *apply, table));
-        MUON_TRY(launch_tc(tc::kBxApply, bxt, sms, s, &table));
+        MUON_TRY(launch_tc(apply->kind == 0 ? tc::kBxApply : tc::kBx, bxt, sms, s, &table));
       } else {
         MUON_TRY(launch_tc(tc::kBx, bxt, sms, s));
       }
@@ -969,10 +983,18 @@ int ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, const float* 
     Workspace* ws = nullptr;
     MUON_TRY(get_workspace(s, off, &ws));
     bf16_layout(mats, groups, static_cast<char*>(ws->ptr), L);
+    // the last step writes X_T straight into the callers' buffers where it can
+    // (only the prep pass reads them, so writing in place is safe)
+    ApplySpec wb;
+    wb.mats = &mats;
+    wb.w = &ys;
+    wb.kind = 1;
+    wb.done.assign(batch, 0);
     MUON_TRY(run_bf16_path(mats, groups, L, src, {}, ew::kFromBf16, 0.f, 0, abc, steps,
-                           ws->status, dev.sms, s));
+                           ws->status, dev.sms, s, &wb));
     for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
-    MUON_TRY(launch_out_chunked(mats, groups, res, ys, 1, 0.f, 0.f, s, steps == 0 ? L.xscale : nullptr));
+    MUON_TRY(launch_out_chunked(mats, groups, res, ys, 1, 0.f, 0.f, s, steps == 0 ? L.xscale : nullptr,
+                                &wb.done));
     return MUON_OK;
   }
   // fp32 verification path: normalised fp32 X, SIMT GEMMs
@@ -1070,12 +1092,18 @@ int muon_ns_orthogonalize_static(int batch, int m, int n, void* const* X_ptrs, f
 
   std::vector<const void*> src(X_ptrs, X_ptrs + batch);
   const std::vector<float> abc = constant_schedule(a, b, c, steps);
+  std::vector<void*> ys(X_ptrs, X_ptrs + batch);
+  ApplySpec wb;  // as in ns_orthogonalize: the last step writes X_T where it can
+  wb.mats = &mats;
+  wb.w = &ys;
+  wb.kind = 1;
+  wb.done.assign(batch, 0);
   MUON_TRY(run_bf16_path(mats, groups, L, src, {}, ew::kFromBf16, 0.f, 0, abc.data(), steps, status,
-                         dev.sms, s));
+                         dev.sms, s, &wb));
   std::vector<Result> res;
   for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
-  std::vector<void*> ys(X_ptrs, X_ptrs + batch);
-  MUON_TRY(launch_out_chunked(mats, groups, res, ys, 1, 0.f, 0.f, s, steps == 0 ? L.xscale : nullptr));
+  MUON_TRY(launch_out_chunked(mats, groups, res, ys, 1, 0.f, 0.f, s, steps == 0 ? L.xscale : nullptr,
+                              &wb.done));
   return MUON_OK;
 }
 

@@ -287,12 +287,10 @@ constexpr int threads_of() {
   return EPI == kGram ? kThreads : kThreads + 32;
 }
 
-template <int EPI>
-using TableOf = ApplyTable<EPI == kBxApply ? kMaxApply : 1>;
-
-template <int EPI>
+// NT: entries of the per-matrix table (1 where the launch has none).
+template <int EPI, int NT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1)
-    gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ TableOf<EPI> tab) {
+    gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ ApplyTable<NT> tab) {
   using C = Cfg<EPI>;
   constexpr int S = C::kStages;
   constexpr int K = C::kSlots;
@@ -599,14 +597,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             mbar_wait(ready_bar(slot), (s / K) & 1, ctl);
             if (kind != kSkip) {  // never start a store wholly outside the matrix
               const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
-              const int j = (EPI == kBxApply) ? apply_entry(tab, G, tc.b) : -1;
+              const int j = (NT > 1) ? apply_entry(tab, G, tc.b) : -1;
               const int mode = j >= 0 ? tab.mat[j].mode : 0;
-              if (mode == 1) {
+              if (EPI == kBxApply && mode == 1) {
                 for (int h = 0; h < 2; ++h)
                   if (col0 + 32 * h < G.n) tma_store_3d(&tab.w[j], hs + C::kWOff + h * (BM * 32 * 4), col0 + 32 * h, row0, 0);
-              } else if (mode == 2) {
+              } else if (EPI == kBxApply && mode == 2) {
                 for (int q = 0; q < 4; ++q)
                   if (row0 + 32 * q < G.m) tma_store_3d(&tab.w[j], hs + C::kWOff + q * (64 * 32 * 4), row0 + 32 * q, col0, 0);
+              } else if (EPI == kBx && mode == 3) {
+                tma_store_3d(&tab.w[j], hs, col0, row0, 0);  // hi' -> the caller's bf16 buffer; no residual
               } else {
                 tma_store_3d(&M.d, hs, col0, row0, tc.b);               // hi' -> the other hi buffer
                 tma_store_3d(&M.mt, hs + C::kLoOff, col0, row0, tc.b);  // lo' -> lo, in place
@@ -933,15 +933,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
   }
 }
 
-template <int EPI>
-static cudaError_t launch_one(const Params& p, const TableOf<EPI>& tab, int max_pairs, cudaStream_t stream) {
+template <int EPI, int NT>
+static cudaError_t launch_one(const Params& p, const ApplyTable<NT>& tab, int max_pairs, cudaStream_t stream) {
   static thread_local int configured_device = -1;
   static thread_local int resident_pairs = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   const size_t smem = Cfg<EPI>::kSmem;
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<EPI>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<EPI, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -951,14 +951,14 @@ static cudaError_t launch_one(const Params& p, const TableOf<EPI>& tab, int max_
     cfg.blockDim = dim3(threads_of<EPI>(), 1, 1);
     cfg.dynamicSmemBytes = smem;
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel<EPI>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, gemm_kernel<EPI, NT>, &cfg);
     if (e != cudaSuccess) return e;
     resident_pairs = n;
     configured_device = dev;
   }
   int pairs = p.total_tiles < max_pairs ? p.total_tiles : max_pairs;
   if (resident_pairs > 0 && pairs > resident_pairs) pairs = resident_pairs;
-  gemm_kernel<EPI><<<2 * pairs, threads_of<EPI>(), smem, stream>>>(p, tab);
+  gemm_kernel<EPI, NT><<<2 * pairs, threads_of<EPI>(), smem, stream>>>(p, tab);
   return cudaGetLastError();
 }
 
@@ -967,12 +967,14 @@ cudaError_t launch(int epi, const Params& p, int max_pairs, cudaStream_t stream,
   if (max_pairs < 1) max_pairs = 1;
   const ApplyTable<1> none{};
   switch (epi) {
-    case kGram: return launch_one<kGram>(p, none, max_pairs, stream);
-    case kPoly: return launch_one<kPoly>(p, none, max_pairs, stream);
-    case kBx: return launch_one<kBx>(p, none, max_pairs, stream);
+    case kGram: return launch_one<kGram, 1>(p, none, max_pairs, stream);
+    case kPoly: return launch_one<kPoly, 1>(p, none, max_pairs, stream);
+    case kBx:  // with a table: the hi of its mode-3 matrices goes to the caller's buffers
+      return apply ? launch_one<kBx, kMaxApply>(p, *apply, max_pairs, stream)
+                   : launch_one<kBx, 1>(p, none, max_pairs, stream);
     case kBxApply:
       if (!apply) return cudaErrorInvalidValue;
-      return launch_one<kBxApply>(p, *apply, max_pairs, stream);
+      return launch_one<kBxApply, kMaxApply>(p, *apply, max_pairs, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -81,8 +81,11 @@ struct Params {
 // box 32 x 64, four per chunk).
 constexpr int kMaxApply = 96;  // matrices per launch with a table entry
 
+// A kBx launch may carry the same table with mode 3: the matrix's X_T goes to
+// the caller's bf16 buffer in X's layout (its tensor map; box 64 x 128) as
+// the hi of the pair, i.e. X_T rounded to nearest, and no residual is kept.
 struct ApplyMat {
-  int mode;  // 0, 1 or 2 as above
+  int mode;  // 0, 1 or 2 as above (kBxApply), 0 or 3 (kBx)
   float ls;  // fl(lr * scale)
 };
 
@@ -114,7 +117,8 @@ inline int sym_tiles(int m) {
 
 size_t smem_bytes(int epi);
 // `max_pairs` bounds the number of CTA pairs (clusters) of the persistent grid;
-// `apply` is the table of a kBxApply launch (ignored by the other kinds).
+// `apply` is the table of a kBxApply launch (required) or of a kBx launch
+// (optional; ignored by the other kinds).
 cudaError_t launch(int epi, const Params& p, int max_pairs, cudaStream_t stream,
                    const LaunchApply* apply = nullptr);
 
