@@ -119,18 +119,22 @@ def _worker(rank, world, port, buckets, out):
         dist.destroy_process_group()
 
 
-def _run_two_ranks(buckets):
+def _run_ranks(world, target, *args):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, buckets, q)) for r in range(2)]
+    procs = [ctx.Process(target=target, args=(r, world, port) + args + (q,)) for r in range(world)]
     for p in procs:
         p.start()
-    res = sorted((q.get(timeout=300) for _ in range(2)), key=lambda t: t[0])
+    res = sorted((q.get(timeout=300) for _ in range(world)), key=lambda t: t[0])
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
     return res
+
+
+def _run_two_ranks(buckets):
+    return _run_ranks(2, _worker, buckets)
 
 
 def _single_process_reference():
@@ -159,3 +163,46 @@ def test_two_gloo_ranks_equal_the_single_process_step(buckets):
         assert sorted(moms) == [i for i in range(len(SHAPES)) if owner[i] == rank]
         for i, m in moms.items():
             np.testing.assert_array_equal(m, M_ref[i].astype(np.float32))
+
+
+# ------------------------------------------- three ranks, one idle in a bucket
+SHAPES3 = [(16, 24), (24, 16), (32, 32), (8, 40)]
+
+
+def exact_grad(i, shape, rank):
+    """Integers times 2^-14: their three-rank sums are exact in any order."""
+    g = torch.Generator().manual_seed(4000 + 10 * rank + i)
+    return torch.round(torch.randn(shape, generator=g) * 160) / 2 ** 14
+
+
+def _worker3(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from newton_schulz_12_b200.sharded import ShardedMuon
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        sm = ShardedMuon(SHAPES3, buckets=2, grad_dtype=torch.float32,
+                         local_step=oracle_local_step, **HYPER)
+        for i, s in enumerate(SHAPES3):
+            sm.params[i].copy_(initial_w(i, s))
+            sm.grads[i].copy_(exact_grad(i, s, rank))
+        sm.step()
+        out.put((rank, [p.clone().numpy() for p in sm.params], sm.owner))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_three_ranks_with_an_idle_rank_in_a_bucket():
+    owner, ranges = plan_ownership(SHAPES3, 3, 2)
+    assert ranges == [(0, 2), (2, 4)]
+    assert 2 not in owner[0:2]  # rank 2 owns nothing in bucket 0 yet joins its collectives
+    res = _run_ranks(3, _worker3)
+    for rank, params, own in res:
+        assert own == owner
+        for i, s in enumerate(SHAPES3):
+            g = (exact_grad(i, s, 0) + exact_grad(i, s, 1) + exact_grad(i, s, 2)) / 3
+            Wn, _, _ = oracle.muon_step(initial_w(i, s).double().numpy(), g.double().numpy(),
+                                        np.zeros(s), **HYPER)
+            np.testing.assert_array_equal(params[i], Wn.astype(np.float32),
+                                          err_msg=f"rank {rank} matrix {i}")
