@@ -70,7 +70,11 @@ typedef enum {
  * X_ptrs  host array of `batch` device pointers, each to an m x n row-major
  *         matrix of bf16 (dtype MUON_BF16) or fp32 (MUON_FP32).  On return
  *         (stream order) each holds NS(X / (||X||_F + 1e-7)) after `steps`
- *         iterations, rounded to the storage type.
+ *         iterations, rounded to the storage type.  (MUON_BF16, steps >= 1:
+ *         with m <= n and n % 8 == 0 the last GEMM stores the fp32 result
+ *         rounded to bf16 straight into the first 96 buffers of each launch;
+ *         the others are written from the bf16 + int8 pair by a separate
+ *         pass, which can differ from that rounding by one bf16 unit.)
  * a, b, c coefficients of the quintic; the speedrun's are 3.4445, -4.7750, 2.0315.
  * steps   number of iterations T (0 <= steps <= 100; 0 = normalise only).
  * dtype   a muon_dtype.
