@@ -250,15 +250,19 @@ int sym_maps(tc::Maps& M, const void* S, int m, int k, long long lds, long long 
 
 // Maps of X' = a X + B X with X carried as the pair bf16 hi + int8 lo: B
 // (m x m), hi of X (m x n: MN-major operand and epilogue chunks), lo of X
-// (read and written in place), hi of X' (written).
+// (read and written in place), hi of X' (written).  Epilogue chunks are
+// `chunk` (64 or 32) columns wide: hi rows of 2 chunk bytes, lo rows of
+// chunk bytes, each swizzled over its full width.
 int bx_maps(tc::Maps& M, const void* B, long long ldb, long long sb, const void* Xhi,
-            void* Xlo, void* Xhi_out, int m, int n, long long ldx, long long sx, int batch) {
+            void* Xlo, void* Xhi_out, int m, int n, long long ldx, long long sx, int batch,
+            int chunk = 64) {
   MUON_TRY(make_map(&M.p, B, 2, m, m, batch, ldb, sb, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
   MUON_TRY(make_map(&M.q, Xhi, 2, n, m, batch, ldx, sx, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
-  // epilogue chunks of 64 columns: 128-byte rows
-  MUON_TRY(make_map(&M.e, Xhi, 2, n, m, batch, ldx, sx, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
-  MUON_TRY(make_map(&M.mt, Xlo, 1, n, m, batch, ldx, sx, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
-  MUON_TRY(make_map(&M.d, Xhi_out, 2, n, m, batch, ldx, sx, 64, tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
+  const CUtensorMapSwizzle hs = chunk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUtensorMapSwizzle ls = chunk == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  MUON_TRY(make_map(&M.e, Xhi, 2, n, m, batch, ldx, sx, chunk, tc::BM, hs));
+  MUON_TRY(make_map(&M.mt, Xlo, 1, n, m, batch, ldx, sx, chunk, tc::BM, ls));
+  MUON_TRY(make_map(&M.d, Xhi_out, 2, n, m, batch, ldx, sx, chunk, tc::BM, hs));
   M.s = M.d;  // unused
   return MUON_OK;
 }
@@ -414,7 +418,7 @@ int build_apply_table(const std::vector<NsGroup>& gs, size_t g0, size_t g1, Appl
                         tc::BM, CU_TENSOR_MAP_SWIZZLE_128B));
     else
       MUON_TRY(make_map(&T.w[j], W, 4, M.cols, M.rows, 1, M.cols, static_cast<uint64_t>(M.rows) * M.cols, 32,
-                        64, CU_TENSOR_MAP_SWIZZLE_128B));
+                        tc::bx_apply_chunk(), CU_TENSOR_MAP_SWIZZLE_128B));
     T.mat[j] = tc::ApplyMat{M.transposed ? 2 : 1, apply_ls(M, A.lr)};
     A.done[i] = 1;
   }
@@ -486,7 +490,21 @@ int run_ns_bf16(std::vector<NsGroup>& gs, int steps, const float* abc, int* stat
       if (apply && t == steps - 1) {
         tc::LaunchApply table;
         MUON_TRY(build_apply_table(gs, g0, g1, *apply, table));
-        MUON_TRY(launch_tc(apply->kind == 0 ? tc::kBxApply : tc::kBx, bxt, sms, s, &table));
+        if (apply->kind == 0) {
+          // kBxApply reads and writes X's pair in chunks of its own width
+          tc::Params bxa = bxt;
+          for (size_t gi = g0; gi < g1; ++gi) {
+            NsGroup& G = gs[gi];
+            const int k = static_cast<int>(gi - g0);
+            const long long xs = static_cast<long long>(G.m) * G.ldn;
+            const long long as = static_cast<long long>(G.m) * G.ldm;
+            MUON_TRY(bx_maps(bxa.map[k], G.B, G.ldm, as, G.xb[cur], G.xlo, G.xb[cur ^ 1], G.m, G.n, G.ldn,
+                             xs, G.batch, tc::bx_apply_chunk()));
+          }
+          MUON_TRY(launch_tc(tc::kBxApply, bxa, sms, s, &table));
+        } else {
+          MUON_TRY(launch_tc(tc::kBx, bxt, sms, s, &table));
+        }
       } else {
         MUON_TRY(launch_tc(tc::kBx, bxt, sms, s));
       }

@@ -82,13 +82,18 @@ constexpr size_t kMaxSmem = 232448;                         // 227 KiB per CTA o
 #ifndef MUON_BX_SLOTS
 #define MUON_BX_SLOTS 4
 #endif
-// kBxApply slots also hold the chunk's 32 KiB of W: fewer stages and slots fit
+// kBxApply slots also hold the chunk's W (fp32): with 32-column chunks a slot
+// is 28 KiB and 4 fit next to 3 stages, so 3 chunks can be in flight
+#ifndef MUON_BXA_CHUNK
+#define MUON_BXA_CHUNK 32
+#endif
 #ifndef MUON_BXA_STAGES
 #define MUON_BXA_STAGES 3
 #endif
 #ifndef MUON_BXA_SLOTS
-#define MUON_BXA_SLOTS 2
+#define MUON_BXA_SLOTS (MUON_BXA_CHUNK == 32 ? 4 : 2)
 #endif
+static_assert(MUON_BXA_CHUNK == 32 || MUON_BXA_CHUNK == 64, "kBxApply chunk width");
 
 // kBx and kBxApply share the operands, the tiling and X's epilogue chunks.
 template <int EPI>
@@ -107,17 +112,19 @@ struct Cfg {
       (EPI == kBx) ? MUON_BX_SLOTS : (EPI == kBxApply ? MUON_BXA_SLOTS : MUON_POLY_SLOTS);
   // kBx works on 64-column chunks (128-byte rows in global memory), the
   // symmetric kernels on kSymChunk-column chunks
-  static constexpr int kCW = is_bx<EPI>() ? 2 * kChunk : kSymChunk;
+  static constexpr int kCW = (EPI == kBx) ? 2 * kChunk : (EPI == kBxApply ? MUON_BXA_CHUNK : kSymChunk);
   static constexpr int kNCh = BN / kCW;  // per tile
   // bytes of one bf16 chunk, 128 rows x kCW columns
   static constexpr uint32_t kChunkBytes = BM * kCW * 2;
-  // kBx slot: hi (bf16, 128 rows x 128 B) then lo (int8, 128 rows x 64 B);
-  // kBxApply: then W's 128 x 64 fp32 chunk (32 KiB); kPoly slot: A's chunk
-  static constexpr uint32_t kLoOff = 2 * kChunkBf16;
-  static constexpr uint32_t kWOff = 3 * kChunkBf16;
-  static constexpr uint32_t kWBytes = BM * 64 * 4;
-  static constexpr uint32_t kSlotBytes = (EPI == kBx)        ? 3 * kChunkBf16
-                                         : (EPI == kBxApply) ? 3 * kChunkBf16 + kWBytes
+  // kBx / kBxApply slot: hi (bf16, 128 rows x 2 kCW bytes) then lo (int8,
+  // 128 rows x kCW bytes); kBxApply: then W's 128 x kCW fp32 chunk; kPoly
+  // slot: A's chunk
+  static constexpr uint32_t kXBytes = BM * kCW * 3;  // the pair of X's chunk
+  static constexpr uint32_t kLoOff = BM * kCW * 2;
+  static constexpr uint32_t kWOff = kXBytes;
+  static constexpr uint32_t kWBytes = BM * kCW * 4;
+  static constexpr uint32_t kSlotBytes = (EPI == kBx)        ? kXBytes
+                                         : (EPI == kBxApply) ? kXBytes + kWBytes
                                          : (EPI == kPoly)    ? kChunkBytes
                                                              : 0;
   static constexpr uint32_t kSlotsBytes = kSlotBytes * kSlots;
@@ -143,6 +150,8 @@ static_assert(Cfg<kBx>::kSmem <= kMaxSmem, "kBx shared memory");
 static_assert(Cfg<kBxApply>::kSmem <= kMaxSmem, "kBxApply shared memory");
 static_assert(Cfg<kBxApply>::kWOff % 1024 == 0 && Cfg<kBxApply>::kSlotBytes % 1024 == 0,
               "W chunks start on the 1 KiB boundary of the 128-byte swizzle");
+
+int bx_apply_chunk() { return Cfg<kBxApply>::kCW; }
 
 size_t smem_bytes(int epi) {
   switch (epi) {
@@ -211,6 +220,11 @@ __device__ __forceinline__ uint32_t sw64(int r, int u) {
   return static_cast<uint32_t>(r * 64 + ((u ^ ((r >> 1) & 3)) << 4));
 }
 
+// Same for a 32-byte-swizzled tile (rows of 32 bytes).
+__device__ __forceinline__ uint32_t sw32(int r, int u) {
+  return static_cast<uint32_t>(r * 32 + ((u ^ ((r >> 2) & 1)) << 4));
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
@@ -254,13 +268,18 @@ __device__ __forceinline__ int apply_entry(const ApplyTable<N>& t, const Group& 
   return (j >= 0 && j < t.nmat && t.mat[j].mode != 0) ? j : -1;
 }
 
-// Bytes of W's chunk at (row0, col0) of X that the loader copies (boxes
-// wholly outside W are neither copied nor stored).
+// Bytes of W's chunk (CW columns of X) at (row0, col0) that the loader
+// copies: mode 1, CW / 32 boxes of 32 x 128; mode 2, four boxes of 32 x CW.
+// Boxes wholly outside W are neither copied nor stored.
+template <int CW>
 __device__ __forceinline__ uint32_t w_chunk_bytes(int mode, const Group& G, int row0, int col0) {
-  if (mode == 1) return (col0 + 32 < G.n ? 2u : 1u) * (BM * 32 * 4);
   uint32_t q = 0;
+  if (mode == 1) {
+    for (int h = 0; h < CW / 32; ++h) q += (col0 + 32 * h < G.n) ? 1u : 0u;
+    return q * (BM * 32 * 4);
+  }
   for (int i = 0; i < 4; ++i) q += (row0 + 32 * i < G.m) ? 1u : 0u;
-  return q * (64 * 32 * 4);
+  return q * (32 * CW * 4);
 }
 
 // W' = (W - lw W) - ls O, each operation rounded to nearest in fp32.
@@ -542,20 +561,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             const uint32_t dst = slots_u32 + slot * C::kSlotBytes;
             const int j = (EPI == kBxApply) ? apply_entry(tab, G, tc.b) : -1;
             const int mode = j >= 0 ? tab.mat[j].mode : 0;
-            const uint32_t bytes = is_bx<EPI>() ? 3 * kChunkBf16 : C::kSlotBytes;
-            mbar_arrive_expect_tx(efull_bar(slot), bytes + (mode ? w_chunk_bytes(mode, G, row0, col0) : 0u));
+            const uint32_t bytes = is_bx<EPI>() ? C::kXBytes : C::kSlotBytes;
+            mbar_arrive_expect_tx(efull_bar(slot), bytes + (mode ? w_chunk_bytes<CW>(mode, G, row0, col0) : 0u));
             tma_load_3d(dst, &p.map[tc.g].e, efull_bar(slot), col0, row0, tc.b);
             if (is_bx<EPI>())  // lo half of X next to its hi half
               tma_load_3d(dst + C::kLoOff, &p.map[tc.g].mt, efull_bar(slot), col0, row0, tc.b);
-            if (mode == 1) {  // W as X: two 32-column boxes of 128 rows
-              for (int h = 0; h < 2; ++h)
+            if (mode == 1) {  // W as X: CW / 32 boxes of 32 columns x 128 rows
+              for (int h = 0; h < CW / 32; ++h)
                 if (col0 + 32 * h < G.n)
                   tma_load_3d(dst + C::kWOff + h * (BM * 32 * 4), &tab.w[j], efull_bar(slot), col0 + 32 * h,
                               row0, 0);
-            } else if (mode == 2) {  // W = X^T: four 32-column boxes of 64 rows
+            } else if (mode == 2) {  // W = X^T: four boxes of 32 columns x CW rows
               for (int q = 0; q < 4; ++q)
                 if (row0 + 32 * q < G.m)
-                  tma_load_3d(dst + C::kWOff + q * (64 * 32 * 4), &tab.w[j], efull_bar(slot), row0 + 32 * q,
+                  tma_load_3d(dst + C::kWOff + q * (32 * CW * 4), &tab.w[j], efull_bar(slot), row0 + 32 * q,
                               col0, 0);
             }
           }
@@ -600,11 +619,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
               const int j = (NT > 1) ? apply_entry(tab, G, tc.b) : -1;
               const int mode = j >= 0 ? tab.mat[j].mode : 0;
               if (EPI == kBxApply && mode == 1) {
-                for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < CW / 32; ++h)
                   if (col0 + 32 * h < G.n) tma_store_3d(&tab.w[j], hs + C::kWOff + h * (BM * 32 * 4), col0 + 32 * h, row0, 0);
               } else if (EPI == kBxApply && mode == 2) {
                 for (int q = 0; q < 4; ++q)
-                  if (row0 + 32 * q < G.m) tma_store_3d(&tab.w[j], hs + C::kWOff + q * (64 * 32 * 4), row0 + 32 * q, col0, 0);
+                  if (row0 + 32 * q < G.m) tma_store_3d(&tab.w[j], hs + C::kWOff + q * (32 * CW * 4), row0 + 32 * q, col0, 0);
               } else if (EPI == kBx && mode == 3) {
                 tma_store_3d(&tab.w[j], hs, col0, row0, 0);  // hi' -> the caller's bf16 buffer; no residual
               } else {
@@ -699,25 +718,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
           const int j = (EPI == kBxApply) ? apply_entry(tab, G, tc.b) : -1;
           const int mode = j >= 0 ? tab.mat[j].mode : 0;
           const float lsc = j >= 0 ? tab.mat[j].ls : 0.f;  // fl(lr * scale)
-          // 64-column chunks c: thread (r, hf) takes accumulator columns
-          // 32 hf .. +31 of the chunk, i.e. 16-byte units 4 hf .. 4 hf + 3 of
-          // its 128-byte row in the slot's hi and lo tiles (128-byte swizzle)
+          // BCW-column chunks c (64 for kBx, MUON_BXA_CHUNK for kBxApply): thread
+          // (r, hf) takes accumulator columns VB hf .. +VB-1 of the chunk
+          constexpr int BCW = C::kCW, VB = BCW / 2;
           const int sr = r;
           for (int c = 0; c < C::kNCh; ++c) {
             if (leader && c > 0) TRACE(k, 4 + c);
             const int s = k * C::kNCh + c;
             const int col0 = tc.tn * BN + c * C::kCW;
             const bool live = chunk_kind<EPI>(G, tc.tm, col0) != kSkip;
-            float v[32];
+            float v[VB];
             if (live) {
-              uint32_t rr[32];
+              uint32_t rr[VB];
               __syncwarp();
-              tmem_ld_32x32(tmem_base + (static_cast<uint32_t>(lane_base) << 16) +
-                                static_cast<uint32_t>(acc * BN + c * C::kCW + hf * 32),
-                            rr);
+              const uint32_t ta = tmem_base + (static_cast<uint32_t>(lane_base) << 16) +
+                                  static_cast<uint32_t>(acc * BN + c * C::kCW + hf * VB);
+              if constexpr (VB == 32)
+                tmem_ld_32x32(ta, rr);
+              else
+                tmem_ld_32x32_x16(ta, rr);
               tmem_ld_wait();
 #pragma unroll
-              for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(rr[q]);
+              for (int q = 0; q < VB; ++q) v[q] = __uint_as_float(rr[q]);
             }
             if (c == C::kNCh - 1) {
               // accumulator fully read: one arrival per warp hands it back (in
@@ -730,16 +752,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             mbar_wait(efull_bar(slot), (s / K) & 1, ctl);
             // X = hi + lo from the slot; X' = a X + acc (times s on the first
             // step) written back in place as the pair (hi', lo') for the IO
-            // thread to store.  Columns 32 hf + 8 uu .. +7: 16-byte unit
-            // 4 hf + uu of the hi row (128-byte swizzle), bytes 8 (uu & 1)..
-            // of unit 2 hf + uu / 2 of the lo row (64-byte swizzle).
+            // thread to store.  Columns VB hf + 8 uu .. +7 are 16-byte unit
+            // (VB / 8) hf + uu of the hi row (2 BCW bytes, swizzled over its
+            // width) and bytes 8 (uu & 1) .. of unit (VB / 16) hf + uu / 2 of
+            // the lo row (BCW bytes, likewise).
             if (live) {
               const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
               const uint32_t ls = hs + C::kLoOff;
 #pragma unroll
-              for (int uu = 0; uu < 4; ++uu) {
-                const uint32_t ha = hs + sw128(sr, 4 * hf + uu);
-                const uint32_t la = ls + sw64(sr, 2 * hf + (uu >> 1)) + 8 * (uu & 1);
+              for (int uu = 0; uu < VB / 8; ++uu) {
+                const uint32_t ha = hs + (BCW == 64 ? sw128(sr, 4 * hf + uu) : sw64(sr, 2 * hf + uu));
+                const uint32_t la = ls + (BCW == 64 ? sw64(sr, 2 * hf + (uu >> 1)) : sw32(sr, hf)) + 8 * (uu & 1);
                 uint4 h4;
                 uint2 l2;
                 ld_shared_v4(ha, h4.x, h4.y, h4.z, h4.w);
@@ -749,12 +772,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
 #pragma unroll
                 for (int e = 0; e < 8; ++e) x[e] = fmaf(p.a, x[e], v[8 * uu + e]) * xs;
                 if (EPI == kBxApply && mode == 1) {
-                  // W's row sr, columns 32 hf + 8 uu ..: 16-byte units 2 uu, 2 uu + 1
-                  // of row sr of box hf (128-byte swizzle)
-                  const uint32_t wb = hs + C::kWOff + hf * (BM * 32 * 4);
+                  // W's row sr, columns VB hf + 8 uu ..: box (VB hf) / 32 (32
+                  // fp32 per 128-byte row, 128-byte swizzle), 16-byte units
+                  // ((VB hf) % 32) / 4 + 2 uu and the next
+                  const uint32_t wb = hs + C::kWOff + ((VB * hf) / 32) * (BM * 32 * 4);
+                  const int u0 = ((VB * hf) % 32) / 4 + 2 * uu;
 #pragma unroll
                   for (int h = 0; h < 2; ++h) {
-                    const uint32_t wa = wb + sw128(sr, 2 * uu + h);
+                    const uint32_t wa = wb + sw128(sr, u0 + h);
                     uint32_t w[4];
                     ld_shared_v4(wa, w[0], w[1], w[2], w[3]);
 #pragma unroll
@@ -763,12 +788,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                     st_shared_v4(wa, w[0], w[1], w[2], w[3]);
                   }
                 } else if (EPI == kBxApply && mode == 2) {
-                  // W = X^T: X's column 32 hf + 8 uu + e is row 32 hf + 8 uu + e of
-                  // box (warp & 3), whose 32 columns are this lane quarter's rows
-                  const uint32_t wb = hs + C::kWOff + (warp & 3) * (64 * 32 * 4);
+                  // W = X^T: X's column VB hf + 8 uu + e is row VB hf + 8 uu + e
+                  // of box (warp & 3) (BCW rows of 128 bytes), whose 32 columns
+                  // are this lane quarter's rows
+                  const uint32_t wb = hs + C::kWOff + (warp & 3) * (32 * BCW * 4);
 #pragma unroll
                   for (int e = 0; e < 8; ++e) {
-                    const int row = 32 * hf + 8 * uu + e;
+                    const int row = VB * hf + 8 * uu + e;
                     const uint32_t wa =
                         wb + static_cast<uint32_t>(row * 128 + ((((lane >> 2) ^ row) & 7) << 4) + (lane & 3) * 4);
                     float w;

@@ -77,8 +77,8 @@ struct Params {
 // as the pair (mode 0; the apply runs as its own pass later), or the caller's
 // fp32 W is updated in place from O = X_T, W' = (W - lw W) - ls O, with W
 // read and written through its own tensor map: mode 1, W has X's layout
-// (box 32 x 128, two per 64-column chunk); mode 2, W = X^T (a tall matrix;
-// box 32 x 64, four per chunk).
+// (boxes of 32 x 128, one per 32 columns of a chunk); mode 2, W = X^T (a tall
+// matrix; box 32 x chunk width, four per chunk).
 constexpr int kMaxApply = 96;  // matrices per launch with a table entry
 
 // A kBx launch may carry the same table with mode 3: the matrix's X_T goes to
@@ -116,6 +116,9 @@ inline int sym_tiles(int m) {
 }
 
 size_t smem_bytes(int epi);
+// Epilogue chunk width (columns) of kBxApply: its launch takes maps of X's
+// pair with boxes this wide, and mode-2 W maps with boxes of 32 x this.
+int bx_apply_chunk();
 // `max_pairs` bounds the number of CTA pairs (clusters) of the persistent grid;
 // `apply` is the table of a kBxApply launch (required) or of a kBx launch
 // (optional; ignored by the other kinds).
