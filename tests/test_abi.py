@@ -31,6 +31,18 @@ def test_header_lists_the_boundary():
     assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
 
 
+def test_kernel_kinds_match_the_header():
+    """The binding's names for muon_profile_end's slots follow the header's enum."""
+    with open(HEADER) as f:
+        text = f.read()
+    kinds = dict((name, int(v)) for name, v in re.findall(r"MUON_KERNEL_([A-Z_]+)\s*=\s*(\d+)", text))
+    count = kinds.pop("KINDS")
+    assert count == len(_lib.KERNEL_KINDS)
+    assert sorted(kinds.values()) == list(range(count))
+    for name, v in kinds.items():
+        assert _lib.KERNEL_KINDS[v] == name.lower(), name
+
+
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
