@@ -175,6 +175,14 @@ class MuonStepPlan:
         self._hyper = (float(beta), int(bool(nesterov)), float(lr), float(wd), int(steps))
         self._fn = _lib.lib().muon_step
 
+    def update(self, beta=None, nesterov=None, lr=None, wd=None, steps=None):
+        """Change hyper-parameters for the following calls (None keeps a value)."""
+        old = self._hyper
+        self._hyper = (float(old[0] if beta is None else beta),
+                       int(bool(old[1] if nesterov is None else nesterov)),
+                       float(old[2] if lr is None else lr), float(old[3] if wd is None else wd),
+                       int(old[4] if steps is None else steps))
+
     def __call__(self, stream=None):
         beta, nest, lr, wd, steps = self._hyper
         check(self._fn(len(self.params), self._p, self._g, self._m, self._s, beta, nest, lr, wd,

@@ -146,8 +146,16 @@ class ShardedMuon:
                                     async_op=True)
 
     # ------------------------------------------------------------------ step
-    def step(self):
-        """One optimizer step over the group (every rank calls it)."""
+    def step(self, lr=None, wd=None):
+        """One optimizer step over the group (every rank calls it, with the same
+        arguments).  ``lr`` / ``wd`` replace the constructor's values from this
+        step on (a learning-rate schedule); None keeps the current one."""
+        if lr is not None or wd is not None:
+            b_, n_, lr_, wd_, st_ = self.hyper
+            self.hyper = (b_, n_, float(lr_ if lr is None else lr), float(wd_ if wd is None else wd), st_)
+            for bk in self._buckets:
+                if bk["plan"] is not None:
+                    bk["plan"].update(lr=self.hyper[2], wd=self.hyper[3])
         for bk in self._buckets:
             self._reduce_scatter_avg(bk["G"], bk["slot"])
         pending = []

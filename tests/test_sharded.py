@@ -76,6 +76,22 @@ def test_longest_first_on_a_small_case():
     assert owner == [1, 0, 0, 1]
 
 
+def test_learning_rate_schedule_per_step():
+    """step(lr=, wd=) changes the values the local step receives from then on."""
+    from newton_schulz_12_b200.sharded import ShardedMuon
+    seen = []
+
+    def record(params, grads, bufs, beta, nesterov, lr, wd, steps):
+        seen.append((lr, wd))
+
+    sm = ShardedMuon(SHAPES[:3], buckets=1, grad_dtype=torch.float32, local_step=record, **HYPER)
+    sm.step()
+    sm.step(lr=0.02)
+    sm.step(wd=0.5)
+    sm.step()
+    assert seen == [(0.05, 0.01), (0.02, 0.01), (0.02, 0.5), (0.02, 0.5)]
+
+
 def test_single_rank_step_equals_oracle_step():
     from newton_schulz_12_b200.sharded import ShardedMuon
     sm = ShardedMuon(SHAPES, buckets=3, grad_dtype=torch.float32, local_step=oracle_local_step,
