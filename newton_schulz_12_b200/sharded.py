@@ -74,13 +74,20 @@ class ShardedMuon:
     def __init__(self, shapes, *, device=None, group=None, buckets=2, beta=0.95, nesterov=True,
                  lr=0.05, wd=0.0, steps=5, grad_dtype=torch.bfloat16, local_step=None):
         import torch.distributed as dist
+        for i, shp in enumerate(shapes):
+            if len(shp) != 2 or int(shp[0]) < 1 or int(shp[1]) < 1:
+                raise ValueError(f"shape {i} must be two positive sizes, got {tuple(shp)}")
+        dev = torch.device(device) if device is not None else torch.device("cpu")
+        if local_step is None and (dev.type != "cuda" or grad_dtype != torch.bfloat16):
+            raise ValueError("the library's muon_step needs device='cuda' and bf16 gradients; "
+                             "pass local_step for anything else")
         self.dist = dist if dist.is_available() and dist.is_initialized() else None
         self.group = group
         self.world = self.dist.get_world_size(group) if self.dist else 1
         self.rank = self.dist.get_rank(group) if self.dist else 0
         self.shapes = [(int(r), int(c)) for r, c in shapes]
         self.hyper = (float(beta), bool(nesterov), float(lr), float(wd), int(steps))
-        self.device = torch.device(device) if device is not None else torch.device("cpu")
+        self.device = dev
         self.owner, self.bucket_ranges = plan_ownership(self.shapes, self.world, buckets, steps)
         self._nccl = bool(self.dist) and self.dist.get_backend(group) == "nccl"
 

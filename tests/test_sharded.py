@@ -76,6 +76,23 @@ def test_longest_first_on_a_small_case():
     assert owner == [1, 0, 0, 1]
 
 
+def test_arguments_are_checked_before_any_allocation():
+    from newton_schulz_12_b200.sharded import ShardedMuon
+    with pytest.raises(ValueError, match="device='cuda'"):
+        ShardedMuon([(8, 8)])  # the CUDA step on a CPU device
+    with pytest.raises(ValueError, match="device='cuda'"):
+        ShardedMuon([(8, 8)], device="cuda", grad_dtype=torch.float32)
+    with pytest.raises(ValueError, match="two positive sizes"):
+        ShardedMuon([(8, 0)], local_step=oracle_local_step)
+
+
+def test_no_matrices_is_a_no_op():
+    from newton_schulz_12_b200.sharded import ShardedMuon
+    sm = ShardedMuon([], local_step=oracle_local_step)
+    sm.step()
+    assert sm.params == [] and sm.bucket_ranges == []
+
+
 def test_learning_rate_schedule_per_step():
     """step(lr=, wd=) changes the values the local step receives from then on."""
     from newton_schulz_12_b200.sharded import ShardedMuon
