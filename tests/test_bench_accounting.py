@@ -46,3 +46,26 @@ def test_per_launch_work():
     assert w["bx_apply"][1] == pytest.approx(1019.3e6, rel=1e-4)
     # a step is 5 gram + 5 poly + 5 BX-like launches: the nominal step FLOPs
     assert 5 * (w["gram"][1] + w["poly"][1] + w["bx"][1]) == bench.nominal_flops(SHAPES)
+
+
+def test_reference_arm_line(capsys, monkeypatch):
+    """`bench.py --impl reference` on rank 0: one JSON line with the arm's own
+    cpu_baseline and an e2e that moves no bytes (the oracle runs on the host)."""
+    import json
+    monkeypatch.delenv("RANK", raising=False)
+
+    class A:
+        steps, warmup, gpus = 1, 1, 1
+
+    bench.run_reference(A())
+    out = capsys.readouterr().out.strip().splitlines()
+    assert len(out) == 1
+    line = json.loads(out[0])
+    assert line["impl"] == "reference"
+    assert (line["metric"], line["unit"]) == (bench.METRIC, bench.UNIT)
+    assert line["higher_is_better"] is True and line["value"] > 0
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["config"]["workload"] == bench.WORKLOAD
