@@ -13,7 +13,9 @@ Citations name the page title and the passage:
   account for most of the speedup" (record #3).
 * [Overview ¶Reading guide] the same page, paragraph "Reading guide": later
   refinements tune the same update, among them Polar Express polynomials
-  (per-step coefficients; none are printed on the pages).
+  (per-step coefficients; none are printed on the pages), NorMuon's
+  per-neuron rescale and cautious weight decay (no formulas on the pages;
+  the readings are stated at ``normuon_rescale`` and ``cautious_mask``).
 """
 from __future__ import annotations
 
@@ -109,11 +111,62 @@ def update_scale(rows, cols):
     return math.sqrt(max(1.0, rows / cols))
 
 
-def apply_update(W, O, lr, wd, scale):
-    """W' = W - lr*wd*W - lr*scale*O (decoupled weight decay from the pre-update W)."""
+#: NorMuon's second-moment coefficient and the guard inside its 1/sqrt
+#: (reading; the pages give neither).
+NORMUON_BETA2 = 0.95
+NORMUON_EPS = 1e-10
+
+
+def cautious_mask(W, O):
+    """Cautious weight decay's mask [Overview ¶Reading guide], fp64.
+
+    Reading: decay acts only where it pushes the same way as the update, i.e.
+    where the weight and the update O (which is subtracted) have the same
+    sign, W*O > 0.  Elements where either is zero are not decayed.
+    """
     W = np.asarray(W, dtype=np.float64)
     O = np.asarray(O, dtype=np.float64)
-    return W - lr * wd * W - lr * scale * O
+    return (W * O > 0).astype(np.float64)
+
+
+def apply_update(W, O, lr, wd, scale, cautious=False):
+    """W' = W - lr*wd*W - lr*scale*O (decoupled weight decay from the pre-update W).
+
+    With ``cautious`` the decay term is multiplied by ``cautious_mask(W, O)``.
+    """
+    W = np.asarray(W, dtype=np.float64)
+    O = np.asarray(O, dtype=np.float64)
+    decay = lr * wd * W
+    if cautious:
+        decay = decay * cautious_mask(W, O)
+    return W - decay - lr * scale * O
+
+
+def normuon_rescale(O, v, beta2=NORMUON_BETA2, eps=NORMUON_EPS):
+    """NorMuon's per-neuron rescale of the orthogonalised update [Overview ¶Reading guide], fp64.
+
+    Reading (the pages name it and give no formula): a neuron is a row of W
+    in the caller's layout.  Each row keeps an exponential moving average of
+    its update's mean square, and the update's rows are divided by the root
+    of that average (an Adam-like second moment per neuron); the result is
+    scaled back to the Frobenius norm of O, so the rescale only changes how
+    the update is split over the neurons, not its size:
+
+        r_i  = mean_j O_ij^2
+        v'_i = beta2 v_i + (1 - beta2) r_i
+        D    = diag(1 / sqrt(v' + eps))
+        O'   = (||O||_F / ||D O||_F) D O        (O' = D O when ||D O||_F = 0)
+
+    Returns (O', v').
+    """
+    O = np.asarray(O, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    r = np.mean(O * O, axis=1)
+    v_new = beta2 * v + (1.0 - beta2) * r
+    DO = O / np.sqrt(v_new + eps)[:, None]
+    n_do = np.linalg.norm(DO)
+    g = np.linalg.norm(O) / n_do if n_do > 0 else 1.0
+    return g * DO, v_new
 
 
 def muon_step(W, grad, buf, beta=0.95, nesterov=True, lr=0.05, wd=0.0,
@@ -128,6 +181,26 @@ def muon_step(W, grad, buf, beta=0.95, nesterov=True, lr=0.05, wd=0.0,
     r, s = O.shape
     W_new = apply_update(W, O, lr, wd, update_scale(r, s))
     return W_new, new_buf, O
+
+
+def muon_step_ex(W, grad, buf, beta=0.95, nesterov=True, lr=0.05, wd=0.0, steps=NS_STEPS,
+                 coeffs=NS_COEFFS, eps=NORM_EPS, cautious=False, neuron_state=None,
+                 beta2=NORMUON_BETA2):
+    """``muon_step`` with the refinements of [Overview ¶Reading guide], fp64.
+
+    Momentum -> orthogonalise -> (NorMuon rescale when ``neuron_state`` is
+    given) -> scale and apply (cautious decay when ``cautious``).  Returns
+    (W', buf', O', v') with O' the update applied and v' the new state (None
+    without NorMuon).
+    """
+    new_buf, u = momentum(grad, buf, beta, nesterov)
+    O = newton_schulz(u, steps, coeffs, eps)
+    v_new = None
+    if neuron_state is not None:
+        O, v_new = normuon_rescale(O, neuron_state, beta2)
+    r, s = O.shape
+    W_new = apply_update(W, O, lr, wd, update_scale(r, s), cautious=cautious)
+    return W_new, new_buf, O, v_new
 
 
 def ns_flops(rows, cols, steps=NS_STEPS):

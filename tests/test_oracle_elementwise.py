@@ -107,3 +107,114 @@ def test_muon_step_composes_the_steps():
     assert np.array_equal(nb, nb_ref) and np.array_equal(O, O_ref)
     assert O.shape == (12, 5)
     assert np.allclose(W2, W - 0.1 * 0.01 * W - 0.1 * np.sqrt(12 / 5) * O, rtol=0, atol=1e-15)
+
+
+# ------------------------------------------------------------------ pair format
+# The pair (hi, q) is how the bf16 path carries X between Newton-Schulz steps;
+# its definition is the library's (header), restated in oracle/fp32_ref.py.
+from fractions import Fraction  # noqa: E402
+
+from oracle.fp32_ref import fma_f32, pair_encode, pair_value  # noqa: E402
+
+
+def _exponent(hi):
+    return int(np.floor(np.log2(abs(float(hi)))))
+
+
+def test_pair_value_closed_form():
+    """value = hi + q 2^(E-15), checked on hand-picked hi (E read off by hand)."""
+    hi = np.float32([1.0, 1.5, -0.75, 3.0, 2.0 ** -20])
+    q = np.int8([1, -3, 127, -128, 5])
+    want = [1.0 + 2.0 ** -15, 1.5 - 3 * 2.0 ** -15, -0.75 + 127 * 2.0 ** -16, 3.0 - 128 * 2.0 ** -14,
+            2.0 ** -20 + 5 * 2.0 ** -35]
+    assert np.array_equal(pair_value(hi, q), np.array(want))
+    # residual unused at 0, for subnormal hi and below 2^-111
+    tiny = np.float32([0.0, -0.0, 2.0 ** -130, 2.0 ** -112, 2.0 ** -111])
+    got = pair_value(tiny, np.int8([9, 9, 9, 9, 1]))
+    assert np.array_equal(got[:4], tiny[:4].astype(np.float64))
+    assert got[4] == 2.0 ** -111 + 2.0 ** -126
+
+
+def test_pair_encode_bound_and_range():
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal(50000) * 2.0 ** rng.integers(-60, 60, 50000)).astype(np.float32)
+    hi, q = pair_encode(x)
+    assert np.array_equal(hi, bf16_round(x))
+    err = np.abs(pair_value(hi, q) - x.astype(np.float64))
+    E = np.floor(np.log2(np.abs(hi.astype(np.float64))))
+    unit = 2.0 ** (E - 15)
+    assert np.all(err <= unit)                                      # 2^(E-15) at most (the clamp)
+    clamped = (q == 127) & (x.astype(np.float64) - hi > 127.5 * unit)
+    assert np.all(err[~clamped] <= unit[~clamped] / 2)              # 2^(E-16) otherwise
+
+
+def test_pair_encode_round_trips_every_residual():
+    """Brute force: for a spread of hi and every q whose value still rounds to
+    hi (not at a bf16 tie), encoding the value gives back exactly (hi, q)."""
+    rng = np.random.default_rng(6)
+    his = bf16_round((rng.standard_normal(64) * 2.0 ** rng.integers(-30, 30, 64)).astype(np.float32))
+    his = np.concatenate([his, np.float32([1.0, -2.0, 0.5, 1.0078125])])
+    for h in his:
+        qs = np.arange(-128, 128, dtype=np.int64)
+        v = pair_value(np.full(qs.shape, h, np.float32), qs)
+        v32 = v.astype(np.float32)
+        assert np.array_equal(v32.astype(np.float64), v)             # exact in fp32
+        keep = bf16_round(v32) == h
+        # a value exactly halfway to a neighbouring bf16 is a tie the encoder may
+        # round either way: leave those out
+        bits = int(np.float32(h).view(np.uint32)) >> 16
+        nb = np.array([(bits - 1) << 16, (bits + 1) << 16], dtype=np.uint32).view(np.float32)
+        mids = (nb.astype(np.float64) + float(h)) / 2.0
+        keep &= (v != mids[0]) & (v != mids[1])
+        hh, qq = pair_encode(v32[keep])
+        assert np.all(hh == h)
+        assert np.array_equal(qq.astype(np.int64), qs[keep]), float(h)
+
+
+def _round_fraction_f32(v):
+    """Nearest-even float32 of an exact rational (normal range), by integers only."""
+    if v == 0:
+        return 0.0
+    sign = -1 if v < 0 else 1
+    v = abs(v)
+    e = v.numerator.bit_length() - v.denominator.bit_length()
+    while Fraction(2) ** e > v:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= v:
+        e += 1
+    t = v * Fraction(2) ** (23 - e)                  # in [2^23, 2^24)
+    n = t.numerator // t.denominator
+    rest = t - n
+    if rest > Fraction(1, 2) or (rest == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return sign * float(Fraction(n) * Fraction(2) ** (e - 23))
+
+
+def test_fma_f32_hand_worked_ties():
+    """a x + c exactly halfway between two float32 values except for a tail
+    below float64's reach: the tail decides the rounding."""
+    one_m = np.float32(1 - 2.0 ** -24)   # a = 1 + 2^-23, x = 1 - 2^-24: a x = 1 + 2^-24 - 2^-47
+    a = np.float32(1 + 2.0 ** -23)
+    up = np.float32(2.0 ** -47 * (1 + 2.0 ** -23))    # exact sum 1 + 2^-24 + 2^-70: rounds up
+    down = np.float32(2.0 ** -47 * (1 - 2.0 ** -24))  # exact sum 1 + 2^-24 - 2^-71: rounds down
+    assert fma_f32(a, one_m, up) == np.float32(1 + 2.0 ** -23)
+    assert fma_f32(a, one_m, down) == np.float32(1.0)
+    # a plain tie (no tail) goes to even
+    assert fma_f32(np.float32(1.0), np.float32(1 + 2.0 ** -23), np.float32(2.0 ** -24)) == np.float32(1 + 2.0 ** -22)
+    assert fma_f32(np.float32(1.0), np.float32(1.0), np.float32(2.0 ** -24)) == np.float32(1.0)
+    # a single product is numpy's float32 multiply
+    assert fma_f32(np.float32(3.4445), np.float32(0.3), np.float32(0.0)) == np.float32(3.4445) * np.float32(0.3)
+
+
+def test_fma_f32_against_exact_rationals():
+    rng = np.random.default_rng(7)
+    n = 3000
+    a = (rng.standard_normal(n) * 2.0 ** rng.integers(-8, 8, n)).astype(np.float32)
+    x = (rng.standard_normal(n) * 2.0 ** rng.integers(-8, 8, n)).astype(np.float32)
+    c = (rng.standard_normal(n) * 2.0 ** rng.integers(-40, 8, n)).astype(np.float32)
+    # near-cancelling and near-tie triples as well
+    c[:500] = -(a[:500].astype(np.float64) * x[:500]).astype(np.float32)
+    got = fma_f32(a, x, c)
+    for i in range(n):
+        want = _round_fraction_f32(Fraction(float(a[i])) * Fraction(float(x[i])) + Fraction(float(c[i])))
+        assert float(got[i]) == want, (i, a[i], x[i], c[i])
