@@ -8,6 +8,7 @@ iid N(0, 0.01^2), fp32 momentum (beta 0.95, Nesterov), lr 0.05, wd 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --ns-cases      # NS-only: batched 768x3072 and the width sweep
+    python bench.py --sharded       # the data-parallel step (ShardedMuon) over the ranks
 
 Prints one JSON line (rank 0).  `value` is matrices/s over all ranks with
 inputs resident in HBM; `e2e` repeats the measurement with the gradients
@@ -15,7 +16,12 @@ copied in from pinned host memory and the updated weights copied back every
 step (the copies of one step overlap the compute of its neighbours).
 Per-kernel device times are taken live with CUDA events on the launching
 stream (the library's timing hooks); `roofline` reports the dominant kernel
-against the measured peaks in MEASURED_PEAKS.json.
+against the measured peaks in MEASURED_PEAKS.json.  After the timed region
+(outside it) the same run adds: `value_sustained`, a loop of at least a
+second without the timing hooks, with its own clock record; `ns_768x3072`,
+muon_ns_orthogonalize on 64 matrices 768x3072 (the three GEMMs and the whole
+call, nominal and executed TFLOP/s); `scaled_set`, the 144-matrix 1024-wide
+set's full muon_step.
 `--impl reference` times the fp64 CPU oracle on a bounded sample instead.
 """
 from __future__ import annotations
@@ -53,6 +59,11 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sharded", action="store_true",
+                    help="time ShardedMuon (reduce-scatter, local step, all-gather) over the ranks "
+                         "instead of independent replicas")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the sustained loop and the NS-only / scaled-set measurements")
     ap.add_argument("--ns-cases", action="store_true",
                     help="instead of the step benchmark: muon_ns_orthogonalize (bf16) on the "
                          "batched 768x3072 case and the square width sweep, one JSON line each")
@@ -81,6 +92,27 @@ def nominal_flops(shapes, steps=5):
     for r, c in shapes:
         m, n = min(r, c), max(r, c)
         tot += steps * (4 * m * m * n + 2 * m ** 3)
+    return tot
+
+
+PAIR_TILE = 256  # rows x columns of one tensor-core pair tile
+K_STAGE = 64     # K of one operand stage
+
+
+def executed_flops(shapes, steps=5):
+    """FLOPs the tensor cores execute per call: whole 256 x 256 pair tiles
+    (padding included), X X^T and A A only on the tiles on or above the
+    diagonal, B X on every tile; K rounded up to the 64-deep stage."""
+    tot = 0
+    for r, c in shapes:
+        m, n = min(r, c), max(r, c)
+        tm = -(-m // PAIR_TILE)
+        tn = -(-n // PAIR_TILE)
+        sym = tm * (tm + 1) // 2
+        kn = -(-n // K_STAGE) * K_STAGE
+        km = -(-m // K_STAGE) * K_STAGE
+        tile = 2 * PAIR_TILE * PAIR_TILE
+        tot += steps * tile * (sym * kn + sym * km + tm * tn * km)
     return tot
 
 
@@ -203,27 +235,36 @@ def cpu_baseline(shapes, budget_s=12.0):
 
 
 def run_reference(args):
-    """`--impl reference`: the fp64 oracle as it stands, on host cores, rank 0 only."""
+    """`--impl reference`: the fp64 oracle as it stands, on host cores, rank 0 only.
+
+    A step is one whole GPT-2-small layer (its 6 hidden matrices: 4x 768x768,
+    768x3072, 3072x768), the same mix and unit as the GPU arm's 72-matrix set."""
     rank = rank_env()[1]
     if rank != 0:
         return
     shapes = gpt2_shapes()
     layer = shapes[:6]
-    for w in range(args.warmup):
-        oracle_matrix_step(layer[w % 6], w % 6)
+
+    def one_layer():
+        for i, s in enumerate(layer):
+            oracle_matrix_step(s, i)
+
+    for _ in range(args.warmup):
+        one_layer()
     t0 = time.perf_counter()
-    for k in range(args.steps):
-        oracle_matrix_step(layer[k % 6], k % 6)
+    for _ in range(args.steps):
+        one_layer()
     dt = time.perf_counter() - t0
-    value = args.steps / dt
+    value = len(layer) * args.steps / dt
     cores = _blas_threads()
-    sample = (f"each step = one matrix of GPT-2-small layer 0, cycling through its 6 shapes "
-              f"(4x 768x768, 768x3072, 3072x768), full Muon step in fp64 numpy")
+    sample = (f"each step = one whole GPT-2-small layer (4x 768x768, 768x3072, 3072x768), "
+              f"full Muon step in fp64 numpy; {args.steps} layers timed")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1000.0 * dt / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "matrices_per_step": 1, "parallelism": "none (host cores)"},
+        "config": {"workload": WORKLOAD, "matrices_per_step": len(layer),
+                   "parallelism": "none (host cores)"},
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -270,6 +311,109 @@ def traffic_record():
     if h.hexdigest() != rec.get("sources_sha256"):
         return None
     return rec
+
+
+# ------------------------------------------------ measurements after the timed region
+def time_steps(fn, n, stream):
+    """Device time (ms) of n calls of fn on `stream`, CUDA events, synchronised on both sides."""
+    import torch
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(n):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
+def measure_sustained(step, stream, dev, ms_hint, units, min_s=1.5):
+    """The same step in a loop of at least `min_s` seconds, timing hooks off:
+    the steady-state rate under the power cap, with its clock record."""
+    n = max(50, int(min_s * 1000.0 / max(ms_hint, 1e-3)) + 1)
+    for _ in range(3):
+        step()
+    with ClockSampler(dev) as clocks:
+        ms = time_steps(step, n, stream)
+    c = clocks.summary()
+    out = {"value": units * n / (ms / 1000.0), "unit": UNIT, "steps": n, "ms_per_step": ms / n,
+           "seconds": ms / 1000.0, "clocks": c}
+    if c.get("sm_mhz"):
+        out["ms_x_sm_ghz"] = ms / n * c["sm_mhz"] / 1000.0
+    return out
+
+
+def measure_ns_768x3072(dev, peaks, reps=20):
+    """muon_ns_orthogonalize (bf16) on 64 matrices 768 x 3072: the three GEMMs
+    (from the timing hooks) and the whole call, nominal and executed TFLOP/s."""
+    import torch
+    import newton_schulz_12_b200 as nsb
+    m, n, batch = 768, 3072, 64
+    g = torch.Generator(device="cpu").manual_seed(3000 + m)
+    xs = [torch.randn(m, n, generator=g).to(torch.bfloat16).to(dev) for _ in range(batch)]
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        nsb.muon_ns_orthogonalize(xs)
+    with ClockSampler(dev) as clocks:
+        nsb.muon_profile_begin()
+        ms = time_steps(lambda: nsb.muon_ns_orthogonalize(xs), reps, stream)
+        prof = nsb.muon_profile_end()
+    if nsb.muon_get_status() != 0:
+        raise RuntimeError("device status in the 768x3072 case: " + nsb.muon_last_error())
+    nominal = nominal_flops([(m, n)] * batch)
+    executed = executed_flops([(m, n)] * batch)
+    gemm_ms = sum(prof[k][0] for k in ("gram", "poly", "bx")) / reps
+    call_ms = ms / reps
+    out = {"batch": batch, "m": m, "n": n, "reps": reps, "call_ms": call_ms, "gemm_ms": gemm_ms,
+           "nominal_gflop": nominal / 1e9, "executed_gflop": executed / 1e9,
+           "gemm_tflops_nominal": nominal / gemm_ms / 1e9, "gemm_tflops_executed": executed / gemm_ms / 1e9,
+           "call_tflops_nominal": nominal / call_ms / 1e9, "call_tflops_executed": executed / call_ms / 1e9,
+           "peak": peaks["bf16_tflops"],
+           "per_kernel_us": {k: v[0] / v[1] * 1e3 for k, v in prof.items() if v[1]},
+           "clocks": clocks.summary()}
+    out["gemm_frac_nominal"] = out["gemm_tflops_nominal"] / peaks["bf16_tflops"]
+    out["gemm_frac_executed"] = out["gemm_tflops_executed"] / peaks["bf16_tflops"]
+    del xs
+    return out
+
+
+def measure_scaled_set(dev, peaks, steps=10):
+    """Full muon_step over the 144-matrix 1024-wide set (24 layers x [4x 1024^2,
+    1024x4096, 4096x1024]), bf16 grads N(0, 0.01^2), fp32 W N(0, 0.02^2),
+    momentum zeros, wd 0.01.  Inputs drawn on the device (seeded)."""
+    import torch
+    import newton_schulz_12_b200 as nsb
+    from newton_schulz_12_b200 import workloads
+    shapes = workloads.scaled_shapes()
+    counts = [r * c for r, c in shapes]
+    total = sum(counts)
+    offs = [0]
+    for k in counts:
+        offs.append(offs[-1] + k)
+    g = torch.Generator(device=dev).manual_seed(5)
+    W_flat = torch.randn(total, generator=g, device=dev) * 0.02
+    G_flat = (torch.randn(total, generator=g, device=dev) * 0.01).to(torch.bfloat16)
+    M_flat = torch.zeros(total, device=dev)
+    view = lambda flat, i: flat[offs[i]:offs[i + 1]].view(shapes[i])  # noqa: E731
+    plan = nsb.MuonStepPlan([view(W_flat, i) for i in range(len(shapes))],
+                            [view(G_flat, i) for i in range(len(shapes))],
+                            [view(M_flat, i) for i in range(len(shapes))], wd=0.01)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        plan(stream)
+    with ClockSampler(dev) as clocks:
+        ms = time_steps(lambda: plan(stream), steps, stream)
+    if nsb.muon_get_status(stream) != 0:
+        raise RuntimeError("device status in the scaled set: " + nsb.muon_last_error())
+    per = ms / steps
+    flops = nominal_flops(shapes)
+    out = {"matrices": len(shapes), "steps": steps, "ms_per_step": per,
+           "value": len(shapes) / (per / 1000.0), "unit": UNIT,
+           "tflops_nominal": flops / per / 1e9, "pct_of_bf16_peak": 100.0 * flops / per / 1e9 / peaks["bf16_tflops"],
+           "l2": "inputs far larger than L2 (W 1.2 GB, momentum 1.2 GB, grads 0.6 GB); no flush",
+           "clocks": clocks.summary()}
+    del plan, W_flat, G_flat, M_flat
+    return out
 
 
 def run_ours(args):
@@ -444,11 +588,95 @@ def run_ours(args):
                     "d2h_bytes_per_step": W_host.numel() * W_host.element_size()},
             "clocks": clocks.summary(),
         }
+        if world == 1 and not args.no_extras:
+            line["value_sustained"] = measure_sustained(step, stream, dev, ms / args.steps, len(shapes))
+            line["ns_768x3072"] = measure_ns_768x3072(dev, peaks)
+            del W_flat, G_flat, M_flat, W, G, M, plan, plans, G_dev, W_stage
+            torch.cuda.empty_cache()
+            line["scaled_set"] = measure_scaled_set(dev, peaks)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(shapes)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------- data-parallel step
+def run_sharded(args):
+    """`--sharded`: ShardedMuon over the ranks -- reduce-scatter of the bf16
+    gradients by owner (NCCL), the local muon_step on the owned matrices, and
+    an asynchronous all-gather of the updated fp32 weights per bucket -- on the
+    72-matrix GPT-2-small set.  A step updates the whole set once, so the work
+    per step is fixed as ranks are added (strong scaling)."""
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    import newton_schulz_12_b200 as nsb
+    from newton_schulz_12_b200 import workloads
+    from newton_schulz_12_b200.sharded import ShardedMuon
+
+    world, rank, local = rank_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    if "MASTER_PORT" not in os.environ:
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            os.environ["MASTER_PORT"] = str(sk.getsockname()[1])
+    dist.init_process_group("nccl", rank=rank, world_size=world, timeout=timedelta(seconds=120),
+                            device_id=dev)
+    peaks, _ = load_peaks()
+    shapes = gpt2_shapes()
+    sm = ShardedMuon(shapes, device=dev, buckets=2, beta=0.95, nesterov=True, lr=0.05, wd=0.0, steps=5)
+    Ws, Gs = workloads.muon_set(shapes, step=0)
+    for i in range(len(shapes)):
+        sm.params[i].copy_(Ws[i])
+        sm.grads[i].copy_(Gs[i])
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        sm.step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev) as clocks:
+        nsb.muon_profile_begin()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            sm.step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        prof = nsb.muon_profile_end()
+    dist.barrier()
+    ms = max_over_ranks(a.elapsed_time(b), dev)
+    kern_ms = sum(t for t, _ in prof.values()) / args.steps
+    kern_max = max_over_ranks(kern_ms, dev)
+    if nsb.muon_get_status(stream) != 0:
+        raise RuntimeError("device status in the sharded run: " + nsb.muon_last_error())
+    owned = sum(1 for o in sm.owner if o == rank)
+    if rank == 0:
+        per = ms / args.steps
+        line = {
+            "metric": METRIC, "value": len(shapes) / (per / 1000.0), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": per,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "matrices_per_step": len(shapes),
+                       "parallelism": f"sharded dp{world}: reduce-scatter of bf16 grads by owner "
+                                      "(NCCL AVG), local muon_step, async all-gather of fp32 W per "
+                                      "bucket (2 buckets)",
+                       "matrices_owned_rank0": owned},
+            "kernel_ms_per_step_max_rank": kern_max,
+            "comm_and_host_ms_per_step": per - kern_max,
+            "tflops": nominal_flops(shapes) / per / 1e9,
+            "gpu_launches": sum(n for _, n in prof.values()),
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
 
 
 # ------------------------------------------------------- NS-only case sweep
@@ -511,6 +739,8 @@ def main():
         args.warmup = 3
     if args.ns_cases:
         run_ns_cases(args)
+    elif args.sharded and args.impl == "ours":
+        run_sharded(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

@@ -141,7 +141,9 @@ int muon_ns_orthogonalize_schedule(int batch, int m, int n, void* const* X_ptrs,
  * events.
  * Set-up: the first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current, and caches it; make that
- * first call before any stream capture begins.
+ * first call before any stream capture begins.  muon_release() forgets the
+ * cached address (the next call looks it up again), which is what a context
+ * re-created after cudaDeviceReset needs.
  * If kernel timing (muon_profile_begin) is on, this call's launches are not
  * timed, so no CUDA event objects are created on its behalf.
  */
@@ -178,6 +180,41 @@ int muon_step(int count, float* const* params, const void* const* grads,
               float* const* momentum_bufs, const int64_t* shapes, float beta, int nesterov,
               float lr, float wd, int steps, void* stream);
 
+/* Option bits of muon_step_ex, muon_apply_ex and muon_bx_apply_bf16. */
+#define MUON_CAUTIOUS_WD 1 /* cautious weight decay (below) */
+
+/*
+ * muon_step_ex -- muon_step with the later refinements of the same update.
+ *
+ * Source: "The NanoGPT speedrun", paragraph "Reading guide", names NorMuon's
+ * per-neuron rescale and cautious weight decay among the refinements that
+ * tune the Muon update; the pages give no formulas, so the library reads them
+ * as follows.
+ *
+ * flags & MUON_CAUTIOUS_WD: the decay term fl(lr*wd)*W is applied only to the
+ *   elements where W and the update O have the same sign (W*O > 0); elsewhere
+ *   W' = fl(W - fl(lr*scale)*O).  Same fp32 operation order otherwise.
+ * neuron_state != NULL: NorMuon's per-neuron rescale.  neuron_state is a HOST
+ *   array of `count` DEVICE pointers, each to `rows` fp32 values (one per row
+ *   of W, the caller's layout; zeros before the first step), updated in place.
+ *   After the iteration, with O the update in W's layout:
+ *     r_i   = mean over row i of O^2
+ *     v_i'  = fl(fl(beta2*v_i) + fl(fl(1-beta2) * fl32(r_i)))      (the state)
+ *     f_i   = 1 / sqrt(v_i' + 1e-10)
+ *     O_i  <- O_i * f_i * g,   g = ||O||_F / ||diag(f) O||_F
+ *   so the update keeps its Frobenius norm and only its split over the rows
+ *   (neurons) changes; then the apply as in muon_step.  Row sums are fp64 in
+ *   a fixed order; the factor f_i g is rounded to fp32 and multiplies O in
+ *   fp32.  This path applies every update in the separate pass.
+ *   beta2 in [0, 1].
+ * neuron_state == NULL and flags == 0 is exactly muon_step.
+ * Returns MUON_OK or a negative muon_status (unknown flag bits: MUON_ERR_ARG).
+ */
+int muon_step_ex(int count, float* const* params, const void* const* grads,
+                 float* const* momentum_bufs, const int64_t* shapes, float beta, int nesterov,
+                 float lr, float wd, int steps, int flags, float* const* neuron_state, float beta2,
+                 void* stream);
+
 /*
  * muon_momentum -- the momentum stage of muon_step on its own.
  *
@@ -202,6 +239,19 @@ int muon_momentum(int count, const void* const* grads, float* const* momentum_bu
  */
 int muon_apply(int count, float* const* params, const float* const* updates,
                const int64_t* shapes, float lr, float wd, void* stream);
+
+/*
+ * muon_apply_ex -- muon_apply with the options of muon_step_ex.
+ *
+ * flags & MUON_CAUTIOUS_WD: decay only where W*O > 0 (as in muon_step_ex).
+ * row_scale: NULL, or a HOST array of `count` DEVICE pointers, each to `rows`
+ *   fp32 factors; row r of matrix i's update is first multiplied by
+ *   row_scale[i][r] in fp32 (the per-neuron factors of muon_step_ex).
+ * Otherwise exactly muon_apply.
+ */
+int muon_apply_ex(int count, float* const* params, const float* const* updates,
+                  const int64_t* shapes, float lr, float wd, int flags,
+                  const float* const* row_scale, void* stream);
 
 /*
  * Stage calls on contiguous bf16 batches (the tensor-core kernels of the
@@ -233,6 +283,43 @@ int muon_bx_bf16(int batch, int m, int n, const void* B, const void* Xhi, void* 
                  void* Xhi_out, float a, void* stream);
 
 /*
+ * muon_bx_apply_bf16 -- the last Newton-Schulz GEMM of muon_step with the
+ * update applied to the weights in its epilogue, on its own.
+ *
+ * Source: "The NanoGPT speedrun", record #3 (the orthogonalised update is
+ * "then scaled and applied"); the apply's operation order is muon_apply's.
+ * muon_step runs exactly this launch for its last step; the call exists so
+ * that the fused epilogue can be checked bit for bit.
+ *
+ * Per matrix i (X_i = the pair Xhi_i, Xlo_i as in muon_bx_bf16, m x n, m <= n):
+ *   O    = fl(a*X + acc),  acc = B_i * hi_i accumulated in fp32 (tensor cores),
+ *          one rounding after a fused multiply-add
+ *   W'   = fl(fl(W - fl(fl(lr*wd)*W)) - fl(fl(lr*scale)*O_W)),  no FMA,
+ *   O_W  = O (tall == 0, W is m x n) or O^T (tall != 0, W is n x m),
+ *   scale = sqrt(max(1, rows/cols)) of W's shape, in fp32;
+ *   with flags & MUON_CAUTIOUS_WD the fl(lr*wd)*W term only where W*O > 0.
+ * batch   number of matrices (>= 0).
+ * ldx     row stride (elements) of Xhi and Xlo; >= n and a multiple of 16.
+ *         Matrix i starts at element i*m*ldx.
+ * B       DEVICE pointer, batch x m x ldb bf16 (row stride ldb >= m, a multiple
+ *         of 8; matrix stride m*ldb).
+ * Xhi     DEVICE pointer, bf16 hi of X; read only.
+ * Xlo     DEVICE pointer, int8 q of X.  Read; overwritten with q of X' for the
+ *         matrices that take the separate pass (below).
+ * W_ptrs  HOST array of `batch` DEVICE pointers to fp32 W (row-major,
+ *         contiguous, 16-byte aligned), updated in place.
+ * The first 96 matrices whose W has a column count that is a multiple of 4
+ * are updated inside the GEMM epilogue with O as above.  The others (past
+ * the first 96, or W columns not a multiple of 4) get X' as the pair (hi in
+ * the library's workspace, q in Xlo) and are updated by the apply pass from
+ * the pair's value, as muon_step does for them.
+ * Returns MUON_OK or a negative muon_status.
+ */
+int muon_bx_apply_bf16(int batch, int m, int n, int ldx, const void* B, int ldb, const void* Xhi,
+                       void* Xlo, float* const* W_ptrs, int tall, float a, float lr, float wd, int flags,
+                       void* stream);
+
+/*
  * muon_get_status -- synchronise `stream`, then return and clear the device
  * status word of (current device, stream): MUON_OK or MUON_ERR_DEVICE_TIMEOUT,
  * or MUON_ERR_CUDA if the synchronisation itself failed.
@@ -245,9 +332,20 @@ const char* muon_last_error(void);
 /*
  * muon_release -- synchronise the device and free every workspace and status
  * word the library holds on the current device.  Safe to call at any time
- * outside stream capture; later calls re-allocate on demand.
+ * outside stream capture; later calls re-allocate on demand.  It also forgets
+ * the cached address of muon_ns_orthogonalize_static's array on this device,
+ * so call it after a device reset (cudaDeviceReset) before using the library
+ * again on that device.
  */
 int muon_release(void);
+
+/*
+ * muon_workspace_bytes -- device memory the library holds for (current
+ * device, stream): its workspace plus the status word, or 0 if it holds
+ * none.  `bytes` is a HOST pointer.  No synchronisation.  The allocation-free
+ * call (muon_ns_orthogonalize_static) never adds to it.
+ */
+int muon_workspace_bytes(void* stream, long long* bytes);
 
 /*
  * muon_set_wait_timeout_ms -- limit of every device-side wait (default 2000 ms).
@@ -288,7 +386,8 @@ typedef enum {
   MUON_KERNEL_PREP = 8, /* momentum + Nesterov blend written as the bf16 + int8 pair (transposing) */
   MUON_KERNEL_SCALE = 9, /* per-matrix 1 / (||u||_F + eps) */
   MUON_KERNEL_BX_APPLY = 10, /* tensor cores: the last step's X' = aX + BX applied to W */
-  MUON_KERNEL_KINDS = 11
+  MUON_KERNEL_NORM = 11,     /* per-neuron rescale: row norms, state, factors */
+  MUON_KERNEL_KINDS = 12
 } muon_kernel_kind;
 
 int muon_profile_begin(void);

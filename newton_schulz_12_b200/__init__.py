@@ -17,14 +17,15 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import MUON_BF16, MUON_FP32, MuonError, check, ptr_array, shape_array
+from ._lib import MUON_BF16, MUON_CAUTIOUS_WD, MUON_FP32, MuonError, check, ptr_array, shape_array
 
 __all__ = [
     "NS_COEFFS", "MuonError", "MuonStepPlan", "muon_ns_orthogonalize",
     "muon_ns_orthogonalize_schedule",
-    "muon_ns_orthogonalize_static", "muon_step", "muon_momentum",
-    "muon_apply", "muon_gram_bf16", "muon_poly_bf16", "muon_bx_bf16", "muon_get_status",
-    "muon_last_error", "muon_release", "muon_set_wait_timeout_ms", "muon_set_fault_injection",
+    "muon_ns_orthogonalize_static", "muon_step", "muon_step_ex", "muon_momentum",
+    "muon_apply", "muon_apply_ex", "MUON_CAUTIOUS_WD", "muon_gram_bf16", "muon_poly_bf16", "muon_bx_bf16",
+    "muon_bx_apply_bf16", "muon_get_status",
+    "muon_last_error", "muon_release", "muon_workspace_bytes", "muon_set_wait_timeout_ms", "muon_set_fault_injection",
     "muon_profile_begin", "muon_profile_end", "muon_version", "MUON_BF16", "MUON_FP32",
 ]
 
@@ -146,6 +147,48 @@ def muon_step(params, grads, momentum_bufs, beta=0.95, nesterov=True, lr=0.05, w
                                beta, int(bool(nesterov)), lr, wd, steps, _stream(stream)))
 
 
+def _step_args(params, grads, momentum_bufs):
+    params, grads, bufs = list(params), list(grads), list(momentum_bufs)
+    if not (len(params) == len(grads) == len(bufs)):
+        raise ValueError("params, grads and momentum_bufs must have the same length")
+    shapes = []
+    for i, (w, g, m) in enumerate(zip(params, grads, bufs)):
+        _check_cuda(w, f"params[{i}]", torch.float32)
+        _check_cuda(g, f"grads[{i}]", torch.bfloat16)
+        _check_cuda(m, f"momentum_bufs[{i}]", torch.float32)
+        if w.dim() != 2 or w.shape != g.shape or w.shape != m.shape:
+            raise ValueError(f"matrix {i}: params, grads and buffers must be equal 2-D shapes")
+        shapes.append(tuple(w.shape))
+    return params, grads, bufs, shapes
+
+
+def muon_step_ex(params, grads, momentum_bufs, beta=0.95, nesterov=True, lr=0.05, wd=0.0, steps=5,
+                 cautious_wd=False, neuron_state=None, beta2=0.95, stream=None):
+    """muon_step with cautious weight decay and / or NorMuon's per-neuron rescale.
+
+    ``neuron_state``: None (off) or a list of fp32 CUDA vectors, one per
+    matrix with one entry per row of W (zeros before the first step), updated
+    in place.
+    """
+    params, grads, bufs, shapes = _step_args(params, grads, momentum_bufs)
+    state = None
+    if neuron_state is not None:
+        neuron_state = list(neuron_state)
+        if len(neuron_state) != len(params):
+            raise ValueError("one neuron_state vector per matrix is required")
+        for i, (v, (r, _)) in enumerate(zip(neuron_state, shapes)):
+            _check_cuda(v, f"neuron_state[{i}]", torch.float32)
+            if v.numel() != r:
+                raise ValueError(f"neuron_state[{i}] must hold {r} values (one per row of W)")
+        state = ptr_array([v.data_ptr() for v in neuron_state])
+    check(_lib.lib().muon_step_ex(len(params), ptr_array([w.data_ptr() for w in params]),
+                                  ptr_array([g.data_ptr() for g in grads]),
+                                  ptr_array([m.data_ptr() for m in bufs]), shape_array(shapes),
+                                  beta, int(bool(nesterov)), lr, wd, steps,
+                                  MUON_CAUTIOUS_WD if cautious_wd else 0, state, beta2,
+                                  _stream(stream)))
+
+
 class MuonStepPlan:
     """muon_step with its arguments marshalled once, for a fixed set of tensors.
 
@@ -225,6 +268,31 @@ def muon_apply(params, updates, lr=0.05, wd=0.0, stream=None):
                                 lr, wd, _stream(stream)))
 
 
+def muon_apply_ex(params, updates, lr=0.05, wd=0.0, cautious_wd=False, row_scale=None, stream=None):
+    """muon_apply with cautious decay and / or per-row factors of the update
+    (``row_scale``: a list of fp32 CUDA vectors, one entry per row of W)."""
+    params, updates = list(params), list(updates)
+    shapes = []
+    for i, (w, o) in enumerate(zip(params, updates)):
+        _check_cuda(w, f"params[{i}]", torch.float32)
+        _check_cuda(o, f"updates[{i}]", torch.float32)
+        if w.shape != o.shape or w.dim() != 2:
+            raise ValueError(f"matrix {i}: params and updates must be equal 2-D shapes")
+        shapes.append(tuple(w.shape))
+    rs = None
+    if row_scale is not None:
+        row_scale = list(row_scale)
+        for i, (f, (r, _)) in enumerate(zip(row_scale, shapes)):
+            _check_cuda(f, f"row_scale[{i}]", torch.float32)
+            if f.numel() != r:
+                raise ValueError(f"row_scale[{i}] must hold {r} values")
+        rs = ptr_array([f.data_ptr() for f in row_scale])
+    check(_lib.lib().muon_apply_ex(len(params), ptr_array([w.data_ptr() for w in params]),
+                                   ptr_array([o.data_ptr() for o in updates]), shape_array(shapes),
+                                   lr, wd, MUON_CAUTIOUS_WD if cautious_wd else 0, rs,
+                                   _stream(stream)))
+
+
 def muon_gram_bf16(X, A=None, stream=None):
     """A = X X^T for a contiguous bf16 batch X (batch, m, k); returns A (batch, m, m)."""
     _check_cuda(X, "X", torch.bfloat16)
@@ -264,6 +332,38 @@ def muon_bx_bf16(B, Xhi, Xlo, a=NS_COEFFS[0], Xhi_out=None, stream=None):
     return Xhi_out
 
 
+def muon_bx_apply_bf16(B, Xhi, Xlo, Ws, n=None, tall=False, a=NS_COEFFS[0], lr=0.05, wd=0.0,
+                       cautious=False, stream=None):
+    """The last step's X' = a X + B X applied to fp32 weights in the GEMM epilogue.
+
+    ``B`` (batch, m, ldb) bf16, ``Xhi`` (batch, m, ldx) bf16 and ``Xlo``
+    (batch, m, ldx) int8 are contiguous batches whose rows may be padded; ``n``
+    is X's logical width (default ldx).  ``Ws`` is a list of ``batch`` fp32
+    CUDA matrices, each (m, n), or (n, m) with ``tall`` (W = O^T).  Updated in
+    place: W <- (W - lr*wd*W) - lr*scale*O (with ``cautious``, the decay only
+    where W and O have the same sign).
+    """
+    _check_cuda(B, "B", torch.bfloat16)
+    _check_cuda(Xhi, "Xhi", torch.bfloat16)
+    _check_cuda(Xlo, "Xlo", torch.int8)
+    bsz, m, ldx = Xhi.shape
+    if tuple(Xlo.shape) != (bsz, m, ldx) or B.dim() != 3 or B.shape[0] != bsz or B.shape[1] != m:
+        raise ValueError("B must be (batch, m, ldb) and Xlo the shape of Xhi")
+    n = ldx if n is None else int(n)
+    Ws = list(Ws)
+    if len(Ws) != bsz:
+        raise ValueError("one weight matrix per batch entry is required")
+    want = (n, m) if tall else (m, n)
+    for i, w in enumerate(Ws):
+        _check_cuda(w, f"Ws[{i}]", torch.float32)
+        if tuple(w.shape) != want:
+            raise ValueError(f"Ws[{i}] must be {want}, got {tuple(w.shape)}")
+    check(_lib.lib().muon_bx_apply_bf16(bsz, m, n, ldx, B.data_ptr(), B.shape[2], Xhi.data_ptr(),
+                                        Xlo.data_ptr(), ptr_array([w.data_ptr() for w in Ws]),
+                                        int(bool(tall)), a, lr, wd,
+                                        MUON_CAUTIOUS_WD if cautious else 0, _stream(stream)))
+
+
 def muon_get_status(stream=None):
     """Synchronise the stream and return (and clear) its device status word."""
     return _lib.lib().muon_get_status(_stream(stream))
@@ -276,6 +376,13 @@ def muon_last_error():
 
 def muon_release():
     check(_lib.lib().muon_release())
+
+
+def muon_workspace_bytes(stream=None):
+    """Device bytes the library holds for (current device, stream)."""
+    out = ctypes.c_longlong(0)
+    check(_lib.lib().muon_workspace_bytes(_stream(stream), ctypes.byref(out)))
+    return out.value
 
 
 def muon_set_wait_timeout_ms(ms):

@@ -18,6 +18,7 @@ LIB_PATH = os.environ.get("MUON_B200_LIB") or os.path.join(
 
 MUON_BF16 = 0
 MUON_FP32 = 1
+MUON_CAUTIOUS_WD = 1
 
 STATUS_NAMES = {
     0: "MUON_OK",
@@ -41,14 +42,18 @@ SIGNATURES = {
     "muon_ns_orthogonalize_static": (_I, [_I, _I, _I, _PP, _F, _F, _F, _I, _P, _P]),
     "muon_ns_orthogonalize_schedule": (_I, [_I, _I, _I, _PP, ctypes.POINTER(_F), _I, _I, _P]),
     "muon_step": (_I, [_I, _PP, _PP, _PP, _I64P, _F, _I, _F, _F, _I, _P]),
+    "muon_step_ex": (_I, [_I, _PP, _PP, _PP, _I64P, _F, _I, _F, _F, _I, _I, _PP, _F, _P]),
     "muon_momentum": (_I, [_I, _PP, _PP, _I64P, _F, _I, _P, _P]),
     "muon_apply": (_I, [_I, _PP, _PP, _I64P, _F, _F, _P]),
+    "muon_apply_ex": (_I, [_I, _PP, _PP, _I64P, _F, _F, _I, _PP, _P]),
     "muon_gram_bf16": (_I, [_I, _I, _I, _P, _P, _P]),
     "muon_poly_bf16": (_I, [_I, _I, _P, _P, _F, _F, _P]),
     "muon_bx_bf16": (_I, [_I, _I, _I, _P, _P, _P, _P, _F, _P]),
+    "muon_bx_apply_bf16": (_I, [_I, _I, _I, _I, _P, _I, _P, _P, _PP, _I, _F, _F, _F, _I, _P]),
     "muon_get_status": (_I, [_P]),
     "muon_last_error": (ctypes.c_char_p, []),
     "muon_release": (_I, []),
+    "muon_workspace_bytes": (_I, [_P, ctypes.POINTER(ctypes.c_longlong)]),
     "muon_set_wait_timeout_ms": (_I, [_I]),
     "muon_set_fault_injection": (_I, [_I]),
     "muon_profile_begin": (_I, []),
@@ -57,7 +62,8 @@ SIGNATURES = {
 }
 
 #: muon_kernel_kind names, in enum order.
-KERNEL_KINDS = ["flat", "cast", "gram", "poly", "bx", "out", "simt", "sums", "prep", "scale", "bx_apply"]
+KERNEL_KINDS = ["flat", "cast", "gram", "poly", "bx", "out", "simt", "sums", "prep", "scale", "bx_apply",
+                "norm"]
 
 _lock = threading.Lock()
 _lib = None

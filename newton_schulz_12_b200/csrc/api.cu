@@ -37,6 +37,7 @@ constexpr int kMaxDim = 32768;
 constexpr int kMaxStepsArg = 100;
 constexpr float kNormEps = 1e-7f;
 constexpr float kCoefA = 3.4445f, kCoefB = -4.7750f, kCoefC = 2.0315f;
+constexpr double kNeuronEps = 1e-10;  // guard inside the per-neuron 1 / sqrt(v + eps)
 
 thread_local std::string t_err;
 
@@ -373,6 +374,7 @@ struct ApplySpec {
   const std::vector<void*>* w = nullptr;  // W (kind 0) or the output (kind 1) of matrix i, caller's layout
   int kind = 0;
   float lr = 0.f, wd = 0.f;
+  int cautious = 0;        // kind 0: decay only where W and O have the same sign
   std::vector<char> done;  // out: matrix i was finished by the GEMM epilogue
 };
 
@@ -393,6 +395,7 @@ int build_apply_table(const std::vector<NsGroup>& gs, size_t g0, size_t g1, Appl
   T.nmat = 0;
   T.mat_base = gs[g0].mat_base;
   T.lw = A.lr * A.wd;
+  T.cautious = A.cautious;
   int span = 0;
   for (size_t gi = g0; gi < g1; ++gi) span += gs[gi].batch;
   T.nmat = std::min(span, tc::kMaxApply);
@@ -838,7 +841,8 @@ int run_bf16_path(const std::vector<MatInfo>& mats, std::vector<NsGroup>& groups
 int launch_out_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGroup>& groups,
                        const std::vector<Result>& res, const std::vector<void*>& ys, int mode,
                        float lr, float wd, cudaStream_t s, const float* oscale = nullptr,
-                       const std::vector<char>* done = nullptr) {
+                       const std::vector<char>* done = nullptr, int cautious = 0,
+                       const std::vector<const float*>* rowf = nullptr) {
   std::vector<int> todo;
   for (int i = 0; i < static_cast<int>(mats.size()); ++i)
     if (!done || !(*done)[i]) todo.push_back(i);
@@ -848,6 +852,7 @@ int launch_out_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGro
     ew::OutParams op{};
     op.mode = mode;
     op.lw = lr * wd;
+    op.cautious = cautious;
     int tiles = 0;
     for (int t = i0; t < i1; ++t) {
       const int i = todo[t];
@@ -868,6 +873,7 @@ int launch_out_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGro
       O.tile_begin = tiles;
       O.ls = apply_ls(M, lr);
       O.oscale = oscale ? oscale + G.mat_base + M.index : nullptr;
+      O.rowf = rowf ? (*rowf)[i] : nullptr;
       O.vec = (M.cols % 8 == 0) && (G.ldn % 8 == 0) && aligned16(ys[i]);
       tiles += ((M.rows + ew::kTile - 1) / ew::kTile) * O.tiles_c;
     }
@@ -875,6 +881,71 @@ int launch_out_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGro
     op.ntiles = tiles;
     ProfScope prof(MUON_KERNEL_OUT, s);
     CUDA_TRY(ew::launch_out(op, s));
+  }
+  return MUON_OK;
+}
+
+// Per-neuron rescale (NorMuon reading): row sums of O^2 of every caller W,
+// then the state update and the row factors.  rsq / rowf hold one entry per
+// W row, matrices in order; rowf_ptrs[i] is matrix i's first factor.
+int launch_norm_chunked(const std::vector<MatInfo>& mats, const std::vector<NsGroup>& groups,
+                        const std::vector<Result>& res, const float* oscale, float* const* state,
+                        float beta2, double* rsq, float* rowf, std::vector<const float*>& rowf_ptrs,
+                        cudaStream_t s) {
+  const int count = static_cast<int>(mats.size());
+  std::vector<long long> base(count);
+  long long rows = 0;
+  for (int i = 0; i < count; ++i) {
+    base[i] = rows;
+    rows += mats[i].rows;
+  }
+  rowf_ptrs.resize(count);
+  for (int i = 0; i < count; ++i) rowf_ptrs[i] = rowf + base[i];
+  for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
+    const int i1 = std::min(count, i0 + ew::kMaxMats);
+    ew::NormStatParams sp{};
+    sp.rsq = rsq;
+    int blk = 0;
+    for (int i = i0; i < i1; ++i) {
+      const MatInfo& M = mats[i];
+      const NsGroup& G = groups[M.group];
+      const Result& R = res[M.group];
+      const long long roff = static_cast<long long>(M.index) * G.m * G.ldn;
+      ew::NormMat& N = sp.mat[i - i0];
+      N.hi = R.hi + roff;
+      N.lo = R.lo + roff;
+      N.oscale = oscale ? oscale + G.mat_base + M.index : nullptr;
+      N.m = G.m;
+      N.n = G.n;
+      N.ld = G.ldn;
+      N.transposed = M.transposed;
+      N.blk_begin = blk;
+      N.row_base = base[i];
+      blk += M.transposed ? (M.rows + ew::kNormRowsTall - 1) / ew::kNormRowsTall
+                          : (M.rows + ew::kNormRowsWide - 1) / ew::kNormRowsWide;
+    }
+    sp.nmat = i1 - i0;
+    sp.nblocks = blk;
+    {
+      ProfScope prof(MUON_KERNEL_NORM, s);
+      CUDA_TRY(ew::launch_norm_stats(sp, s));
+    }
+    ew::NormFacParams fp{};
+    fp.rsq = rsq;
+    fp.rowf = rowf;
+    fp.beta2 = beta2;
+    fp.omb2 = 1.0f - beta2;
+    fp.eps = kNeuronEps;
+    for (int i = i0; i < i1; ++i) {
+      ew::NormFacMat& F = fp.mat[i - i0];
+      F.v = state[i];
+      F.rows = mats[i].rows;
+      F.cols = mats[i].cols;
+      F.row_base = base[i];
+    }
+    fp.nmat = i1 - i0;
+    ProfScope prof(MUON_KERNEL_NORM, s);
+    CUDA_TRY(ew::launch_norm_factors(fp, s));
   }
   return MUON_OK;
 }
@@ -1040,6 +1111,136 @@ int ns_orthogonalize(int batch, int m, int n, void* const* X_ptrs, const float* 
   return MUON_OK;
 }
 
+std::vector<float> constant_schedule(float a, float b, float c, int steps);
+
+// muon_step with its options: flags (MUON_CAUTIOUS_WD) and, when
+// neuron_state is given, the per-neuron rescale of the update (NorMuon
+// reading) with second-moment coefficient beta2.
+int step_impl(int count, float* const* params, const void* const* grads, float* const* momentum_bufs,
+              const int64_t* shapes, float beta, int nesterov, float lr, float wd, int steps, int flags,
+              float* const* neuron_state, float beta2, void* stream) {
+  if (count < 0) return set_err(MUON_ERR_ARG, "count %d < 0", count);
+  if (steps < 0 || steps > kMaxStepsArg) return set_err(MUON_ERR_ARG, "steps %d out of range 0..%d", steps, kMaxStepsArg);
+  if (!finite(beta) || beta < 0.f || beta > 1.f) return set_err(MUON_ERR_ARG, "beta must be in [0, 1]");
+  if (!finite(lr) || !finite(wd)) return set_err(MUON_ERR_ARG, "lr and wd must be finite");
+  if (flags & ~MUON_CAUTIOUS_WD) return set_err(MUON_ERR_ARG, "unknown flags 0x%x", flags);
+  if (neuron_state && (!finite(beta2) || beta2 < 0.f || beta2 > 1.f))
+    return set_err(MUON_ERR_ARG, "beta2 must be in [0, 1]");
+  if (count == 0) return MUON_OK;
+  if (!params || !grads || !momentum_bufs || !shapes)
+    return set_err(MUON_ERR_ARG, "params, grads, momentum_bufs and shapes must be non-NULL");
+  std::vector<std::pair<int, int>> shp(count);
+  for (int i = 0; i < count; ++i) {
+    MUON_TRY(check_shape(shapes[2 * i], shapes[2 * i + 1], i));
+    shp[i] = std::make_pair(static_cast<int>(shapes[2 * i]), static_cast<int>(shapes[2 * i + 1]));
+    MUON_TRY(check_ptr(params[i], "params", i));
+    MUON_TRY(check_ptr(grads[i], "grads", i));
+    MUON_TRY(check_ptr(momentum_bufs[i], "momentum_bufs", i));
+    if (neuron_state) {
+      if (!neuron_state[i]) return set_err(MUON_ERR_ARG, "neuron_state[%d] is NULL", i);
+      if (reinterpret_cast<uintptr_t>(neuron_state[i]) & 3u)
+        return set_err(MUON_ERR_ARG, "neuron_state[%d] is not 4-byte aligned", i);
+    }
+  }
+  DevInfo dev;
+  MUON_TRY(device_info(&dev));
+  cudaStream_t s = as_stream(stream);
+
+  std::vector<MatInfo> mats;
+  std::vector<NsGroup> groups;
+  group_shapes(shp, mats, groups);
+  assign_mat_base(groups);
+  BfLayout L;
+  size_t off = bf16_layout(mats, groups, nullptr, L);
+  long long wrows = 0;
+  for (const MatInfo& M : mats) wrows += M.rows;
+  const size_t norm_off = align_up(off, 1024);
+  if (neuron_state) off = align_up(norm_off + static_cast<size_t>(wrows) * 8, 1024) + static_cast<size_t>(wrows) * 4;
+  Workspace* ws = nullptr;
+  MUON_TRY(get_workspace(s, off, &ws));
+  char* base = static_cast<char*>(ws->ptr);
+  bf16_layout(mats, groups, base, L);
+
+  std::vector<const void*> gsrc(grads, grads + count);
+  std::vector<float*> bufs(momentum_bufs, momentum_bufs + count);
+  const std::vector<float> abc = constant_schedule(kCoefA, kCoefB, kCoefC, steps);
+  std::vector<void*> ys(params, params + count);
+  const int cautious = (flags & MUON_CAUTIOUS_WD) ? 1 : 0;
+  // the last step applies the update to W in its epilogue where it can; the
+  // per-neuron rescale needs every row's norm first, so it takes the pass
+  ApplySpec apply;
+  apply.mats = &mats;
+  apply.w = &ys;
+  apply.lr = lr;
+  apply.wd = wd;
+  apply.cautious = cautious;
+  apply.done.assign(count, 0);
+  MUON_TRY(run_bf16_path(mats, groups, L, gsrc, bufs, ew::kFromMomentum, beta, nesterov,
+                         abc.data(), steps, ws->status, dev.sms, s, neuron_state ? nullptr : &apply));
+  std::vector<Result> res;
+  for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
+  const float* oscale = steps == 0 ? L.xscale : nullptr;
+  if (!neuron_state)
+    return launch_out_chunked(mats, groups, res, ys, 0, lr, wd, s, oscale, &apply.done, cautious);
+  double* rsq = reinterpret_cast<double*>(base + norm_off);
+  float* rowf = reinterpret_cast<float*>(base + align_up(norm_off + static_cast<size_t>(wrows) * 8, 1024));
+  std::vector<const float*> rowf_ptrs;
+  MUON_TRY(launch_norm_chunked(mats, groups, res, oscale, neuron_state, beta2, rsq, rowf, rowf_ptrs, s));
+  return launch_out_chunked(mats, groups, res, ys, 0, lr, wd, s, oscale, nullptr, cautious, &rowf_ptrs);
+}
+
+// muon_apply with its options: flags (MUON_CAUTIOUS_WD) and optional per-row
+// factors of O (row_scale[i][r] multiplies row r of matrix i's update first).
+int apply_impl(int count, float* const* params, const float* const* updates, const int64_t* shapes,
+               float lr, float wd, int flags, const float* const* row_scale, void* stream) {
+  if (count < 0) return set_err(MUON_ERR_ARG, "count %d < 0", count);
+  if (!finite(lr) || !finite(wd)) return set_err(MUON_ERR_ARG, "lr and wd must be finite");
+  if (flags & ~MUON_CAUTIOUS_WD) return set_err(MUON_ERR_ARG, "unknown flags 0x%x", flags);
+  if (count == 0) return MUON_OK;
+  if (!params || !updates || !shapes) return set_err(MUON_ERR_ARG, "params, updates and shapes must be non-NULL");
+  for (int i = 0; i < count; ++i) {
+    MUON_TRY(check_shape(shapes[2 * i], shapes[2 * i + 1], i));
+    MUON_TRY(check_ptr(params[i], "params", i));
+    MUON_TRY(check_ptr(updates[i], "updates", i));
+    if (row_scale && (!row_scale[i] || (reinterpret_cast<uintptr_t>(row_scale[i]) & 3u)))
+      return set_err(MUON_ERR_ARG, "row_scale[%d] is NULL or not 4-byte aligned", i);
+  }
+  DevInfo dev;
+  MUON_TRY(device_info(&dev));
+  cudaStream_t s = as_stream(stream);
+  for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
+    const int i1 = std::min(count, i0 + ew::kMaxMats);
+    ew::OutParams op{};
+    op.mode = 0;
+    op.lw = lr * wd;
+    op.cautious = (flags & MUON_CAUTIOUS_WD) ? 1 : 0;
+    int tiles = 0;
+    for (int i = i0; i < i1; ++i) {
+      const int r = static_cast<int>(shapes[2 * i]), c = static_cast<int>(shapes[2 * i + 1]);
+      ew::OutMat& O = op.mat[i - i0];
+      O.y = params[i];
+      O.o = updates[i];
+      O.rows = r;
+      O.cols = c;
+      O.o_transposed = 0;
+      O.ld = c;
+      O.tiles_c = (c + ew::kTile - 1) / ew::kTile;
+      O.tile_begin = tiles;
+      const float ratio = static_cast<float>(r) / static_cast<float>(c);
+      const float scale = ratio > 1.0f ? sqrtf(ratio) : 1.0f;
+      O.ls = lr * scale;
+      O.rowf = row_scale ? row_scale[i] : nullptr;
+      O.vec = (c % 8 == 0) && aligned16(params[i]) && aligned16(updates[i]);
+      tiles += ((r + ew::kTile - 1) / ew::kTile) * O.tiles_c;
+    }
+    op.nmat = i1 - i0;
+    op.ntiles = tiles;
+    ProfScope prof(MUON_KERNEL_OUT, s);
+    CUDA_TRY(ew::launch_out(op, s));
+  }
+  return MUON_OK;
+}
+
 // The fixed triple as a table of `steps` rows.
 std::vector<float> constant_schedule(float a, float b, float c, int steps) {
   std::vector<float> t;
@@ -1129,53 +1330,17 @@ int muon_step(int count, float* const* params, const void* const* grads,
               float* const* momentum_bufs, const int64_t* shapes, float beta, int nesterov,
               float lr, float wd, int steps, void* stream) {
   t_err.clear();
-  if (count < 0) return set_err(MUON_ERR_ARG, "count %d < 0", count);
-  if (steps < 0 || steps > kMaxStepsArg) return set_err(MUON_ERR_ARG, "steps %d out of range 0..%d", steps, kMaxStepsArg);
-  if (!finite(beta) || beta < 0.f || beta > 1.f) return set_err(MUON_ERR_ARG, "beta must be in [0, 1]");
-  if (!finite(lr) || !finite(wd)) return set_err(MUON_ERR_ARG, "lr and wd must be finite");
-  if (count == 0) return MUON_OK;
-  if (!params || !grads || !momentum_bufs || !shapes)
-    return set_err(MUON_ERR_ARG, "params, grads, momentum_bufs and shapes must be non-NULL");
-  std::vector<std::pair<int, int>> shp(count);
-  for (int i = 0; i < count; ++i) {
-    MUON_TRY(check_shape(shapes[2 * i], shapes[2 * i + 1], i));
-    shp[i] = std::make_pair(static_cast<int>(shapes[2 * i]), static_cast<int>(shapes[2 * i + 1]));
-    MUON_TRY(check_ptr(params[i], "params", i));
-    MUON_TRY(check_ptr(grads[i], "grads", i));
-    MUON_TRY(check_ptr(momentum_bufs[i], "momentum_bufs", i));
-  }
-  DevInfo dev;
-  MUON_TRY(device_info(&dev));
-  cudaStream_t s = as_stream(stream);
+  return step_impl(count, params, grads, momentum_bufs, shapes, beta, nesterov, lr, wd, steps, 0,
+                   nullptr, 0.f, stream);
+}
 
-  std::vector<MatInfo> mats;
-  std::vector<NsGroup> groups;
-  group_shapes(shp, mats, groups);
-  assign_mat_base(groups);
-  BfLayout L;
-  size_t off = bf16_layout(mats, groups, nullptr, L);
-  Workspace* ws = nullptr;
-  MUON_TRY(get_workspace(s, off, &ws));
-  bf16_layout(mats, groups, static_cast<char*>(ws->ptr), L);
-
-  std::vector<const void*> gsrc(grads, grads + count);
-  std::vector<float*> bufs(momentum_bufs, momentum_bufs + count);
-  const std::vector<float> abc = constant_schedule(kCoefA, kCoefB, kCoefC, steps);
-  std::vector<void*> ys(params, params + count);
-  // the last step applies the update to W in its epilogue where it can
-  ApplySpec apply;
-  apply.mats = &mats;
-  apply.w = &ys;
-  apply.lr = lr;
-  apply.wd = wd;
-  apply.done.assign(count, 0);
-  MUON_TRY(run_bf16_path(mats, groups, L, gsrc, bufs, ew::kFromMomentum, beta, nesterov,
-                         abc.data(), steps, ws->status, dev.sms, s, &apply));
-  std::vector<Result> res;
-  for (NsGroup& g : groups) res.push_back(bf16_result(g, steps));
-  MUON_TRY(launch_out_chunked(mats, groups, res, ys, 0, lr, wd, s, steps == 0 ? L.xscale : nullptr,
-                              &apply.done));
-  return MUON_OK;
+int muon_step_ex(int count, float* const* params, const void* const* grads,
+                 float* const* momentum_bufs, const int64_t* shapes, float beta, int nesterov,
+                 float lr, float wd, int steps, int flags, float* const* neuron_state, float beta2,
+                 void* stream) {
+  t_err.clear();
+  return step_impl(count, params, grads, momentum_bufs, shapes, beta, nesterov, lr, wd, steps, flags,
+                   neuron_state, beta2, stream);
 }
 
 int muon_momentum(int count, const void* const* grads, float* const* momentum_bufs,
@@ -1226,47 +1391,13 @@ int muon_momentum(int count, const void* const* grads, float* const* momentum_bu
 int muon_apply(int count, float* const* params, const float* const* updates, const int64_t* shapes,
                float lr, float wd, void* stream) {
   t_err.clear();
-  if (count < 0) return set_err(MUON_ERR_ARG, "count %d < 0", count);
-  if (!finite(lr) || !finite(wd)) return set_err(MUON_ERR_ARG, "lr and wd must be finite");
-  if (count == 0) return MUON_OK;
-  if (!params || !updates || !shapes) return set_err(MUON_ERR_ARG, "params, updates and shapes must be non-NULL");
-  for (int i = 0; i < count; ++i) {
-    MUON_TRY(check_shape(shapes[2 * i], shapes[2 * i + 1], i));
-    MUON_TRY(check_ptr(params[i], "params", i));
-    MUON_TRY(check_ptr(updates[i], "updates", i));
-  }
-  DevInfo dev;
-  MUON_TRY(device_info(&dev));
-  cudaStream_t s = as_stream(stream);
-  for (int i0 = 0; i0 < count; i0 += ew::kMaxMats) {
-    const int i1 = std::min(count, i0 + ew::kMaxMats);
-    ew::OutParams op{};
-    op.mode = 0;
-    op.lw = lr * wd;
-    int tiles = 0;
-    for (int i = i0; i < i1; ++i) {
-      const int r = static_cast<int>(shapes[2 * i]), c = static_cast<int>(shapes[2 * i + 1]);
-      ew::OutMat& O = op.mat[i - i0];
-      O.y = params[i];
-      O.o = updates[i];
-      O.rows = r;
-      O.cols = c;
-      O.o_transposed = 0;
-      O.ld = c;
-      O.tiles_c = (c + ew::kTile - 1) / ew::kTile;
-      O.tile_begin = tiles;
-      const float ratio = static_cast<float>(r) / static_cast<float>(c);
-      const float scale = ratio > 1.0f ? sqrtf(ratio) : 1.0f;
-      O.ls = lr * scale;
-      O.vec = (c % 8 == 0) && aligned16(params[i]) && aligned16(updates[i]);
-      tiles += ((r + ew::kTile - 1) / ew::kTile) * O.tiles_c;
-    }
-    op.nmat = i1 - i0;
-    op.ntiles = tiles;
-    ProfScope prof(MUON_KERNEL_OUT, s);
-    CUDA_TRY(ew::launch_out(op, s));
-  }
-  return MUON_OK;
+  return apply_impl(count, params, updates, shapes, lr, wd, 0, nullptr, stream);
+}
+
+int muon_apply_ex(int count, float* const* params, const float* const* updates, const int64_t* shapes,
+                  float lr, float wd, int flags, const float* const* row_scale, void* stream) {
+  t_err.clear();
+  return apply_impl(count, params, updates, shapes, lr, wd, flags, row_scale, stream);
 }
 
 static int stage_common(int batch, int m, int k, DevInfo* dev, Workspace** ws, cudaStream_t s) {
@@ -1341,6 +1472,81 @@ int muon_bx_bf16(int batch, int m, int n, const void* B, const void* Xhi, void* 
   return launch_tc(tc::kBx, P, dev.sms, s);
 }
 
+int muon_bx_apply_bf16(int batch, int m, int n, int ldx, const void* B, int ldb, const void* Xhi,
+                       void* Xlo, float* const* W_ptrs, int tall, float a, float lr, float wd, int flags,
+                       void* stream) {
+  t_err.clear();
+  if (flags & ~MUON_CAUTIOUS_WD) return set_err(MUON_ERR_ARG, "unknown flags 0x%x", flags);
+  if (batch < 0 || batch > 65535) return set_err(MUON_ERR_ARG, "batch %d out of range 0..65535", batch);
+  if (!finite(a) || !finite(lr) || !finite(wd)) return set_err(MUON_ERR_ARG, "a, lr and wd must be finite");
+  if (batch == 0) return MUON_OK;
+  MUON_TRY(check_shape(m, n, 0));
+  if (m > n) return set_err(MUON_ERR_SHAPE, "muon_bx_apply_bf16 expects m <= n (got %dx%d)", m, n);
+  if (ldx < n || ldx % 16 || ldb < m || ldb % 8)
+    return set_err(MUON_ERR_SHAPE,
+                   "row strides: ldx (%d) must be >= n (%d) and a multiple of 16, ldb (%d) >= m (%d) "
+                   "and a multiple of 8", ldx, n, ldb, m);
+  if (!B || !Xhi || !Xlo || !aligned16(B) || !aligned16(Xhi) || !aligned16(Xlo))
+    return set_err(MUON_ERR_ARG, "B, Xhi and Xlo must be non-NULL and 16-byte aligned");
+  if (!W_ptrs) return set_err(MUON_ERR_ARG, "W_ptrs is NULL");
+  for (int i = 0; i < batch; ++i) MUON_TRY(check_ptr(W_ptrs[i], "W_ptrs", i));
+  DevInfo dev;
+  MUON_TRY(device_info(&dev));
+  MUON_TRY(get_encoder());
+  cudaStream_t s = as_stream(stream);
+
+  // One shape group over the caller's contiguous batch, laid out as the
+  // iteration's workspace would be (matrix strides m * ldx and m * ldb).
+  std::vector<NsGroup> gs(1);
+  NsGroup& G = gs[0];
+  G.batch = batch;
+  G.m = m;
+  G.n = n;
+  G.ldn = ldx;
+  G.ldm = ldb;
+  G.mat_base = 0;
+  G.B = static_cast<bf16*>(const_cast<void*>(B));
+  G.xb[0] = static_cast<bf16*>(const_cast<void*>(Xhi));
+  G.xlo = static_cast<int8_t*>(Xlo);
+  std::vector<MatInfo> mats(batch);
+  for (int i = 0; i < batch; ++i)
+    mats[i] = MatInfo{tall ? n : m, tall ? m : n, m, n, tall ? 1 : 0, 0, i};
+  std::vector<void*> ws_ptrs(W_ptrs, W_ptrs + batch);
+  ApplySpec apply;
+  apply.mats = &mats;
+  apply.w = &ws_ptrs;
+  apply.kind = 0;
+  apply.lr = lr;
+  apply.wd = wd;
+  apply.cautious = (flags & MUON_CAUTIOUS_WD) ? 1 : 0;
+  apply.done.assign(batch, 0);
+  tc::LaunchApply table;
+  MUON_TRY(build_apply_table(gs, 0, 1, apply, table));
+  // Matrices the epilogue cannot update (past the table, or W rows not 16-byte
+  // strided) get X' as the pair: hi into a workspace buffer, q into Xlo.
+  bool any_pair = false;
+  for (int i = 0; i < batch; ++i) any_pair |= !apply.done[i];
+  Workspace* ws = nullptr;
+  const size_t hi_bytes = static_cast<size_t>(batch) * m * ldx * 2;
+  MUON_TRY(get_workspace(s, any_pair ? hi_bytes : 0, &ws));
+  G.xb[1] = any_pair ? static_cast<bf16*>(ws->ptr) : G.xb[0];
+
+  tc::Params P;
+  init_tc_params(P, ws->status, a, 0.f, 0.f);
+  P.grp[0] = tc_group(batch, m, n, m, false, 0);
+  const long long xs = static_cast<long long>(m) * ldx, as = static_cast<long long>(m) * ldb;
+  MUON_TRY(bx_maps(P.map[0], G.B, ldb, as, G.xb[0], G.xlo, G.xb[1], m, n, ldx, xs, batch,
+                   tc::bx_apply_chunk()));
+  P.ngroups = 1;
+  P.total_tiles = batch * P.grp[0].tiles_per_mat;
+  MUON_TRY(launch_tc(tc::kBxApply, P, dev.sms, s, &table));
+  if (!any_pair) return MUON_OK;
+  std::vector<Result> res(1);
+  res[0].hi = G.xb[1];
+  res[0].lo = G.xlo;
+  return launch_out_chunked(mats, gs, res, ws_ptrs, 0, lr, wd, s, nullptr, &apply.done, apply.cautious);
+}
+
 int muon_get_status(void* stream) {
   t_err.clear();
   cudaStream_t s = as_stream(stream);
@@ -1411,11 +1617,28 @@ int muon_profile_end(int kinds, double* total_ms, int* launches) {
   return rc == MUON_OK ? n : rc;
 }
 
+int muon_workspace_bytes(void* stream, long long* bytes) {
+  t_err.clear();
+  if (!bytes) return set_err(MUON_ERR_ARG, "bytes is NULL");
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_ws.find({dev, reinterpret_cast<uintptr_t>(stream)});
+  *bytes = 0;
+  if (it != g_ws.end()) *bytes = static_cast<long long>(it->second.bytes) + (it->second.status ? 256 : 0);
+  return MUON_OK;
+}
+
 int muon_release(void) {
   t_err.clear();
   int dev = 0;
   CUDA_TRY(cudaGetDevice(&dev));
   CUDA_TRY(cudaDeviceSynchronize());
+  {
+    // a context re-created after a reset places the static scratch anew
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    g_static_addr.erase(dev);
+  }
   std::lock_guard<std::mutex> lk(g_mu);
   for (auto it = g_ws.begin(); it != g_ws.end();) {
     if (it->first.first == dev) {

@@ -17,12 +17,17 @@
 //                 result into the caller's bf16 / fp32 buffer, with O read
 //                 (from fp32 or from the pair) through the same transposing tile.
 //   sums_kernel   per-matrix sum of flat_kernel's partials.
+//   norm_stats_kernel / norm_factor_kernel
+//                 the per-neuron rescale (NorMuon reading): row sums of O^2 of
+//                 the caller's W rows, the fp32 second-moment state and the
+//                 factor each row of O is multiplied by before the apply.
 //
 // Operation order of momentum and apply is fixed with explicit round-to-nearest
 // intrinsics (no contraction into FMA) so that they are bit-exact against an
 // fp32 computation of the same order:
 //   buf' = (beta*buf) + (omb*g),  u = (omb*g) + (beta*buf'),  omb = 1 - beta
 //   W'   = (W - lw*W) - ls*O,     lw = lr*wd,  ls = lr*scale
+//          (cautious decay: the lw*W term only where W and O have the same sign)
 // ("NanoGPT Speedrun: The Ultimate Guide...", section "Optimizer and Training
 // Strategy Tuning": orthogonalise after the Nesterov-momentum update.)
 #include "common.cuh"
@@ -329,19 +334,34 @@ __device__ __forceinline__ void load_o8(const OutMat& M, int r, int c, int orows
   for (int k = 0; k < 8; ++k) o[k] = k < cnt ? M.o[idx + k] : 0.f;
 }
 
+// One weight after the apply: W' = (W - d) - ls O with d = fl(lw W), or d = 0
+// where cautious decay masks it (W and O not of the same sign), each
+// operation rounded to nearest, no fused multiply-add.
+__device__ __forceinline__ float apply_one(float w, float o, float lw, float ls, int cautious) {
+  const bool decay = !cautious || (w > 0.f && o > 0.f) || (w < 0.f && o < 0.f);
+  const float d = decay ? __fmul_rn(lw, w) : 0.0f;
+  return __fsub_rn(__fsub_rn(w, d), __fmul_rn(ls, o));
+}
+
 // Y[r][c + k] op= o[k]: the apply W' = (W - lw W) - ls O, or a write-back.
+// With a row factor (NorMuon), O's row r is fl(O * rowf[r]) first.
 __device__ __forceinline__ void update_y8(const OutParams& p, const OutMat& M, int r, int c,
-                                          const float (&o)[8]) {
+                                          float (&o)[8]) {
   if (r >= M.rows || c >= M.cols) return;
   const long long idx = static_cast<long long>(r) * M.cols + c;
   const int cnt = min(8, M.cols - c);
+  if (p.mode == 0 && M.rowf) {
+    const float f = M.rowf[r];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) o[k] = __fmul_rn(o[k], f);
+  }
   if (cnt == 8 && M.vec) {
     if (p.mode == 0) {
       float4* w4 = reinterpret_cast<float4*>(static_cast<float*>(M.y) + idx);
       const float4 a = w4[0], b = w4[1];
       float w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-      for (int k = 0; k < 8; ++k) w[k] = __fsub_rn(__fsub_rn(w[k], __fmul_rn(p.lw, w[k])), __fmul_rn(M.ls, o[k]));
+      for (int k = 0; k < 8; ++k) w[k] = apply_one(w[k], o[k], p.lw, M.ls, p.cautious);
       w4[0] = make_float4(w[0], w[1], w[2], w[3]);
       w4[1] = make_float4(w[4], w[5], w[6], w[7]);
     } else if (p.mode == 1) {
@@ -361,8 +381,7 @@ __device__ __forceinline__ void update_y8(const OutParams& p, const OutMat& M, i
   for (int k = 0; k < cnt; ++k) {
     if (p.mode == 0) {
       float* W = static_cast<float*>(M.y);
-      const float w = W[idx + k];
-      W[idx + k] = __fsub_rn(__fsub_rn(w, __fmul_rn(p.lw, w)), __fmul_rn(M.ls, o[k]));
+      W[idx + k] = apply_one(W[idx + k], o[k], p.lw, M.ls, p.cautious);
     } else if (p.mode == 1) {
       static_cast<bf16*>(M.y)[idx + k] = __float2bfloat16_rn(o[k]);
     } else {
@@ -623,6 +642,142 @@ __global__ void __launch_bounds__(kScaleThreads) scale_kernel(const __grid_const
     for (int k = 0; k < 4; ++k) oh[k] = pack_bf16x2((h[2 * k] * f1) * f2, (h[2 * k + 1] * f1) * f2);
     *ph = make_uint4(oh[0], oh[1], oh[2], oh[3]);
   }
+}
+
+// ------------------------------------------------------- per-neuron rescale
+// Row sums of O^2 over the caller's W rows (NorMuon reading), O read from the
+// result pair as the apply pass reads it: O = fl(oscale * pair) or the pair's
+// value.  W = X: a block takes kNormRowsWide rows of X, four per warp, the
+// lanes running along the row with 16-byte loads; W = X^T: a block takes
+// kNormRowsTall columns of X, eight threads per row segment, 32 row groups
+// summed in shared memory in a fixed order.  Sums are fp64.
+constexpr int kNormThreads = 256;
+
+__device__ __forceinline__ void load_pair8(const NormMat& M, int i, int c, float (&v)[8]) {
+  const long long idx = static_cast<long long>(i) * M.ld + c;
+  const float f = M.oscale ? *M.oscale : 1.0f;
+  if (c + 8 <= M.n) {  // rows are 16-byte strided (ld % 16 == 0) and c % 8 == 0: aligned
+    pair_decode8(*reinterpret_cast<const uint4*>(static_cast<const bf16*>(M.hi) + idx),
+                 *reinterpret_cast<const uint2*>(static_cast<const int8_t*>(M.lo) + idx), v);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = M.oscale ? v[k] * f : v[k];
+    return;
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float x = 0.f;
+    if (c + k < M.n) {
+      const uint32_t fb = static_cast<uint32_t>(static_cast<const uint16_t*>(M.hi)[idx + k]) << 16;
+      const int q = static_cast<const int8_t*>(M.lo)[idx + k];
+      x = fmaf(static_cast<float>(q), lo8_unit(fb), __uint_as_float(fb));
+      if (M.oscale) x = x * f;
+    }
+    v[k] = x;
+  }
+}
+
+__global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_constant__ NormStatParams p) {
+  __shared__ double red[32][kNormRowsTall + 1];
+  int lo = 0, hi = p.nmat - 1;  // last matrix whose first block is <= blockIdx.x
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.mat[mid].blk_begin <= static_cast<int>(blockIdx.x)) lo = mid; else hi = mid - 1;
+  }
+  const NormMat& M = p.mat[lo];
+  const int local = blockIdx.x - M.blk_begin;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (!M.transposed) {
+    for (int j = 0; j < kNormRowsWide / 8; ++j) {
+      const int i = local * kNormRowsWide + warp * (kNormRowsWide / 8) + j;
+      if (i >= M.m) break;  // warp-uniform
+      double acc = 0.0;
+      for (int c = 8 * lane; c < M.n; c += 256) {
+        float v[8];
+        load_pair8(M, i, c, v);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc = fma(static_cast<double>(v[k]), static_cast<double>(v[k]), acc);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) p.rsq[M.row_base + i] = acc;
+    }
+    return;
+  }
+  const int u = threadIdx.x & 7, g = threadIdx.x >> 3;
+  const int c0 = local * kNormRowsTall;
+  double acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = 0.0;
+  if (c0 + 8 * u < M.n) {
+    for (int i = g; i < M.m; i += 32) {
+      float v[8];
+      load_pair8(M, i, c0 + 8 * u, v);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[k] = fma(static_cast<double>(v[k]), static_cast<double>(v[k]), acc[k]);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) red[g][8 * u + k] = acc[k];
+  __syncthreads();
+  if (threadIdx.x < kNormRowsTall && c0 + static_cast<int>(threadIdx.x) < M.n) {
+    double s = 0.0;
+    for (int q = 0; q < 32; ++q) s += red[q][threadIdx.x];
+    p.rsq[M.row_base + c0 + threadIdx.x] = s;
+  }
+}
+
+// One block per matrix: the state update and the row factors (see NormFacParams).
+__global__ void __launch_bounds__(kNormThreads) norm_factor_kernel(const __grid_constant__ NormFacParams p) {
+  __shared__ double red[2][kNormThreads / 32];
+  __shared__ double s_g;
+  const NormFacMat& M = p.mat[blockIdx.x];
+  const double* rsq = p.rsq + M.row_base;
+  double s0 = 0.0, s1 = 0.0;
+  for (int i = threadIdx.x; i < M.rows; i += kNormThreads) {
+    const double rs = rsq[i];
+    const float r32 = __double2float_rn(rs / static_cast<double>(M.cols));
+    const float v = __fadd_rn(__fmul_rn(p.beta2, M.v[i]), __fmul_rn(p.omb2, r32));
+    M.v[i] = v;
+    const double f = 1.0 / sqrt(static_cast<double>(v) + p.eps);
+    s0 += rs;
+    s1 += f * f * rs;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    red[0][threadIdx.x >> 5] = s0;
+    red[1][threadIdx.x >> 5] = s1;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t0 = 0.0, t1 = 0.0;
+    for (int w = 0; w < kNormThreads / 32; ++w) {
+      t0 += red[0][w];
+      t1 += red[1][w];
+    }
+    s_g = t1 > 0.0 ? sqrt(t0 / t1) : 1.0;
+  }
+  __syncthreads();
+  const double gsc = s_g;
+  for (int i = threadIdx.x; i < M.rows; i += kNormThreads) {
+    const double f = 1.0 / sqrt(static_cast<double>(M.v[i]) + p.eps);  // this thread wrote v[i]
+    p.rowf[M.row_base + i] = __double2float_rn(f * gsc);
+  }
+}
+
+cudaError_t launch_norm_stats(const NormStatParams& p, cudaStream_t s) {
+  if (p.nblocks <= 0) return cudaSuccess;
+  norm_stats_kernel<<<p.nblocks, kNormThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_norm_factors(const NormFacParams& p, cudaStream_t s) {
+  if (p.nmat <= 0) return cudaSuccess;
+  norm_factor_kernel<<<p.nmat, kNormThreads, 0, s>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_prep(const PrepParams& p, cudaStream_t s) {

@@ -282,9 +282,12 @@ __device__ __forceinline__ uint32_t w_chunk_bytes(int mode, const Group& G, int 
   return q * (32 * CW * 4);
 }
 
-// W' = (W - lw W) - ls O, each operation rounded to nearest in fp32.
-__device__ __forceinline__ float apply_w(float w, float o, float lw, float ls) {
-  return __fsub_rn(__fsub_rn(w, __fmul_rn(lw, w)), __fmul_rn(ls, o));
+// W' = (W - d) - ls O with d = fl(lw W) -- or d = 0 under cautious decay where
+// W and O do not have the same sign -- each operation rounded to nearest in fp32.
+__device__ __forceinline__ float apply_w(float w, float o, float lw, float ls, int cautious) {
+  const bool decay = !cautious || (w > 0.f && o > 0.f) || (w < 0.f && o < 0.f);
+  const float d = decay ? __fmul_rn(lw, w) : 0.0f;
+  return __fsub_rn(__fsub_rn(w, d), __fmul_rn(ls, o));
 }
 
 #ifdef MUON_TRACE
@@ -784,7 +787,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                     ld_shared_v4(wa, w[0], w[1], w[2], w[3]);
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                      w[e] = __float_as_uint(apply_w(__uint_as_float(w[e]), x[4 * h + e], tab.lw, lsc));
+                      w[e] = __float_as_uint(apply_w(__uint_as_float(w[e]), x[4 * h + e], tab.lw, lsc, tab.cautious));
                     st_shared_v4(wa, w[0], w[1], w[2], w[3]);
                   }
                 } else if (EPI == kBxApply && mode == 2) {
@@ -799,7 +802,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                         wb + static_cast<uint32_t>(row * 128 + ((((lane >> 2) ^ row) & 7) << 4) + (lane & 3) * 4);
                     float w;
                     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(w) : "r"(wa) : "memory");
-                    w = apply_w(w, x[e], tab.lw, lsc);
+                    w = apply_w(w, x[e], tab.lw, lsc, tab.cautious);
                     asm volatile("st.shared.f32 [%0], %1;" ::"r"(wa), "f"(w) : "memory");
                   }
                 } else {

@@ -96,6 +96,7 @@ struct ApplyTable {
   int nmat;      // entries in use; matrices past them take mode 0
   int mat_base;  // Group::mat_base value of entry 0
   float lw;      // fl(lr * wd)
+  int cautious;  // 1: decay only where W and O have the same sign
 };
 using LaunchApply = ApplyTable<kMaxApply>;
 
@@ -211,6 +212,7 @@ struct OutMat {
   int tile_begin;
   float ls;           // fl(lr * scale)
   const float* oscale;  // O = oscale[0] * (hi + lo) when set (result of zero steps)
+  const float* rowf;  // apply only: O's row r (caller layout) is multiplied by rowf[r] first, or null
   int vec;            // cols % 8 == 0 and ld % 8 == 0: 128-bit accesses
 };
 
@@ -219,7 +221,53 @@ struct OutParams {
   int nmat, ntiles;
   int mode;           // 0: apply, 1: write bf16, 2: write f32
   float lw;           // fl(lr * wd)
+  int cautious;       // apply only: decay only where W and O have the same sign
 };
+
+// Per-neuron rescale of the update (NorMuon reading).  For each row r of the
+// caller's W (rows x cols) with O its update:
+//   rsq_r  = sum over the row of O^2                    (fp64, fixed order)
+//   v'_r   = fl(fl(beta2 v_r) + fl(omb2 fl32(rsq_r / cols)))     (fp32 state)
+//   f_r    = 1 / sqrt(v'_r + eps)                        (fp64)
+//   g      = sqrt(sum_r rsq_r / sum_r f_r^2 rsq_r)       (1 if the sum is 0)
+//   rowf_r = fl32(f_r g)      -- O's row r is multiplied by rowf_r before the apply,
+// so the update keeps its Frobenius norm and only its split over rows changes.
+// O is read from the result pair in X's layout (W = X, or W = X^T when
+// transposed), as the apply pass reads it.
+struct NormMat {
+  const void* hi;     // the pair of O (X layout, m x n, row stride ld)
+  const void* lo;
+  const float* oscale;  // O = fl(oscale[0] * pair) when set, else the pair's value
+  int m, n;
+  long long ld;
+  int transposed;     // W rows are X's columns
+  int blk_begin;
+  long long row_base; // index of the matrix's first W row in rsq / rowf
+};
+
+struct NormStatParams {
+  NormMat mat[kMaxMats];
+  int nmat, nblocks;
+  double* rsq;
+};
+
+struct NormFacMat {
+  float* v;           // the caller's second-moment state, one fp32 per W row (in/out)
+  int rows, cols;     // W
+  long long row_base;
+};
+
+struct NormFacParams {
+  NormFacMat mat[kMaxMats];
+  int nmat;
+  const double* rsq;
+  float* rowf;
+  float beta2, omb2;
+  double eps;
+};
+
+constexpr int kNormRowsWide = 32;   // W rows per stats block when W = X (rows of X)
+constexpr int kNormRowsTall = 64;   // W rows per stats block when W = X^T (columns of X)
 
 // One pass over the caller's matrices: momentum (or a plain read of X), the
 // Nesterov blend u, and u written to the workspace as the pair bf16 hi + int8 lo
@@ -282,6 +330,8 @@ cudaError_t launch_out(const OutParams& p, cudaStream_t s);
 cudaError_t launch_sums(const SumParams& p, cudaStream_t s);
 cudaError_t launch_prep(const PrepParams& p, cudaStream_t s);
 cudaError_t launch_scale(const ScaleParams& p, cudaStream_t s);
+cudaError_t launch_norm_stats(const NormStatParams& p, cudaStream_t s);
+cudaError_t launch_norm_factors(const NormFacParams& p, cudaStream_t s);
 
 }  // namespace ew
 

@@ -131,15 +131,25 @@ class ShardedMuon:
         return flat[self.rank * slot:(self.rank + 1) * slot]
 
     def _reduce_scatter_avg(self, G, slot):
-        """This rank's slot of G := the group mean of every rank's slot."""
+        """This rank's slot of G := the group mean of every rank's slot.
+
+        NCCL: one reduce-scatter with AVG in the gradient dtype; for bf16 each
+        partial sum NCCL forms is rounded to bf16, so the mean is within about
+        (world - 1) * 2^-8 of the mean of |g| of the exact mean.  Other
+        backends (no reduce-scatter): an all-reduce of the gradients widened to
+        fp32, the mean divided in fp32 and rounded once to the gradient dtype.
+        """
         if self.dist is None:
             return
         if self._nccl:
             self.dist.reduce_scatter_tensor(self._mine(G, slot), G, op=self.dist.ReduceOp.AVG,
                                             group=self.group)
-        else:  # backends without reduce-scatter: the same result through an all-reduce
-            self.dist.all_reduce(G, op=self.dist.ReduceOp.SUM, group=self.group)
-            self._mine(G, slot).div_(self.world)
+        else:
+            acc = G if G.dtype == torch.float32 else G.float()
+            self.dist.all_reduce(acc, op=self.dist.ReduceOp.SUM, group=self.group)
+            mean = self._mine(acc, slot).div_(self.world)
+            if acc is not G:
+                self._mine(G, slot).copy_(mean)
 
     def _all_gather(self, W, slot):
         """Every rank's slot of W := its owner's; returns the pending work or None."""

@@ -118,6 +118,17 @@ def test_step_argument_errors(lib):
     assert "grads[0]" in _err(lib)
     assert lib.muon_momentum(1, p, p, shapes, -0.1, 1, None, null) == -1
     assert lib.muon_apply(1, p, None, shapes, 0.1, 0.0, null) == -1
+    # the extended step and apply: unknown option bits, beta2, state pointers
+    assert lib.muon_step_ex(1, p, p, p, shapes, 0.9, 1, 0.1, 0.0, 5, 2, None, 0.95, null) == -1
+    assert "flags" in _err(lib)
+    assert lib.muon_step_ex(1, p, p, p, shapes, 0.9, 1, 0.1, 0.0, 5, 1, p, 1.5, null) == -1
+    assert "beta2" in _err(lib)
+    assert lib.muon_step_ex(1, p, p, p, shapes, 0.9, 1, 0.1, 0.0, 5, 0, _lib.ptr_array([0]), 0.95, null) == -1
+    assert "neuron_state[0]" in _err(lib)
+    assert lib.muon_step_ex(0, None, None, None, None, 0.9, 1, 0.1, 0.0, 5, 1, None, 0.95, null) == 0
+    assert lib.muon_apply_ex(1, p, p, shapes, 0.1, 0.0, 8, None, null) == -1
+    assert lib.muon_apply_ex(1, p, p, shapes, 0.1, 0.0, 1, _lib.ptr_array([0x1002]), null) == -1
+    assert "row_scale[0]" in _err(lib)
 
 
 def test_stage_argument_errors(lib):
@@ -129,6 +140,19 @@ def test_stage_argument_errors(lib):
     assert lib.muon_bx_bf16(1, 8, 24, 0x1000, 0x2000, 0x3000, 0x4000, 1.0, null) == -2
     assert "multiple of 16" in _err(lib)
     assert lib.muon_gram_bf16(0, 8, 8, None, None, null) == 0
+    # fused last product + apply: strides, shape order and pointers are checked on the host
+    w = _lib.ptr_array([0x1000])
+    assert lib.muon_bx_apply_bf16(1, 8, 24, 24, 0x1000, 8, 0x2000, 0x3000, w, 0, 1.0, 0.1, 0.0, 0, null) == -2
+    assert "ldx" in _err(lib)
+    assert lib.muon_bx_apply_bf16(1, 8, 24, 32, 0x1000, 4, 0x2000, 0x3000, w, 0, 1.0, 0.1, 0.0, 0, null) == -2
+    assert lib.muon_bx_apply_bf16(1, 32, 16, 16, 0x1000, 32, 0x2000, 0x3000, w, 0, 1.0, 0.1, 0.0, 0, null) == -2
+    assert lib.muon_bx_apply_bf16(1, 8, 24, 32, 0x1000, 8, 0x2000, 0x3008, w, 0, 1.0, 0.1, 0.0, 0, null) == -1
+    assert lib.muon_bx_apply_bf16(1, 8, 24, 32, 0x1000, 8, 0x2000, 0x3000, None, 0, 1.0, 0.1, 0.0, 0, null) == -1
+    assert lib.muon_bx_apply_bf16(1, 8, 24, 32, 0x1000, 8, 0x2000, 0x3000, w, 0, 1.0, float("nan"), 0.0,
+                                  0, null) == -1
+    assert lib.muon_bx_apply_bf16(1, 8, 32, 32, 0x1000, 8, 0x2000, 0x3000, w, 0, 1.0, 0.1, 0.0, 4, null) == -1
+    assert "flags" in _err(lib)
+    assert lib.muon_bx_apply_bf16(0, 8, 24, 32, None, 8, None, None, None, 0, 1.0, 0.1, 0.0, 0, null) == 0
 
 
 def test_setters(lib):

@@ -69,3 +69,20 @@ def test_reference_arm_line(capsys, monkeypatch):
     assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert line["config"]["workload"] == bench.WORKLOAD
+
+
+def test_executed_flops_of_the_pair_tiles():
+    """Executed work counts whole 256 x 256 pair tiles: for m = 768 (3 x 3
+    tiles) the symmetric products run 6 of 9 tiles, B X all 9, so a step
+    executes (2/3 * 2 m^2 n + 2/3 * 2 m^3 + 2 m^2 n); worked by hand."""
+    m, n = 768, 3072
+    want = 5 * (2 / 3 * 2 * m * m * n + 2 / 3 * 2 * m ** 3 + 2 * m * m * n)
+    assert bench.executed_flops([(m, n)]) == pytest.approx(want, rel=1e-12)
+    assert bench.executed_flops([(n, m)]) == bench.executed_flops([(m, n)])
+    # one ragged 200 x 328 matrix: 1 pair tile row (padded to 256), 2 tile columns,
+    # K padded to 64: 328 -> 384, 200 -> 256
+    t = 2 * 256 * 256
+    assert bench.executed_flops([(200, 328)], steps=1) == t * (1 * 384 + 1 * 256 + 2 * 256)
+    # for large m the symmetric share tends to one half of the nominal work
+    big = bench.executed_flops([(4096, 4096)], steps=1)
+    assert big / bench.nominal_flops([(4096, 4096)], steps=1) == pytest.approx((136 / 256 * 4 + 2) / 6)

@@ -9,6 +9,7 @@ import pytest
 import torch
 
 import newton_schulz_12_b200 as nsb
+from blockcheck import assert_blocks
 from newton_schulz_12_b200 import workloads
 from oracle import muon as oracle
 
@@ -16,6 +17,9 @@ pytestmark = pytest.mark.gpu
 
 TOL_BF16 = 3e-2
 TOL_FP32 = 1e-4
+# every 32 x 32 block within 4x the whole-matrix bound (tests/blockcheck.py)
+BLOCK_TOL_BF16 = 4 * TOL_BF16
+BLOCK_TOL_FP32 = 4 * TOL_FP32
 
 
 def rel_fro(got, ref):
@@ -36,10 +40,12 @@ def test_config1_single_768_fp32_and_bf16():
     ref = oracle.newton_schulz(X.double().numpy())
     got32 = run_ns([X])[0]
     assert rel_fro(got32, ref) <= TOL_FP32
+    assert_blocks(got32, ref, BLOCK_TOL_FP32, "fp32 768x768")
     Xb = X.to(torch.bfloat16)
     ref_b = oracle.newton_schulz(Xb.double().numpy())
     got16 = run_ns([Xb])[0]
     assert rel_fro(got16, ref_b) <= TOL_BF16
+    assert_blocks(got16, ref_b, BLOCK_TOL_BF16, "bf16 768x768")
 
 
 @pytest.mark.parametrize("rows,cols,batch", [
@@ -51,14 +57,18 @@ def test_bf16_shapes(rows, cols, batch):
     got = run_ns(mats)
     for g, x in zip(got, mats):
         assert g.shape == (rows, cols)
-        assert rel_fro(g, oracle.newton_schulz(x.double().numpy())) <= TOL_BF16
+        ref = oracle.newton_schulz(x.double().numpy())
+        assert rel_fro(g, ref) <= TOL_BF16
+        assert_blocks(g, ref, BLOCK_TOL_BF16, f"{rows}x{cols}")
 
 
 @pytest.mark.parametrize("rows,cols", [(768, 3072), (200, 328), (328, 200), (8, 8), (1, 5), (96, 96)])
 def test_fp32_shapes(rows, cols):
     X = workloads.gaussian((rows, cols), 1.0, seed=rows + cols)
     got = run_ns([X])[0]
-    assert rel_fro(got, oracle.newton_schulz(X.double().numpy())) <= TOL_FP32
+    ref = oracle.newton_schulz(X.double().numpy())
+    assert rel_fro(got, ref) <= TOL_FP32
+    assert_blocks(got, ref, BLOCK_TOL_FP32, f"fp32 {rows}x{cols}")
 
 
 @pytest.mark.parametrize("steps", [0, 1, 2, 7])
@@ -122,7 +132,9 @@ def test_hard_spectrum_band():
     """Log-uniform spectrum with a x100 spike: still within tolerance of the oracle."""
     G = workloads.hard_spectrum(768, 768, seed=5, spike=True)
     ref = oracle.newton_schulz(G.double().numpy())
-    assert rel_fro(run_ns([G])[0], ref) <= TOL_BF16
+    got = run_ns([G])[0]
+    assert rel_fro(got, ref) <= TOL_BF16
+    assert_blocks(got, ref, BLOCK_TOL_BF16, "hard spectrum")
 
 
 def test_deterministic():
@@ -144,3 +156,4 @@ def test_last_step_writes_outputs_directly_or_through_the_pass(rows, cols, batch
     for i in sorted({0, batch // 2, batch - 1} | ({95, 96} if batch > 96 else set())):
         ref = oracle.newton_schulz(mats[i].double().numpy())
         assert rel_fro(got[i], ref) <= TOL_BF16, i
+        assert_blocks(got[i], ref, BLOCK_TOL_BF16, f"matrix {i}")

@@ -3,7 +3,8 @@
 * momentum buffers: bit-exact against the fp32 restatement of the same order;
 * apply: bit-exact against the fp32 restatement given the same update;
 * the full step: the weight update W' - W within relative Frobenius 3e-2 of the
-  fp64 oracle run on the GPU's own pre-step state (so no drift accumulates);
+  fp64 oracle run on the GPU's own pre-step state (so no drift accumulates),
+  and every 32 x 32 block of it within 4 x 3e-2 of the same block;
 * the GPT-2-small hidden set (72 matrices, 768 wide) at full size, with
   Gaussian and with hard (log-uniform, spiked) gradient spectra.
 """
@@ -12,6 +13,7 @@ import pytest
 import torch
 
 import newton_schulz_12_b200 as nsb
+from blockcheck import assert_blocks
 from newton_schulz_12_b200 import workloads
 from oracle import muon as oracle
 from oracle.fp32_ref import apply_f32, momentum_f32, update_scale_f32
@@ -19,6 +21,7 @@ from oracle.fp32_ref import apply_f32, momentum_f32, update_scale_f32
 pytestmark = pytest.mark.gpu
 
 TOL = 3e-2
+BLOCK_TOL = 4 * TOL  # every 32 x 32 block of W' - W (tests/blockcheck.py)
 
 
 def rel_fro(got, ref):
@@ -59,6 +62,7 @@ def check_step(st, step, beta=0.95, nesterov=True, lr=0.05, wd=0.0, steps=5, che
         err = rel_fro(dW, dW_ref)
         worst = max(worst, err)
         assert err <= TOL, f"matrix {i} {st.shapes[i]}: rel err {err:.3e}"
+        assert_blocks(dW, dW_ref, BLOCK_TOL, f"matrix {i} {st.shapes[i]}")
     return worst
 
 

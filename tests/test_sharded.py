@@ -239,3 +239,41 @@ def test_three_ranks_with_an_idle_rank_in_a_bucket():
                                         np.zeros(s), **HYPER)
             np.testing.assert_array_equal(params[i], Wn.astype(np.float32),
                                           err_msg=f"rank {rank} matrix {i}")
+
+
+# ------------------------------------------- bf16 gradients on a backend without reduce-scatter
+def _worker_bf16(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from newton_schulz_12_b200.sharded import ShardedMuon
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        seen = {}
+
+        def record(params, grads, bufs, beta, nesterov, lr, wd, steps):
+            for g in grads:
+                seen[g.data_ptr()] = g.clone()
+
+        sm = ShardedMuon(SHAPES, buckets=2, grad_dtype=torch.bfloat16, local_step=record, **HYPER)
+        for i, s in enumerate(SHAPES):
+            sm.grads[i].copy_(rank_grad(i, s, rank, 0) * 37.0)  # bf16 values of mixed exponents
+        ptr = {i: sm.grads[i].data_ptr() for i in range(len(SHAPES))}
+        sm.step()
+        out.put((rank, {i: seen[ptr[i]].float().numpy() for i in range(len(SHAPES)) if ptr[i] in seen}))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bf16_gradients_are_averaged_in_fp32():
+    """Without reduce-scatter (gloo) the owner receives the fp32 mean of the
+    bf16 gradients rounded once to bf16 -- not a bf16 sum divided afterwards."""
+    res = _run_ranks(2, _worker_bf16)
+    owner, _ = plan_ownership(SHAPES, 2, 2)
+    for rank, got in res:
+        assert sorted(got) == [i for i in range(len(SHAPES)) if owner[i] == rank]
+        for i, g in got.items():
+            a = (rank_grad(i, SHAPES[i], 0, 0) * 37.0).to(torch.bfloat16).float()
+            b = (rank_grad(i, SHAPES[i], 1, 0) * 37.0).to(torch.bfloat16).float()
+            want = ((a + b) / 2).to(torch.bfloat16).float().numpy()
+            np.testing.assert_array_equal(g, want, err_msg=f"matrix {i}")
