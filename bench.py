@@ -21,7 +21,9 @@ against the measured peaks in MEASURED_PEAKS.json.  After the timed region
 second without the timing hooks, with its own clock record; `ns_768x3072`,
 muon_ns_orthogonalize on 64 matrices 768x3072 (the three GEMMs and the whole
 call, nominal and executed TFLOP/s); `scaled_set`, the 144-matrix 1024-wide
-set's full muon_step.
+set's full muon_step; `refinements`, muon_step_ex with cautious weight decay
+and NorMuon's per-neuron rescale on the GPT-2-small set; `square_sweep`, the
+square width sweep m = 256 .. 4096 (batch 64 (768/m)^2).
 `--impl reference` times the fp64 CPU oracle on a bounded sample instead.
 """
 from __future__ import annotations
@@ -377,6 +379,66 @@ def measure_ns_768x3072(dev, peaks, reps=20):
     return out
 
 
+def measure_refinements(W, G, M, shapes, stream, dev, steps=20):
+    """muon_step_ex on the GPT-2 set with both refinements on: cautious weight
+    decay (wd 0.01) and NorMuon's per-neuron rescale (beta2 0.95); the
+    rescale needs every row's norm first, so every update takes the apply
+    pass (no fused apply).  Same tensors as the main run (W and momentum keep
+    evolving)."""
+    import torch
+    import newton_schulz_12_b200 as nsb
+    V = [torch.zeros(r, device=dev) for r, _ in shapes]
+
+    def step():
+        nsb.muon_step_ex(W, G, M, wd=0.01, cautious_wd=True, neuron_state=V, beta2=0.95, stream=stream)
+
+    for _ in range(3):
+        step()
+    with ClockSampler(dev) as clocks:
+        nsb.muon_profile_begin()
+        ms = time_steps(step, steps, stream)
+        prof = nsb.muon_profile_end()
+    if nsb.muon_get_status(stream) != 0:
+        raise RuntimeError("device status in the refinements run: " + nsb.muon_last_error())
+    per = ms / steps
+    return {"options": "cautious_wd + NorMuon (beta2 0.95), wd 0.01", "steps": steps,
+            "ms_per_step": per, "value": len(shapes) / (per / 1000.0), "unit": UNIT,
+            "per_kernel_us": {k: v[0] / v[1] * 1e3 for k, v in prof.items() if v[1]},
+            "launches_per_step": sum(v[1] for v in prof.values()) / steps,
+            "clocks": clocks.summary()}
+
+
+def measure_square_sweep(dev, peaks, reps=10):
+    """muon_ns_orthogonalize (bf16) on the square width sweep: m in {256 .. 4096}
+    with batch 64 (768/m)^2 (>= 1), bf16 N(0, 1) drawn on the device; GEMM
+    and whole-call TFLOP/s, nominal and executed, per width."""
+    import torch
+    import newton_schulz_12_b200 as nsb
+    from newton_schulz_12_b200 import workloads
+    stream = torch.cuda.current_stream(dev)
+    out = []
+    for m, batch in workloads.sweep_cases():
+        g = torch.Generator(device=dev).manual_seed(3000 + m)
+        xs = [torch.randn(m, m, generator=g, device=dev).to(torch.bfloat16) for _ in range(batch)]
+        for _ in range(2):
+            nsb.muon_ns_orthogonalize(xs)
+        nsb.muon_profile_begin()
+        ms = time_steps(lambda: nsb.muon_ns_orthogonalize(xs), reps, stream)
+        prof = nsb.muon_profile_end()
+        if nsb.muon_get_status() != 0:
+            raise RuntimeError(f"device status in the sweep at m={m}: " + nsb.muon_last_error())
+        nominal = nominal_flops([(m, m)] * batch)
+        executed = executed_flops([(m, m)] * batch)
+        gemm_ms = sum(prof[k][0] for k in ("gram", "poly", "bx")) / reps
+        out.append({"m": m, "batch": batch, "call_ms": ms / reps, "gemm_ms": gemm_ms,
+                    "gemm_tflops_nominal": nominal / gemm_ms / 1e9,
+                    "gemm_tflops_executed": executed / gemm_ms / 1e9,
+                    "call_tflops_nominal": nominal / (ms / reps) / 1e9,
+                    "gemm_frac_executed": executed / gemm_ms / 1e9 / peaks["bf16_tflops"]})
+        del xs
+    return out
+
+
 def measure_scaled_set(dev, peaks, steps=10):
     """Full muon_step over the 144-matrix 1024-wide set (24 layers x [4x 1024^2,
     1024x4096, 4096x1024]), bf16 grads N(0, 0.01^2), fp32 W N(0, 0.02^2),
@@ -590,7 +652,9 @@ def run_ours(args):
         }
         if world == 1 and not args.no_extras:
             line["value_sustained"] = measure_sustained(step, stream, dev, ms / args.steps, len(shapes))
+            line["refinements"] = measure_refinements(W, G, M, shapes, stream, dev)
             line["ns_768x3072"] = measure_ns_768x3072(dev, peaks)
+            line["square_sweep"] = measure_square_sweep(dev, peaks)
             del W_flat, G_flat, M_flat, W, G, M, plan, plans, G_dev, W_stage
             torch.cuda.empty_cache()
             line["scaled_set"] = measure_scaled_set(dev, peaks)

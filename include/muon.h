@@ -72,7 +72,7 @@ typedef enum {
  *         (stream order) each holds NS(X / (||X||_F + 1e-7)) after `steps`
  *         iterations, rounded to the storage type.  (MUON_BF16, steps >= 1:
  *         with m <= n and n % 8 == 0 the last GEMM stores the fp32 result
- *         rounded to bf16 straight into the first 96 buffers of each launch;
+ *         rounded to bf16 straight into the first 160 buffers of each launch;
  *         the others are written from the bf16 + int8 pair by a separate
  *         pass, which can differ from that rounding by one bf16 unit.)
  * a, b, c coefficients of the quintic; the speedrun's are 3.4445, -4.7750, 2.0315.
@@ -170,7 +170,7 @@ int muon_ns_orthogonalize_static(int batch, int m, int n, void* const* X_ptrs, f
  * shapes         host array of 2*count int64: rows, cols of each matrix.
  * Matrices of equal (min, max) dimensions are batched into one group; any mix
  * of shapes is accepted.  With steps >= 1 the update of a weight whose column
- * count is a multiple of 4 (among the first 96 matrices of each launch of the
+ * count is a multiple of 4 (among the first 160 matrices of each launch of the
  * last step) is applied inside the last Newton-Schulz GEMM, with O its fp32
  * value; the others are applied by a separate pass from O carried as the
  * bf16 + int8 pair.  Both stay within the same tolerance of the definition.
@@ -305,12 +305,15 @@ int muon_bx_bf16(int batch, int m, int n, const void* B, const void* Xhi, void* 
  *         of 8; matrix stride m*ldb).
  * Xhi     DEVICE pointer, bf16 hi of X; read only.
  * Xlo     DEVICE pointer, int8 q of X.  Read; overwritten with q of X' for the
- *         matrices that take the separate pass (below).
+ *         matrices that take the separate pass (below).  For those the bulk
+ *         copies write whole 16-byte units, so when n is not a multiple of 16
+ *         the row's padding bytes n .. (n rounded up to 16) - 1 may change
+ *         too (they are inside the ldx-wide row; nothing past it is written).
  * W_ptrs  HOST array of `batch` DEVICE pointers to fp32 W (row-major,
  *         contiguous, 16-byte aligned), updated in place.
- * The first 96 matrices whose W has a column count that is a multiple of 4
+ * The first 160 matrices whose W has a column count that is a multiple of 4
  * are updated inside the GEMM epilogue with O as above.  The others (past
- * the first 96, or W columns not a multiple of 4) get X' as the pair (hi in
+ * the first 160, or W columns not a multiple of 4) get X' as the pair (hi in
  * the library's workspace, q in Xlo) and are updated by the apply pass from
  * the pair's value, as muon_step does for them.
  * Returns MUON_OK or a negative muon_status.

@@ -285,6 +285,15 @@ __device__ __forceinline__ void tmem_ld_32x32_x16(uint32_t taddr, uint32_t (&r)[
       : "r"(taddr)
       : "memory");
 }
+// 32 lanes x 8 columns: thread t receives lane (base lane + t), columns [col, col+8).
+__device__ __forceinline__ void tmem_ld_32x32_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -363,33 +372,47 @@ __device__ __forceinline__ uint32_t bf16_word_bits(uint32_t w, int k) {
 
 // Eight values -> eight bf16 (uint4) and eight int8 (uint2) of the pair.
 // d = x - hi is exact in fp32 and scaling by 2^(15 - E) is exact, so q is
-// the nearest-even rounding of d / 2^(E - 15), clamped to [-128, 127].
+// the nearest-even rounding of t = d / 2^(E - 15), clamped to [-128, 127].
+// t lies in [-128, 128] (|d| is at most half a bf16 unit of hi), so only 128
+// needs the clamp; adding 1.5 * 2^23 then rounds t to the nearest integer
+// (ties to even, the fp32 unit at that magnitude is 1) and leaves it, two's
+// complement, in the low byte of the sum's bits.  No int/float conversion
+// instruction is used (those run at an eighth of the fp32 rate).
 __device__ __forceinline__ void pair_encode8(const float (&v)[8], uint4& hi, uint2& lo) {
   uint32_t h[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) h[k] = pack_bf16x2(v[2 * k], v[2 * k + 1]);
-  uint32_t qb[8];
+  uint32_t m[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const uint32_t fb = bf16_word_bits(h[k >> 1], k & 1);
-    const float t = (v[k] - __uint_as_float(fb)) * lo8_inv_unit(fb);
-    const int q = min(max(__float2int_rn(t), -128), 127);
-    qb[k] = static_cast<uint32_t>(q) & 0xFFu;
+    const float t = fminf((v[k] - __uint_as_float(fb)) * lo8_inv_unit(fb), 127.0f);
+    m[k] = __float_as_uint(t + 12582912.0f);
   }
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(w[k]) : "r"(m[2 * k]), "r"(m[2 * k + 1]));
   hi = make_uint4(h[0], h[1], h[2], h[3]);
-  lo = make_uint2(qb[0] | (qb[1] << 8) | (qb[2] << 16) | (qb[3] << 24),
-                  qb[4] | (qb[5] << 8) | (qb[6] << 16) | (qb[7] << 24));
+  uint32_t l0, l1;
+  asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(l0) : "r"(w[0]), "r"(w[1]));
+  asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(l1) : "r"(w[2]), "r"(w[3]));
+  lo = make_uint2(l0, l1);
 }
 
-// Eight values of the pair back to fp32: hi + q * 2^(E - 15).
+// Eight values of the pair back to fp32: hi + q * 2^(E - 15).  q is
+// sign-extended from its byte with one byte permute, and turned into a float
+// exactly as the bits of 1.5 * 2^23 + q minus 1.5 * 2^23.
 __device__ __forceinline__ void pair_decode8(const uint4 hi, const uint2 lo, float (&v)[8]) {
   const uint32_t h[4] = {hi.x, hi.y, hi.z, hi.w};
   const uint32_t l[2] = {lo.x, lo.y};
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const uint32_t fb = bf16_word_bits(h[k >> 1], k & 1);
-    const int q = static_cast<int>(l[k >> 2] << (24 - 8 * (k & 3))) >> 24;  // sign-extended byte
-    v[k] = fmaf(static_cast<float>(q), lo8_unit(fb), __uint_as_float(fb));
+    uint32_t q;
+    const uint32_t sel = (k & 3) | ((8 | (k & 3)) * 0x1110);  // byte k & 3, its sign in bytes 1..3
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(q) : "r"(l[k >> 2]), "r"(sel));
+    const float qf = __int_as_float(static_cast<int>(q) + 0x4B400000) - 12582912.0f;
+    v[k] = fmaf(qf, lo8_unit(fb), __uint_as_float(fb));
   }
 }
 

@@ -303,10 +303,34 @@ __device__ __forceinline__ void trace_stamp(const Params& p, int tile, int slot)
 #endif
 
 // ---------------------------------------------------------------------- kernel
-// kPoly and kBx add warp 11, their operand loader.
+// Epilogue math warps per kernel kind: 8 (two per TMEM lane quarter), and 16
+// for the fused apply, whose epilogue (W's stream) bounds it.  Measured on
+// the GPT-2-small set: 16 warps slow kBx by 11 % (its epilogue is off the
+// critical path, and more warps contend with the copy and MMA threads) and
+// speed kBxApply up by 12 %.
+#ifndef MUON_EPI_WARPS
+#define MUON_EPI_WARPS 8
+#endif
+#ifndef MUON_BXA_EPI_WARPS
+#define MUON_BXA_EPI_WARPS 16
+#endif
 template <int EPI>
-constexpr int threads_of() {
-  return EPI == kGram ? kThreads : kThreads + 32;
+__host__ __device__ constexpr int epi_warps() {
+  return EPI == kBxApply ? MUON_BXA_EPI_WARPS : MUON_EPI_WARPS;
+}
+template <int EPI>
+__host__ __device__ constexpr int epi_threads() {
+  return 32 * epi_warps<EPI>();
+}
+// The IO warp follows the epilogue warps; kPoly and kBx add a loader warp after it.
+template <int EPI>
+__host__ __device__ constexpr int io_warp() {
+  return 2 + epi_warps<EPI>();
+}
+template <int EPI>
+__host__ __device__ constexpr int threads_of() {
+  static_assert(epi_warps<EPI>() == 8 || epi_warps<EPI>() == 16, "epilogue warps: 8 or 16");
+  return 32 * (io_warp<EPI>() + 1) + (EPI == kGram ? 0 : 32);
 }
 
 // NT: entries of the per-matrix table (1 where the launch has none).
@@ -314,6 +338,8 @@ template <int EPI, int NT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1)
     gemm_kernel(const __grid_constant__ Params p, const __grid_constant__ ApplyTable<NT> tab) {
   using C = Cfg<EPI>;
+  constexpr int kEpiThreads = epi_threads<EPI>();
+  constexpr int kIoWarp = io_warp<EPI>();
   constexpr int S = C::kStages;
   constexpr int K = C::kSlots;
   extern __shared__ uint8_t smem_raw[];
@@ -523,22 +549,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-9) and IO (warp 10)
+    // ------------------------------------------------------------ epilogue warps and IO (warp kIoWarp)
     constexpr int NCH = C::kNCh, CW = C::kCW;
     const int total_chunks = my_tiles * NCH;
     const uint32_t slots_u32 = smem_u32(slots);
     const uint32_t stage_u32 = smem_u32(staging);
 
-    if (warp >= 10) {
+    if (warp >= kIoWarp) {
       // ---------------------------------------------------------- IO threads
-      // Warp 10 issues the epilogue's bulk stores of what the compute warps
+      // Warp kIoWarp issues the epilogue's bulk stores of what the compute warps
       // finished, draining each store before the buffer it read is handed
-      // back.  The operand chunk copies into the slot ring come from warp 11,
+      // back.  The operand chunk copies into the slot ring come from the next warp,
       // so that a copy issue stalled on the tensor-copy unit never delays a
       // store: kPoly refills a slot once the compute warps have read it, kBx
       // (whose results are stored from the slot itself) once its stores have.
       constexpr bool kLoaderWarp = (EPI != kGram);
-      const bool loads_here = (EPI != kGram) && (kLoaderWarp ? warp == 11 : warp == 10);
+      const bool loads_here = (EPI != kGram) && (kLoaderWarp ? warp == kIoWarp + 1 : warp == kIoWarp);
       if (lane == 0) {
         for (int g = 0; g < p.ngroups; ++g) {
           tma_prefetch_map(&p.map[g].e);
@@ -584,7 +610,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
         };
         if (loads_here)
           for (int s = 0; s < K; ++s) issue_eload(s);
-        if (kLoaderWarp && warp == 11) {
+        if (kLoaderWarp && warp == kIoWarp + 1) {
           if (EPI == kPoly) {
             // refill each slot as soon as every compute thread has read it
             for (int s = 0; s < total_chunks; ++s) {
@@ -593,14 +619,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
               issue_eload(s + K);
             }
           } else {
-            // kBx: chunk s + K - 1 goes into chunk s - 1's slot once its stores have read it
-            for (int s = 1; s + K - 1 < total_chunks; ++s) {
-              mbar_wait(econs_bar((s - 1) % K), ((s - 1) / K) & 1, ctl);
-              issue_eload(s + K - 1);
+            // kBx: chunk s + K goes into chunk s's slot as soon as chunk s's own
+            // stores have read it (the store thread waits for that right after
+            // issuing them), so the loader runs K chunks ahead
+            for (int s = 0; s + K < total_chunks; ++s) {
+              mbar_wait(econs_bar(s % K), (s / K) & 1, ctl);
+              issue_eload(s + K);
             }
           }
         }
-        const int io_chunks = (kLoaderWarp && warp == 11) ? 0 : total_chunks;
+        const int io_chunks = (kLoaderWarp && warp == kIoWarp + 1) ? 0 : total_chunks;
         int njob[NB + 1];  // kGram / kPoly: jobs seen per ready barrier (staging pairs, then the block)
         for (int q = 0; q <= NB; ++q) njob[q] = 0;
         int nup = 0;       // strictly-upper chunks so far (staging pair = nup % NB)
@@ -634,11 +662,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                 tma_store_3d(&M.mt, hs + C::kLoOff, col0, row0, tc.b);  // lo' -> lo, in place
               }
               bulk_commit();
-              asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");  // chunk s-1 drained
+              asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // chunk s drained
             } else {
               bulk_wait_read_all();
             }
-            if (s >= 1) mbar_arrive(econs_bar((s - 1) % K));  // the loader may refill chunk s-1's slot
+            mbar_arrive(econs_bar(s % K));  // the loader may refill chunk s's slot
             continue;
           }
           if (kind == kUpper) {
@@ -689,11 +717,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
       }
       __syncwarp();
     } else {
-      // ---------------------------------------------------------- compute (warps 2-9)
-      // Two warps per TMEM lane quarter: warp w reads lanes 32*(w%4).. and
-      // the half `hf` of each chunk's columns.  A failed (timed-out) wait is
-      // recorded and the schedule continues -- every later wait then returns
-      // at once -- so the compute warps always meet at the same barriers.
+      // ---------------------------------------------------------- compute warps
+      // NP = epi_warps / 4 warps per TMEM lane quarter: warp w reads lanes
+      // 32*(w%4).. and the part `hf` (of NP) of each chunk's columns.  A failed
+      // (timed-out) wait is recorded and the schedule continues -- every later
+      // wait then returns at once -- so the compute warps always meet at the
+      // same barriers.
+      constexpr int NP = epi_warps<EPI>() / 4;
       const int lane_base = 32 * (warp & 3);
       const int hf = (warp - 2) >> 2;
       const int r = lane_base + lane;  // tile row owned by this thread
@@ -723,7 +753,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
           const float lsc = j >= 0 ? tab.mat[j].ls : 0.f;  // fl(lr * scale)
           // BCW-column chunks c (64 for kBx, MUON_BXA_CHUNK for kBxApply): thread
           // (r, hf) takes accumulator columns VB hf .. +VB-1 of the chunk
-          constexpr int BCW = C::kCW, VB = BCW / 2;
+          constexpr int BCW = C::kCW, VB = BCW / NP;
           const int sr = r;
           for (int c = 0; c < C::kNCh; ++c) {
             if (leader && c > 0) TRACE(k, 4 + c);
@@ -738,8 +768,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                                   static_cast<uint32_t>(acc * BN + c * C::kCW + hf * VB);
               if constexpr (VB == 32)
                 tmem_ld_32x32(ta, rr);
-              else
+              else if constexpr (VB == 16)
                 tmem_ld_32x32_x16(ta, rr);
+              else
+                tmem_ld_32x32_x8(ta, rr);
               tmem_ld_wait();
 #pragma unroll
               for (int q = 0; q < VB; ++q) v[q] = __uint_as_float(rr[q]);
@@ -757,15 +789,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             // step) written back in place as the pair (hi', lo') for the IO
             // thread to store.  Columns VB hf + 8 uu .. +7 are 16-byte unit
             // (VB / 8) hf + uu of the hi row (2 BCW bytes, swizzled over its
-            // width) and bytes 8 (uu & 1) .. of unit (VB / 16) hf + uu / 2 of
-            // the lo row (BCW bytes, likewise).
+            // width) and the 8 bytes at offset VB hf + 8 uu of the lo row
+            // (BCW bytes, likewise: unit (VB hf + 8 uu) / 16, half by bit 3).
             if (live) {
               const uint32_t hs = slots_u32 + slot * C::kSlotBytes;
               const uint32_t ls = hs + C::kLoOff;
 #pragma unroll
               for (int uu = 0; uu < VB / 8; ++uu) {
-                const uint32_t ha = hs + (BCW == 64 ? sw128(sr, 4 * hf + uu) : sw64(sr, 2 * hf + uu));
-                const uint32_t la = ls + (BCW == 64 ? sw64(sr, 2 * hf + (uu >> 1)) : sw32(sr, hf)) + 8 * (uu & 1);
+                const int hu = (VB / 8) * hf + uu;  // 16-byte unit of the hi row
+                const int lb = VB * hf + 8 * uu;    // byte offset in the lo row
+                const uint32_t ha = hs + (BCW == 64 ? sw128(sr, hu) : sw64(sr, hu));
+                const uint32_t la = ls + (BCW == 64 ? sw64(sr, lb >> 4) : sw32(sr, lb >> 4)) + (lb & 8);
                 uint4 h4;
                 uint2 l2;
                 ld_shared_v4(ha, h4.x, h4.y, h4.z, h4.w);
@@ -820,7 +854,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
         // VPT hf .. VPT hf + VPT-1 of the chunk, i.e. 16-byte units
         // UPT hf .. UPT hf + UPT-1 of the chunk's swizzled row (64-byte
         // swizzle for 32-column chunks, 128-byte for 64-column ones)
-        constexpr int SCW = C::kCW, VPT = SCW / 2, UPT = VPT / 8;
+        constexpr int SCW = C::kCW, VPT = SCW / NP, UPT = VPT / 8;
         auto swz = [](int row, int u) { return SCW == 64 ? sw128(row, u) : sw64(row, u); };
         for (int c = 0; c < C::kNCh; ++c) {
           if (leader && c > 0) TRACE(k, 4 + c);
@@ -835,8 +869,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                                 static_cast<uint32_t>(acc * BN + c * SCW + hf * VPT);
             if constexpr (VPT == 32)
               tmem_ld_32x32(ta, rr);
-            else
+            else if constexpr (VPT == 16)
               tmem_ld_32x32_x16(ta, rr);
+            else
+              tmem_ld_32x32_x8(ta, rr);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < VPT; ++q) v[q] = __uint_as_float(rr[q]);
@@ -885,13 +921,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             if (leader && c == C::kNCh - 3) TRACE(k, 15);
             const uint32_t ds = stg_direct(stage_u32, b);  // direct [128][SCW]
             const uint32_t ms = stg_mirror(stage_u32, b);  // mirror [SCW][128]
+            uint32_t pk[VPT / 2];  // each value rounded to bf16 once, for both copies
+#pragma unroll
+            for (int q = 0; q < VPT / 2; ++q) pk[q] = pack_bf16x2(v[2 * q], v[2 * q + 1]);
 #pragma unroll
             for (int uu = 0; uu < UPT; ++uu)
-              st_shared_v4(ds + swz(r, UPT * hf + uu), pack_bf16x2(v[8 * uu + 0], v[8 * uu + 1]),
-                           pack_bf16x2(v[8 * uu + 2], v[8 * uu + 3]), pack_bf16x2(v[8 * uu + 4], v[8 * uu + 5]),
-                           pack_bf16x2(v[8 * uu + 6], v[8 * uu + 7]));
+              st_shared_v4(ds + swz(r, UPT * hf + uu), pk[4 * uu], pk[4 * uu + 1], pk[4 * uu + 2], pk[4 * uu + 3]);
 #pragma unroll
-            for (int q = 0; q < VPT; ++q) st_shared_u16(ms + (VPT * hf + q) * 256 + r * 2, bf16_bits(v[q]));
+            for (int q = 0; q < VPT; ++q)
+              st_shared_u16(ms + (VPT * hf + q) * 256 + r * 2, static_cast<uint16_t>(pk[q >> 1] >> (16 * (q & 1))));
             fence_async_smem();
             mbar_arrive(ready_bar(b));
             if (leader && c == C::kNCh - 3) TRACE(k, 16);
@@ -915,13 +953,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
             if (dq == BM / SCW - 1 || col0 + SCW >= G.m) {
               // block complete: lower half := transpose of the upper half.
               // Row r takes S[r][j] = S[j][r] for j < r, eight columns per
-              // 16-byte write; the two warps of a lane quarter split the groups.
+              // 16-byte write; the NP warps of a lane quarter split the groups.
               named_bar(1, kEpiThreads);
               auto s_addr = [&](int row, int col) {
                 return stg_half(stage_u32, col >> 6) +
                        static_cast<uint32_t>(row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2);
               };
-              for (int j0 = 8 * hf; j0 < r; j0 += 16) {
+              for (int j0 = 8 * hf; j0 < r; j0 += 8 * NP) {
                 uint32_t t[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {

@@ -23,9 +23,10 @@ constexpr int kChunk = 32;           // base epilogue chunk width (columns)
 // Epilogue chunk width of the symmetric-output kernels (kGram / kPoly): 32 or 64.
 constexpr int kSymChunk = MUON_SYM_CHUNK;
 static_assert(kSymChunk == 32 || kSymChunk == 64, "symmetric chunk width");
-constexpr int kThreads = 352;        // warp 0 copies, warp 1 MMAs, warps 2-9 epilogue math,
-                                     // warp 10 epilogue loads and stores
-constexpr int kEpiThreads = 256;     // warps 2-9
+// Warp roles: warp 0 copies operands, warp 1 issues the MMAs, warps
+// 2 .. 1 + epilogue warps do the epilogue math (their count per kernel kind
+// is in gemm_tc.cu), then the IO warp (stores) and, for kPoly / kBx /
+// kBxApply, a loader warp (epilogue operand copies).
 
 // kBxApply: the last step's kBx, whose epilogue also applies the result to
 // the caller's weights (ApplyTable) instead of writing X_T.
@@ -79,7 +80,8 @@ struct Params {
 // read and written through its own tensor map: mode 1, W has X's layout
 // (boxes of 32 x 128, one per 32 columns of a chunk); mode 2, W = X^T (a tall
 // matrix; box 32 x chunk width, four per chunk).
-constexpr int kMaxApply = 96;  // matrices per launch with a table entry
+constexpr int kMaxApply = 160;  // matrices per launch with a table entry (the table is a
+                                // __grid_constant__ parameter: about 22 KB at 160)
 
 // A kBx launch may carry the same table with mode 3: the matrix's X_T goes to
 // the caller's bf16 buffer in X's layout (its tensor map; box 64 x 128) as

@@ -11,7 +11,7 @@ the apply (oracle/fp32_ref.apply_f32) given the O the epilogue forms:
   sum of B hi is a multiple of 2^-12 below 2^5, so the fp32 accumulation is
   exact whatever its order and O = fl(a X + B hi) is one rounding of an exact
   value (oracle/fp32_ref.fma_f32);
-* matrices past the epilogue's 96-entry table, or whose W has a column count
+* matrices past the epilogue's 160-entry table, or whose W has a column count
   that is not a multiple of 4, take the pair write and the apply pass: their
   O is the pair's value of that same fp32 O (oracle/fp32_ref.pair_encode).
 
@@ -76,7 +76,7 @@ def run_case(batch, m, n, tall, lr, wd, seed, grid, cautious=False):
     O = expected_O(B, hi, q, m, n)
     scale = update_scale_f32(rows, cols)
     for i in range(batch):
-        fused = i < 96 and cols % 4 == 0
+        fused = i < 160 and cols % 4 == 0
         Oi = O[i] if fused else pair_value(*pair_encode(O[i])).astype(np.float32)
         ref = apply_f32(W0[i], Oi.T if tall else Oi, lr, wd, scale, cautious=cautious)
         got = W[i].cpu().numpy()
@@ -123,8 +123,8 @@ def test_weight_decay_dominant():
 
 @pytest.mark.parametrize("tall", [False, True])
 def test_more_than_the_table(tall):
-    """104 matrices in one launch: 96 applied in the epilogue, 8 by the pass."""
-    run_case(104, 64, 192, tall, lr=0.05, wd=0.5, seed=13 + tall, grid=True)
+    """168 matrices in one launch: 160 applied in the epilogue, 8 by the pass."""
+    run_case(168, 64, 192, tall, lr=0.05, wd=0.5, seed=13 + tall, grid=True)
 
 
 def test_rejects_bad_strides():

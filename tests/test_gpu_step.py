@@ -135,10 +135,10 @@ def test_fused_apply_few_steps(steps):
 
 
 def test_fused_apply_table_overflow():
-    """104 matrices in one launch: the first 96 (wide and tall alternating)
+    """168 matrices in one launch: the first 160 (wide and tall alternating)
     are applied in the epilogue, the rest written as X_T and applied by the
     separate pass."""
-    st = State([(64, 192), (192, 64)] * 52)
+    st = State([(64, 192), (192, 64)] * 84)
     check_step(st, 0, wd=0.5)
 
 
