@@ -652,6 +652,7 @@ __global__ void __launch_bounds__(kScaleThreads) scale_kernel(const __grid_const
 // kNormRowsTall columns of X, eight threads per row segment, 32 row groups
 // summed in shared memory in a fixed order.  Sums are fp64.
 constexpr int kNormThreads = 256;
+constexpr int kNormFactorThreads = 1024;  // one block per matrix: up to 4096 rows
 
 __device__ __forceinline__ void load_pair8(const NormMat& M, int i, int c, float (&v)[8]) {
   const long long idx = static_cast<long long>(i) * M.ld + c;
@@ -687,19 +688,34 @@ __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_c
   const int local = blockIdx.x - M.blk_begin;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (!M.transposed) {
-    for (int j = 0; j < kNormRowsWide / 8; ++j) {
-      const int i = local * kNormRowsWide + warp * (kNormRowsWide / 8) + j;
-      if (i >= M.m) break;  // warp-uniform
-      double acc = 0.0;
-      for (int c = 8 * lane; c < M.n; c += 256) {
-        float v[8];
-        load_pair8(M, i, c, v);
+    // the warp's rows side by side, so each lane has one load per row in flight
+    constexpr int R = kNormRowsWide / 8;
+    const int i0 = local * kNormRowsWide + warp * R;
+    double acc[R];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) acc = fma(static_cast<double>(v[k]), static_cast<double>(v[k]), acc);
+    for (int j = 0; j < R; ++j) acc[j] = 0.0;
+#pragma unroll 2
+    for (int c = 8 * lane; c < M.n; c += 256) {
+      float v[R][8];
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        if (i0 + j < M.m) {
+          load_pair8(M, i0 + j, c, v[j]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[j][k] = 0.f;
+        }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) p.rsq[M.row_base + i] = acc;
+      for (int j = 0; j < R; ++j)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[j] = fma(static_cast<double>(v[j][k]), static_cast<double>(v[j][k]), acc[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+      if (lane == 0 && i0 + j < M.m) p.rsq[M.row_base + i0 + j] = acc[j];
     }
     return;
   }
@@ -709,6 +725,7 @@ __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_c
 #pragma unroll
   for (int k = 0; k < 8; ++k) acc[k] = 0.0;
   if (c0 + 8 * u < M.n) {
+#pragma unroll 8
     for (int i = g; i < M.m; i += 32) {
       float v[8];
       load_pair8(M, i, c0 + 8 * u, v);
@@ -727,13 +744,13 @@ __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_c
 }
 
 // One block per matrix: the state update and the row factors (see NormFacParams).
-__global__ void __launch_bounds__(kNormThreads) norm_factor_kernel(const __grid_constant__ NormFacParams p) {
-  __shared__ double red[2][kNormThreads / 32];
+__global__ void __launch_bounds__(kNormFactorThreads) norm_factor_kernel(const __grid_constant__ NormFacParams p) {
+  __shared__ double red[2][kNormFactorThreads / 32];
   __shared__ double s_g;
   const NormFacMat& M = p.mat[blockIdx.x];
   const double* rsq = p.rsq + M.row_base;
   double s0 = 0.0, s1 = 0.0;
-  for (int i = threadIdx.x; i < M.rows; i += kNormThreads) {
+  for (int i = threadIdx.x; i < M.rows; i += kNormFactorThreads) {
     const double rs = rsq[i];
     const float r32 = __double2float_rn(rs / static_cast<double>(M.cols));
     const float v = __fadd_rn(__fmul_rn(p.beta2, M.v[i]), __fmul_rn(p.omb2, r32));
@@ -754,7 +771,7 @@ __global__ void __launch_bounds__(kNormThreads) norm_factor_kernel(const __grid_
   __syncthreads();
   if (threadIdx.x == 0) {
     double t0 = 0.0, t1 = 0.0;
-    for (int w = 0; w < kNormThreads / 32; ++w) {
+    for (int w = 0; w < kNormFactorThreads / 32; ++w) {
       t0 += red[0][w];
       t1 += red[1][w];
     }
@@ -762,7 +779,7 @@ __global__ void __launch_bounds__(kNormThreads) norm_factor_kernel(const __grid_
   }
   __syncthreads();
   const double gsc = s_g;
-  for (int i = threadIdx.x; i < M.rows; i += kNormThreads) {
+  for (int i = threadIdx.x; i < M.rows; i += kNormFactorThreads) {
     const double f = 1.0 / sqrt(static_cast<double>(M.v[i]) + p.eps);  // this thread wrote v[i]
     p.rowf[M.row_base + i] = __double2float_rn(f * gsc);
   }
@@ -776,7 +793,7 @@ cudaError_t launch_norm_stats(const NormStatParams& p, cudaStream_t s) {
 
 cudaError_t launch_norm_factors(const NormFacParams& p, cudaStream_t s) {
   if (p.nmat <= 0) return cudaSuccess;
-  norm_factor_kernel<<<p.nmat, kNormThreads, 0, s>>>(p);
+  norm_factor_kernel<<<p.nmat, kNormFactorThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
