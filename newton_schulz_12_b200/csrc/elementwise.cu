@@ -688,34 +688,21 @@ __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_c
   const int local = blockIdx.x - M.blk_begin;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (!M.transposed) {
-    // the warp's rows side by side, so each lane has one load per row in flight
-    constexpr int R = kNormRowsWide / 8;
-    const int i0 = local * kNormRowsWide + warp * R;
-    double acc[R];
+    for (int j = 0; j < kNormRowsWide / 8; ++j) {
+      const int i = local * kNormRowsWide + warp * (kNormRowsWide / 8) + j;
+      if (i >= M.m) break;  // warp-uniform
+      double acc = 0.0;
+      // four independent loads in flight per lane, summed in order
+#pragma unroll 4
+      for (int c = 8 * lane; c < M.n; c += 256) {
+        float v[8];
+        load_pair8(M, i, c, v);
 #pragma unroll
-    for (int j = 0; j < R; ++j) acc[j] = 0.0;
-#pragma unroll 2
-    for (int c = 8 * lane; c < M.n; c += 256) {
-      float v[R][8];
-#pragma unroll
-      for (int j = 0; j < R; ++j) {
-        if (i0 + j < M.m) {
-          load_pair8(M, i0 + j, c, v[j]);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) v[j][k] = 0.f;
-        }
+        for (int k = 0; k < 8; ++k) acc = fma(static_cast<double>(v[k]), static_cast<double>(v[k]), acc);
       }
 #pragma unroll
-      for (int j = 0; j < R; ++j)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[j] = fma(static_cast<double>(v[j][k]), static_cast<double>(v[j][k]), acc[j]);
-    }
-#pragma unroll
-    for (int j = 0; j < R; ++j) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
-      if (lane == 0 && i0 + j < M.m) p.rsq[M.row_base + i0 + j] = acc[j];
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) p.rsq[M.row_base + i] = acc;
     }
     return;
   }
@@ -725,7 +712,7 @@ __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_c
 #pragma unroll
   for (int k = 0; k < 8; ++k) acc[k] = 0.0;
   if (c0 + 8 * u < M.n) {
-#pragma unroll 8
+#pragma unroll 4
     for (int i = g; i < M.m; i += 32) {
       float v[8];
       load_pair8(M, i, c0 + 8 * u, v);
