@@ -650,7 +650,9 @@ __global__ void __launch_bounds__(kScaleThreads) scale_kernel(const __grid_const
 // value.  W = X: a block takes kNormRowsWide rows of X, four per warp, the
 // lanes running along the row with 16-byte loads; W = X^T: a block takes
 // kNormRowsTall columns of X, eight threads per row segment, 32 row groups
-// summed in shared memory in a fixed order.  Sums are fp64.
+// summed in shared memory in a fixed order.  Each thread sums its own squares
+// in fp32 (at most max(m, n) / 32 of them: relative error below 1e-5), the
+// threads' partials are combined in fp64; every order is fixed.
 constexpr int kNormThreads = 256;
 constexpr int kNormFactorThreads = 1024;  // one block per matrix: up to 4096 rows
 
@@ -691,15 +693,17 @@ __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_c
     for (int j = 0; j < kNormRowsWide / 8; ++j) {
       const int i = local * kNormRowsWide + warp * (kNormRowsWide / 8) + j;
       if (i >= M.m) break;  // warp-uniform
-      double acc = 0.0;
-      // four independent loads in flight per lane, summed in order
+      // four independent loads in flight per lane; the lane's squares (at
+      // most n / 32 of them) summed in fp32 in order, the lanes in fp64
+      float part = 0.f;
 #pragma unroll 4
       for (int c = 8 * lane; c < M.n; c += 256) {
         float v[8];
         load_pair8(M, i, c, v);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) acc = fma(static_cast<double>(v[k]), static_cast<double>(v[k]), acc);
+        for (int k = 0; k < 8; ++k) part = fmaf(v[k], v[k], part);
       }
+      double acc = static_cast<double>(part);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (lane == 0) p.rsq[M.row_base + i] = acc;
@@ -708,20 +712,22 @@ __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_c
   }
   const int u = threadIdx.x & 7, g = threadIdx.x >> 3;
   const int c0 = local * kNormRowsTall;
-  double acc[8];
+  // each thread's squares of a column (at most m / 32 of them) summed in
+  // fp32 in order, the 32 row groups in fp64
+  float acc[8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) acc[k] = 0.0;
+  for (int k = 0; k < 8; ++k) acc[k] = 0.f;
   if (c0 + 8 * u < M.n) {
 #pragma unroll 4
     for (int i = g; i < M.m; i += 32) {
       float v[8];
       load_pair8(M, i, c0 + 8 * u, v);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) acc[k] = fma(static_cast<double>(v[k]), static_cast<double>(v[k]), acc[k]);
+      for (int k = 0; k < 8; ++k) acc[k] = fmaf(v[k], v[k], acc[k]);
     }
   }
 #pragma unroll
-  for (int k = 0; k < 8; ++k) red[g][8 * u + k] = acc[k];
+  for (int k = 0; k < 8; ++k) red[g][8 * u + k] = static_cast<double>(acc[k]);
   __syncthreads();
   if (threadIdx.x < kNormRowsTall && c0 + static_cast<int>(threadIdx.x) < M.n) {
     double s = 0.0;
