@@ -18,7 +18,8 @@ Per-kernel device times are taken live with CUDA events on the launching
 stream (the library's timing hooks); `roofline` reports the dominant kernel
 against the measured peaks in MEASURED_PEAKS.json.  After the timed region
 (outside it) the same run adds: `value_sustained`, a loop of at least a
-second without the timing hooks, with its own clock record; `ns_768x3072`,
+second without the timing hooks, with its own clock record; `value_graph`,
+the same step recorded once in a CUDA graph and replayed (hooks off); `ns_768x3072`,
 muon_ns_orthogonalize on 64 matrices 768x3072 (the three GEMMs and the whole
 call, nominal and executed TFLOP/s); `scaled_set`, the 144-matrix 1024-wide
 set's full muon_step; `refinements`, muon_step_ex with cautious weight decay
@@ -379,6 +380,26 @@ def measure_ns_768x3072(dev, peaks, reps=20):
     return out
 
 
+def measure_graph(plan, dev, ms_hint, units, min_s=1.0):
+    """The same step recorded once in a CUDA graph (MuonStepPlan.capture) and
+    replayed for at least `min_s` seconds, timing hooks off: the launch gaps
+    of 17 stream launches per step mostly disappear.  capture() itself runs
+    one step (outside the timing)."""
+    import torch
+    import newton_schulz_12_b200 as nsb
+    plan.capture()
+    stream = torch.cuda.current_stream(dev)
+    n = max(50, int(min_s * 1000.0 / max(ms_hint, 1e-3)) + 1)
+    for _ in range(3):
+        plan.replay()
+    with ClockSampler(dev) as clocks:
+        ms = time_steps(plan.replay, n, stream)
+    if nsb.muon_get_status(stream) != 0:
+        raise RuntimeError("device status in the graph replay: " + nsb.muon_last_error())
+    return {"value": units * n / (ms / 1000.0), "unit": UNIT, "steps": n, "ms_per_step": ms / n,
+            "clocks": clocks.summary()}
+
+
 def measure_refinements(W, G, M, shapes, stream, dev, steps=20):
     """muon_step_ex on the GPT-2 set with both refinements on: cautious weight
     decay (wd 0.01) and NorMuon's per-neuron rescale (beta2 0.95); the
@@ -652,6 +673,7 @@ def run_ours(args):
         }
         if world == 1 and not args.no_extras:
             line["value_sustained"] = measure_sustained(step, stream, dev, ms / args.steps, len(shapes))
+            line["value_graph"] = measure_graph(plan, dev, ms / args.steps, len(shapes))
             line["refinements"] = measure_refinements(W, G, M, shapes, stream, dev)
             line["ns_768x3072"] = measure_ns_768x3072(dev, peaks)
             line["square_sweep"] = measure_square_sweep(dev, peaks)

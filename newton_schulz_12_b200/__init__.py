@@ -231,6 +231,35 @@ class MuonStepPlan:
         check(self._fn(len(self.params), self._p, self._g, self._m, self._s, beta, nest, lr, wd,
                        steps, _stream(stream)))
 
+    def capture(self, stream=None):
+        """Record one step into a CUDA graph (returned; also kept for ``replay``).
+
+        One step runs first on ``stream`` (default: a new side stream) so the
+        library's workspace for that stream exists; the next step is only
+        recorded (capture does not run it).  Each replay then performs one step,
+        launching the step's kernels without the per-launch host and scheduling
+        gaps.  The graph bakes in the tensors' addresses, the
+        hyper-parameters of this moment and that stream's workspace: call
+        ``capture`` again after ``update``, and do not call ``muon_release``
+        or a larger library call on that stream while the graph is in use.
+        """
+        s = stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self(s)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            self(s)
+        torch.cuda.current_stream().wait_stream(s)
+        self._graph = graph
+        return graph
+
+    def replay(self):
+        """One step by replaying the graph recorded by ``capture`` (on the current stream)."""
+        if getattr(self, "_graph", None) is None:
+            raise RuntimeError("capture() first")
+        self._graph.replay()
+
 
 def muon_momentum(grads, momentum_bufs, beta=0.95, nesterov=True, sumsq_out=None, stream=None):
     """Momentum stage alone: buffers updated in place; optional per-matrix sum(u^2) (fp32 CUDA)."""
