@@ -340,6 +340,7 @@ void init_tc_params(tc::Params& P, int* status, float a, float b, float c) {
   P.status = status;
   P.timeout_ns = g_timeout_ns;
   P.inject = 0;
+  P.reverse = 0;
   P.trace = nullptr;
 #ifdef MUON_TRACE
   P.trace = g_trace;
@@ -481,6 +482,11 @@ int run_ns_bf16(std::vector<NsGroup>& gs, int steps, const float* abc, int* stat
     tc::Params gram0 = gram[0], bx0 = bx[0];
     gram0.xscale = xscale;
     bx0.xscale = xscale;
+    // Each launch reads what the one before it wrote (X -> A -> B -> X'), and
+    // the tail of that output is what L2 still holds: consecutive launches
+    // walk the tiles in opposite directions, the first Gram backwards (the
+    // pass that wrote X_0 went forwards).
+    int backwards = 1;
     int cur = 0;
     for (int t = 0; t < steps; ++t) {
       // the step's own (a, b, c): B = b A + c A^2 in kPoly, a X in kBx
@@ -488,7 +494,12 @@ int run_ns_bf16(std::vector<NsGroup>& gs, int steps, const float* abc, int* stat
       poly.c = abc[3 * t + 2];
       tc::Params& bxt = t == 0 ? bx0 : bx[cur];
       bxt.a = abc[3 * t];
-      MUON_TRY(launch_tc(tc::kGram, t == 0 ? gram0 : gram[cur], sms, s));
+      tc::Params& gramt = t == 0 ? gram0 : gram[cur];
+      gramt.reverse = backwards;
+      poly.reverse = backwards ^ 1;
+      bxt.reverse = backwards;
+      backwards ^= 1;
+      MUON_TRY(launch_tc(tc::kGram, gramt, sms, s));
       MUON_TRY(launch_tc(tc::kPoly, poly, sms, s));
       if (apply && t == steps - 1) {
         tc::LaunchApply table;

@@ -171,6 +171,7 @@ struct TileCoord {
 template <int EPI>
 __device__ __forceinline__ TileCoord decode_tile(const Params& p, int t, int rank) {
   TileCoord c;
+  if (p.reverse) t = p.total_tiles - 1 - t;
   int g = 0;
   while (g + 1 < p.ngroups && t >= p.grp[g + 1].tile_begin) ++g;
   const Group& G = p.grp[g];

@@ -72,6 +72,9 @@ struct Params {
   unsigned long long timeout_ns;
   int inject;  // 1: withhold one operand copy in CTA 0 (timeout-path test)
   unsigned long long* trace;  // timestamps (only recorded in builds with MUON_TRACE)
+  // 1: the pairs take the tiles in descending order, so a launch starts on
+  // the matrices whose operands the previous launch touched last (still in L2)
+  int reverse;
 };
 
 // Final-step apply (kBxApply): per matrix of the launch, either X_T is written
