@@ -98,11 +98,12 @@ def test_gpt2_small_hard_spectra():
     check_step(st, 0)
 
 
-def test_scaled_set_sampled():
-    """144-matrix 1024-wide set with wd 0.01; one matrix of each shape checked."""
+def test_scaled_set_full():
+    """144-matrix 1024-wide set with wd 0.01, every matrix checked (all 144
+    take the fused apply of the last launch)."""
     shapes = workloads.scaled_shapes()
     st = State(shapes)
-    check_step(st, 0, wd=0.01, check=[0, 4, 5, 142, 143])
+    check_step(st, 0, wd=0.01)
 
 
 # The last step's BX applies its result to W in the GEMM epilogue.  These
