@@ -355,11 +355,12 @@ def measure_ns_768x3072(dev, peaks, reps=20):
     g = torch.Generator(device="cpu").manual_seed(3000 + m)
     xs = [torch.randn(m, n, generator=g).to(torch.bfloat16).to(dev) for _ in range(batch)]
     stream = torch.cuda.current_stream(dev)
+    plan = nsb.MuonNsPlan(xs)
     for _ in range(3):
-        nsb.muon_ns_orthogonalize(xs)
+        plan(stream)
     with ClockSampler(dev) as clocks:
         nsb.muon_profile_begin()
-        ms = time_steps(lambda: nsb.muon_ns_orthogonalize(xs), reps, stream)
+        ms = time_steps(lambda: plan(stream), reps, stream)
         prof = nsb.muon_profile_end()
     if nsb.muon_get_status() != 0:
         raise RuntimeError("device status in the 768x3072 case: " + nsb.muon_last_error())
@@ -432,7 +433,9 @@ def measure_refinements(W, G, M, shapes, stream, dev, steps=20):
 def measure_square_sweep(dev, peaks, reps=10):
     """muon_ns_orthogonalize (bf16) on the square width sweep: m in {256 .. 4096}
     with batch 64 (768/m)^2 (>= 1), bf16 N(0, 1) drawn on the device; GEMM
-    and whole-call TFLOP/s, nominal and executed, per width."""
+    and whole-call TFLOP/s, nominal and executed, per width.  The call goes
+    through MuonNsPlan (arguments marshalled once); `call_ms_graph` is the same
+    call replayed from a CUDA graph."""
     import torch
     import newton_schulz_12_b200 as nsb
     from newton_schulz_12_b200 import workloads
@@ -441,17 +444,24 @@ def measure_square_sweep(dev, peaks, reps=10):
     for m, batch in workloads.sweep_cases():
         g = torch.Generator(device=dev).manual_seed(3000 + m)
         xs = [torch.randn(m, m, generator=g, device=dev).to(torch.bfloat16) for _ in range(batch)]
+        plan = nsb.MuonNsPlan(xs)
         for _ in range(2):
-            nsb.muon_ns_orthogonalize(xs)
+            plan(stream)
         nsb.muon_profile_begin()
-        ms = time_steps(lambda: nsb.muon_ns_orthogonalize(xs), reps, stream)
+        ms = time_steps(lambda: plan(stream), reps, stream)
         prof = nsb.muon_profile_end()
         if nsb.muon_get_status() != 0:
             raise RuntimeError(f"device status in the sweep at m={m}: " + nsb.muon_last_error())
+        gs = torch.cuda.Stream(dev)
+        plan.capture(gs)
+        with torch.cuda.stream(gs):
+            ms_graph = time_steps(plan.replay, reps, gs)
+        del plan
         nominal = nominal_flops([(m, m)] * batch)
         executed = executed_flops([(m, m)] * batch)
         gemm_ms = sum(prof[k][0] for k in ("gram", "poly", "bx")) / reps
-        out.append({"m": m, "batch": batch, "call_ms": ms / reps, "gemm_ms": gemm_ms,
+        out.append({"m": m, "batch": batch, "call_ms": ms / reps, "call_ms_graph": ms_graph / reps,
+                    "gemm_ms": gemm_ms,
                     "gemm_tflops_nominal": nominal / gemm_ms / 1e9,
                     "gemm_tflops_executed": executed / gemm_ms / 1e9,
                     "call_tflops_nominal": nominal / (ms / reps) / 1e9,
@@ -786,8 +796,9 @@ def run_ns_cases(args):
         g = torch.Generator(device="cpu").manual_seed(3000 + m)
         xs = [torch.randn(m, n, generator=g).to(torch.bfloat16).to(dev) for _ in range(batch)]
         flops = nominal_flops([(m, n)] * batch)
+        plan = nsb.MuonNsPlan(xs)
         for _ in range(args.warmup):
-            nsb.muon_ns_orthogonalize(xs)
+            plan()
         torch.cuda.synchronize()
         reps = max(3, min(args.steps, 50))
         nsb.muon_profile_begin()
@@ -795,7 +806,7 @@ def run_ns_cases(args):
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record()
         for _ in range(reps):
-            nsb.muon_ns_orthogonalize(xs)
+            plan()
         t1.record()
         torch.cuda.synchronize()
         prof = nsb.muon_profile_end()

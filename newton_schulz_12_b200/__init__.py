@@ -20,7 +20,7 @@ from . import _lib
 from ._lib import MUON_BF16, MUON_CAUTIOUS_WD, MUON_FP32, MuonError, check, ptr_array, shape_array
 
 __all__ = [
-    "NS_COEFFS", "MuonError", "MuonStepPlan", "muon_ns_orthogonalize",
+    "NS_COEFFS", "MuonError", "MuonStepPlan", "MuonNsPlan", "muon_ns_orthogonalize",
     "muon_ns_orthogonalize_schedule",
     "muon_ns_orthogonalize_static", "muon_step", "muon_step_ex", "muon_momentum",
     "muon_apply", "muon_apply_ex", "MUON_CAUTIOUS_WD", "muon_gram_bf16", "muon_poly_bf16", "muon_bx_bf16",
@@ -189,12 +189,46 @@ def muon_step_ex(params, grads, momentum_bufs, beta=0.95, nesterov=True, lr=0.05
                                   _stream(stream)))
 
 
-class MuonStepPlan:
+class _Replayable:
+    """capture / replay for a plan whose call takes a stream."""
+
+    def capture(self, stream=None):
+        """Record one call into a CUDA graph (returned; also kept for ``replay``).
+
+        One call runs first on ``stream`` (default: a new side stream) so the
+        library's workspace for that stream exists; the next call is only
+        recorded (capture does not run it).  Each replay then performs one call,
+        launching its kernels without the per-launch host and scheduling gaps.
+        The graph bakes in the tensors' addresses, the parameters of this
+        moment and that stream's workspace: call ``capture`` again after
+        ``update``, and do not call ``muon_release`` or a larger library call on
+        that stream while the graph is in use.
+        """
+        s = stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self(s)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            self(s)
+        torch.cuda.current_stream().wait_stream(s)
+        self._graph = graph
+        return graph
+
+    def replay(self):
+        """One call by replaying the graph recorded by ``capture`` (on the current stream)."""
+        if getattr(self, "_graph", None) is None:
+            raise RuntimeError("capture() first")
+        self._graph.replay()
+
+
+class MuonStepPlan(_Replayable):
     """muon_step with its arguments marshalled once, for a fixed set of tensors.
 
     Checks dtypes, shapes and contiguity at construction; each call then passes
     the cached pointer arrays straight to the C ABI.  The tensors must stay
-    alive and keep their storage while the plan is used.
+    alive and keep their storage while the plan is used.  ``capture`` records a
+    step in a CUDA graph and ``replay`` runs it (one step per replay).
     """
 
     def __init__(self, params, grads, momentum_bufs, beta=0.95, nesterov=True, lr=0.05, wd=0.0,
@@ -231,34 +265,28 @@ class MuonStepPlan:
         check(self._fn(len(self.params), self._p, self._g, self._m, self._s, beta, nest, lr, wd,
                        steps, _stream(stream)))
 
-    def capture(self, stream=None):
-        """Record one step into a CUDA graph (returned; also kept for ``replay``).
+class MuonNsPlan(_Replayable):
+    """muon_ns_orthogonalize with its arguments marshalled once, for a fixed
+    list of equal-shape matrices (orthogonalised in place by every call).
 
-        One step runs first on ``stream`` (default: a new side stream) so the
-        library's workspace for that stream exists; the next step is only
-        recorded (capture does not run it).  Each replay then performs one step,
-        launching the step's kernels without the per-launch host and scheduling
-        gaps.  The graph bakes in the tensors' addresses, the
-        hyper-parameters of this moment and that stream's workspace: call
-        ``capture`` again after ``update``, and do not call ``muon_release``
-        or a larger library call on that stream while the graph is in use.
-        """
-        s = stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.Stream()
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            self(s)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=s):
-            self(s)
-        torch.cuda.current_stream().wait_stream(s)
-        self._graph = graph
-        return graph
+    For many small matrices the per-call checks and pointer marshalling cost
+    about as much host time as the GPU spends on them; the plan pays it once.
+    ``capture`` / ``replay`` as for MuonStepPlan.
+    """
 
-    def replay(self):
-        """One step by replaying the graph recorded by ``capture`` (on the current stream)."""
-        if getattr(self, "_graph", None) is None:
-            raise RuntimeError("capture() first")
-        self._graph.replay()
+    def __init__(self, xs, a=NS_COEFFS[0], b=NS_COEFFS[1], c=NS_COEFFS[2], steps=5):
+        self.xs = list(xs)
+        if not self.xs:
+            raise ValueError("no matrices")
+        self.shape, self._mode, self._arr = _ns_batch(self.xs)
+        self._args = (float(a), float(b), float(c), int(steps))
+        self._fn = _lib.lib().muon_ns_orthogonalize
+
+    def __call__(self, stream=None):
+        a, b, c, steps = self._args
+        check(self._fn(len(self.xs), self.shape[0], self.shape[1], self._arr, a, b, c, steps,
+                       self._mode, _stream(stream)))
+        return self.xs
 
 
 def muon_momentum(grads, momentum_bufs, beta=0.95, nesterov=True, sumsq_out=None, stream=None):

@@ -34,3 +34,26 @@ def test_graph_replay_equals_direct_calls(shapes):
     assert nsb.muon_get_status() == 0
     for x, y in zip(Wa + Ma, Wb + Mb):
         assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("m,n,batch", [(256, 256, 200), (130, 68, 3), (768, 3072, 2)])
+def test_ns_plan_and_its_replay_equal_direct_calls(m, n, batch):
+    """MuonNsPlan: a call equals muon_ns_orthogonalize; capture (one call) plus
+    two replays equal three direct calls, bit for bit."""
+    xs = [workloads.gaussian((m, n), 1.0, seed=40 + i, dtype=torch.bfloat16).cuda() for i in range(batch)]
+    a = [x.clone() for x in xs]
+    b = [x.clone() for x in xs]
+    c = [x.clone() for x in xs]
+    nsb.MuonNsPlan(a)()
+    nsb.muon_ns_orthogonalize(b)
+    torch.cuda.synchronize()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+    plan = nsb.MuonNsPlan(c)
+    plan.capture()
+    for _ in range(2):
+        plan.replay()
+    for _ in range(2):
+        nsb.muon_ns_orthogonalize(b)
+    torch.cuda.synchronize()
+    assert nsb.muon_get_status() == 0
+    assert all(torch.equal(x, y) for x, y in zip(c, b))
