@@ -19,7 +19,9 @@ stream (the library's timing hooks); `roofline` reports the dominant kernel
 against the measured peaks in MEASURED_PEAKS.json.  After the timed region
 (outside it) the same run adds: `value_sustained`, a loop of at least a
 second without the timing hooks, with its own clock record; `value_graph`,
-the same step recorded once in a CUDA graph and replayed (hooks off); `ns_768x3072`,
+the same step recorded once in a CUDA graph and replayed (hooks off);
+`step_distribution`, median / p10 / p90 of single-step times, warm and with L2
+flushed before each step; `ns_768x3072`,
 muon_ns_orthogonalize on 64 matrices 768x3072 (the three GEMMs and the whole
 call, nominal and executed TFLOP/s); `scaled_set`, the 144-matrix 1024-wide
 set's full muon_step; `refinements`, muon_step_ex with cautious weight decay
@@ -343,6 +345,34 @@ def measure_sustained(step, stream, dev, ms_hint, units, min_s=1.5):
            "seconds": ms / 1000.0, "clocks": c}
     if c.get("sm_mhz"):
         out["ms_x_sm_ghz"] = ms / n * c["sm_mhz"] / 1000.0
+    return out
+
+
+def measure_step_distribution(step, stream, dev, reps=50):
+    """Per-step device times (timing hooks off), each step between its own
+    pair of events: median, p10 and p90 over `reps` steps, once warm (inputs
+    already larger than L2) and once with L2 flushed before every step (a
+    256 MB buffer, twice L2, written between the steps, outside their events)."""
+    import torch
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    out = {}
+    for kind in ("warm", "l2_flushed"):
+        for _ in range(3):
+            step()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        torch.cuda.synchronize(dev)
+        for a, b in evs:
+            if kind == "l2_flushed":
+                flush.fill_(1.0)
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        t = sorted(a.elapsed_time(b) for a, b in evs)
+        q = lambda f: t[min(len(t) - 1, int(round(f * (len(t) - 1))))]  # noqa: E731
+        out[kind] = {"median_ms": q(0.5), "p10_ms": q(0.1), "p90_ms": q(0.9), "steps": reps}
+    del flush
     return out
 
 
@@ -684,6 +714,7 @@ def run_ours(args):
         if world == 1 and not args.no_extras:
             line["value_sustained"] = measure_sustained(step, stream, dev, ms / args.steps, len(shapes))
             line["value_graph"] = measure_graph(plan, dev, ms / args.steps, len(shapes))
+            line["step_distribution"] = measure_step_distribution(step, stream, dev)
             line["refinements"] = measure_refinements(W, G, M, shapes, stream, dev)
             line["ns_768x3072"] = measure_ns_768x3072(dev, peaks)
             line["square_sweep"] = measure_square_sweep(dev, peaks)
