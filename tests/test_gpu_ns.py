@@ -157,3 +157,17 @@ def test_last_step_writes_outputs_directly_or_through_the_pass(rows, cols, batch
         ref = oracle.newton_schulz(mats[i].double().numpy())
         assert rel_fro(got[i], ref) <= TOL_BF16, i
         assert_blocks(got[i], ref, BLOCK_TOL_BF16, f"matrix {i}")
+
+
+@pytest.mark.parametrize("bad", [float("nan"), float("inf")])
+def test_non_finite_matrix_leaves_the_others_unchanged(bad):
+    """Matrices are independent (the iteration is per matrix): a NaN or an inf
+    in one matrix of a batch changes no bit of the other matrices' results,
+    so no reduction, tile or table entry mixes them."""
+    mats = [workloads.gaussian((300, 1000), 1.0, seed=7500 + i, dtype=torch.bfloat16) for i in range(4)]
+    clean = run_ns(mats)
+    dirty = [m.clone() for m in mats]
+    dirty[1][5, 7] = bad
+    got = run_ns(dirty)
+    for i in (0, 2, 3):
+        assert np.array_equal(got[i], clean[i]), i

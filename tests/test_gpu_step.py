@@ -182,3 +182,24 @@ def test_step_is_deterministic():
 def test_empty_count_is_noop():
     nsb.muon_step([], [], [])
     assert nsb.muon_get_status() == 0
+
+
+@pytest.mark.parametrize("bad", [float("nan"), float("inf")])
+def test_non_finite_gradient_leaves_the_other_matrices_unchanged(bad):
+    """A NaN or inf in one matrix's gradient changes no bit of any other
+    matrix's weights or momentum (same shape group and other groups)."""
+    shapes = [(256, 256), (256, 1024), (1024, 256), (256, 256), (256, 1024)]
+    Ws, Gs = workloads.muon_set(shapes, step=0)
+    runs = []
+    for poison in (False, True):
+        W = [w.cuda() for w in Ws]
+        M = [torch.zeros(s, device="cuda") for s in shapes]
+        G = [g.clone().cuda() for g in Gs]
+        if poison:
+            G[1][3, 9] = bad
+        nsb.muon_step(W, G, M, wd=0.01)
+        torch.cuda.synchronize()
+        runs.append(([w.cpu() for w in W], [m.cpu() for m in M]))
+    (Wc, Mc), (Wp, Mp) = runs
+    for i in (0, 2, 3, 4):
+        assert torch.equal(Wc[i], Wp[i]) and torch.equal(Mc[i], Mp[i]), i
