@@ -170,3 +170,41 @@ def test_python_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError):
         nsb.muon_step([torch.zeros(4, 4)], [torch.zeros(4, 4, dtype=torch.bfloat16)],
                       [torch.zeros(4, 4)])
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "muon.h"
+int main(void) {
+  if (muon_version() != 100) return 1;
+  /* argument errors come back synchronously, before any device work */
+  if (muon_ns_orthogonalize(-1, 8, 8, NULL, 3.4445f, -4.775f, 2.0315f, 5, MUON_BF16, NULL) != MUON_ERR_ARG)
+    return 2;
+  if (strlen(muon_last_error()) == 0) return 3;
+  if (muon_step(-1, NULL, NULL, NULL, NULL, 0.95f, 1, 0.05f, 0.0f, 5, NULL) != MUON_ERR_ARG) return 4;
+  printf("ok\n");
+  return 0;
+}
+"""
+
+
+@pytest.mark.parametrize("compiler,std", [("gcc", "-std=c11"), ("g++", "-std=c++17")])
+def test_plain_c_client_builds_and_runs(tmp_path, compiler, std):
+    """The header compiles on its own as C11 and C++17 (no CUDA headers) and a
+    program linked against the library gets its version and its synchronous
+    argument errors without a GPU."""
+    import shutil
+    import subprocess
+    if shutil.which(compiler) is None:
+        pytest.skip(f"{compiler} not available")
+    src = tmp_path / ("client.c" if compiler == "gcc" else "client.cpp")
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    libname = os.path.basename(_lib.LIB_PATH)
+    subprocess.run([compiler, std, "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                    "-o", str(exe), os.path.join(libdir, libname), f"-Wl,-rpath,{libdir}"],
+                   check=True, capture_output=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stdout, out.stderr)
