@@ -6,7 +6,9 @@
   fp64 oracle run on the GPU's own pre-step state (so no drift accumulates),
   and every 32 x 32 block of it within 4 x 3e-2 of the same block;
 * the GPT-2-small hidden set (72 matrices, 768 wide) at full size, with
-  Gaussian and with hard (log-uniform, spiked) gradient spectra.
+  Gaussian and with hard (log-uniform, spiked) gradient spectra;
+* ten consecutive steps against the oracle run on its own state (no drift),
+  and a non-finite gradient isolated to its own matrix.
 """
 import numpy as np
 import pytest
@@ -203,3 +205,29 @@ def test_non_finite_gradient_leaves_the_other_matrices_unchanged(bad):
     (Wc, Mc), (Wp, Mp) = runs
     for i in (0, 2, 3, 4):
         assert torch.equal(Wc[i], Wp[i]) and torch.equal(Mc[i], Mp[i]), i
+
+
+def test_ten_steps_track_the_oracle():
+    """Ten consecutive steps from the same start, the GPU on its own state and
+    the fp64 oracle on its own (momentum and weights never re-synchronised):
+    the total change of W stays within 3e-2 of the oracle's, relative in
+    Frobenius norm, for every matrix, and within 4 x 3e-2 on every 32 x 32
+    block -- no error builds up in the momentum or the weights over steps."""
+    shapes = workloads.gpt2_small_shapes(layers=1, width=256) + [(130, 68)]
+    Ws, _ = workloads.muon_set(shapes, step=0)
+    W = [w.cuda() for w in Ws]
+    M = [torch.zeros(s, device="cuda") for s in shapes]
+    Wo = [w.double().numpy() for w in Ws]
+    Mo = [np.zeros(s) for s in shapes]
+    for step in range(10):
+        _, Gs = workloads.muon_set(shapes, step=step)
+        nsb.muon_step(W, [g.cuda() for g in Gs], M, wd=0.01)
+        for i in range(len(shapes)):
+            Wo[i], Mo[i], _ = oracle.muon_step(Wo[i], Gs[i].double().numpy(), Mo[i], beta=np.float32(0.95),
+                                               lr=np.float32(0.05), wd=np.float32(0.01))
+    assert nsb.muon_get_status() == 0
+    for i in range(len(shapes)):
+        dW_ref = Wo[i] - Ws[i].double().numpy()
+        dW = W[i].double().cpu().numpy() - Ws[i].double().numpy()
+        assert rel_fro(dW, dW_ref) <= TOL, (i, shapes[i], rel_fro(dW, dW_ref))
+        assert_blocks(dW, dW_ref, BLOCK_TOL, f"matrix {i} after ten steps")
