@@ -153,7 +153,7 @@ def test_last_step_writes_outputs_directly_or_through_the_pass(rows, cols, batch
     mats = [workloads.gaussian((rows, cols), 1.0, seed=7300 + i, dtype=torch.bfloat16)
             for i in range(batch)]
     got = run_ns(mats)
-    for i in sorted({0, batch // 2, batch - 1} | ({159, 160} if batch > 160 else set())):
+    for i in range(batch):
         ref = oracle.newton_schulz(mats[i].double().numpy())
         assert rel_fro(got[i], ref) <= TOL_BF16, i
         assert_blocks(got[i], ref, BLOCK_TOL_BF16, f"matrix {i}")
