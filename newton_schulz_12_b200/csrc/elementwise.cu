@@ -645,39 +645,45 @@ __global__ void __launch_bounds__(kScaleThreads) scale_kernel(const __grid_const
 }
 
 // ------------------------------------------------------- per-neuron rescale
-// Row sums of O^2 over the caller's W rows (NorMuon reading), O read from the
-// result pair as the apply pass reads it: O = fl(oscale * pair) or the pair's
-// value.  W = X: a block takes kNormRowsWide rows of X, four per warp, the
-// lanes running along the row with 16-byte loads; W = X^T: a block takes
-// kNormRowsTall columns of X, eight threads per row segment, 32 row groups
-// summed in shared memory in a fixed order.  Each thread sums its own squares
-// in fp32 (at most max(m, n) / 32 of them: relative error below 1e-5), the
-// threads' partials are combined in fp64; every order is fixed.
+// Row sums of O^2 over the caller's W rows (NorMuon reading), from the bf16
+// part of O's pair: hi is O rounded to nearest bf16, |O - hi| <= 2^-9 |hi|,
+// so every square, and with it every row sum, is within a factor 1 +- 2^-8
+// of O's (the update itself carries a 3e-2 tolerance).  Reading 2 B per
+// element instead of 3, with no residual to decode, keeps the pass at the
+// memory's rate.  O = oscale * pair when oscale is set (zero steps): the
+// sums are then scaled by oscale^2.  W = X: a block takes kNormRowsWide rows
+// of X, four per warp, the lanes running along the row with 16-byte loads;
+// W = X^T: a block takes kNormRowsTall columns of X, eight threads per row
+// segment, 32 row groups summed in shared memory in a fixed order.  Each
+// thread sums its own squares in fp32 (at most max(m, n) / 32 of them:
+// relative error below 1e-5), the threads' partials are combined in fp64;
+// every order is fixed.
 constexpr int kNormThreads = 256;
 constexpr int kNormFactorThreads = 1024;  // one block per matrix: up to 4096 rows
 
-__device__ __forceinline__ void load_pair8(const NormMat& M, int i, int c, float (&v)[8]) {
-  const long long idx = static_cast<long long>(i) * M.ld + c;
-  const float f = M.oscale ? *M.oscale : 1.0f;
-  if (c + 8 <= M.n) {  // rows are 16-byte strided (ld % 16 == 0) and c % 8 == 0: aligned
-    pair_decode8(*reinterpret_cast<const uint4*>(static_cast<const bf16*>(M.hi) + idx),
-                 *reinterpret_cast<const uint2*>(static_cast<const int8_t*>(M.lo) + idx), v);
+// Squares of eight bf16 values (one 16-byte word of hi) added to acc[0..7].
+__device__ __forceinline__ void add_squares8(const uint4 w, float (&acc)[8]) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int k = 0; k < 8; ++k) v[k] = M.oscale ? v[k] * f : v[k];
-    return;
-  }
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    float x = 0.f;
-    if (c + k < M.n) {
-      const uint32_t fb = static_cast<uint32_t>(static_cast<const uint16_t*>(M.hi)[idx + k]) << 16;
-      const int q = static_cast<const int8_t*>(M.lo)[idx + k];
-      x = fmaf(static_cast<float>(q), lo8_unit(fb), __uint_as_float(fb));
-      if (M.oscale) x = x * f;
-    }
-    v[k] = x;
+  for (int h = 0; h < 4; ++h) {
+    const float a = __uint_as_float(ws[h] << 16), b = __uint_as_float(ws[h] & 0xFFFF0000u);
+    acc[2 * h] = fmaf(a, a, acc[2 * h]);
+    acc[2 * h + 1] = fmaf(b, b, acc[2 * h + 1]);
   }
 }
+
+// The 16-byte word of hi at (row i, columns c .. c+7), zeros past column n
+// (rows are 16-byte strided, ld % 16 == 0, and c % 8 == 0).
+__device__ __forceinline__ uint4 load_hi8(const NormMat& M, int i, int c) {
+  const bf16* row = static_cast<const bf16*>(M.hi) + static_cast<long long>(i) * M.ld;
+  if (c + 8 <= M.n) return *reinterpret_cast<const uint4*>(row + c);
+  uint32_t h[4] = {0u, 0u, 0u, 0u};
+  const uint16_t* r16 = reinterpret_cast<const uint16_t*>(row);
+  for (int k = 0; k < 8 && c + k < M.n; ++k) h[k >> 1] |= static_cast<uint32_t>(r16[c + k]) << (16 * (k & 1));
+  return make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+constexpr int kNormBatch = 8;  // 16-byte loads a thread has in flight
 
 __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_constant__ NormStatParams p) {
   __shared__ double red[32][kNormRowsTall + 1];
@@ -689,24 +695,30 @@ __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_c
   const NormMat& M = p.mat[lo];
   const int local = blockIdx.x - M.blk_begin;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const double s2 = M.oscale ? static_cast<double>(*M.oscale) * static_cast<double>(*M.oscale) : 1.0;
   if (!M.transposed) {
     for (int j = 0; j < kNormRowsWide / 8; ++j) {
       const int i = local * kNormRowsWide + warp * (kNormRowsWide / 8) + j;
       if (i >= M.m) break;  // warp-uniform
-      // four independent loads in flight per lane; the lane's squares (at
-      // most n / 32 of them) summed in fp32 in order, the lanes in fp64
-      float part = 0.f;
-#pragma unroll 4
-      for (int c = 8 * lane; c < M.n; c += 256) {
-        float v[8];
-        load_pair8(M, i, c, v);
+      // the lanes along the row, kNormBatch words each in flight; each
+      // lane's squares summed in fp32 in a fixed order, the lanes in fp64
+      float part[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) part = fmaf(v[k], v[k], part);
+      for (int k = 0; k < 8; ++k) part[k] = 0.f;
+      for (int c0 = 8 * lane; c0 < M.n; c0 += 256 * kNormBatch) {
+        uint4 w[kNormBatch];
+#pragma unroll
+        for (int q = 0; q < kNormBatch; ++q)
+          w[q] = c0 + 256 * q < M.n ? load_hi8(M, i, c0 + 256 * q) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int q = 0; q < kNormBatch; ++q) add_squares8(w[q], part);
       }
-      double acc = static_cast<double>(part);
+      double acc = 0.0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc += static_cast<double>(part[k]);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) p.rsq[M.row_base + i] = acc;
+      if (lane == 0) p.rsq[M.row_base + i] = acc * s2;
     }
     return;
   }
@@ -718,12 +730,13 @@ __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_c
 #pragma unroll
   for (int k = 0; k < 8; ++k) acc[k] = 0.f;
   if (c0 + 8 * u < M.n) {
-#pragma unroll 4
-    for (int i = g; i < M.m; i += 32) {
-      float v[8];
-      load_pair8(M, i, c0 + 8 * u, v);
+    for (int i0 = g; i0 < M.m; i0 += 32 * kNormBatch) {
+      uint4 w[kNormBatch];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) acc[k] = fmaf(v[k], v[k], acc[k]);
+      for (int q = 0; q < kNormBatch; ++q)
+        w[q] = i0 + 32 * q < M.m ? load_hi8(M, i0 + 32 * q, c0 + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int q = 0; q < kNormBatch; ++q) add_squares8(w[q], acc);
     }
   }
 #pragma unroll
@@ -732,7 +745,7 @@ __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_c
   if (threadIdx.x < kNormRowsTall && c0 + static_cast<int>(threadIdx.x) < M.n) {
     double s = 0.0;
     for (int q = 0; q < 32; ++q) s += red[q][threadIdx.x];
-    p.rsq[M.row_base + c0 + threadIdx.x] = s;
+    p.rsq[M.row_base + c0 + threadIdx.x] = s * s2;
   }
 }
 

@@ -231,17 +231,18 @@ struct OutParams {
 
 // Per-neuron rescale of the update (NorMuon reading).  For each row r of the
 // caller's W (rows x cols) with O its update:
-//   rsq_r  = sum over the row of O^2                    (fp64, fixed order)
+//   rsq_r  = sum over the row of bf16(O)^2              (fp64, fixed order)
 //   v'_r   = fl(fl(beta2 v_r) + fl(omb2 fl32(rsq_r / cols)))     (fp32 state)
 //   f_r    = 1 / sqrt(v'_r + eps)                        (fp64)
 //   g      = sqrt(sum_r rsq_r / sum_r f_r^2 rsq_r)       (1 if the sum is 0)
 //   rowf_r = fl32(f_r g)      -- O's row r is multiplied by rowf_r before the apply,
 // so the update keeps its Frobenius norm and only its split over rows changes.
-// O is read from the result pair in X's layout (W = X, or W = X^T when
-// transposed), as the apply pass reads it.
+// The row sums read the bf16 part of the result pair (O rounded to nearest
+// bf16) in X's layout (W = X, or W = X^T when transposed); the apply pass
+// then multiplies the pair's value.
 struct NormMat {
-  const void* hi;     // the pair of O (X layout, m x n, row stride ld)
-  const void* lo;
+  const void* hi;     // bf16 part of O's pair (X layout, m x n, row stride ld)
+  const void* lo;     // its int8 residual (not read by the row sums)
   const float* oscale;  // O = fl(oscale[0] * pair) when set, else the pair's value
   int m, n;
   long long ld;
