@@ -685,7 +685,7 @@ __device__ __forceinline__ uint4 load_hi8(const NormMat& M, int i, int c) {
 
 constexpr int kNormBatch = 8;  // 16-byte loads a thread has in flight
 
-__global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_constant__ NormStatParams p) {
+__global__ void __launch_bounds__(kNormThreads, 4) norm_stats_kernel(const __grid_constant__ NormStatParams p) {
   __shared__ double red[32][kNormRowsTall + 1];
   int lo = 0, hi = p.nmat - 1;  // last matrix whose first block is <= blockIdx.x
   while (lo < hi) {
@@ -697,28 +697,47 @@ __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const double s2 = M.oscale ? static_cast<double>(*M.oscale) * static_cast<double>(*M.oscale) : 1.0;
   if (!M.transposed) {
-    for (int j = 0; j < kNormRowsWide / 8; ++j) {
-      const int i = local * kNormRowsWide + warp * (kNormRowsWide / 8) + j;
-      if (i >= M.m) break;  // warp-uniform
-      // the lanes along the row, kNormBatch words each in flight; each
-      // lane's squares summed in fp32 in a fixed order, the lanes in fp64
-      float part[8];
+    // two of the warp's rows at a time, the lanes along them, four words of
+    // each row in flight per lane; each lane's squares of a row summed in
+    // fp32 in a fixed order, the lanes in fp64
+    constexpr int kB = kNormBatch / 2;
+    for (int j = 0; j < kNormRowsWide / 8; j += 2) {
+      const int ia = local * kNormRowsWide + warp * (kNormRowsWide / 8) + j, ib = ia + 1;
+      if (ia >= M.m) break;  // warp-uniform
+      const bool has_b = ib < M.m;
+      float pa[8], pb[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) part[k] = 0.f;
-      for (int c0 = 8 * lane; c0 < M.n; c0 += 256 * kNormBatch) {
-        uint4 w[kNormBatch];
+      for (int k = 0; k < 8; ++k) pa[k] = pb[k] = 0.f;
+      for (int c0 = 8 * lane; c0 < M.n; c0 += 256 * kB) {
+        uint4 wa[kB], wb[kB];
 #pragma unroll
-        for (int q = 0; q < kNormBatch; ++q)
-          w[q] = c0 + 256 * q < M.n ? load_hi8(M, i, c0 + 256 * q) : make_uint4(0u, 0u, 0u, 0u);
+        for (int q = 0; q < kB; ++q) {
+          const int c = c0 + 256 * q;
+          wa[q] = c < M.n ? load_hi8(M, ia, c) : make_uint4(0u, 0u, 0u, 0u);
+          wb[q] = (has_b && c < M.n) ? load_hi8(M, ib, c) : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
-        for (int q = 0; q < kNormBatch; ++q) add_squares8(w[q], part);
+        for (int q = 0; q < kB; ++q)
+          if (c0 + 256 * q < M.n) {  // rows shorter than a batch: no idle squares
+            add_squares8(wa[q], pa);
+            add_squares8(wb[q], pb);
+          }
       }
-      double acc = 0.0;
+      double a = 0.0, b = 0.0;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) acc += static_cast<double>(part[k]);
+      for (int k = 0; k < 8; ++k) {
+        a += static_cast<double>(pa[k]);
+        b += static_cast<double>(pb[k]);
+      }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) p.rsq[M.row_base + i] = acc * s2;
+      for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        b += __shfl_xor_sync(0xffffffffu, b, o);
+      }
+      if (lane == 0) {
+        p.rsq[M.row_base + ia] = a * s2;
+        if (has_b) p.rsq[M.row_base + ib] = b * s2;
+      }
     }
     return;
   }
@@ -736,7 +755,8 @@ __global__ void __launch_bounds__(kNormThreads) norm_stats_kernel(const __grid_c
       for (int q = 0; q < kNormBatch; ++q)
         w[q] = i0 + 32 * q < M.m ? load_hi8(M, i0 + 32 * q, c0 + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-      for (int q = 0; q < kNormBatch; ++q) add_squares8(w[q], acc);
+      for (int q = 0; q < kNormBatch; ++q)
+        if (i0 + 32 * q < M.m) add_squares8(w[q], acc);
     }
   }
 #pragma unroll
