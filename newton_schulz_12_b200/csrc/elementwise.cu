@@ -685,6 +685,8 @@ __device__ __forceinline__ uint4 load_hi8(const NormMat& M, int i, int c) {
 
 constexpr int kNormBatch = 8;  // 16-byte loads a thread has in flight
 
+// At most 64 registers, so that four blocks (32 warps) share an SM: the pass
+// is bound by the loads each SM keeps in flight.
 __global__ void __launch_bounds__(kNormThreads, 4) norm_stats_kernel(const __grid_constant__ NormStatParams p) {
   __shared__ double red[32][kNormRowsTall + 1];
   int lo = 0, hi = p.nmat - 1;  // last matrix whose first block is <= blockIdx.x
