@@ -134,10 +134,10 @@ def test_normuon_few_steps(steps):
 
 def test_gpt2_small_set_refinements():
     """The GPT-2-small hidden set (72 matrices) with both refinements, two
-    steps; one layer's six matrices and the last layer checked."""
+    steps, every matrix checked."""
     st = State(workloads.gpt2_small_shapes(), normuon=True)
     for step in range(2):
-        check_step_ex(st, step, cautious=True, wd=0.1, check=list(range(6)) + list(range(66, 72)))
+        check_step_ex(st, step, cautious=True, wd=0.1)
 
 
 def test_no_options_is_muon_step():
