@@ -204,8 +204,8 @@ int muon_step(int count, float* const* params, const void* const* grads,
  *     O_i  <- O_i * f_i * g,   g = ||O||_F / ||diag(f) O||_F
  *   so the update keeps its Frobenius norm and only its split over the rows
  *   (neurons) changes; then the apply as in muon_step.  The row sums of O^2
- *   are taken over O rounded to bf16 (each within a factor 1 +- 2^-8 of the
- *   exact sum), in a fixed order (fp32 within a thread, fp64 across
+ *   are taken over O rounded to bf16 (each within a relative 2^-7 + 2^-14 of
+ *   the exact sum), in a fixed order (fp32 within a thread, fp64 across
  *   threads); the factor f_i g is rounded to fp32 and multiplies O in fp32.  This path applies every update in the separate pass.
  *   beta2 in [0, 1].
  * neuron_state == NULL and flags == 0 is exactly muon_step.

@@ -646,9 +646,10 @@ __global__ void __launch_bounds__(kScaleThreads) scale_kernel(const __grid_const
 
 // ------------------------------------------------------- per-neuron rescale
 // Row sums of O^2 over the caller's W rows (NorMuon reading), from the bf16
-// part of O's pair: hi is O rounded to nearest bf16, |O - hi| <= 2^-9 |hi|,
-// so every square, and with it every row sum, is within a factor 1 +- 2^-8
-// of O's (the update itself carries a 3e-2 tolerance).  Reading 2 B per
+// part of O's pair: hi is O rounded to nearest bf16, |O - hi| <= 2^-8 |hi|
+// (half a bf16 unit), so every square, and with it every row sum, is within
+// a relative 2^-7 + 2^-14 of O's (the update itself carries a 3e-2
+// tolerance).  Reading 2 B per
 // element instead of 3, with no residual to decode, keeps the pass at the
 // memory's rate.  O = oscale * pair when oscale is set (zero steps): the
 // sums are then scaled by oscale^2.  W = X: a block takes kNormRowsWide rows
