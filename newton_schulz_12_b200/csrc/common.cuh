@@ -399,6 +399,90 @@ __device__ __forceinline__ void pair_encode8(const float (&v)[8], uint4& hi, uin
   lo = make_uint2(l0, l1);
 }
 
+// Packed pairs of fp32 (f32x2 arithmetic, each lane rounded to nearest as
+// its scalar form would be).
+__device__ __forceinline__ unsigned long long f2(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_sub(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// x' = fl(fl(a x + acc) * s) for eight values of the pair (hi, lo), decoded
+// and updated two at a time with packed fp32 arithmetic: per value the same
+// operations, in the same order, as pair_decode8 then fmaf and *.
+__device__ __forceinline__ void pair_axpy8(const uint4 hi, const uint2 lo, const float* acc, float a, float s,
+                                           float (&x)[8]) {
+  const uint32_t h[4] = {hi.x, hi.y, hi.z, hi.w};
+  const uint32_t l[2] = {lo.x, lo.y};
+  const unsigned long long magic2 = f2(12582912.0f, 12582912.0f), a2 = f2(a, a), s2 = f2(s, s);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t fb0 = h[j] << 16, fb1 = h[j] & 0xFFFF0000u;
+    const int k0 = 2 * j, k1 = 2 * j + 1;
+    const uint32_t sel0 = (k0 & 3) | ((8 | (k0 & 3)) * 0x1110), sel1 = (k1 & 3) | ((8 | (k1 & 3)) * 0x1110);
+    uint32_t q0, q1;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(q0) : "r"(l[k0 >> 2]), "r"(sel0));
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(q1) : "r"(l[k1 >> 2]), "r"(sel1));
+    const unsigned long long qf = f2_sub(f2(__int_as_float(static_cast<int>(q0) + 0x4B400000),
+                                             __int_as_float(static_cast<int>(q1) + 0x4B400000)),
+                                          magic2);
+    const unsigned long long v =
+        f2_fma(qf, f2(lo8_unit(fb0), lo8_unit(fb1)), f2(__uint_as_float(fb0), __uint_as_float(fb1)));
+    f2_split(f2_mul(f2_fma(a2, v, f2(acc[k0], acc[k1])), s2), x[k0], x[k1]);
+  }
+}
+
+// pair_encode8 with its fp32 arithmetic two values at a time (same result).
+__device__ __forceinline__ void pair_encode8_x2(const float (&x)[8], uint4& hi, uint2& lo) {
+  const unsigned long long magic2 = f2(12582912.0f, 12582912.0f);
+  uint32_t hh[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) hh[k] = pack_bf16x2(x[2 * k], x[2 * k + 1]);
+  uint32_t m[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t fb0 = hh[j] << 16, fb1 = hh[j] & 0xFFFF0000u;
+    const unsigned long long d = f2_sub(f2(x[2 * j], x[2 * j + 1]), f2(__uint_as_float(fb0), __uint_as_float(fb1)));
+    float t0, t1;
+    f2_split(f2_mul(d, f2(lo8_inv_unit(fb0), lo8_inv_unit(fb1))), t0, t1);
+    float m0, m1;
+    f2_split(f2_add(f2(fminf(t0, 127.0f), fminf(t1, 127.0f)), magic2), m0, m1);
+    m[2 * j] = __float_as_uint(m0);
+    m[2 * j + 1] = __float_as_uint(m1);
+  }
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) asm("prmt.b32 %0, %1, %2, 0x0040;" : "=r"(w[k]) : "r"(m[2 * k]), "r"(m[2 * k + 1]));
+  uint32_t l0, l1;
+  asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(l0) : "r"(w[0]), "r"(w[1]));
+  asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(l1) : "r"(w[2]), "r"(w[3]));
+  hi = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+  lo = make_uint2(l0, l1);
+}
+
 // Eight values of the pair back to fp32: hi + q * 2^(E - 15).  q is
 // sign-extended from its byte with one byte permute, and turned into a float
 // exactly as the bits of 1.5 * 2^23 + q minus 1.5 * 2^23.

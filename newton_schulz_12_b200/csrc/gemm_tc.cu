@@ -806,9 +806,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                 ld_shared_v4(ha, h4.x, h4.y, h4.z, h4.w);
                 asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(l2.x), "=r"(l2.y) : "r"(la) : "memory");
                 float x[8];
-                pair_decode8(h4, l2, x);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = fmaf(p.a, x[e], v[8 * uu + e]) * xs;
+                pair_axpy8(h4, l2, v + 8 * uu, p.a, xs, x);  // two values per fp32 instruction
                 if (EPI == kBxApply && mode == 1) {
                   // W's row sr, columns VB hf + 8 uu ..: box (VB hf) / 32 (32
                   // fp32 per 128-byte row, 128-byte swizzle), 16-byte units
@@ -841,7 +839,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of<EPI>(), 1
                     asm volatile("st.shared.f32 [%0], %1;" ::"r"(wa), "f"(w) : "memory");
                   }
                 } else {
-                  pair_encode8(x, h4, l2);
+                  pair_encode8_x2(x, h4, l2);
                   st_shared_v4(ha, h4.x, h4.y, h4.z, h4.w);
                   asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(la), "r"(l2.x), "r"(l2.y) : "memory");
                 }
