@@ -186,10 +186,16 @@ int muon_step(int count, float* const* params, const void* const* grads,
 /*
  * muon_step_ex -- muon_step with the later refinements of the same update.
  *
- * Source: "The NanoGPT speedrun", paragraph "Reading guide", names NorMuon's
- * per-neuron rescale and cautious weight decay among the refinements that
- * tune the Muon update; the pages give no formulas, so the library reads them
- * as follows.
+ * Source: "The NanoGPT speedrun", paragraph "Reading guide", names Polar
+ * Express polynomials, NorMuon's per-neuron rescale and cautious weight decay
+ * among the refinements that tune the Muon update; the pages give no
+ * formulas, so the library reads them as follows.
+ *
+ * schedule: NULL for the default triple (3.4445, -4.7750, 2.0315) at every
+ *   step, else a HOST array of 3 * steps floats, (a_t, b_t, c_t) for step
+ *   t = 1 .. steps, as in muon_ns_orthogonalize_schedule (Polar Express
+ *   reading: the same iteration with per-step coefficients).  Every value
+ *   must be finite (else MUON_ERR_ARG).
  *
  * flags & MUON_CAUTIOUS_WD: the decay term fl(lr*wd)*W is applied only to the
  *   elements where W and the update O have the same sign (W*O > 0); elsewhere
@@ -206,15 +212,15 @@ int muon_step(int count, float* const* params, const void* const* grads,
  *   (neurons) changes; then the apply as in muon_step.  The row sums of O^2
  *   are taken over O rounded to bf16 (each within a relative 2^-7 + 2^-14 of
  *   the exact sum), in a fixed order (fp32 within a thread, fp64 across
- *   threads); the factor f_i g is rounded to fp32 and multiplies O in fp32.  This path applies every update in the separate pass.
- *   beta2 in [0, 1].
- * neuron_state == NULL and flags == 0 is exactly muon_step.
+ *   threads); the factor f_i g is rounded to fp32 and multiplies O in fp32.
+ *   This path applies every update in the separate pass.  beta2 in [0, 1].
+ * schedule == NULL, neuron_state == NULL and flags == 0 is exactly muon_step.
  * Returns MUON_OK or a negative muon_status (unknown flag bits: MUON_ERR_ARG).
  */
 int muon_step_ex(int count, float* const* params, const void* const* grads,
                  float* const* momentum_bufs, const int64_t* shapes, float beta, int nesterov,
-                 float lr, float wd, int steps, int flags, float* const* neuron_state, float beta2,
-                 void* stream);
+                 float lr, float wd, int steps, const float* schedule, int flags,
+                 float* const* neuron_state, float beta2, void* stream);
 
 /*
  * muon_momentum -- the momentum stage of muon_step on its own.

@@ -163,14 +163,24 @@ def _step_args(params, grads, momentum_bufs):
 
 
 def muon_step_ex(params, grads, momentum_bufs, beta=0.95, nesterov=True, lr=0.05, wd=0.0, steps=5,
-                 cautious_wd=False, neuron_state=None, beta2=0.95, stream=None):
-    """muon_step with cautious weight decay and / or NorMuon's per-neuron rescale.
+                 cautious_wd=False, neuron_state=None, beta2=0.95, schedule=None, stream=None):
+    """muon_step with per-step coefficients, cautious weight decay and / or
+    NorMuon's per-neuron rescale.
 
+    ``schedule``: None (the default triple at every step) or a sequence of
+    (a, b, c) triples, one per Newton-Schulz step; it then sets the step count.
     ``neuron_state``: None (off) or a list of fp32 CUDA vectors, one per
     matrix with one entry per row of W (zeros before the first step), updated
     in place.
     """
     params, grads, bufs, shapes = _step_args(params, grads, momentum_bufs)
+    table = None
+    if schedule is not None:
+        flat = [float(v) for triple in schedule for v in triple]
+        if len(flat) != 3 * len(schedule):
+            raise ValueError("schedule must be a sequence of (a, b, c) triples")
+        steps = len(schedule)
+        table = (ctypes.c_float * max(1, len(flat)))(*flat)
     state = None
     if neuron_state is not None:
         neuron_state = list(neuron_state)
@@ -184,7 +194,7 @@ def muon_step_ex(params, grads, momentum_bufs, beta=0.95, nesterov=True, lr=0.05
     check(_lib.lib().muon_step_ex(len(params), ptr_array([w.data_ptr() for w in params]),
                                   ptr_array([g.data_ptr() for g in grads]),
                                   ptr_array([m.data_ptr() for m in bufs]), shape_array(shapes),
-                                  beta, int(bool(nesterov)), lr, wd, steps,
+                                  beta, int(bool(nesterov)), lr, wd, steps, table,
                                   MUON_CAUTIOUS_WD if cautious_wd else 0, state, beta2,
                                   _stream(stream)))
 

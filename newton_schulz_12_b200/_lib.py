@@ -42,7 +42,7 @@ SIGNATURES = {
     "muon_ns_orthogonalize_static": (_I, [_I, _I, _I, _PP, _F, _F, _F, _I, _P, _P]),
     "muon_ns_orthogonalize_schedule": (_I, [_I, _I, _I, _PP, ctypes.POINTER(_F), _I, _I, _P]),
     "muon_step": (_I, [_I, _PP, _PP, _PP, _I64P, _F, _I, _F, _F, _I, _P]),
-    "muon_step_ex": (_I, [_I, _PP, _PP, _PP, _I64P, _F, _I, _F, _F, _I, _I, _PP, _F, _P]),
+    "muon_step_ex": (_I, [_I, _PP, _PP, _PP, _I64P, _F, _I, _F, _F, _I, ctypes.POINTER(_F), _I, _PP, _F, _P]),
     "muon_momentum": (_I, [_I, _PP, _PP, _I64P, _F, _I, _P, _P]),
     "muon_apply": (_I, [_I, _PP, _PP, _I64P, _F, _F, _P]),
     "muon_apply_ex": (_I, [_I, _PP, _PP, _I64P, _F, _F, _I, _PP, _P]),

@@ -1128,10 +1128,14 @@ std::vector<float> constant_schedule(float a, float b, float c, int steps);
 // neuron_state is given, the per-neuron rescale of the update (NorMuon
 // reading) with second-moment coefficient beta2.
 int step_impl(int count, float* const* params, const void* const* grads, float* const* momentum_bufs,
-              const int64_t* shapes, float beta, int nesterov, float lr, float wd, int steps, int flags,
-              float* const* neuron_state, float beta2, void* stream) {
+              const int64_t* shapes, float beta, int nesterov, float lr, float wd, int steps,
+              const float* schedule, int flags, float* const* neuron_state, float beta2, void* stream) {
   if (count < 0) return set_err(MUON_ERR_ARG, "count %d < 0", count);
   if (steps < 0 || steps > kMaxStepsArg) return set_err(MUON_ERR_ARG, "steps %d out of range 0..%d", steps, kMaxStepsArg);
+  if (schedule)
+    for (int i = 0; i < 3 * steps; ++i)
+      if (!finite(schedule[i]))
+        return set_err(MUON_ERR_ARG, "coefficient %d of step %d is not finite", i % 3, i / 3);
   if (!finite(beta) || beta < 0.f || beta > 1.f) return set_err(MUON_ERR_ARG, "beta must be in [0, 1]");
   if (!finite(lr) || !finite(wd)) return set_err(MUON_ERR_ARG, "lr and wd must be finite");
   if (flags & ~MUON_CAUTIOUS_WD) return set_err(MUON_ERR_ARG, "unknown flags 0x%x", flags);
@@ -1174,7 +1178,8 @@ int step_impl(int count, float* const* params, const void* const* grads, float* 
 
   std::vector<const void*> gsrc(grads, grads + count);
   std::vector<float*> bufs(momentum_bufs, momentum_bufs + count);
-  const std::vector<float> abc = constant_schedule(kCoefA, kCoefB, kCoefC, steps);
+  const std::vector<float> abc = schedule ? std::vector<float>(schedule, schedule + 3 * steps)
+                                          : constant_schedule(kCoefA, kCoefB, kCoefC, steps);
   std::vector<void*> ys(params, params + count);
   const int cautious = (flags & MUON_CAUTIOUS_WD) ? 1 : 0;
   // the last step applies the update to W in its epilogue where it can; the
@@ -1341,17 +1346,17 @@ int muon_step(int count, float* const* params, const void* const* grads,
               float* const* momentum_bufs, const int64_t* shapes, float beta, int nesterov,
               float lr, float wd, int steps, void* stream) {
   t_err.clear();
-  return step_impl(count, params, grads, momentum_bufs, shapes, beta, nesterov, lr, wd, steps, 0,
-                   nullptr, 0.f, stream);
+  return step_impl(count, params, grads, momentum_bufs, shapes, beta, nesterov, lr, wd, steps, nullptr,
+                   0, nullptr, 0.f, stream);
 }
 
 int muon_step_ex(int count, float* const* params, const void* const* grads,
                  float* const* momentum_bufs, const int64_t* shapes, float beta, int nesterov,
-                 float lr, float wd, int steps, int flags, float* const* neuron_state, float beta2,
-                 void* stream) {
+                 float lr, float wd, int steps, const float* schedule, int flags,
+                 float* const* neuron_state, float beta2, void* stream) {
   t_err.clear();
-  return step_impl(count, params, grads, momentum_bufs, shapes, beta, nesterov, lr, wd, steps, flags,
-                   neuron_state, beta2, stream);
+  return step_impl(count, params, grads, momentum_bufs, shapes, beta, nesterov, lr, wd, steps, schedule,
+                   flags, neuron_state, beta2, stream);
 }
 
 int muon_momentum(int count, const void* const* grads, float* const* momentum_bufs,

@@ -185,16 +185,17 @@ def muon_step(W, grad, buf, beta=0.95, nesterov=True, lr=0.05, wd=0.0,
 
 def muon_step_ex(W, grad, buf, beta=0.95, nesterov=True, lr=0.05, wd=0.0, steps=NS_STEPS,
                  coeffs=NS_COEFFS, eps=NORM_EPS, cautious=False, neuron_state=None,
-                 beta2=NORMUON_BETA2):
+                 beta2=NORMUON_BETA2, schedule=None):
     """``muon_step`` with the refinements of [Overview ¶Reading guide], fp64.
 
-    Momentum -> orthogonalise -> (NorMuon rescale when ``neuron_state`` is
-    given) -> scale and apply (cautious decay when ``cautious``).  Returns
-    (W', buf', O', v') with O' the update applied and v' the new state (None
-    without NorMuon).
+    Momentum -> orthogonalise (per-step triples when ``schedule`` is given,
+    the Polar Express reading of ``newton_schulz``) -> (NorMuon rescale when
+    ``neuron_state`` is given) -> scale and apply (cautious decay when
+    ``cautious``).  Returns (W', buf', O', v') with O' the update applied and
+    v' the new state (None without NorMuon).
     """
     new_buf, u = momentum(grad, buf, beta, nesterov)
-    O = newton_schulz(u, steps, coeffs, eps)
+    O = newton_schulz(u, steps, coeffs, eps, schedule=schedule)
     v_new = None
     if neuron_state is not None:
         O, v_new = normuon_rescale(O, neuron_state, beta2)

@@ -119,13 +119,16 @@ def test_step_argument_errors(lib):
     assert lib.muon_momentum(1, p, p, shapes, -0.1, 1, None, null) == -1
     assert lib.muon_apply(1, p, None, shapes, 0.1, 0.0, null) == -1
     # the extended step and apply: unknown option bits, beta2, state pointers
-    assert lib.muon_step_ex(1, p, p, p, shapes, 0.9, 1, 0.1, 0.0, 5, 2, None, 0.95, null) == -1
+    assert lib.muon_step_ex(1, p, p, p, shapes, 0.9, 1, 0.1, 0.0, 5, None, 2, None, 0.95, null) == -1
     assert "flags" in _err(lib)
-    assert lib.muon_step_ex(1, p, p, p, shapes, 0.9, 1, 0.1, 0.0, 5, 1, p, 1.5, null) == -1
+    assert lib.muon_step_ex(1, p, p, p, shapes, 0.9, 1, 0.1, 0.0, 5, None, 1, p, 1.5, null) == -1
     assert "beta2" in _err(lib)
-    assert lib.muon_step_ex(1, p, p, p, shapes, 0.9, 1, 0.1, 0.0, 5, 0, _lib.ptr_array([0]), 0.95, null) == -1
+    assert lib.muon_step_ex(1, p, p, p, shapes, 0.9, 1, 0.1, 0.0, 5, None, 0, _lib.ptr_array([0]), 0.95, null) == -1
     assert "neuron_state[0]" in _err(lib)
-    assert lib.muon_step_ex(0, None, None, None, None, 0.9, 1, 0.1, 0.0, 5, 1, None, 0.95, null) == 0
+    assert lib.muon_step_ex(0, None, None, None, None, 0.9, 1, 0.1, 0.0, 5, None, 1, None, 0.95, null) == 0
+    sched = (ctypes.c_float * 15)(*([1.5, -0.5, 0.0] * 4 + [1.5, float("nan"), 0.0]))
+    assert lib.muon_step_ex(1, p, p, p, shapes, 0.9, 1, 0.1, 0.0, 5, sched, 0, None, 0.95, null) == -1
+    assert "coefficient 1 of step 4" in _err(lib)
     assert lib.muon_apply_ex(1, p, p, shapes, 0.1, 0.0, 8, None, null) == -1
     assert lib.muon_apply_ex(1, p, p, shapes, 0.1, 0.0, 1, _lib.ptr_array([0x1002]), null) == -1
     assert "row_scale[0]" in _err(lib)

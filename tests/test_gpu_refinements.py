@@ -1,4 +1,5 @@
-"""Cautious weight decay and NorMuon's per-neuron rescale on the GPU.
+"""Cautious weight decay, NorMuon's per-neuron rescale and per-step
+coefficients in the full step on the GPU.
 
 The pages name both refinements of the Muon update without formulas ("The
 NanoGPT speedrun", paragraph "Reading guide"); the readings are those of
@@ -76,13 +77,15 @@ class State:
         self.V = [torch.zeros(r, device="cuda") for r, _ in shapes] if normuon else None
 
 
-def check_step_ex(st, step, cautious, beta2=0.95, lr=0.05, wd=0.0, steps=5, check=None):
+def check_step_ex(st, step, cautious, beta2=0.95, lr=0.05, wd=0.0, steps=5, check=None, schedule=None):
     _, Gs = workloads.muon_set(st.shapes, step=step)
     W0 = [w.cpu().numpy() for w in st.W]
     M0 = [m.cpu().numpy() for m in st.M]
     V0 = [v.cpu().numpy() for v in st.V] if st.V is not None else None
     nsb.muon_step_ex(st.W, [g.cuda() for g in Gs], st.M, lr=lr, wd=wd, steps=steps,
-                     cautious_wd=cautious, neuron_state=st.V, beta2=beta2)
+                     cautious_wd=cautious, neuron_state=st.V, beta2=beta2, schedule=schedule)
+    if schedule is not None:  # the triples as the library received them (fp32)
+        schedule = [tuple(float(np.float32(v)) for v in t) for t in schedule]
     assert nsb.muon_get_status() == 0
     for i in (range(len(st.shapes)) if check is None else check):
         g32 = Gs[i].float().numpy()
@@ -91,7 +94,7 @@ def check_step_ex(st, step, cautious, beta2=0.95, lr=0.05, wd=0.0, steps=5, chec
         Wn, _, _, vn = oracle.muon_step_ex(
             W0[i], g32, M0[i], beta=np.float32(0.95), lr=np.float32(lr), wd=np.float32(wd),
             steps=steps, cautious=cautious, neuron_state=None if V0 is None else V0[i],
-            beta2=np.float32(beta2))
+            beta2=np.float32(beta2), schedule=schedule)
         dW_ref = Wn - W0[i]
         dW = st.W[i].cpu().numpy().astype(np.float64) - W0[i]
         err = rel_fro(dW, dW_ref)
@@ -131,6 +134,36 @@ def test_normuon_few_steps(steps):
     """steps = 0: O is the normalised update itself (the scaled pair)."""
     st = State(MIX[:4], normuon=True)
     check_step_ex(st, 0, cautious=False, steps=steps)
+
+
+# Per-step coefficients in the full step (the Polar Express reading: the
+# pages print no coefficients, so the triples are the speedrun quintic, the
+# flat quintic 15/8, -10/8, 3/8 and the classic cubic).
+QUINTIC = (3.4445, -4.7750, 2.0315)
+SCHEDULE = [QUINTIC, QUINTIC, (15 / 8, -10 / 8, 3 / 8), (1.5, -0.5, 0.0), (15 / 8, -10 / 8, 3 / 8)]
+
+
+def test_schedule_step_mixed_shapes():
+    """muon_step_ex with a schedule, alone and with both refinements, two
+    steps, against the oracle step with the same triples."""
+    st = State(MIX, normuon=False)
+    for step in range(2):
+        check_step_ex(st, step, cautious=False, wd=0.1, schedule=SCHEDULE)
+    st = State(MIX[:5], normuon=True)
+    for step in range(2):
+        check_step_ex(st, step, cautious=True, wd=0.5, schedule=SCHEDULE[:4])
+
+
+def test_default_schedule_is_muon_step():
+    """The default triple at every step gives muon_step's bits (weights and momentum)."""
+    shapes = MIX + workloads.gpt2_small_shapes()[:6]
+    a, b = State(shapes, normuon=False), State(shapes, normuon=False)
+    _, Gs = workloads.muon_set(shapes, step=0)
+    nsb.muon_step(a.W, [g.cuda() for g in Gs], a.M, wd=0.1)
+    nsb.muon_step_ex(b.W, [g.cuda() for g in Gs], b.M, wd=0.1, schedule=[QUINTIC] * 5)
+    assert nsb.muon_get_status() == 0
+    for i in range(len(shapes)):
+        assert torch.equal(a.W[i], b.W[i]) and torch.equal(a.M[i], b.M[i]), shapes[i]
 
 
 def test_gpt2_small_set_refinements():

@@ -183,6 +183,28 @@ def test_step_ex_composes_the_refinements():
     assert all(np.array_equal(x, y) for x, y in zip(a[:3], b)) and a[3] is None
 
 
+def test_step_ex_schedule_is_the_ns_schedule():
+    """A schedule only changes the orthogonalisation: the step with it is
+    momentum -> newton_schulz(schedule) -> apply, and the default triple at
+    every step is the plain step."""
+    rng = np.random.default_rng(12)
+    W = rng.standard_normal((10, 18)) * 0.02
+    g = rng.standard_normal((10, 18)) * 0.01
+    buf = rng.standard_normal((10, 18)) * 0.01
+    sched = [(3.4445, -4.7750, 2.0315), (15 / 8, -10 / 8, 3 / 8), (1.5, -0.5, 0.0)]
+    W2, nb, O2, _ = muon.muon_step_ex(W, g, buf, lr=0.1, wd=0.2, schedule=sched)
+    _, u = muon.momentum(g, buf, 0.95, True)
+    O = muon.newton_schulz(u, schedule=sched)
+    assert np.array_equal(O2, O)
+    assert np.array_equal(W2, muon.apply_update(W, O, 0.1, 0.2, muon.update_scale(10, 18)))
+    a = muon.muon_step_ex(W, g, buf, lr=0.1, wd=0.2, schedule=[muon.NS_COEFFS] * muon.NS_STEPS)
+    b = muon.muon_step_ex(W, g, buf, lr=0.1, wd=0.2)
+    assert all(np.array_equal(x, y) for x, y in zip(a[:3], b[:3]))
+    # and the order of the triples matters (the cubic first differs)
+    c = muon.muon_step_ex(W, g, buf, lr=0.1, wd=0.2, schedule=sched[::-1])
+    assert not np.allclose(c[2], O2, rtol=0, atol=1e-6)
+
+
 def _mut_per_column(O, v, b2, eps):
     """statistics per column instead of per row (the wrong neuron axis)"""
     return muon.normuon_rescale(O.T, np.resize(v, O.shape[1]), b2, eps)[0].T
