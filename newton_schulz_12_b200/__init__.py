@@ -238,11 +238,13 @@ class MuonStepPlan(_Replayable):
     Checks dtypes, shapes and contiguity at construction; each call then passes
     the cached pointer arrays straight to the C ABI.  The tensors must stay
     alive and keep their storage while the plan is used.  ``capture`` records a
-    step in a CUDA graph and ``replay`` runs it (one step per replay).
+    step in a CUDA graph and ``replay`` runs it (one step per replay).  With
+    any of ``cautious_wd``, ``neuron_state`` or ``schedule`` the calls go to
+    muon_step_ex (options as there; a schedule fixes the step count).
     """
 
     def __init__(self, params, grads, momentum_bufs, beta=0.95, nesterov=True, lr=0.05, wd=0.0,
-                 steps=5):
+                 steps=5, cautious_wd=False, neuron_state=None, beta2=0.95, schedule=None):
         self.params, self.grads, self.bufs = list(params), list(grads), list(momentum_bufs)
         if not (len(self.params) == len(self.grads) == len(self.bufs)):
             raise ValueError("params, grads and momentum_bufs must have the same length")
@@ -259,11 +261,35 @@ class MuonStepPlan(_Replayable):
         self._g = ptr_array([g.data_ptr() for g in self.grads])
         self._m = ptr_array([m.data_ptr() for m in self.bufs])
         self._s = shape_array(shapes)
+        # the refinements (muon_step_ex): per-step triples, cautious decay, NorMuon state
+        self._table = None
+        if schedule is not None:
+            flat = [float(v) for triple in schedule for v in triple]
+            if len(flat) != 3 * len(schedule):
+                raise ValueError("schedule must be a sequence of (a, b, c) triples")
+            steps = len(schedule)
+            self._table = (ctypes.c_float * max(1, len(flat)))(*flat)
+        self._state = None
+        if neuron_state is not None:
+            self.neuron_state = list(neuron_state)
+            if len(self.neuron_state) != len(self.params):
+                raise ValueError("one neuron_state vector per matrix is required")
+            for i, (v, (r, _)) in enumerate(zip(self.neuron_state, shapes)):
+                _check_cuda(v, f"neuron_state[{i}]", torch.float32)
+                if v.numel() != r:
+                    raise ValueError(f"neuron_state[{i}] must hold {r} values (one per row of W)")
+            self._state = ptr_array([v.data_ptr() for v in self.neuron_state])
+        self._ex = (MUON_CAUTIOUS_WD if cautious_wd else 0, float(beta2))
         self._hyper = (float(beta), int(bool(nesterov)), float(lr), float(wd), int(steps))
         self._fn = _lib.lib().muon_step
+        self._fn_ex = None
+        if self._table is not None or self._state is not None or cautious_wd:
+            self._fn_ex = _lib.lib().muon_step_ex
 
     def update(self, beta=None, nesterov=None, lr=None, wd=None, steps=None):
         """Change hyper-parameters for the following calls (None keeps a value)."""
+        if steps is not None and self._table is not None and int(steps) != self._hyper[4]:
+            raise ValueError("the step count is fixed by the plan's schedule")
         old = self._hyper
         self._hyper = (float(old[0] if beta is None else beta),
                        int(bool(old[1] if nesterov is None else nesterov)),
@@ -272,6 +298,11 @@ class MuonStepPlan(_Replayable):
 
     def __call__(self, stream=None):
         beta, nest, lr, wd, steps = self._hyper
+        if self._fn_ex is not None:
+            flags, beta2 = self._ex
+            check(self._fn_ex(len(self.params), self._p, self._g, self._m, self._s, beta, nest, lr,
+                              wd, steps, self._table, flags, self._state, beta2, _stream(stream)))
+            return
         check(self._fn(len(self.params), self._p, self._g, self._m, self._s, beta, nest, lr, wd,
                        steps, _stream(stream)))
 

@@ -69,10 +69,19 @@ class ShardedMuon:
     ``muon_step`` (bf16 gradients on the CUDA device), prepared once per
     bucket.  Without an initialised process group the object runs as a
     single rank.
+
+    The refinements of ``muon_step_ex`` ("The NanoGPT speedrun", paragraph
+    "Reading guide"): ``cautious_wd``, ``normuon`` (NorMuon's per-neuron
+    state, one fp32 vector per owned matrix in ``neuron_state``, kept by the
+    owner like the momentum; ``beta2``) and ``schedule`` (one (a, b, c) per
+    Newton-Schulz step; it sets ``steps``).  With any of them on, a custom
+    ``local_step`` also receives the keywords ``cautious_wd``,
+    ``neuron_state``, ``beta2`` and ``schedule``.
     """
 
     def __init__(self, shapes, *, device=None, group=None, buckets=2, beta=0.95, nesterov=True,
-                 lr=0.05, wd=0.0, steps=5, grad_dtype=torch.bfloat16, local_step=None):
+                 lr=0.05, wd=0.0, steps=5, grad_dtype=torch.bfloat16, local_step=None,
+                 cautious_wd=False, normuon=False, beta2=0.95, schedule=None):
         import torch.distributed as dist
         for i, shp in enumerate(shapes):
             if len(shp) != 2 or int(shp[0]) < 1 or int(shp[1]) < 1:
@@ -86,6 +95,14 @@ class ShardedMuon:
         self.world = self.dist.get_world_size(group) if self.dist else 1
         self.rank = self.dist.get_rank(group) if self.dist else 0
         self.shapes = [(int(r), int(c)) for r, c in shapes]
+        if schedule is not None:
+            schedule = [tuple(float(v) for v in t) for t in schedule]
+            if any(len(t) != 3 for t in schedule):
+                raise ValueError("schedule must be a sequence of (a, b, c) triples")
+            steps = len(schedule)
+        self.options = None
+        if cautious_wd or normuon or schedule is not None:
+            self.options = dict(cautious_wd=bool(cautious_wd), beta2=float(beta2), schedule=schedule)
         self.hyper = (float(beta), bool(nesterov), float(lr), float(wd), int(steps))
         self.device = dev
         self.owner, self.bucket_ranges = plan_ownership(self.shapes, self.world, buckets, steps)
@@ -94,6 +111,7 @@ class ShardedMuon:
         self.params = [None] * len(self.shapes)
         self.grads = [None] * len(self.shapes)
         self.momentum = [None] * len(self.shapes)
+        self.neuron_state = [None] * len(self.shapes)
         self._buckets = []
         for lo, hi in self.bucket_ranges:
             offs, used = {}, [0] * self.world
@@ -112,6 +130,8 @@ class ShardedMuon:
                 self.grads[i] = G[a:a + rows * cols].view(rows, cols)
                 if r == self.rank:
                     self.momentum[i] = torch.zeros(rows, cols, dtype=torch.float32, device=self.device)
+                    if normuon:
+                        self.neuron_state[i] = torch.zeros(rows, dtype=torch.float32, device=self.device)
                     owned.append(i)
             self._buckets.append({"W": W, "G": G, "slot": slot, "owned": owned, "plan": None})
 
@@ -119,12 +139,23 @@ class ShardedMuon:
         if local_step is None:
             from . import MuonStepPlan
             beta_, nest_, lr_, wd_, steps_ = self.hyper
+            opts = self._local_options
             for bk in self._buckets:
                 if bk["owned"]:
                     bk["plan"] = MuonStepPlan([self.params[i] for i in bk["owned"]],
                                               [self.grads[i] for i in bk["owned"]],
                                               [self.momentum[i] for i in bk["owned"]],
-                                              beta=beta_, nesterov=nest_, lr=lr_, wd=wd_, steps=steps_)
+                                              beta=beta_, nesterov=nest_, lr=lr_, wd=wd_, steps=steps_,
+                                              **opts(bk["owned"]))
+
+    def _local_options(self, owned):
+        """Keywords of the local step for the matrices ``owned`` (none with no refinement on)."""
+        if self.options is None:
+            return {}
+        state = None
+        if self.neuron_state[owned[0]] is not None:
+            state = [self.neuron_state[i] for i in owned]
+        return dict(self.options, neuron_state=state)
 
     # ------------------------------------------------------------ collectives
     def _mine(self, flat, slot):
@@ -184,7 +215,8 @@ class ShardedMuon:
                 else:
                     own = bk["owned"]
                     self._local_step([self.params[i] for i in own], [self.grads[i] for i in own],
-                                     [self.momentum[i] for i in own], beta, nest, lr, wd, steps)
+                                     [self.momentum[i] for i in own], beta, nest, lr, wd, steps,
+                                     **self._local_options(own))
             work = self._all_gather(bk["W"], bk["slot"])
             if work is not None:
                 pending.append(work)

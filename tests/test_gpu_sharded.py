@@ -64,3 +64,38 @@ def test_one_nccl_rank_reproduces_muon_step():
                 assert err <= 3e-2, (i, err)
     finally:
         dist.destroy_process_group()
+
+
+def test_one_nccl_rank_with_refinements_reproduces_muon_step_ex():
+    """Cautious decay, NorMuon (state kept by the owner) and a per-step
+    schedule through the sharded object: bit for bit muon_step_ex on the same
+    inputs, weights, momentum and state."""
+    import torch.distributed as dist
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        shapes = workloads.gpt2_small_shapes(layers=1) + [(300, 1000), (77, 5)]
+        sched = [(3.4445, -4.7750, 2.0315)] * 3 + [(15 / 8, -10 / 8, 3 / 8), (1.5, -0.5, 0.0)]
+        Ws, _ = workloads.muon_set(shapes, step=0)
+        sm = ShardedMuon(shapes, device="cuda", buckets=2, lr=0.05, wd=0.3, cautious_wd=True,
+                         normuon=True, beta2=0.9, schedule=sched)
+        for i in range(len(shapes)):
+            sm.params[i].copy_(Ws[i])
+        W_ref = [w.cuda() for w in Ws]
+        M_ref = [torch.zeros_like(w) for w in W_ref]
+        V_ref = [torch.zeros(w.shape[0], device="cuda") for w in W_ref]
+        for step in range(2):
+            _, Gs = workloads.muon_set(shapes, step=step)
+            for i in range(len(shapes)):
+                sm.grads[i].copy_(Gs[i])
+            sm.step()
+            nsb.muon_step_ex(W_ref, [g.cuda() for g in Gs], M_ref, lr=0.05, wd=0.3, cautious_wd=True,
+                             neuron_state=V_ref, beta2=0.9, schedule=sched)
+            torch.cuda.synchronize()
+            assert nsb.muon_get_status() == 0
+            for i in range(len(shapes)):
+                assert torch.equal(sm.params[i], W_ref[i]), (step, i)
+                assert torch.equal(sm.momentum[i], M_ref[i]), (step, i)
+                assert torch.equal(sm.neuron_state[i], V_ref[i]), (step, i)
+    finally:
+        dist.destroy_process_group()

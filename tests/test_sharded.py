@@ -33,6 +33,21 @@ def oracle_local_step(params, grads, bufs, beta, nesterov, lr, wd, steps):
         M.copy_(torch.from_numpy(Mn).float())
 
 
+def oracle_local_step_ex(params, grads, bufs, beta, nesterov, lr, wd, steps, cautious_wd=False,
+                         neuron_state=None, beta2=0.95, schedule=None):
+    """The oracle's step with the refinements; the NorMuon state updated in place."""
+    for k, (W, G, M) in enumerate(zip(params, grads, bufs)):
+        v = None if neuron_state is None else neuron_state[k].double().numpy()
+        Wn, Mn, _, vn = oracle.muon_step_ex(W.double().numpy(), G.double().numpy(), M.double().numpy(),
+                                            beta=beta, nesterov=nesterov, lr=lr, wd=wd, steps=steps,
+                                            cautious=cautious_wd, neuron_state=v, beta2=beta2,
+                                            schedule=schedule)
+        W.copy_(torch.from_numpy(Wn).float())
+        M.copy_(torch.from_numpy(Mn).float())
+        if neuron_state is not None:
+            neuron_state[k].copy_(torch.from_numpy(vn).float())
+
+
 def initial_w(i, shape):
     g = torch.Generator().manual_seed(2000 + i)
     return torch.randn(shape, generator=g) * 0.02
@@ -196,6 +211,80 @@ def test_two_gloo_ranks_equal_the_single_process_step(buckets):
         assert sorted(moms) == [i for i in range(len(SHAPES)) if owner[i] == rank]
         for i, m in moms.items():
             np.testing.assert_array_equal(m, M_ref[i].astype(np.float32))
+
+
+# ------------------------------------- two gloo ranks with the refinements on
+REFINE = dict(cautious_wd=True, normuon=True, beta2=0.9,
+              schedule=[(3.4445, -4.7750, 2.0315)] * 3 + [(15 / 8, -10 / 8, 3 / 8), (1.5, -0.5, 0.0)])
+HYPER_R = dict(HYPER, wd=0.3)
+del HYPER_R["steps"]
+
+
+def _worker_refined(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from newton_schulz_12_b200.sharded import ShardedMuon
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        sm = ShardedMuon(SHAPES, buckets=2, grad_dtype=torch.float32,
+                         local_step=oracle_local_step_ex, **HYPER_R, **REFINE)
+        for i, s in enumerate(SHAPES):
+            sm.params[i].copy_(initial_w(i, s))
+        for step in range(2):
+            for i, s in enumerate(SHAPES):
+                sm.grads[i].copy_(rank_grad(i, s, rank, step))
+            sm.step()
+        out.put((rank, [p.clone().numpy() for p in sm.params],
+                 {i: v.clone().numpy() for i, v in enumerate(sm.neuron_state) if v is not None}))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_with_refinements_equal_the_single_process_step():
+    """Cautious decay, NorMuon's state (kept by the owner) and a per-step
+    schedule: the group step equals the single-process step_ex on the
+    averaged gradients, state included."""
+    res = _run_ranks(2, _worker_refined)
+    W = [initial_w(i, s).double().numpy() for i, s in enumerate(SHAPES)]
+    M = [np.zeros(s) for s in SHAPES]
+    V = [np.zeros(s[0]) for s in SHAPES]
+    for step in range(2):
+        for i, s in enumerate(SHAPES):
+            g = (rank_grad(i, s, 0, step) + rank_grad(i, s, 1, step)) / 2
+            Wn, Mn, _, vn = oracle.muon_step_ex(W[i], g.double().numpy(), M[i], **HYPER_R,
+                                                cautious=True, neuron_state=V[i], beta2=0.9,
+                                                schedule=REFINE["schedule"])
+            W[i] = Wn.astype(np.float32).astype(np.float64)
+            M[i] = Mn.astype(np.float32).astype(np.float64)
+            V[i] = vn.astype(np.float32).astype(np.float64)
+    owner, _ = plan_ownership(SHAPES, 2, 2, steps=5)
+    for rank, params, states in res:
+        for i in range(len(SHAPES)):
+            np.testing.assert_array_equal(params[i], W[i].astype(np.float32),
+                                          err_msg=f"rank {rank} matrix {i}")
+        assert sorted(states) == [i for i in range(len(SHAPES)) if owner[i] == rank]
+        for i, v in states.items():
+            np.testing.assert_array_equal(v, V[i].astype(np.float32))
+
+
+def test_refinement_options_reach_the_local_step():
+    from newton_schulz_12_b200.sharded import ShardedMuon
+    seen = []
+
+    def record(params, grads, bufs, beta, nesterov, lr, wd, steps, **kw):
+        seen.append((steps, kw))
+
+    ShardedMuon(SHAPES[:2], buckets=1, grad_dtype=torch.float32, local_step=record, **HYPER).step()
+    assert seen == [(5, {})]  # nothing on: the plain call
+    seen.clear()
+    sm = ShardedMuon(SHAPES[:2], buckets=1, grad_dtype=torch.float32, local_step=record,
+                     **HYPER_R, **REFINE)
+    sm.step()
+    steps, kw = seen[0]
+    assert steps == 5 and kw["cautious_wd"] and kw["beta2"] == 0.9
+    assert kw["schedule"] == [tuple(float(v) for v in t) for t in REFINE["schedule"]]
+    assert [tuple(v.shape) for v in kw["neuron_state"]] == [(16,), (24,)]
 
 
 # ------------------------------------------- three ranks, one idle in a bucket
