@@ -222,3 +222,42 @@ class ShardedMuon:
                 pending.append(work)
         for work in pending:
             work.wait()
+
+    # ------------------------------------------------------------ checkpoint
+    def state_dict(self):
+        """This rank's optimizer state: the current hyper-parameters and, for
+        every matrix it owns, its momentum buffer (and NorMuon state), keyed by
+        matrix index.  The weights are ``params`` (every rank holds them all)."""
+        own = [i for i, m in enumerate(self.momentum) if m is not None]
+        out = {"hyper": self.hyper, "shapes": list(self.shapes),
+               "momentum": {i: self.momentum[i].detach().clone() for i in own}}
+        if any(v is not None for v in self.neuron_state):
+            out["neuron_state"] = {i: self.neuron_state[i].detach().clone() for i in own}
+        return out
+
+    def load_state_dict(self, state):
+        """Restore from ``state_dict()``, or from several ranks' dicts merged
+        (their ``momentum`` / ``neuron_state`` maps joined): the saving group
+        may have had another size or ownership, as long as every matrix this
+        rank owns is present.  Every rank calls it before its next step."""
+        if [tuple(s) for s in state["shapes"]] != self.shapes:
+            raise ValueError("the state is for another set of matrix shapes")
+        if tuple(state["hyper"])[4] != self.hyper[4]:
+            raise ValueError("the state is for another Newton-Schulz step count")
+        b_, n_, lr_, wd_, st_ = (float(state["hyper"][0]), bool(state["hyper"][1]),
+                                 float(state["hyper"][2]), float(state["hyper"][3]), int(state["hyper"][4]))
+        has_state = any(v is not None for v in self.neuron_state)
+        if has_state != ("neuron_state" in state):
+            raise ValueError("NorMuon state present in one of the optimizer and the checkpoint only")
+        for i, m in enumerate(self.momentum):
+            if m is None:
+                continue
+            if i not in state["momentum"]:
+                raise ValueError(f"matrix {i} is owned by this rank but missing from the state")
+            m.copy_(state["momentum"][i])
+            if has_state:
+                self.neuron_state[i].copy_(state["neuron_state"][i])
+        self.hyper = (b_, n_, lr_, wd_, st_)
+        for bk in self._buckets:
+            if bk["plan"] is not None:
+                bk["plan"].update(beta=b_, nesterov=n_, lr=lr_, wd=wd_)

@@ -287,6 +287,89 @@ def test_refinement_options_reach_the_local_step():
     assert [tuple(v.shape) for v in kw["neuron_state"]] == [(16,), (24,)]
 
 
+# ------------------------------------------------------- checkpoint / resume
+def _worker_ckpt(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from newton_schulz_12_b200.sharded import ShardedMuon
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        sm = ShardedMuon(SHAPES, buckets=2, grad_dtype=torch.float32,
+                         local_step=oracle_local_step_ex, **HYPER_R, **REFINE)
+        for i, s in enumerate(SHAPES):
+            sm.params[i].copy_(initial_w(i, s))
+        for step in range(2):
+            for i, s in enumerate(SHAPES):
+                sm.grads[i].copy_(rank_grad(i, s, rank, step))
+            sm.step(lr=0.04 if step == 1 else None)
+        st = sm.state_dict()  # tensors leave the process as arrays
+        st = dict(st, momentum={i: t.numpy() for i, t in st["momentum"].items()},
+                  neuron_state={i: t.numpy() for i, t in st["neuron_state"].items()})
+        out.put((rank, [p.clone().numpy() for p in sm.params], st))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_checkpoint_from_two_ranks_resumes_on_one():
+    """Two gloo ranks take two steps (the second with a new lr) and save;
+    their states, merged, resume on a single rank: the third step equals
+    three uninterrupted single-process steps on the averaged gradients, bit
+    for bit (weights, momentum, NorMuon state)."""
+    from newton_schulz_12_b200.sharded import ShardedMuon
+    res = _run_ranks(2, _worker_ckpt)
+    merged = {"momentum": {}, "neuron_state": {}}
+    for _, _, st in res:
+        merged["hyper"], merged["shapes"] = st["hyper"], st["shapes"]
+        merged["momentum"].update({i: torch.from_numpy(a) for i, a in st["momentum"].items()})
+        merged["neuron_state"].update({i: torch.from_numpy(a) for i, a in st["neuron_state"].items()})
+    assert sorted(merged["momentum"]) == list(range(len(SHAPES)))
+    sm = ShardedMuon(SHAPES, buckets=3, grad_dtype=torch.float32, local_step=oracle_local_step_ex,
+                     **HYPER_R, **REFINE)
+    sm.load_state_dict(merged)
+    assert sm.hyper[2] == 0.04
+    for i, p in enumerate(res[0][1]):
+        sm.params[i].copy_(torch.from_numpy(p))
+    for i, s in enumerate(SHAPES):
+        sm.grads[i].copy_((rank_grad(i, s, 0, 2) + rank_grad(i, s, 1, 2)) / 2)
+    sm.step()
+    W = [initial_w(i, s).double().numpy() for i, s in enumerate(SHAPES)]
+    M = [np.zeros(s) for s in SHAPES]
+    V = [np.zeros(s[0]) for s in SHAPES]
+    for step in range(3):
+        hyper = dict(HYPER_R, lr=0.05 if step == 0 else 0.04)
+        for i, s in enumerate(SHAPES):
+            g = (rank_grad(i, s, 0, step) + rank_grad(i, s, 1, step)) / 2
+            Wn, Mn, _, vn = oracle.muon_step_ex(W[i], g.double().numpy(), M[i], **hyper, cautious=True,
+                                                neuron_state=V[i], beta2=0.9,
+                                                schedule=REFINE["schedule"])
+            W[i] = Wn.astype(np.float32).astype(np.float64)
+            M[i] = Mn.astype(np.float32).astype(np.float64)
+            V[i] = vn.astype(np.float32).astype(np.float64)
+    for i in range(len(SHAPES)):
+        np.testing.assert_array_equal(sm.params[i].numpy(), W[i].astype(np.float32))
+        np.testing.assert_array_equal(sm.momentum[i].numpy(), M[i].astype(np.float32))
+        np.testing.assert_array_equal(sm.neuron_state[i].numpy(), V[i].astype(np.float32))
+
+
+def test_load_state_dict_checks():
+    from newton_schulz_12_b200.sharded import ShardedMuon
+    sm = ShardedMuon(SHAPES[:3], buckets=1, grad_dtype=torch.float32, local_step=oracle_local_step,
+                     **HYPER)
+    st = sm.state_dict()
+    assert sorted(st["momentum"]) == [0, 1, 2] and "neuron_state" not in st
+    with pytest.raises(ValueError, match="shapes"):
+        ShardedMuon(SHAPES[:2], buckets=1, grad_dtype=torch.float32,
+                    local_step=oracle_local_step, **HYPER).load_state_dict(st)
+    partial = dict(st, momentum={0: st["momentum"][0]})
+    with pytest.raises(ValueError, match="missing"):
+        sm.load_state_dict(partial)
+    refined = ShardedMuon(SHAPES[:3], buckets=1, grad_dtype=torch.float32,
+                          local_step=oracle_local_step_ex, normuon=True, **HYPER)
+    with pytest.raises(ValueError, match="NorMuon"):
+        refined.load_state_dict(st)
+
+
 # ------------------------------------------- three ranks, one idle in a bucket
 SHAPES3 = [(16, 24), (24, 16), (32, 32), (8, 40)]
 
