@@ -14,6 +14,7 @@ import numpy as np
 import pytest
 import torch
 import torch.multiprocessing as mp
+from hypothesis import given, settings, strategies as st
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
@@ -80,6 +81,29 @@ def test_every_matrix_has_one_owner_and_buckets_are_balanced(world, buckets):
         # greedy longest-first: no rank exceeds the mean by more than one item
         assert max(load) <= sum(load) / world + biggest
     assert plan_ownership(shapes, world, buckets) == (owner, ranges)  # deterministic
+
+
+@settings(max_examples=200, deadline=None)
+@given(shapes=st.lists(st.tuples(st.integers(1, 4096), st.integers(1, 4096)), min_size=0, max_size=40),
+       world=st.integers(1, 9), buckets=st.integers(1, 6), steps=st.integers(0, 7))
+def test_ownership_properties(shapes, world, buckets, steps):
+    """Any shapes, group size and bucket count: one owner per matrix, buckets
+    tile the list in order, every bucket within one item of its mean load."""
+    owner, ranges = plan_ownership(shapes, world, buckets, steps)
+    assert len(owner) == len(shapes) and all(0 <= r < world for r in owner)
+    if not shapes:
+        assert ranges == [(0, 0)] or ranges == []
+        return
+    assert ranges[0][0] == 0 and ranges[-1][1] == len(shapes)
+    assert all(a[1] == b[0] and a[0] < a[1] for a, b in zip(ranges, ranges[1:]))
+    assert len(ranges) == min(buckets, len(shapes))
+    for lo, hi in ranges:
+        load = [0] * world
+        for i in range(lo, hi):
+            load[owner[i]] += ns_flops(shapes[i], steps)
+        biggest = max(ns_flops(shapes[i], steps) for i in range(lo, hi))
+        assert max(load) <= sum(load) / world + biggest
+    assert plan_ownership(shapes, world, buckets, steps) == (owner, ranges)
 
 
 def test_longest_first_on_a_small_case():
