@@ -218,7 +218,8 @@ def _mut_no_renorm(O, v, b2, eps):
 def _mut_swapped_ema(O, v, b2, eps):
     """the moving average with its two weights swapped"""
     v_bad = (1 - b2) * v + b2 * np.mean(O * O, axis=1)
-    DO = O / np.sqrt(v_bad + eps)[:, None]
+    with np.errstate(divide="ignore", invalid="ignore"):  # a mutant may divide by zero
+        DO = O / np.sqrt(v_bad + eps)[:, None]
     return np.linalg.norm(O) / np.linalg.norm(DO) * DO
 
 
