@@ -57,3 +57,29 @@ def test_ns_plan_and_its_replay_equal_direct_calls(m, n, batch):
     torch.cuda.synchronize()
     assert nsb.muon_get_status() == 0
     assert all(torch.equal(x, y) for x, y in zip(c, b))
+
+
+def test_refined_plan_replay_equals_muon_step_ex():
+    """MuonStepPlan with the refinements (cautious decay, NorMuon state, a
+    per-step schedule) calls muon_step_ex; recorded and replayed it gives the
+    bits of direct muon_step_ex calls, weights, momentum and state."""
+    shapes = workloads.gpt2_small_shapes(layers=1) + [(130, 68), (77, 5)]
+    sched = [(3.4445, -4.7750, 2.0315)] * 4 + [(1.5, -0.5, 0.0)]
+    Wa, Ga, Ma = _set(shapes)
+    Wb, Gb, Mb = [w.clone() for w in Wa], [g.clone() for g in Ga], [m.clone() for m in Ma]
+    Va = [torch.zeros(w.shape[0], device="cuda") for w in Wa]
+    Vb = [v.clone() for v in Va]
+    plan = nsb.MuonStepPlan(Wa, Ga, Ma, wd=0.2, cautious_wd=True, neuron_state=Va, beta2=0.9,
+                            schedule=sched)
+    plan.capture()
+    for _ in range(2):
+        plan.replay()
+    for _ in range(3):
+        nsb.muon_step_ex(Wb, Gb, Mb, wd=0.2, cautious_wd=True, neuron_state=Vb, beta2=0.9,
+                         schedule=sched)
+    torch.cuda.synchronize()
+    assert nsb.muon_get_status() == 0
+    for x, y in zip(Wa + Ma + Va, Wb + Mb + Vb):
+        assert torch.equal(x, y)
+    with pytest.raises(ValueError, match="schedule"):
+        plan.update(steps=3)
